@@ -1,0 +1,33 @@
+"""Oracle: analytic FLOP count of a per-tile and a shared layer.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).
+
+[TileShare] Tab. 1 and Tab. S7 report block FLOPs of partly or fully shared
+layers relative to per-tile layers; Tab. S6 notes that per-token work shrinks
+with the token count while attention is unchanged.  Counted here: the four
+linear layers (2 FLOPs per multiply-add) and the two attention contractions;
+norms, softmax, GELU and the blend are not counted.
+"""
+
+
+def linear_flops_per_row(d: int, f: int) -> int:
+    return 2 * (3 * d * d + d * d + 2 * d * f)
+
+
+def attention_flops(T: int, N: int, d: int) -> int:
+    return 4 * T * N * N * d
+
+
+def tiled_layer_flops(T: int, N: int, d: int, f: int) -> int:
+    return T * N * linear_flops_per_row(d, f) + attention_flops(T, N, d)
+
+
+def shared_layer_flops(U: int, T: int, N: int, d: int, f: int) -> int:
+    return (U + T) * linear_flops_per_row(d, f) + attention_flops(T, N, d)
+
+
+def stack_flop_ratio(U: int, T: int, N: int, d: int, f: int, L: int, k: int) -> float:
+    """FLOPs of TileShare-k over FLOPs of L per-tile layers."""
+    tiled = tiled_layer_flops(T, N, d, f)
+    shared = shared_layer_flops(U, T, N, d, f)
+    return (k * tiled + (L - k) * shared) / (L * tiled)

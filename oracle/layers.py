@@ -1,0 +1,248 @@
+"""Oracle: the per-tile layer, the shared layer and the TileShare-k stack.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).  float64 NumPy, no
+blocking, fusion or reordering beyond what the pages state.
+
+What the pages fix
+    * [TileShare] Tab. S1 (each operation of a block under TileShare):
+        - Norm1, QKV projection and QK-RMSNorm run once per token on the shared
+          state (exact: identical inputs give identical results);
+        - RoPE runs per tile on tile coordinates, as released;
+        - attention is dense and per tile, with the tile's own registers (here one
+          global token per tile) that attend only to their own tile; keys and
+          values come from the shared states;
+        - the blend of attention outputs of overlap tokens is the only
+          approximation and happens in every shared layer.
+    * [TileShare] Fig. 2: out-projection and MLP also run once per token; overlap
+      tokens are stored once but attended in every window covering them; their
+      attention outputs are blended with w-bar.
+    * [TileShare] abstract and Tab. 1: TileShare-k keeps the first k layers per
+      tile (each tile its own residual stream), the rest shared.
+    * [TileShare] Fig. 3b: the per-tile states can be merged into one state.
+
+Readings taken where the pages are silent (also listed in the design doc)
+    R4 block: pre-LN ViT block  x += W_o Attn(RoPE(QKnorm(W_qkv LN1(x)))) + b_o;
+       x += W_2 GELU(W_1 LN2(x) + b_1) + b_2; LayerNorm and QK-RMSNorm eps 1e-6
+       with learnable gain (and LN bias); exact erf GELU; attention scale
+       1/sqrt(hd), no mask.  QKV columns: [q | k | v], head h at h*hd.
+    R5 the global token is not rotated by RoPE.
+    R6 RoPE: the head dimension is split into consecutive blocks of
+       rope_dims = (D_f, D_y, D_x) channels for the three axes; inside a block of
+       D channels, channel j pairs with j + D/2 (j < D/2) and is rotated by angle
+       pos * base^(-2j/D), pos being the integer tile-local coordinate.
+    R7 the blend acts on the attention outputs, before the out-projection
+       (Fig. 2 says the attention outputs are blended).  Because w-bar sums to 1,
+       blending before or after the out-projection and residual is the same map.
+    R8 the transition at layer k merges the per-tile states with the same w-bar
+       (Fig. 3b); each global token keeps its own tile's state.
+"""
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+from scipy.special import erf
+
+from . import fp8 as _fp8
+
+
+@dataclass(frozen=True)
+class Model:
+    d: int
+    heads: int
+    mlp: int
+    rope_dims: tuple          # (D_f, D_y, D_x), sum = head dim, each even
+    eps_ln: float = 1e-6
+    eps_qk: float = 1e-6
+    rope_base: float = 10000.0
+    fp8: bool = False         # e4m3 GEMMs with per-channel / per-token scales
+
+    @property
+    def hd(self):
+        return self.d // self.heads
+
+
+# ---------------------------------------------------------------------------
+# elementary operations
+# ---------------------------------------------------------------------------
+
+def layer_norm(x, g, b, eps):
+    mu = x.mean(axis=-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps) * g + b
+
+
+def rms_norm(x, g, eps):
+    return x / np.sqrt((x * x).mean(axis=-1, keepdims=True) + eps) * g
+
+
+def gelu(x):
+    return 0.5 * x * (1.0 + erf(x / math.sqrt(2.0)))
+
+
+def rope(x, pos, m: Model):
+    """Rotate x [n, heads, hd] of rows at integer coordinates pos [n, 3] (R6)."""
+    out = x.copy()
+    off = 0
+    for axis, D in enumerate(m.rope_dims):
+        half = D // 2
+        for j in range(half):
+            theta = m.rope_base ** (-2.0 * j / D)
+            ang = pos[:, axis].astype(np.float64) * theta          # [n]
+            c = np.cos(ang)[:, None]
+            s = np.sin(ang)[:, None]
+            a = x[:, :, off + j]
+            b = x[:, :, off + j + half]
+            out[:, :, off + j] = a * c - b * s
+            out[:, :, off + j + half] = a * s + b * c
+        off += D
+    return out
+
+
+def linear(x, w, b, m: Model):
+    """x @ w.T + b; with m.fp8 the product is the e4m3 scaled GEMM of fp8.scaled_matmul."""
+    if m.fp8:
+        y = _fp8.scaled_matmul(x, w)
+    else:
+        y = x @ w.T
+    return y + b
+
+
+def attention(q, k, v):
+    """Dense softmax attention of one tile, all heads: q, k, v [n, heads, hd] -> [n, heads*hd]."""
+    n, h, hd = q.shape
+    s = np.einsum("qhc,khc->hqk", q, k) / math.sqrt(hd)
+    s = s - s.max(axis=-1, keepdims=True)
+    p = np.exp(s)
+    p = p / p.sum(axis=-1, keepdims=True)
+    o = np.einsum("hqk,khc->qhc", p, v)
+    return o.reshape(n, h * hd)
+
+
+# ---------------------------------------------------------------------------
+# the pieces of a block
+# ---------------------------------------------------------------------------
+
+def qkv_project(x, p, m: Model):
+    """Norm1, QKV projection and QK-RMSNorm of rows x [n, d] -> q, k, v [n, heads, hd]."""
+    n = x.shape[0]
+    h = layer_norm(x, p["ln1_g"], p["ln1_b"], m.eps_ln)
+    qkv = linear(h, p["w_qkv"], p["b_qkv"], m)
+    q = qkv[:, 0 * m.d:1 * m.d].reshape(n, m.heads, m.hd)
+    k = qkv[:, 1 * m.d:2 * m.d].reshape(n, m.heads, m.hd)
+    v = qkv[:, 2 * m.d:3 * m.d].reshape(n, m.heads, m.hd)
+    q = rms_norm(q, p["q_g"], m.eps_qk)
+    k = rms_norm(k, p["k_g"], m.eps_qk)
+    return q, k, v
+
+
+def tile_attention(q, k, v, slot_pos, m: Model):
+    """Attention of one tile: rows [global token, window slot 0..Nw-1].
+
+    RoPE on tile-local coordinates for the window rows only (R5, R6).
+    Returns the attention output [N, d] before the out-projection.
+    """
+    q = q.copy()
+    k = k.copy()
+    q[1:] = rope(q[1:], slot_pos, m)
+    k[1:] = rope(k[1:], slot_pos, m)
+    return attention(q, k, v)
+
+
+def mlp_residual(x, p, m: Model):
+    """x + W_2 GELU(W_1 LN2(x) + b_1) + b_2, once per row."""
+    h = layer_norm(x, p["ln2_g"], p["ln2_b"], m.eps_ln)
+    h = gelu(linear(h, p["w_1"], p["b_1"], m))
+    return x + linear(h, p["w_2"], p["b_2"], m)
+
+
+# ---------------------------------------------------------------------------
+# tile <-> token maps
+# ---------------------------------------------------------------------------
+
+def gather(S, plan):
+    """Per-tile copies X [T, N, d] of a shared state S [U + T, d]."""
+    T, N, U = plan.T, plan.N, plan.U
+    X = np.empty((T, N, S.shape[1]), dtype=S.dtype)
+    for t in range(T):
+        X[t, 0] = S[U + t]
+        X[t, 1:] = S[plan.tile_tok[t]]
+    return X
+
+
+def merge(P, plan):
+    """Blend per-tile rows P [T, N, d] into one row per token (Fig. 2, R8).
+
+    S[u] = sum over the tiles t covering u, in ascending t, of w-bar[t, u] *
+    P[t, slot of u]; S[U + t] = P[t, 0] (each global token keeps its tile's row).
+    """
+    T, N, U = plan.T, plan.N, plan.U
+    flat = P.reshape(T * N, -1)
+    S = np.zeros((U + T, P.shape[2]), dtype=np.float64)
+    for u in range(U):
+        for e in range(plan.tok_ptr[u], plan.tok_ptr[u + 1]):
+            S[u] += plan.tok_w[e] * flat[plan.tok_ent[e]]
+    for t in range(T):
+        S[U + t] = P[t, 0]
+    return S
+
+
+# ---------------------------------------------------------------------------
+# layers and the stack
+# ---------------------------------------------------------------------------
+
+def block_tiled(X, p, m: Model, plan):
+    """One released (per-tile) layer on per-tile states X [T, N, d] (Tab. S1, layer 0)."""
+    out = np.empty_like(X, dtype=np.float64)
+    for t in range(X.shape[0]):
+        x = X[t].astype(np.float64)
+        q, k, v = qkv_project(x, p, m)
+        o = tile_attention(q, k, v, plan.slot_pos, m)
+        x = x + linear(o, p["w_o"], p["b_o"], m)
+        out[t] = mlp_residual(x, p, m)
+    return out
+
+
+def shared_attention_outputs(S, p, m: Model, plan):
+    """Per-tile attention outputs O [T, N, d] of a shared layer on S [U + T, d].
+
+    Norm1/QKV/QK-norm once per token; then, per tile, the rows of the tile's global
+    token and window tokens are taken from the shared q, k, v (Tab. S1).
+    """
+    U, T, N = plan.U, plan.T, plan.N
+    q, k, v = qkv_project(S, p, m)
+    O = np.empty((T, N, m.d), dtype=np.float64)
+    for t in range(T):
+        rows = np.concatenate([[U + t], plan.tile_tok[t]])
+        O[t] = tile_attention(q[rows], k[rows], v[rows], plan.slot_pos, m)
+    return O
+
+
+def block_shared(S, p, m: Model, plan):
+    """One TileShare shared layer on the shared state S [U + T, d] (Fig. 2, Tab. S1)."""
+    S = S.astype(np.float64)
+    O = shared_attention_outputs(S, p, m, plan)
+    A = merge(O, plan)
+    S = S + linear(A, p["w_o"], p["b_o"], m)
+    return mlp_residual(S, p, m)
+
+
+def decode_stack(S0, G0, layers, m: Model, plan, k: int):
+    """TileShare-k: layers 0..k-1 per tile, the rest shared; returns the U token rows.
+
+    S0 [U, d] are the grid tokens entering layer 0, G0 [T, d] the global tokens.
+    With k = L this is overlapping tiled decoding with the tiles blended by w-bar at
+    the end (abstract; R8).
+    """
+    L = len(layers)
+    if not 0 <= k <= L:
+        raise ValueError("k must lie in [0, L]")
+    S = np.concatenate([np.asarray(S0, np.float64), np.asarray(G0, np.float64)], axis=0)
+    if k > 0:
+        X = gather(S, plan)
+        for li in range(k):
+            X = block_tiled(X, layers[li], m, plan)
+        S = merge(X, plan)
+    for li in range(k, L):
+        S = block_shared(S, layers[li], m, plan)
+    return S[: plan.U]
