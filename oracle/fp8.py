@@ -53,11 +53,20 @@ def round_e4m3_scalar(x: float) -> float:
     return math.copysign(lo * quantum, x)
 
 
-_round_vec = np.vectorize(round_e4m3_scalar, otypes=[np.float64])
-
-
 def round_e4m3(x: np.ndarray) -> np.ndarray:
-    return _round_vec(np.asarray(x, dtype=np.float64))
+    """Array form of round_e4m3_scalar (same steps, elementwise, exact in float64)."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    _, E = np.frexp(a)
+    quantum = np.where(a < 2.0 ** -6, 2.0 ** -9, np.ldexp(1.0, E - 4))
+    q = a / quantum
+    lo = np.floor(q)
+    rem = q - lo
+    up = (rem > 0.5) | ((rem == 0.5) & (np.mod(lo, 2) == 1))
+    r = (lo + up) * quantum
+    r = np.where(a >= E4M3_MAX, E4M3_MAX, r)
+    r = np.where(np.isnan(x), x, np.copysign(r, x))
+    return r
 
 
 def row_scales(x: np.ndarray) -> np.ndarray:

@@ -1,0 +1,335 @@
+// rowops.cuh -- memory-bound row kernels: LayerNorm, the w-bar blend / merge, the
+// tile gather of the stack input, per-row e4m3 quantisation, and the fp32 path's
+// QK-RMSNorm + RoPE.  One warp per row, 16-byte vector accesses, fp32 arithmetic.
+#pragma once
+
+#include "common.cuh"
+
+namespace ts {
+
+// ---------------------------------------------------------------------------
+// element access: bf16 or fp32 rows, 16-byte vectors (8 bf16 / 4 fp32)
+// ---------------------------------------------------------------------------
+template <typename T>
+struct Vec;
+template <>
+struct Vec<bf16> {
+  static constexpr int E = 8;
+  __device__ static void load(const bf16* p, float* f) { bf16x8_to_f32(*reinterpret_cast<const uint4*>(p), f); }
+  __device__ static void store(bf16* p, const float* f) { *reinterpret_cast<uint4*>(p) = f32_to_bf16x8(f); }
+};
+template <>
+struct Vec<float> {
+  static constexpr int E = 4;
+  __device__ static void load(const float* p, float* f) {
+    const float4 v = *reinterpret_cast<const float4*>(p);
+    f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+  }
+  __device__ static void store(float* p, const float* f) { *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]); }
+};
+
+// Write one row held by a warp (NV vectors of E elements per lane, lane-strided) in
+// the output format: T (bf16 / fp32), or e4m3 bytes + per-row scale absmax / 448.
+template <typename T, int NV, bool Q8>
+__device__ __forceinline__ void store_row(const float (&v)[NV][Vec<T>::E], int lane, T* out, uint8_t* q8,
+                                          float* qscale, size_t row, int d) {
+  constexpr int E = Vec<T>::E;
+  if (!Q8) {
+#pragma unroll
+    for (int i = 0; i < NV; ++i) Vec<T>::store(out + row * d + (i * 32 + lane) * E, v[i]);
+  } else {
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+#pragma unroll
+      for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(v[i][e]));
+    amax = warp_max(amax);
+    const float s = amax > 0.f ? amax / 448.0f : 1.0f;
+    if (lane == 0) qscale[row] = s;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      uint16_t pk[E / 2];
+#pragma unroll
+      for (int e = 0; e < E; e += 2) pk[e / 2] = f32x2_to_e4m3x2(v[i][e] / s, v[i][e + 1] / s);
+      uint8_t* dst = q8 + row * d + (i * 32 + lane) * E;
+      if (E == 8)
+        *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(pk);
+      else
+        *reinterpret_cast<uint32_t*>(dst) = *reinterpret_cast<const uint32_t*>(pk);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// LayerNorm (pre-LN block, [TileShare] Tab. S1 Norm1 / Norm2): population variance,
+// two passes over the row held in registers.  NV = d / (32 * E) vectors per lane.
+// ---------------------------------------------------------------------------
+template <typename T, int NV, bool Q8>
+__global__ void __launch_bounds__(256) layernorm_kernel(const T* __restrict__ x, int rows, int d,
+                                                        const float* __restrict__ g, const float* __restrict__ b,
+                                                        float eps, T* __restrict__ y, uint8_t* __restrict__ q8,
+                                                        float* __restrict__ qscale) {
+  constexpr int E = Vec<T>::E;
+  const int lane = threadIdx.x & 31;
+  const size_t row = static_cast<size_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= static_cast<size_t>(rows)) return;
+  float v[NV][E];
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    Vec<T>::load(x + row * d + (i * 32 + lane) * E, v[i]);
+#pragma unroll
+    for (int e = 0; e < E; ++e) s += v[i][e];
+  }
+  const float mean = warp_sum(s) / d;
+  float q = 0.f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i)
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float c = v[i][e] - mean;
+      q = fmaf(c, c, q);
+    }
+  const float rstd = rsqrtf(warp_sum(q) / d + eps);
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c0 = (i * 32 + lane) * E;
+#pragma unroll
+    for (int e = 0; e < E; ++e) v[i][e] = (v[i][e] - mean) * rstd * __ldg(g + c0 + e) + __ldg(b + c0 + e);
+  }
+  store_row<T, NV, Q8>(v, lane, y, q8, qscale, row, d);
+}
+
+// generic fallback: any d (one warp per row, scalar, two passes over global memory)
+template <typename T>
+__global__ void __launch_bounds__(256) layernorm_generic_kernel(const T* __restrict__ x, int rows, int d,
+                                                                const float* __restrict__ g,
+                                                                const float* __restrict__ b, float eps,
+                                                                T* __restrict__ y) {
+  const int lane = threadIdx.x & 31;
+  const size_t row = static_cast<size_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= static_cast<size_t>(rows)) return;
+  const T* xr = x + row * d;
+  float s = 0.f;
+  for (int c = lane; c < d; c += 32) s += static_cast<float>(xr[c]);
+  const float mean = warp_sum(s) / d;
+  float q = 0.f;
+  for (int c = lane; c < d; c += 32) {
+    const float t = static_cast<float>(xr[c]) - mean;
+    q = fmaf(t, t, q);
+  }
+  const float rstd = rsqrtf(warp_sum(q) / d + eps);
+  for (int c = lane; c < d; c += 32) y[row * d + c] = static_cast<T>((static_cast<float>(xr[c]) - mean) * rstd * g[c] + b[c]);
+}
+
+// ---------------------------------------------------------------------------
+// Blend / merge ([TileShare] Fig. 2: overlap tokens' attention outputs blended with
+// w-bar; Fig. 3b: per-tile states merged).  Row u < U: fp32 sum over the token's
+// CSR entries in ascending tile order of wbar * P[ent]; row U + t: P[t*N].  One
+// warp writes each output row once; no atomics, so the result is deterministic.
+// ---------------------------------------------------------------------------
+template <typename T, int NV, bool Q8>
+__global__ void __launch_bounds__(256) merge_kernel(const T* __restrict__ P, int rows, int U, int N, int d,
+                                                    const int* __restrict__ tok_ptr, const int* __restrict__ tok_ent,
+                                                    const float* __restrict__ wbar, T* __restrict__ A,
+                                                    uint8_t* __restrict__ q8, float* __restrict__ qscale) {
+  constexpr int E = Vec<T>::E;
+  const int lane = threadIdx.x & 31;
+  const size_t row = static_cast<size_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= static_cast<size_t>(rows)) return;
+  float v[NV][E];
+  if (row < static_cast<size_t>(U)) {
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+#pragma unroll
+      for (int e = 0; e < E; ++e) v[i][e] = 0.f;
+    const int e0 = __ldg(tok_ptr + row), e1 = __ldg(tok_ptr + row + 1);
+    for (int e = e0; e < e1; ++e) {
+      const float w = __ldg(wbar + e);
+      const T* src = P + static_cast<size_t>(__ldg(tok_ent + e)) * d;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        float f[E];
+        Vec<T>::load(src + (i * 32 + lane) * E, f);
+#pragma unroll
+        for (int k = 0; k < E; ++k) v[i][k] = fmaf(w, f[k], v[i][k]);
+      }
+    }
+  } else {
+    const T* src = P + (row - U) * static_cast<size_t>(N) * d;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) Vec<T>::load(src + (i * 32 + lane) * E, v[i]);
+  }
+  store_row<T, NV, Q8>(v, lane, A, q8, qscale, row, d);
+}
+
+// generic fallback of the blend for any d (scalar)
+template <typename T>
+__global__ void __launch_bounds__(256) merge_generic_kernel(const T* __restrict__ P, int rows, int U, int N, int d,
+                                                            const int* __restrict__ tok_ptr,
+                                                            const int* __restrict__ tok_ent,
+                                                            const float* __restrict__ wbar, T* __restrict__ A) {
+  const int lane = threadIdx.x & 31;
+  const size_t row = static_cast<size_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= static_cast<size_t>(rows)) return;
+  for (int c = lane; c < d; c += 32) {
+    float acc = 0.f;
+    if (row < static_cast<size_t>(U)) {
+      for (int e = tok_ptr[row]; e < tok_ptr[row + 1]; ++e)
+        acc = fmaf(wbar[e], static_cast<float>(P[static_cast<size_t>(tok_ent[e]) * d + c]), acc);
+    } else {
+      acc = static_cast<float>(P[(row - U) * static_cast<size_t>(N) * d + c]);
+    }
+    A[row * d + c] = static_cast<T>(acc);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Stack input: per-tile copies X[t*N + s] of grid tokens S0 and global tokens G0
+// (row map of the shared layout: < U grid token, >= U global token).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint8_t* __restrict__ S0,
+                                                          const uint8_t* __restrict__ G0,
+                                                          const int* __restrict__ rowmap, int nrows, int U,
+                                                          size_t row_bytes, uint8_t* __restrict__ X) {
+  const int lane = threadIdx.x & 31;
+  const size_t r = static_cast<size_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= static_cast<size_t>(nrows)) return;
+  const int src = __ldg(rowmap + r);
+  const uint8_t* s = src < U ? S0 + static_cast<size_t>(src) * row_bytes : G0 + static_cast<size_t>(src - U) * row_bytes;
+  for (size_t c = lane * 16; c < row_bytes; c += 32 * 16)
+    *reinterpret_cast<uint4*>(X + r * row_bytes + c) = *reinterpret_cast<const uint4*>(s + c);
+}
+
+// ---------------------------------------------------------------------------
+// Per-row e4m3 quantisation of a bf16 matrix: scale = absmax / 448 (1 if zero),
+// q = e4m3(x / scale), nearest-even, saturating.  cols % 8 == 0.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) quantize_rows_kernel(const bf16* __restrict__ x, int rows, int cols,
+                                                            uint8_t* __restrict__ q, float* __restrict__ scale) {
+  const int lane = threadIdx.x & 31;
+  const size_t row = static_cast<size_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= static_cast<size_t>(rows)) return;
+  const bf16* xr = x + row * cols;
+  float amax = 0.f;
+  for (int c = lane * 8; c < cols; c += 256) {
+    float f[8];
+    bf16x8_to_f32(*reinterpret_cast<const uint4*>(xr + c), f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+  }
+  amax = warp_max(amax);
+  const float s = amax > 0.f ? amax / 448.0f : 1.0f;
+  if (lane == 0) scale[row] = s;
+  for (int c = lane * 8; c < cols; c += 256) {
+    float f[8];
+    bf16x8_to_f32(*reinterpret_cast<const uint4*>(xr + c), f);
+    uint16_t pk[4];
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) pk[e / 2] = f32x2_to_e4m3x2(f[e] / s, f[e + 1] / s);
+    *reinterpret_cast<uint2*>(q + row * cols + c) = *reinterpret_cast<const uint2*>(pk);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// fp32 path: QK-RMSNorm (gain) then RoPE at the row's coordinates, in place on the
+// q and k parts of qkv [rows, 3d].  One thread per (row, head, q|k).
+// ---------------------------------------------------------------------------
+struct RopeF32 {
+  int dims[3];
+  float th_hi[32];
+  float th_lo[32];
+};
+
+__global__ void __launch_bounds__(128) qk_norm_rope_f32_kernel(float* __restrict__ qkv, int rows, int d, int heads,
+                                                               const float* __restrict__ q_g,
+                                                               const float* __restrict__ k_g, float eps,
+                                                               const int4* __restrict__ pos, const RopeF32 rope) {
+  const int hd = d / heads;
+  const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<size_t>(rows) * heads * 2) return;
+  const int part = static_cast<int>(idx % 2);
+  const int h = static_cast<int>((idx / 2) % heads);
+  const size_t row = idx / (2 * heads);
+  float* v = qkv + row * 3 * d + part * d + h * hd;
+  const float* g = part ? k_g : q_g;
+  float x[64];
+  float ss = 0.f;
+  for (int c = 0; c < hd; ++c) {
+    x[c] = v[c];
+    ss = fmaf(x[c], x[c], ss);
+  }
+  const float r = rsqrtf(ss / hd + eps);
+  for (int c = 0; c < hd; ++c) x[c] = x[c] * r * g[c];
+  const int4 p4 = pos[row];
+  const float p[3] = {static_cast<float>(p4.x), static_cast<float>(p4.y), static_cast<float>(p4.z)};
+  int off = 0, pair = 0;
+  for (int a = 0; a < 3; ++a) {
+    const int half = rope.dims[a] / 2;
+    for (int j = 0; j < half; ++j) {
+      float c, s;
+      rope_cos_sin(p[a], rope.th_hi[pair + j], rope.th_lo[pair + j], c, s);
+      const float xa = x[off + j], xb = x[off + j + half];
+      x[off + j] = xa * c - xb * s;
+      x[off + j + half] = xa * s + xb * c;
+    }
+    off += rope.dims[a];
+    pair += half;
+  }
+  for (int c = 0; c < hd; ++c) v[c] = x[c];
+}
+
+// ---------------------------------------------------------------------------
+// fp32 path: SIMT GEMM Y = A W^T (+ b) with the same epilogues as the tensor-core
+// kernel (bias, GELU, residual).  64 x 64 tiles, K slices of 16, 4 x 4 per thread.
+// ---------------------------------------------------------------------------
+template <int EPI>
+__global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__ A, const float* __restrict__ W,
+                                                       const float* __restrict__ bias, float* __restrict__ Y, int M,
+                                                       int N, int K) {
+  __shared__ float sA[16][64 + 4];
+  __shared__ float sW[16][64 + 4];
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  const int m0 = blockIdx.x * 64, n0 = blockIdx.y * 64;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    for (int i = threadIdx.x; i < 64 * 16; i += 256) {
+      const int r = i / 16, c = i % 16;
+      const int gm = m0 + r, gn = n0 + r, gk = k0 + c;
+      sA[c][r] = (gm < M && gk < K) ? A[static_cast<size_t>(gm) * K + gk] : 0.f;
+      sW[c][r] = (gn < N && gk < K) ? W[static_cast<size_t>(gn) * K + gk] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[4], w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        a[i] = sA[kk][ty * 4 + i];
+        w[i] = sW[kk][tx * 4 + i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], w[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = m0 + ty * 4 + i;
+    if (m >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx * 4 + j;
+      if (n >= N) continue;
+      float v = acc[i][j] + (bias ? bias[n] : 0.f);
+      float* y = Y + static_cast<size_t>(m) * N + n;
+      if (EPI == 1) v = gelu_erf(v);
+      if (EPI == 2) v += *y;
+      *y = v;
+    }
+  }
+}
+
+}  // namespace ts

@@ -1,0 +1,814 @@
+// tileshare.cu -- libtileshare.so: the C ABI declared in include/tileshare.h and
+// include/tileshare_ops.h, the host-side launchers and the layer orchestration.
+//
+// One translation unit: the kernels live in the included .cuh files.
+//
+// [TileShare] = "TileShare: Training-Free Acceleration of Overlapping Tiled ViT
+// Decoding" (arXiv 2610.32233).  Data flow of one shared layer (Fig. 2, Tab. S1):
+//   S --LN1--> xn --QKV GEMM + QK-RMSNorm + RoPE--> qkv --gathered attention--> O
+//     --w-bar blend--> A --out-proj GEMM (+= S)--> S --LN2--> xn --up GEMM + GELU--> h
+//     --down GEMM (+= S)--> S
+// A per-tile layer is the same on X [T*N, d] with contiguous rows and no blend.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "../../include/tileshare.h"
+#include "../../include/tileshare_ops.h"
+#include "attention.cuh"
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "plan.inl"
+#include "rowops.cuh"
+
+using ts::bf16;
+
+// ============================================================================
+// errors
+// ============================================================================
+static thread_local std::string g_last_error;
+
+static ts_status fail(ts_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+static ts_status fail(ts_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+#define TS_CUDA_CHECK(expr)                                                                        \
+  do {                                                                                             \
+    cudaError_t e_ = (expr);                                                                       \
+    if (e_ != cudaSuccess) return fail(TS_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(e_));       \
+  } while (0)
+
+#define TS_TRY(expr)               \
+  do {                             \
+    ts_status s_ = (expr);         \
+    if (s_ != TS_OK) return s_;    \
+  } while (0)
+
+static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static ts_status launched(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(TS_ERR_CUDA, "launch of %s failed: %s", what, cudaGetErrorString(e));
+  return TS_OK;
+}
+
+// ============================================================================
+// tensor maps (driver entry point fetched through the runtime, no -lcuda)
+// ============================================================================
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static ts_status encode_fn(EncodeTiledFn* out) {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p)
+      return fail(TS_ERR_CUDA, "cuTensorMapEncodeTiled not available");
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  *out = fn;
+  return TS_OK;
+}
+
+// 2-D K-major operand [rows, K] (element size esz), box of 128 bytes x box_rows,
+// 128-byte swizzle, out-of-bounds rows read as zero.
+static ts_status make_tmap(CUtensorMap* map, const void* base, int rows, int K, int esz, int box_rows) {
+  EncodeTiledFn enc;
+  TS_TRY(encode_fn(&enc));
+  const CUtensorMapDataType dt = esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * esz};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esz), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return TS_OK;
+}
+
+// ============================================================================
+// model checks and RoPE tables
+// ============================================================================
+static int esize(ts_dtype dt) { return dt == TS_F32 ? 4 : 2; }
+
+static ts_status check_model(const ts_model_desc* m) {
+  if (!m) return fail(TS_ERR_INVALID_ARG, "model is NULL");
+  if (m->d <= 0 || m->heads <= 0 || m->mlp <= 0 || m->d % m->heads)
+    return fail(TS_ERR_INVALID_ARG, "bad model sizes d=%d heads=%d mlp=%d", m->d, m->heads, m->mlp);
+  if (m->dtype != TS_F32 && m->dtype != TS_BF16 && m->dtype != TS_FP8_E4M3)
+    return fail(TS_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(m->dtype));
+  const int hd = m->d / m->heads;
+  int sum = 0;
+  for (int a = 0; a < 3; ++a) {
+    if (m->rope_dims[a] < 0 || (m->rope_dims[a] & 1)) return fail(TS_ERR_INVALID_ARG, "rope_dims must be even and >= 0");
+    sum += m->rope_dims[a];
+  }
+  if (sum != hd) return fail(TS_ERR_INVALID_ARG, "rope_dims sum %d != head dim %d", sum, hd);
+  if (!(m->eps_ln > 0.f) || !(m->eps_qk > 0.f) || !(m->rope_base > 0.f))
+    return fail(TS_ERR_INVALID_ARG, "eps and rope_base must be positive");
+  if (m->dtype == TS_F32) {
+    if (hd != 16 && hd != 32 && hd != 64) return fail(TS_ERR_UNSUPPORTED, "fp32 path supports head dim 16, 32, 64");
+    if (m->d % 4 || m->mlp % 4) return fail(TS_ERR_UNSUPPORTED, "fp32 path needs d, mlp multiples of 4");
+  } else {
+    if (hd != 64) return fail(TS_ERR_UNSUPPORTED, "bf16/e4m3 path supports head dim 64 only");
+    if (m->d % 256 || m->d > 2048) return fail(TS_ERR_UNSUPPORTED, "bf16/e4m3 path needs d %% 256 == 0, d <= 2048");
+    if (m->mlp % 256) return fail(TS_ERR_UNSUPPORTED, "bf16/e4m3 path needs mlp %% 256 == 0");
+    const int* r = m->rope_dims;
+    const bool s2 = r[0] == 0 && r[1] == 32 && r[2] == 32;
+    const bool s3 = r[0] == 16 && r[1] == 24 && r[2] == 24;
+    if (!s2 && !s3) return fail(TS_ERR_UNSUPPORTED, "bf16/e4m3 path supports rope_dims (0,32,32) or (16,24,24)");
+  }
+  return TS_OK;
+}
+
+template <typename Tab>
+static void fill_theta(const ts_model_desc* m, Tab* hi, Tab* lo) {
+  int pair = 0;
+  for (int a = 0; a < 3; ++a) {
+    const int D = m->rope_dims[a];
+    for (int j = 0; j < D / 2; ++j, ++pair) {
+      const double th = std::pow(static_cast<double>(m->rope_base), -2.0 * j / D);
+      hi[pair] = static_cast<float>(th);
+      lo[pair] = static_cast<float>(th - static_cast<double>(hi[pair]));
+    }
+  }
+}
+
+static ts_status check_plan(ts_plan_t p) {
+  if (!p) return fail(TS_ERR_INVALID_ARG, "plan is NULL");
+  int dev = -1;
+  TS_CUDA_CHECK(cudaGetDevice(&dev));
+  if (dev != p->device) return fail(TS_ERR_INVALID_ARG, "current device %d differs from the plan's device %d", dev, p->device);
+  return TS_OK;
+}
+
+static ts_status check_weights(const ts_model_desc* m, const ts_layer_weights* w) {
+  if (!w) return fail(TS_ERR_INVALID_ARG, "weights are NULL");
+  const void* ptrs[] = {w->ln1_g, w->ln1_b, w->w_qkv, w->b_qkv, w->q_g, w->k_g, w->w_o, w->b_o,
+                        w->ln2_g, w->ln2_b, w->w_1,   w->b_1,   w->w_2, w->b_2};
+  for (const void* p : ptrs) {
+    if (!p) return fail(TS_ERR_INVALID_ARG, "a weight pointer is NULL");
+    if (!aligned16(p)) return fail(TS_ERR_INVALID_ARG, "weight pointers must be 16-byte aligned");
+  }
+  if (m->dtype == TS_FP8_E4M3) {
+    const void* s[] = {w->s_qkv, w->s_o, w->s_1, w->s_2};
+    for (const void* p : s)
+      if (!p || !aligned16(p)) return fail(TS_ERR_INVALID_ARG, "e4m3 weights need 16-byte aligned scales s_*");
+  }
+  return TS_OK;
+}
+
+// ============================================================================
+// workspace layout
+// ============================================================================
+struct Workspace {
+  void* xn;      // [Mx, d]   normalised rows
+  void* qkv;     // [Mx, 3d]
+  void* o;       // [T*N, d]  attention output
+  void* a;       // [U+T, d]  blended attention output
+  void* h;       // [Mx, f]   MLP hidden
+  uint8_t* q8;   // [Mx, max(d, f)] e4m3 GEMM operand
+  float* qs;     // [Mx]      its per-row scales
+  void* X;       // [T*N, d]  per-tile state (stack)
+  void* S;       // [U+T, d]  shared state (stack)
+  size_t bytes;
+};
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static Workspace layout(const ts_plan_s* p, const ts_model_desc* m, bool stack, char* base) {
+  const size_t Mt = static_cast<size_t>(p->T) * p->N, Ms = static_cast<size_t>(p->U) + p->T;
+  const size_t Mx = std::max(Mt, Ms);
+  const size_t e = esize(m->dtype), d = m->d, f = m->mlp;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* r = base ? base + off : nullptr;
+    off += align256(bytes);
+    return r;
+  };
+  Workspace w{};
+  w.xn = take(Mx * d * e);
+  w.qkv = take(Mx * 3 * d * e);
+  w.o = take(Mt * d * e);
+  w.a = take(Ms * d * e);
+  w.h = take(Mx * f * e);
+  if (m->dtype == TS_FP8_E4M3) {
+    w.q8 = reinterpret_cast<uint8_t*>(take(Mx * std::max(d, f)));
+    w.qs = reinterpret_cast<float*>(take(Mx * 4));
+  }
+  if (stack) {
+    w.X = take(Mt * d * e);
+    w.S = take(Ms * d * e);
+  }
+  w.bytes = off;
+  return w;
+}
+
+// ============================================================================
+// launchers
+// ============================================================================
+static inline unsigned rows_grid(size_t rows) { return static_cast<unsigned>((rows + 7) / 8); }
+
+template <typename T, bool Q8>
+static ts_status launch_layernorm_vec(const void* x, int rows, int d, const float* g, const float* b, float eps,
+                                      void* y, uint8_t* q8, float* qs, cudaStream_t st) {
+  constexpr int E = ts::Vec<T>::E;
+  const int nv = d / (32 * E);
+  const T* xx = static_cast<const T*>(x);
+  T* yy = static_cast<T*>(y);
+#define TS_LN_CASE(NV) \
+  case NV: ts::layernorm_kernel<T, NV, Q8><<<rows_grid(rows), 256, 0, st>>>(xx, rows, d, g, b, eps, yy, q8, qs); break;
+  switch (nv) {
+    TS_LN_CASE(1) TS_LN_CASE(2) TS_LN_CASE(3) TS_LN_CASE(4) TS_LN_CASE(5) TS_LN_CASE(6) TS_LN_CASE(7) TS_LN_CASE(8)
+    default: return fail(TS_ERR_UNSUPPORTED, "layernorm width %d", d);
+  }
+#undef TS_LN_CASE
+  return launched("layernorm");
+}
+
+// y = LN(x); for e4m3 writes q8/qs instead of y.
+static ts_status run_layernorm(const ts_model_desc* m, const void* x, int rows, const float* g, const float* b,
+                               void* y, uint8_t* q8, float* qs, cudaStream_t st) {
+  if (rows == 0) return TS_OK;
+  const int d = m->d;
+  if (m->dtype == TS_F32) {
+    if (d % 128 == 0 && d <= 1024) return launch_layernorm_vec<float, false>(x, rows, d, g, b, m->eps_ln, y, nullptr, nullptr, st);
+    ts::layernorm_generic_kernel<float><<<rows_grid(rows), 256, 0, st>>>(static_cast<const float*>(x), rows, d, g, b,
+                                                                        m->eps_ln, static_cast<float*>(y));
+    return launched("layernorm_generic");
+  }
+  if (q8) return launch_layernorm_vec<bf16, true>(x, rows, d, g, b, m->eps_ln, nullptr, q8, qs, st);
+  return launch_layernorm_vec<bf16, false>(x, rows, d, g, b, m->eps_ln, y, nullptr, nullptr, st);
+}
+
+template <typename T, bool Q8>
+static ts_status launch_merge_vec(const ts_plan_s* p, const void* P, int rows, int d, void* A, uint8_t* q8,
+                                  float* qs, cudaStream_t st) {
+  constexpr int E = ts::Vec<T>::E;
+  const int nv = d / (32 * E);
+  const T* pp = static_cast<const T*>(P);
+  T* aa = static_cast<T*>(A);
+#define TS_MG_CASE(NV)                                                                                    \
+  case NV:                                                                                                \
+    ts::merge_kernel<T, NV, Q8><<<rows_grid(rows), 256, 0, st>>>(pp, rows, p->U, p->N, d, p->d_tok_ptr,  \
+                                                                 p->d_tok_ent, p->d_wbar, aa, q8, qs);    \
+    break;
+  switch (nv) {
+    TS_MG_CASE(1) TS_MG_CASE(2) TS_MG_CASE(3) TS_MG_CASE(4) TS_MG_CASE(5) TS_MG_CASE(6) TS_MG_CASE(7) TS_MG_CASE(8)
+    default: return fail(TS_ERR_UNSUPPORTED, "merge width %d", d);
+  }
+#undef TS_MG_CASE
+  return launched("merge");
+}
+
+static ts_status run_merge(const ts_plan_s* p, const ts_model_desc* m, const void* P, int rows, void* A, uint8_t* q8,
+                           float* qs, cudaStream_t st) {
+  if (rows == 0) return TS_OK;
+  const int d = m->d;
+  if (m->dtype == TS_F32) {
+    if (d % 128 == 0 && d <= 1024) return launch_merge_vec<float, false>(p, P, rows, d, A, nullptr, nullptr, st);
+    ts::merge_generic_kernel<float><<<rows_grid(rows), 256, 0, st>>>(static_cast<const float*>(P), rows, p->U, p->N, d,
+                                                                    p->d_tok_ptr, p->d_tok_ent, p->d_wbar,
+                                                                    static_cast<float*>(A));
+    return launched("merge_generic");
+  }
+  if (q8) return launch_merge_vec<bf16, true>(p, P, rows, d, nullptr, q8, qs, st);
+  return launch_merge_vec<bf16, false>(p, P, rows, d, A, nullptr, nullptr, st);
+}
+
+static ts_status run_quantize(const void* x, int rows, int cols, uint8_t* q, float* s, cudaStream_t st) {
+  if (rows == 0) return TS_OK;
+  ts::quantize_rows_kernel<<<rows_grid(rows), 256, 0, st>>>(static_cast<const bf16*>(x), rows, cols, q, s);
+  return launched("quantize_rows");
+}
+
+// ---------------------------------------------------------------------------
+// tensor-core GEMM
+// ---------------------------------------------------------------------------
+static int g_num_sms = 0;
+
+static int num_sms() {
+  if (!g_num_sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_num_sms <= 0) g_num_sms = 148;
+  }
+  return g_num_sms;
+}
+
+template <int BN, int STAGES, int EPI, bool FP8, int R0, int R1, int R2>
+static ts_status launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, const ts::GemmArgs& args,
+                                cudaStream_t st) {
+  using SM = ts::GemmSmem<BN, STAGES>;
+  auto kern = ts::gemm_tc_kernel<BN, STAGES, EPI, FP8, R0, R1, R2>;
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    TS_CUDA_CHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::LAUNCH_BYTES));
+    configured[dev] = 1;
+  }
+  dim3 grid((args.M + 127) / 128, args.N / BN);
+  kern<<<grid, 192, SM::LAUNCH_BYTES, st>>>(ta, tb, args);
+  return launched("gemm_tc");
+}
+
+template <int EPI, bool FP8, int R0, int R1, int R2>
+static ts_status dispatch_gemm_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const ts::GemmArgs& args,
+                                  cudaStream_t st) {
+  switch (bn) {
+    case 256: return launch_gemm_tc<256, 4, EPI, FP8, R0, R1, R2>(ta, tb, args, st);
+    case 128: return launch_gemm_tc<128, 6, EPI, FP8, R0, R1, R2>(ta, tb, args, st);
+    default: return launch_gemm_tc<64, 8, EPI, FP8, R0, R1, R2>(ta, tb, args, st);
+  }
+}
+
+// Output tile width: the widest of 256/128/64 dividing N that still gives at
+// least one CTA per SM; else the narrowest (most CTAs).
+static int pick_bn(int M, int N) {
+  const int mt = (M + 127) / 128;
+  const int sms = num_sms();
+  for (int bn : {256, 128, 64})
+    if (N % bn == 0 && mt * (N / bn) >= sms) return bn;
+  return 64;
+}
+
+// Y[M, N] = A[M, K] W[N, K]^T with epilogue; A bf16 (or e4m3 + a_scale), W bf16 (or e4m3 + w_scale).
+static ts_status run_gemm_tc(const ts_model_desc* m, int epi, const void* A, const float* a_scale, const void* W,
+                             const float* w_scale, int M, int N, int K, const float* bias, bf16* out,
+                             const ts_layer_weights* qk, const int* pos, cudaStream_t st) {
+  if (M == 0) return TS_OK;
+  const bool fp8 = m->dtype == TS_FP8_E4M3;
+  if (K % (fp8 ? 128 : 64) || N % 64) return fail(TS_ERR_UNSUPPORTED, "GEMM sizes K=%d N=%d not tiled", K, N);
+  const int bn = pick_bn(M, N);
+  CUtensorMap ta, tb;
+  TS_TRY(make_tmap(&ta, A, M, K, fp8 ? 1 : 2, 128));
+  TS_TRY(make_tmap(&tb, W, N, K, fp8 ? 1 : 2, bn));
+  ts::GemmArgs g{};
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.bias = bias;
+  g.out = out;
+  g.ldo = N;
+  g.a_scale = a_scale;
+  g.w_scale = w_scale;
+  g.d = m->d;
+  g.eps_qk = m->eps_qk;
+  if (epi == ts::EPI_QKV) {
+    g.q_g = qk->q_g;
+    g.k_g = qk->k_g;
+    g.pos = reinterpret_cast<const int4*>(pos);
+    fill_theta(m, g.theta.hi, g.theta.lo);
+  }
+  const bool r3 = m->rope_dims[0] == 16;
+#define TS_GEMM_EPI(E, R0, R1, R2) \
+  (fp8 ? dispatch_gemm_bn<E, true, R0, R1, R2>(bn, ta, tb, g, st) : dispatch_gemm_bn<E, false, R0, R1, R2>(bn, ta, tb, g, st))
+  switch (epi) {
+    case ts::EPI_BIAS: return TS_GEMM_EPI(ts::EPI_BIAS, 0, 32, 32);
+    case ts::EPI_GELU: return TS_GEMM_EPI(ts::EPI_GELU, 0, 32, 32);
+    case ts::EPI_RESID: return TS_GEMM_EPI(ts::EPI_RESID, 0, 32, 32);
+    case ts::EPI_QKV: return r3 ? TS_GEMM_EPI(ts::EPI_QKV, 16, 24, 24) : TS_GEMM_EPI(ts::EPI_QKV, 0, 32, 32);
+  }
+#undef TS_GEMM_EPI
+  return fail(TS_ERR_INVALID_ARG, "unknown epilogue");
+}
+
+// fp32 SIMT GEMM
+static ts_status run_gemm_f32(int epi, const float* A, const float* W, int M, int N, int K, const float* bias, float* Y,
+                              cudaStream_t st) {
+  if (M == 0) return TS_OK;
+  dim3 grid((M + 63) / 64, (N + 63) / 64);
+  switch (epi) {
+    case ts::EPI_GELU: ts::gemm_f32_kernel<1><<<grid, 256, 0, st>>>(A, W, bias, Y, M, N, K); break;
+    case ts::EPI_RESID: ts::gemm_f32_kernel<2><<<grid, 256, 0, st>>>(A, W, bias, Y, M, N, K); break;
+    default: ts::gemm_f32_kernel<0><<<grid, 256, 0, st>>>(A, W, bias, Y, M, N, K); break;
+  }
+  return launched("gemm_f32");
+}
+
+// ---------------------------------------------------------------------------
+// attention
+// ---------------------------------------------------------------------------
+static ts_status run_attention(const ts_plan_s* p, const ts_model_desc* m, bool shared, const void* qkv, void* O,
+                               cudaStream_t st) {
+  const int hd = m->d / m->heads;
+  ts::AttnArgs a{};
+  a.qkv = qkv;
+  a.rowmap = shared ? p->d_rowmap : nullptr;
+  a.O = O;
+  a.N = p->N;
+  a.Nw = p->Nw;
+  a.d = m->d;
+  a.heads = m->heads;
+  a.T = p->T;
+  a.scale = 1.0f / std::sqrt(static_cast<float>(hd));
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(hd)));
+  if (m->dtype == TS_F32) {
+    dim3 grid((p->N + 63) / 64, m->heads, p->T);
+    switch (hd) {
+      case 16: ts::attn_f32_kernel<16><<<grid, 64, 0, st>>>(a); break;
+      case 32: ts::attn_f32_kernel<32><<<grid, 64, 0, st>>>(a); break;
+      default: ts::attn_f32_kernel<64><<<grid, 64, 0, st>>>(a); break;
+    }
+    return launched("attn_f32");
+  }
+  const int nqb = (p->Nw + ts::kAttnBQ - 1) / ts::kAttnBQ;
+  dim3 grid(nqb + 1, m->heads, p->T);
+  ts::attn_bf16_kernel<<<grid, 128, ts::kAttnBf16SmemMax, st>>>(a);
+  return launched("attn_bf16");
+}
+
+// ---------------------------------------------------------------------------
+// QKV step: LN1 + QKV GEMM + QK-RMSNorm + RoPE
+// ---------------------------------------------------------------------------
+static ts_status run_qkv(const ts_plan_s* p, const ts_model_desc* m, const ts_layer_weights* w, bool shared,
+                         const void* state, void* qkv, const Workspace& ws, cudaStream_t st) {
+  const int rows = shared ? p->U + p->T : p->T * p->N;
+  const int* pos = shared ? p->d_pos_shared : p->d_pos_tiled;
+  const int d = m->d;
+  if (m->dtype == TS_F32) {
+    TS_TRY(run_layernorm(m, state, rows, w->ln1_g, w->ln1_b, ws.xn, nullptr, nullptr, st));
+    TS_TRY(run_gemm_f32(ts::EPI_BIAS, static_cast<const float*>(ws.xn), static_cast<const float*>(w->w_qkv), rows,
+                        3 * d, d, w->b_qkv, static_cast<float*>(qkv), st));
+    ts::RopeF32 r{};
+    for (int a = 0; a < 3; ++a) r.dims[a] = m->rope_dims[a];
+    fill_theta(m, r.th_hi, r.th_lo);
+    const size_t n = static_cast<size_t>(rows) * m->heads * 2;
+    ts::qk_norm_rope_f32_kernel<<<static_cast<unsigned>((n + 127) / 128), 128, 0, st>>>(
+        static_cast<float*>(qkv), rows, d, m->heads, w->q_g, w->k_g, m->eps_qk, reinterpret_cast<const int4*>(pos), r);
+    return launched("qk_norm_rope_f32");
+  }
+  if (m->dtype == TS_FP8_E4M3) {
+    TS_TRY(run_layernorm(m, state, rows, w->ln1_g, w->ln1_b, nullptr, ws.q8, ws.qs, st));
+    return run_gemm_tc(m, ts::EPI_QKV, ws.q8, ws.qs, w->w_qkv, w->s_qkv, rows, 3 * d, d, w->b_qkv,
+                       static_cast<bf16*>(qkv), w, pos, st);
+  }
+  TS_TRY(run_layernorm(m, state, rows, w->ln1_g, w->ln1_b, ws.xn, nullptr, nullptr, st));
+  return run_gemm_tc(m, ts::EPI_QKV, ws.xn, nullptr, w->w_qkv, nullptr, rows, 3 * d, d, w->b_qkv,
+                     static_cast<bf16*>(qkv), w, pos, st);
+}
+
+// out-proj (+= state) from attention/blend output `att` [rows, d]
+static ts_status run_out_proj(const ts_model_desc* m, const ts_layer_weights* w, const void* att, bool att_quantised,
+                              int rows, void* state, const Workspace& ws, cudaStream_t st) {
+  const int d = m->d;
+  if (m->dtype == TS_F32)
+    return run_gemm_f32(ts::EPI_RESID, static_cast<const float*>(att), static_cast<const float*>(w->w_o), rows, d, d,
+                        w->b_o, static_cast<float*>(state), st);
+  if (m->dtype == TS_FP8_E4M3) {
+    if (!att_quantised) TS_TRY(run_quantize(att, rows, d, ws.q8, ws.qs, st));
+    return run_gemm_tc(m, ts::EPI_RESID, ws.q8, ws.qs, w->w_o, w->s_o, rows, d, d, w->b_o, static_cast<bf16*>(state),
+                       nullptr, nullptr, st);
+  }
+  return run_gemm_tc(m, ts::EPI_RESID, att, nullptr, w->w_o, nullptr, rows, d, d, w->b_o, static_cast<bf16*>(state),
+                     nullptr, nullptr, st);
+}
+
+// state += W2 GELU(W1 LN2(state) + b1) + b2
+static ts_status run_mlp(const ts_model_desc* m, const ts_layer_weights* w, int rows, void* state, const Workspace& ws,
+                         cudaStream_t st) {
+  const int d = m->d, f = m->mlp;
+  if (m->dtype == TS_F32) {
+    TS_TRY(run_layernorm(m, state, rows, w->ln2_g, w->ln2_b, ws.xn, nullptr, nullptr, st));
+    TS_TRY(run_gemm_f32(ts::EPI_GELU, static_cast<const float*>(ws.xn), static_cast<const float*>(w->w_1), rows, f, d,
+                        w->b_1, static_cast<float*>(ws.h), st));
+    return run_gemm_f32(ts::EPI_RESID, static_cast<const float*>(ws.h), static_cast<const float*>(w->w_2), rows, d, f,
+                        w->b_2, static_cast<float*>(state), st);
+  }
+  if (m->dtype == TS_FP8_E4M3) {
+    TS_TRY(run_layernorm(m, state, rows, w->ln2_g, w->ln2_b, nullptr, ws.q8, ws.qs, st));
+    TS_TRY(run_gemm_tc(m, ts::EPI_GELU, ws.q8, ws.qs, w->w_1, w->s_1, rows, f, d, w->b_1, static_cast<bf16*>(ws.h),
+                       nullptr, nullptr, st));
+    TS_TRY(run_quantize(ws.h, rows, f, ws.q8, ws.qs, st));
+    return run_gemm_tc(m, ts::EPI_RESID, ws.q8, ws.qs, w->w_2, w->s_2, rows, d, f, w->b_2, static_cast<bf16*>(state),
+                       nullptr, nullptr, st);
+  }
+  TS_TRY(run_layernorm(m, state, rows, w->ln2_g, w->ln2_b, ws.xn, nullptr, nullptr, st));
+  TS_TRY(run_gemm_tc(m, ts::EPI_GELU, ws.xn, nullptr, w->w_1, nullptr, rows, f, d, w->b_1, static_cast<bf16*>(ws.h),
+                     nullptr, nullptr, st));
+  return run_gemm_tc(m, ts::EPI_RESID, ws.h, nullptr, w->w_2, nullptr, rows, d, f, w->b_2, static_cast<bf16*>(state),
+                     nullptr, nullptr, st);
+}
+
+// ============================================================================
+// layers
+// ============================================================================
+static ts_status layer_tiled(const ts_plan_s* p, const ts_model_desc* m, const ts_layer_weights* w, void* X,
+                             const Workspace& ws, cudaStream_t st) {
+  const int rows = p->T * p->N;
+  TS_TRY(run_qkv(p, m, w, false, X, ws.qkv, ws, st));
+  TS_TRY(run_attention(p, m, false, ws.qkv, ws.o, st));
+  TS_TRY(run_out_proj(m, w, ws.o, false, rows, X, ws, st));
+  return run_mlp(m, w, rows, X, ws, st);
+}
+
+static ts_status layer_shared(const ts_plan_s* p, const ts_model_desc* m, const ts_layer_weights* w, void* S,
+                              const Workspace& ws, cudaStream_t st) {
+  const int rows = p->U + p->T;
+  TS_TRY(run_qkv(p, m, w, true, S, ws.qkv, ws, st));
+  TS_TRY(run_attention(p, m, true, ws.qkv, ws.o, st));
+  const bool q = m->dtype == TS_FP8_E4M3;
+  TS_TRY(run_merge(p, m, ws.o, rows, q ? nullptr : ws.a, q ? ws.q8 : nullptr, q ? ws.qs : nullptr, st));
+  TS_TRY(run_out_proj(m, w, ws.a, q, rows, S, ws, st));
+  return run_mlp(m, w, rows, S, ws, st);
+}
+
+static ts_status check_ws(const ts_plan_s* p, const ts_model_desc* m, bool stack, void* ws, size_t ws_bytes,
+                          Workspace* out) {
+  const Workspace need = layout(p, m, stack, nullptr);
+  if (!ws) return fail(TS_ERR_INVALID_ARG, "workspace is NULL");
+  if (!aligned16(ws)) return fail(TS_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  if (ws_bytes < need.bytes) return fail(TS_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need.bytes);
+  *out = layout(p, m, stack, static_cast<char*>(ws));
+  return TS_OK;
+}
+
+// ============================================================================
+// C ABI
+// ============================================================================
+extern "C" {
+
+const char* ts_status_string(ts_status s) {
+  switch (s) {
+    case TS_OK: return "ok";
+    case TS_ERR_INVALID_ARG: return "invalid argument";
+    case TS_ERR_UNSUPPORTED: return "unsupported";
+    case TS_ERR_WORKSPACE: return "workspace too small";
+    case TS_ERR_CUDA: return "CUDA error";
+    case TS_ERR_DEVICE_CHECK: return "device-side check failed";
+    case TS_ERR_TIMEOUT: return "device-side wait timed out";
+    case TS_ERR_ALLOC: return "allocation failed";
+  }
+  return "unknown status";
+}
+
+const char* ts_last_error(void) { return g_last_error.c_str(); }
+
+static ts_status plan_build_host(const int grid[3], const int win[3], const int stride[3], ts_blend_rule rule,
+                                 ts_plan_s** out) {
+  if (!grid || !win || !stride || !out) return fail(TS_ERR_INVALID_ARG, "NULL argument");
+  *out = nullptr;
+  if (rule != TS_BLEND_LINEAR_RAMP) return fail(TS_ERR_UNSUPPORTED, "unknown blend rule %d", static_cast<int>(rule));
+  for (int a = 0; a < 3; ++a) {
+    if (grid[a] < 1 || win[a] < 1 || win[a] > grid[a] || stride[a] < 1 || stride[a] > win[a])
+      return fail(TS_ERR_INVALID_ARG, "axis %d: need 1 <= win <= grid and 1 <= stride <= win", a);
+  }
+  if (static_cast<double>(grid[0]) * grid[1] * grid[2] > (1 << 28)) return fail(TS_ERR_UNSUPPORTED, "grid too large");
+  if (static_cast<double>(win[0]) * win[1] * win[2] > (1 << 24)) return fail(TS_ERR_UNSUPPORTED, "window too large");
+  ts_plan_s* P = new (std::nothrow) ts_plan_s();
+  if (!P) return fail(TS_ERR_ALLOC, "host allocation failed");
+  for (int a = 0; a < 3; ++a) {
+    P->grid[a] = grid[a];
+    P->win[a] = win[a];
+    P->stride[a] = stride[a];
+  }
+  P->device = -1;
+  if (!tsplan::build(*P)) {
+    delete P;
+    return fail(TS_ERR_INVALID_ARG, "tiling leaves a token uncovered");
+  }
+  if (static_cast<double>(P->T) * P->N > 2.0e9) {
+    delete P;
+    return fail(TS_ERR_UNSUPPORTED, "too many tile rows");
+  }
+  *out = P;
+  return TS_OK;
+}
+
+ts_status ts_plan_create_host(const int grid[3], const int win[3], const int stride[3], ts_blend_rule rule,
+                              ts_plan_t* out) {
+  return plan_build_host(grid, win, stride, rule, out);
+}
+
+ts_status ts_plan_create(const int grid[3], const int win[3], const int stride[3], ts_blend_rule rule,
+                         ts_plan_t* out) {
+  ts_plan_s* P = nullptr;
+  TS_TRY(plan_build_host(grid, win, stride, rule, &P));
+  cudaError_t e = cudaGetDevice(&P->device);
+  auto upload = [&](auto** dst, const auto& vec) -> bool {
+    using E = typename std::decay<decltype(vec)>::type::value_type;
+    if (e != cudaSuccess) return false;
+    const size_t bytes = std::max<size_t>(vec.size(), 1) * sizeof(E);
+    e = cudaMalloc(reinterpret_cast<void**>(dst), bytes);
+    if (e != cudaSuccess) return false;
+    if (!vec.empty()) e = cudaMemcpy(*dst, vec.data(), vec.size() * sizeof(E), cudaMemcpyHostToDevice);
+    return e == cudaSuccess;
+  };
+  const bool ok = upload(&P->d_tok_ptr, P->tok_ptr) && upload(&P->d_tok_ent, P->tok_ent) &&
+                  upload(&P->d_wbar, P->wbar) && upload(&P->d_rowmap, P->rowmap) &&
+                  upload(&P->d_pos_shared, P->pos_shared) && upload(&P->d_pos_tiled, P->pos_tiled);
+  if (!ok) {
+    if (P->device < 0) P->device = 0;
+    ts_plan_destroy(P);
+    return fail(e == cudaErrorMemoryAllocation ? TS_ERR_ALLOC : TS_ERR_CUDA, "plan upload failed: %s",
+                cudaGetErrorString(e));
+  }
+  *out = P;
+  return TS_OK;
+}
+
+ts_status ts_plan_info(ts_plan_t p, ts_plan_desc* out) {
+  if (!p || !out) return fail(TS_ERR_INVALID_ARG, "NULL argument");
+  for (int a = 0; a < 3; ++a) {
+    out->grid[a] = p->grid[a];
+    out->win[a] = p->win[a];
+    out->stride[a] = p->stride[a];
+  }
+  out->T = p->T;
+  out->U = p->U;
+  out->Nw = p->Nw;
+  out->N = p->N;
+  out->nnz = p->nnz;
+  out->max_cover = p->max_cover;
+  out->device = p->device;
+  out->origins = p->origins.data();
+  out->tile_tok = p->tile_tok.data();
+  out->slot_pos = p->slot_pos.data();
+  out->tok_ptr = p->tok_ptr.data();
+  out->tok_ent = p->tok_ent.data();
+  out->wbar = p->wbar.data();
+  return TS_OK;
+}
+
+void ts_plan_destroy(ts_plan_t p) {
+  if (!p) return;
+  if (p->device < 0) {
+    delete p;
+    return;
+  }
+  int prev = -1;
+  cudaGetDevice(&prev);
+  cudaSetDevice(p->device);
+  cudaFree(p->d_tok_ptr);
+  cudaFree(p->d_tok_ent);
+  cudaFree(p->d_wbar);
+  cudaFree(p->d_rowmap);
+  cudaFree(p->d_pos_shared);
+  cudaFree(p->d_pos_tiled);
+  if (prev >= 0) cudaSetDevice(prev);
+  delete p;
+}
+
+ts_status ts_workspace_size(ts_plan_t p, const ts_model_desc* m, int L, int k, size_t* bytes) {
+  if (!p || !bytes) return fail(TS_ERR_INVALID_ARG, "NULL argument");
+  TS_TRY(check_model(m));
+  if (L < 0 || k < 0 || k > L) return fail(TS_ERR_INVALID_ARG, "need L >= 0 and 0 <= k <= L");
+  *bytes = layout(p, m, L > 0, nullptr).bytes;
+  return TS_OK;
+}
+
+ts_status ts_block_tiled(ts_plan_t p, const ts_model_desc* m, const ts_layer_weights* w, void* X, void* ws,
+                         size_t ws_bytes, void* stream) {
+  TS_TRY(check_plan(p));
+  TS_TRY(check_model(m));
+  TS_TRY(check_weights(m, w));
+  if (!X || !aligned16(X)) return fail(TS_ERR_INVALID_ARG, "X must be a 16-byte aligned device pointer");
+  Workspace W;
+  TS_TRY(check_ws(p, m, false, ws, ws_bytes, &W));
+  return layer_tiled(p, m, w, X, W, static_cast<cudaStream_t>(stream));
+}
+
+ts_status ts_block_shared(ts_plan_t p, const ts_model_desc* m, const ts_layer_weights* w, void* S, void* ws,
+                          size_t ws_bytes, void* stream) {
+  TS_TRY(check_plan(p));
+  TS_TRY(check_model(m));
+  TS_TRY(check_weights(m, w));
+  if (!S || !aligned16(S)) return fail(TS_ERR_INVALID_ARG, "S must be a 16-byte aligned device pointer");
+  Workspace W;
+  TS_TRY(check_ws(p, m, false, ws, ws_bytes, &W));
+  return layer_shared(p, m, w, S, W, static_cast<cudaStream_t>(stream));
+}
+
+ts_status ts_decode_stack(ts_plan_t p, const ts_model_desc* m, const ts_layer_weights* w, int L, int k, const void* S0,
+                          const void* G0, void* out, void* ws, size_t ws_bytes, void* stream) {
+  TS_TRY(check_plan(p));
+  TS_TRY(check_model(m));
+  if (!w) return fail(TS_ERR_INVALID_ARG, "weights are NULL");
+  if (L < 1 || k < 0 || k > L) return fail(TS_ERR_INVALID_ARG, "need L >= 1 and 0 <= k <= L");
+  for (int l = 0; l < L; ++l) TS_TRY(check_weights(m, w + l));
+  if (!S0 || !G0 || !out || !aligned16(S0) || !aligned16(G0) || !aligned16(out))
+    return fail(TS_ERR_INVALID_ARG, "S0, G0, out must be 16-byte aligned device pointers");
+  Workspace W;
+  TS_TRY(check_ws(p, m, true, ws, ws_bytes, &W));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t rb = static_cast<size_t>(m->d) * esize(m->dtype);
+  if (k > 0) {
+    const int nrows = p->T * p->N;
+    ts::gather_rows_kernel<<<rows_grid(nrows), 256, 0, st>>>(static_cast<const uint8_t*>(S0),
+                                                             static_cast<const uint8_t*>(G0), p->d_rowmap, nrows, p->U,
+                                                             rb, static_cast<uint8_t*>(W.X));
+    TS_TRY(launched("gather_rows"));
+    for (int l = 0; l < k; ++l) TS_TRY(layer_tiled(p, m, w + l, W.X, W, st));
+    if (k == L) return run_merge(p, m, W.X, p->U, out, nullptr, nullptr, st);
+    TS_TRY(run_merge(p, m, W.X, p->U + p->T, W.S, nullptr, nullptr, st));
+  } else {
+    TS_CUDA_CHECK(cudaMemcpyAsync(W.S, S0, rb * p->U, cudaMemcpyDeviceToDevice, st));
+    TS_CUDA_CHECK(cudaMemcpyAsync(static_cast<char*>(W.S) + rb * p->U, G0, rb * p->T, cudaMemcpyDeviceToDevice, st));
+  }
+  for (int l = k; l < L; ++l) TS_TRY(layer_shared(p, m, w + l, W.S, W, st));
+  TS_CUDA_CHECK(cudaMemcpyAsync(out, W.S, rb * p->U, cudaMemcpyDeviceToDevice, st));
+  return TS_OK;
+}
+
+ts_status ts_quantize_rows_e4m3(const void* x, int rows, int cols, void* q, float* scale, void* stream) {
+  if (!x || !q || !scale) return fail(TS_ERR_INVALID_ARG, "NULL argument");
+  if (rows < 0 || cols <= 0 || cols % 8) return fail(TS_ERR_INVALID_ARG, "need rows >= 0, cols %% 8 == 0");
+  if (!aligned16(x) || !aligned16(q) || !aligned16(scale)) return fail(TS_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  return run_quantize(x, rows, cols, static_cast<uint8_t*>(q), scale, static_cast<cudaStream_t>(stream));
+}
+
+ts_status ts_device_status(void) {
+  int v = 0;
+  TS_CUDA_CHECK(cudaDeviceSynchronize());
+  TS_CUDA_CHECK(cudaMemcpyFromSymbol(&v, ts::g_status, sizeof(int)));
+  const int zero = 0;
+  TS_CUDA_CHECK(cudaMemcpyToSymbol(ts::g_status, &zero, sizeof(int)));
+  if (v == 0) return TS_OK;
+  return fail(static_cast<ts_status>(v), "device status %d", v);
+}
+
+// ---------------------------------------------------------------------------
+// op-level entry points (include/tileshare_ops.h)
+// ---------------------------------------------------------------------------
+ts_status ts_op_layernorm(const ts_model_desc* m, const void* x, int rows, const float* g, const float* b, void* y,
+                          void* stream) {
+  TS_TRY(check_model(m));
+  if (!x || !y || !g || !b || rows < 0) return fail(TS_ERR_INVALID_ARG, "bad argument");
+  if (!aligned16(x) || !aligned16(y) || !aligned16(g) || !aligned16(b)) return fail(TS_ERR_INVALID_ARG, "alignment");
+  return run_layernorm(m, x, rows, g, b, y, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+ts_status ts_op_linear(const ts_model_desc* m, const void* x, int rows, int K, const void* W, const float* w_scale,
+                       int N, const float* bias, ts_epilogue epi, void* y, void* scratch, void* stream) {
+  TS_TRY(check_model(m));
+  if (!x || !W || !y || !bias || rows < 0 || K <= 0 || N <= 0) return fail(TS_ERR_INVALID_ARG, "bad argument");
+  if (!aligned16(x) || !aligned16(W) || !aligned16(y) || !aligned16(bias)) return fail(TS_ERR_INVALID_ARG, "alignment");
+  if (epi != TS_EPI_BIAS && epi != TS_EPI_BIAS_GELU && epi != TS_EPI_BIAS_RESID)
+    return fail(TS_ERR_INVALID_ARG, "unknown epilogue");
+  const int e = epi == TS_EPI_BIAS ? ts::EPI_BIAS : epi == TS_EPI_BIAS_GELU ? ts::EPI_GELU : ts::EPI_RESID;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (m->dtype == TS_F32)
+    return run_gemm_f32(e, static_cast<const float*>(x), static_cast<const float*>(W), rows, N, K, bias,
+                        static_cast<float*>(y), st);
+  if (m->dtype == TS_FP8_E4M3) {
+    if (!scratch || !aligned16(scratch) || !w_scale) return fail(TS_ERR_INVALID_ARG, "e4m3 linear needs scratch and w_scale");
+    uint8_t* q8 = static_cast<uint8_t*>(scratch);
+    float* qs = reinterpret_cast<float*>(q8 + align256(static_cast<size_t>(rows) * K));
+    TS_TRY(run_quantize(x, rows, K, q8, qs, st));
+    return run_gemm_tc(m, e, q8, qs, W, w_scale, rows, N, K, bias, static_cast<bf16*>(y), nullptr, nullptr, st);
+  }
+  return run_gemm_tc(m, e, x, nullptr, W, nullptr, rows, N, K, bias, static_cast<bf16*>(y), nullptr, nullptr, st);
+}
+
+ts_status ts_op_qkv(ts_plan_t p, const ts_model_desc* m, const ts_layer_weights* w, ts_rows_mode mode,
+                    const void* state, void* qkv, void* scratch, void* stream) {
+  TS_TRY(check_plan(p));
+  TS_TRY(check_model(m));
+  TS_TRY(check_weights(m, w));
+  if (!state || !qkv || !scratch || !aligned16(state) || !aligned16(qkv) || !aligned16(scratch))
+    return fail(TS_ERR_INVALID_ARG, "bad argument");
+  const bool shared = mode == TS_ROWS_SHARED;
+  const size_t rows = shared ? p->U + p->T : static_cast<size_t>(p->T) * p->N;
+  Workspace ws{};
+  ws.xn = scratch;
+  ws.q8 = static_cast<uint8_t*>(scratch) + align256(rows * m->d * esize(m->dtype));
+  ws.qs = reinterpret_cast<float*>(ws.q8 + align256(rows * m->d));
+  return run_qkv(p, m, w, shared, state, qkv, ws, static_cast<cudaStream_t>(stream));
+}
+
+ts_status ts_op_attention(ts_plan_t p, const ts_model_desc* m, ts_rows_mode mode, const void* qkv, void* O,
+                          void* stream) {
+  TS_TRY(check_plan(p));
+  TS_TRY(check_model(m));
+  if (!qkv || !O || !aligned16(qkv) || !aligned16(O)) return fail(TS_ERR_INVALID_ARG, "bad argument");
+  return run_attention(p, m, mode == TS_ROWS_SHARED, qkv, O, static_cast<cudaStream_t>(stream));
+}
+
+ts_status ts_op_merge(ts_plan_t p, const ts_model_desc* m, const void* P, int rows, void* A, void* stream) {
+  TS_TRY(check_plan(p));
+  TS_TRY(check_model(m));
+  if (!P || !A || !aligned16(P) || !aligned16(A)) return fail(TS_ERR_INVALID_ARG, "bad argument");
+  if (rows != p->U && rows != p->U + p->T) return fail(TS_ERR_INVALID_ARG, "rows must be U or U + T");
+  return run_merge(p, m, P, rows, A, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

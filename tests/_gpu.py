@@ -1,0 +1,79 @@
+"""Helpers of the GPU parity tests: device copies of the seeded inputs, the oracle
+run on the same inputs, and the error measure used by the tolerances."""
+
+import numpy as np
+import torch
+
+from oracle import layers as OL
+from oracle import plan as OP
+from shared_token_transformer_b200 import binding as B
+from shared_token_transformer_b200 import workloads as W
+
+TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.bfloat16}
+BIG = ("w_qkv", "w_o", "w_1", "w_2")
+SCALE = {"w_qkv": "s_qkv", "w_o": "s_o", "w_1": "s_1", "w_2": "s_2"}
+
+
+def rel_l2(got, want):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    return float(np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-300))
+
+
+def oracle_model(cfg):
+    return OL.Model(cfg.d, cfg.heads, cfg.mlp, cfg.rope_dims, fp8=(cfg.dtype == "fp8"))
+
+
+def model_desc(cfg):
+    return B.model_desc(cfg.d, cfg.heads, cfg.mlp, cfg.dtype, cfg.rope_dims)
+
+
+def dev(a, dtype):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device="cuda", dtype=dtype)
+
+
+def host(t):
+    return t.detach().to(torch.float64).cpu().numpy()
+
+
+def dev_layer(cfg, p):
+    """Device tensors of one layer; e4m3 weights quantised on the device, per row."""
+    out = {}
+    for k, v in p.items():
+        if k in BIG:
+            t = dev(v, TORCH_DT[cfg.dtype])
+            if cfg.dtype == "fp8":
+                q = torch.empty(t.shape, dtype=torch.uint8, device="cuda")
+                s = torch.empty(t.shape[0], dtype=torch.float32, device="cuda")
+                B.quantize_rows_e4m3(t, q, s)
+                out[k], out[SCALE[k]] = q, s
+            else:
+                out[k] = t
+        else:
+            out[k] = dev(v, torch.float32)
+    return out
+
+
+class Case:
+    """Seeded inputs of a configuration, on both sides."""
+
+    def __init__(self, cfg, seed=0, affine=True, L=None):
+        self.cfg = cfg
+        self.oplan = OP.make_plan(cfg.grid, cfg.win, cfg.stride)
+        self.plan = B.Plan(cfg.grid, cfg.win, cfg.stride)
+        dr = W.Draw(cfg, self.oplan.T, seed=seed, affine=affine)
+        self.S0, self.G0 = dr.states()
+        self.layers = dr.layers(L)
+        self.m = model_desc(cfg)
+        self.om = oracle_model(cfg)
+        self.dlayers = [dev_layer(cfg, p) for p in self.layers]
+        self.wlist = [B.layer_weights(t) for t in self.dlayers]
+        self.dt = TORCH_DT[cfg.dtype]
+
+    @property
+    def S(self):
+        return np.concatenate([self.S0, self.G0])
+
+    def workspace(self, L=0, k=0):
+        n = B.workspace_size(self.plan, self.m, L, k)
+        return torch.empty(n, dtype=torch.uint8, device="cuda")

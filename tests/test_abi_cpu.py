@@ -1,0 +1,120 @@
+"""The C-ABI library on the CPU: it loads, exports every declared entry point, its
+host planner equals the oracle's plan bit for bit, and bad arguments are refused.
+No CUDA compute call is made here."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import plan as OP
+from shared_token_transformer_b200 import binding as B
+from shared_token_transformer_b200 import build as Bd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    Bd.build()
+
+
+def _declared():
+    names = set()
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        txt = open(os.path.join(ROOT, "include", h)).read()
+        names |= set(re.findall(r"^(?:ts_status|void|const char\*)\s+(ts_\w+)\s*\(", txt, re.M))
+    return names
+
+
+def test_exports_every_declared_symbol():
+    names = _declared()
+    assert len(names) >= 16
+    L = ctypes.CDLL(B.LIB_PATH)
+    for n in sorted(names):
+        assert hasattr(L, n), n
+    assert names <= set(B.exported_symbols()), names - set(B.exported_symbols())
+
+
+GEOMS = [
+    ((1, 14, 14), (1, 8, 8), (1, 6, 6)),
+    ((1, 16, 16), (1, 8, 8), (1, 8, 8)),
+    ((1, 48, 48), (1, 16, 16), (1, 12, 12)),
+    ((4, 44, 80), (4, 32, 32), (4, 24, 24)),
+    ((1, 128, 128), (1, 32, 32), (1, 24, 24)),
+    ((1, 11, 13), (1, 8, 8), (1, 5, 6)),
+    ((3, 7, 9), (2, 4, 5), (1, 1, 2)),
+    ((1, 20, 9), (1, 8, 3), (1, 3, 1)),
+    ((1, 5, 5), (1, 5, 5), (1, 2, 2)),
+]
+
+
+@pytest.mark.parametrize("grid,win,stride", GEOMS)
+def test_host_planner_bit_exact_against_oracle(grid, win, stride):
+    o = OP.make_plan(grid, win, stride)
+    p = B.Plan(grid, win, stride, host_only=True)
+    try:
+        assert (p.T, p.U, p.Nw, p.N, p.nnz) == (o.T, o.U, o.Nw, o.N, o.nnz)
+        assert p.device == -1
+        np.testing.assert_array_equal(p.origins, o.origins)
+        np.testing.assert_array_equal(p.tile_tok, o.tile_tok)
+        np.testing.assert_array_equal(p.slot_pos, o.slot_pos)
+        np.testing.assert_array_equal(p.tok_ptr, o.tok_ptr)
+        np.testing.assert_array_equal(p.tok_ent, o.tok_ent)
+        # w-bar: the planner rounds its double weights to float once
+        np.testing.assert_array_equal(p.wbar, o.tok_w.astype(np.float32))
+        assert p.max_cover == int(o.coverage.max())
+    finally:
+        p.close()
+
+
+def test_image4k_plan_counts():
+    p = B.Plan((1, 256, 256), (1, 32, 32), (1, 24, 24), host_only=True)
+    assert (p.T, p.U, p.N, p.nnz, p.max_cover) == (121, 65536, 1025, 123904, 4)
+    p.close()
+
+
+@pytest.mark.parametrize("grid,win,stride", [
+    ((1, 8, 8), (1, 9, 8), (1, 1, 1)),     # window larger than grid
+    ((1, 8, 8), (1, 4, 4), (1, 5, 4)),     # stride larger than window
+    ((1, 8, 8), (1, 4, 4), (1, 0, 4)),     # zero stride
+    ((0, 8, 8), (1, 4, 4), (1, 4, 4)),     # empty axis
+])
+def test_plan_rejects_bad_geometry(grid, win, stride):
+    with pytest.raises(B.TileShareError) as e:
+        B.Plan(grid, win, stride, host_only=True)
+    assert e.value.status == 1
+
+
+def test_status_strings_and_workspace_on_host_plan():
+    L = B.lib()
+    assert L.ts_status_string(0) == b"ok"
+    assert L.ts_status_string(3) == b"workspace too small"
+    p = B.Plan((1, 48, 48), (1, 16, 16), (1, 12, 12), host_only=True)
+    m = B.model_desc(512, 8, 2048, "bf16", (0, 32, 32))
+    n0 = B.workspace_size(p, m, 0, 0)
+    n8 = B.workspace_size(p, m, 8, 2)
+    assert n8 > n0 > 0
+    # unsupported head dim on the bf16 path, bad k, bad rope split
+    with pytest.raises(B.TileShareError) as e:
+        B.workspace_size(p, B.model_desc(512, 4, 2048, "bf16", (0, 64, 64)), 0, 0)
+    assert e.value.status == 2
+    with pytest.raises(B.TileShareError) as e:
+        B.workspace_size(p, m, 4, 5)
+    assert e.value.status == 1
+    with pytest.raises(B.TileShareError) as e:
+        B.workspace_size(p, B.model_desc(512, 8, 2048, "bf16", (0, 30, 32)), 0, 0)
+    assert e.value.status == 1
+    p.close()
+
+
+def test_compute_calls_refuse_host_plan():
+    # a host-only plan is refused before any launch (device -1 never matches)
+    p = B.Plan((1, 14, 14), (1, 8, 8), (1, 6, 6), host_only=True)
+    m = B.model_desc(64, 4, 256, "f32", (0, 8, 8))
+    w = B.LayerWeights()
+    st = B.lib().ts_block_shared(p.handle, ctypes.byref(m), ctypes.byref(w), None, None, 0, None)
+    assert st in (1, 4)     # invalid argument (or CUDA unavailable when querying the device)
+    p.close()

@@ -1,0 +1,293 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Op level first (LayerNorm, linear epilogues, QKV + QK-norm + RoPE, gathered
+attention, blend), then layers, stacks, determinism and error paths.  Inputs are
+the seeded draws of ``workloads`` (with nonzero biases and gains: affine=True);
+the oracle consumes the same dtype-rounded values in float64.
+
+Tolerances (relative L2 against the oracle): fp32 path 1e-5 per layer; bf16 path
+1e-2 on stack outputs (and per layer); e4m3 path 3e-2.  Op-level bf16 checks use
+the rounding of one bf16 store (2^-8 relative per element) as their scale.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import layers as OL
+from shared_token_transformer_b200 import binding as B
+from shared_token_transformer_b200 import workloads as W
+
+from _gpu import Case, dev, host, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+SMALL = W.small_config("small_bf16", grid=(1, 11, 13), win=(1, 8, 8), stride=(1, 5, 6), d=256, heads=4, mlp=512,
+                       dtype="bf16", L=3, k=1)
+RAGGED = W.small_config("ragged_bf16", grid=(1, 40, 37), win=(1, 15, 21), stride=(1, 12, 9), d=256, heads=4,
+                        mlp=512, dtype="bf16", L=2, k=1)
+VOL = W.small_config("vol_bf16", grid=(3, 12, 14), win=(2, 8, 8), stride=(1, 4, 6), d=256, heads=4, mlp=768,
+                     dtype="bf16", L=2, k=1)
+SMALL_FP8 = W.small_config("small_fp8", grid=(1, 11, 13), win=(1, 8, 8), stride=(1, 5, 6), d=256, heads=4,
+                           mlp=512, dtype="fp8", L=2, k=1)
+VIT14 = W.CONFIGS["vit14_fp32"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from shared_token_transformer_b200 import build
+    build.build()
+    torch.manual_seed(0)
+    yield
+    B.device_status()
+
+
+_cases = {}
+
+
+def case(cfg, **kw):
+    key = (cfg.name, tuple(sorted(kw.items())))
+    if key not in _cases:
+        _cases[key] = Case(cfg, **kw)
+    return _cases[key]
+
+
+# ---------------------------------------------------------------------------
+# op level
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("cfg", [SMALL, RAGGED, VIT14], ids=lambda c: c.name)
+def test_layernorm(cfg):
+    c = case(cfg)
+    x = dev(c.S, c.dt)
+    y = torch.empty_like(x)
+    p = c.layers[0]
+    B.op_layernorm(c.m, x, c.dlayers[0]["ln1_g"], c.dlayers[0]["ln1_b"], y)
+    want = OL.layer_norm(c.S, p["ln1_g"], p["ln1_b"], 1e-6)
+    tol = 1e-6 if cfg.dtype == "f32" else 3e-3
+    assert rel_l2(host(y), want) < tol
+
+
+@pytest.mark.parametrize("M,K,N", [(300, 256, 512), (128, 512, 768), (129, 256, 192), (1, 256, 64), (2320, 512, 1536),
+                                   (777, 2048, 512)])
+@pytest.mark.parametrize("epi", [B.TS_EPI_BIAS, B.TS_EPI_BIAS_GELU, B.TS_EPI_BIAS_RESID])
+def test_linear_bf16(M, K, N, epi):
+    rng = np.random.default_rng(M * 7 + N + epi)
+    x = W.round_to(rng.standard_normal((M, K)), "bf16")
+    w = W.round_to(0.05 * rng.standard_normal((N, K)), "bf16")
+    b = W.round_to(0.1 * rng.standard_normal(N), "f32")
+    y0 = W.round_to(rng.standard_normal((M, N)), "bf16")
+    m = B.model_desc(256, 4, 256, "bf16", (0, 32, 32))
+    y = dev(y0, torch.bfloat16)
+    B.op_linear(m, dev(x, torch.bfloat16), dev(w, torch.bfloat16), dev(b, torch.float32), y, epi=epi)
+    want = x @ w.T + b
+    if epi == B.TS_EPI_BIAS_GELU:
+        want = OL.gelu(want)
+    if epi == B.TS_EPI_BIAS_RESID:
+        want = want + y0
+    assert rel_l2(host(y), want) < 3e-3
+
+
+@pytest.mark.parametrize("M,K,N", [(300, 256, 512), (129, 512, 256), (64, 1536, 4608)])
+def test_linear_fp8(M, K, N):
+    from oracle import fp8 as F8
+    rng = np.random.default_rng(M + K)
+    x = W.round_to(rng.standard_normal((M, K)), "bf16")
+    w = W.round_to(0.02 * rng.standard_normal((N, K)), "bf16")
+    b = W.round_to(0.1 * rng.standard_normal(N), "f32")
+    m = B.model_desc(256, 4, 256, "fp8", (0, 32, 32))
+    wd = dev(w, torch.bfloat16)
+    q = torch.empty((N, K), dtype=torch.uint8, device="cuda")
+    s = torch.empty(N, dtype=torch.float32, device="cuda")
+    B.quantize_rows_e4m3(wd, q, s)
+    # the weight codes equal the oracle's rounding of the same bf16 values
+    qo, so = F8.quantize_rows(w)
+    got_codes = q.cpu().view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_allclose(host(s), so, rtol=1e-6)
+    assert np.mean(got_codes == qo) > 0.999
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    scratch = torch.empty(M * K + 4 * M + 512, dtype=torch.uint8, device="cuda")
+    B.op_linear(m, dev(x, torch.bfloat16), q, dev(b, torch.float32), y, epi=B.TS_EPI_BIAS, w_scale=s,
+                scratch=scratch)
+    want = F8.scaled_matmul(x, w) + b
+    assert rel_l2(host(y), want) < 1e-2
+
+
+def _qkv_oracle(c, state, rows_pos, unrot):
+    """LN1 + QKV + QK-norm (oracle), then RoPE at the given per-row coordinates."""
+    p = c.layers[0]
+    q, k, v = OL.qkv_project(state, p, c.om)
+    rot = ~unrot
+    q[rot] = OL.rope(q[rot], rows_pos[rot], c.om)
+    k[rot] = OL.rope(k[rot], rows_pos[rot], c.om)
+    n = state.shape[0]
+    return np.concatenate([q.reshape(n, -1), k.reshape(n, -1), v.reshape(n, -1)], axis=1)
+
+
+@pytest.mark.parametrize("cfg", [SMALL, VOL, VIT14], ids=lambda c: c.name)
+@pytest.mark.parametrize("mode", [B.TS_ROWS_SHARED, B.TS_ROWS_TILED])
+def test_qkv_norm_rope(cfg, mode):
+    c = case(cfg)
+    op = c.oplan
+    if mode == B.TS_ROWS_SHARED:
+        state = c.S
+        F, H, Wd = cfg.grid
+        u = np.arange(op.U)
+        pos = np.concatenate([np.stack([u // (H * Wd), (u // Wd) % H, u % Wd], 1), op.origins])
+        unrot = np.zeros(len(state), bool)
+    else:
+        state = OL.gather(c.S, op).reshape(op.T * op.N, -1)
+        pos = np.tile(np.concatenate([[[0, 0, 0]], op.slot_pos]), (op.T, 1))
+        unrot = np.zeros(len(state), bool)
+        unrot[::op.N] = True
+    want = _qkv_oracle(c, state, pos, unrot)
+    qkv = torch.empty((len(state), 3 * cfg.d), dtype=c.dt, device="cuda")
+    scratch = torch.empty(len(state) * cfg.d * 6 + 4096, dtype=torch.uint8, device="cuda")
+    B.op_qkv(c.plan, c.m, c.wlist[0], mode, dev(state, c.dt), qkv, scratch)
+    got = host(qkv)
+    tol = 1e-5 if cfg.dtype == "f32" else 8e-3
+    for part in range(3):
+        sl = slice(part * cfg.d, (part + 1) * cfg.d)
+        assert rel_l2(got[:, sl], want[:, sl]) < tol, part
+
+
+@pytest.mark.parametrize("cfg", [SMALL, RAGGED, VOL, VIT14], ids=lambda c: c.name)
+@pytest.mark.parametrize("mode", [B.TS_ROWS_SHARED, B.TS_ROWS_TILED])
+def test_attention(cfg, mode):
+    c = case(cfg)
+    op = c.oplan
+    rows = op.U + op.T if mode == B.TS_ROWS_SHARED else op.T * op.N
+    rng = np.random.default_rng(3)
+    qkv = W.round_to(rng.standard_normal((rows, 3 * cfg.d)), cfg.dtype if cfg.dtype != "fp8" else "bf16")
+    O = torch.empty((op.T * op.N, cfg.d), dtype=c.dt, device="cuda")
+    B.op_attention(c.plan, c.m, mode, dev(qkv, c.dt), O)
+    hd = cfg.hd
+    want = np.empty((op.T * op.N, cfg.d))
+    for t in range(op.T):
+        if mode == B.TS_ROWS_SHARED:
+            r = np.concatenate([[op.U + t], op.tile_tok[t]])
+        else:
+            r = t * op.N + np.arange(op.N)
+        q = qkv[r, :cfg.d].reshape(op.N, cfg.heads, hd)
+        k = qkv[r, cfg.d:2 * cfg.d].reshape(op.N, cfg.heads, hd)
+        v = qkv[r, 2 * cfg.d:].reshape(op.N, cfg.heads, hd)
+        want[t * op.N:(t + 1) * op.N] = OL.attention(q, k, v)
+    tol = 1e-5 if cfg.dtype == "f32" else 1e-2
+    got = host(O)
+    assert rel_l2(got, want) < tol
+    # global-token rows (handled by their own code path) checked separately
+    assert rel_l2(got[::op.N], want[::op.N]) < tol
+
+
+@pytest.mark.parametrize("cfg", [SMALL, RAGGED, VOL, VIT14], ids=lambda c: c.name)
+def test_merge(cfg):
+    c = case(cfg)
+    op = c.oplan
+    rng = np.random.default_rng(4)
+    P = W.round_to(rng.standard_normal((op.T, op.N, cfg.d)), cfg.dtype if cfg.dtype != "fp8" else "bf16")
+    for rows in (op.U, op.U + op.T):
+        A = torch.empty((rows, cfg.d), dtype=c.dt, device="cuda")
+        B.op_merge(c.plan, c.m, dev(P.reshape(op.T * op.N, -1), c.dt), rows, A)
+        want = OL.merge(P, op)[:rows]
+        tol = 1e-6 if cfg.dtype == "f32" else 3e-3
+        assert rel_l2(host(A), want) < tol
+
+
+# ---------------------------------------------------------------------------
+# layers
+# ---------------------------------------------------------------------------
+def _tol(cfg):
+    return {"f32": 1e-5, "bf16": 1e-2, "fp8": 3e-2}[cfg.dtype]
+
+
+@pytest.mark.parametrize("cfg", [SMALL, RAGGED, VOL, VIT14, SMALL_FP8], ids=lambda c: c.name)
+def test_block_shared(cfg):
+    c = case(cfg)
+    S_in = c.S
+    S = dev(S_in, c.dt)
+    ws = c.workspace()
+    B.block_shared(c.plan, c.m, c.wlist[0], S, ws)
+    want = OL.block_shared(S_in, c.layers[0], c.om, c.oplan)
+    got = host(S)
+    assert rel_l2(got, want) < _tol(cfg)
+    assert rel_l2(got - S_in, want - S_in) < 3 * _tol(cfg)
+
+
+@pytest.mark.parametrize("cfg", [SMALL, RAGGED, VOL, VIT14, SMALL_FP8], ids=lambda c: c.name)
+def test_block_tiled(cfg):
+    c = case(cfg)
+    X_in = OL.gather(c.S, c.oplan)
+    X = dev(X_in.reshape(c.oplan.T * c.oplan.N, -1), c.dt)
+    ws = c.workspace()
+    B.block_tiled(c.plan, c.m, c.wlist[0], X, ws)
+    want = OL.block_tiled(X_in, c.layers[0], c.om, c.oplan).reshape(X.shape)
+    got = host(X)
+    X_in = X_in.reshape(X.shape)
+    assert rel_l2(got, want) < _tol(cfg)
+    assert rel_l2(got - X_in, want - X_in) < 3 * _tol(cfg)
+
+
+# ---------------------------------------------------------------------------
+# stacks
+# ---------------------------------------------------------------------------
+def _run_stack(c, k):
+    op = c.oplan
+    L = len(c.wlist)
+    out = torch.empty((op.U, c.cfg.d), dtype=c.dt, device="cuda")
+    ws = c.workspace(L, k)
+    B.decode_stack(c.plan, c.m, c.wlist, k, dev(c.S0, c.dt), dev(c.G0, c.dt), out, ws)
+    return out
+
+
+@pytest.mark.parametrize("cfg,ks", [(SMALL, (0, 1, 3)), (RAGGED, (1,)), (VOL, (0, 2)), (VIT14, (0, 1)),
+                                    (SMALL_FP8, (0, 1, 2))], ids=lambda x: getattr(x, "name", str(x)))
+def test_decode_stack(cfg, ks):
+    c = case(cfg)
+    for k in ks:
+        got = host(_run_stack(c, k))
+        want = OL.decode_stack(c.S0, c.G0, c.layers, c.om, c.oplan, k)
+        assert rel_l2(got, want) < _tol(cfg), k
+
+
+def test_stack48_bf16_full():
+    """The benchmark stack (48x48 tokens, d=512, L=8, k=2) against the full oracle."""
+    cfg = W.CONFIGS["stack48_bf16"]
+    c = case(cfg, affine=False)
+    got = host(_run_stack(c, cfg.k))
+    want = OL.decode_stack(c.S0, c.G0, c.layers, c.om, c.oplan, cfg.k)
+    assert rel_l2(got, want) < 1e-2
+
+
+def test_stack_deterministic():
+    c = case(SMALL)
+    a = _run_stack(c, 1).clone()
+    b = _run_stack(c, 1)
+    assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------------------
+# error paths: refused on the host, nothing written
+# ---------------------------------------------------------------------------
+def test_error_paths():
+    c = case(SMALL)
+    S = dev(c.S, c.dt)
+    before = S.clone()
+    ws = c.workspace()
+    with pytest.raises(B.TileShareError) as e:
+        B.block_shared(c.plan, c.m, c.wlist[0], S, ws[:-1024])
+    assert e.value.status == 3
+    with pytest.raises(B.TileShareError) as e:
+        B.block_shared(c.plan, c.m, c.wlist[0], S.view(torch.uint8)[2:], ws)
+    assert e.value.status == 1
+    bad = dict(c.dlayers[0])
+    bad["w_o"] = None
+    with pytest.raises(B.TileShareError) as e:
+        B.block_shared(c.plan, c.m, B.layer_weights(bad), S, ws)
+    assert e.value.status == 1
+    with pytest.raises(B.TileShareError) as e:
+        B.decode_stack(c.plan, c.m, c.wlist, 7, dev(c.S0, c.dt), dev(c.G0, c.dt),
+                       torch.empty((c.oplan.U, 256), dtype=c.dt, device="cuda"), c.workspace(3, 1))
+    assert e.value.status == 1
+    torch.cuda.synchronize()
+    assert torch.equal(S, before)

@@ -43,6 +43,14 @@ def test_e4m3_rounding_against_library_cast():
     assert F8.round_e4m3_scalar(1e6) == 448.0 and F8.round_e4m3_scalar(-500.0) == -448.0
 
 
+def test_array_rounding_equals_scalar_rounding():
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.standard_normal(3000) * s for s in (1e-4, 3e-3, 0.3, 7, 100, 600)])
+    grid = [F8.decode_e4m3(c) for c in range(127)]
+    x = np.concatenate([x, grid, -np.array(grid), [(a + b) / 2 for a, b in zip(grid[:-1], grid[1:])]])
+    np.testing.assert_array_equal(F8.round_e4m3(x), [F8.round_e4m3_scalar(v) for v in x])
+
+
 def test_scaled_matmul_exact_on_grid_inputs():
     # rows whose absmax is 448 * 2^e and whose entries lie on the scaled grid quantise exactly
     rng = np.random.default_rng(2)
