@@ -1,0 +1,516 @@
+#!/usr/bin/env python
+"""Benchmark of the TileShare shared layer on B200: unique tokens/s per shared layer.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tileshare|reference] [--config NAME]
+
+A step is one TileShare-k decode of the configuration's seeded synthetic input
+(default: the 48x48-token, d=512, L=8, k=2 bf16 stack): per-tile copies of the
+input, k per-tile layers, the merge of the per-tile states, L-k shared layers and
+the copy of the output rows.  It runs through the library's public calls,
+captured as CUDA graphs (one for the per-tile part, one for the shared part) so
+that the shared layers are timed on their own by CUDA events on the launching
+stream; L2 is flushed (512 MiB write) before every step, outside the events.
+
+value  = unique tokens per second per shared layer = U * (L - k) * K * N_ranks /
+         (max over ranks of the summed shared-part time of the K steps).
+e2e    = the same metric through the public call with host buffers: pinned host
+         state -> device, one ts_block_shared, device -> pinned host, timed with
+         CUDA events around the copies and the call.
+roofline  per kernel class from a traced pass (library kernel trace: CUDA events
+         around each launch, algorithmic FLOPs / HBM bytes per launch); the
+         dominant class (most time) is reported against MEASURED_PEAKS.json.
+cpu_baseline  the float64 CPU oracle's shared layer on the same inputs (rank 0,
+         N = 1).  --impl reference times that oracle alone as the reference arm.
+
+Multi-GPU (torchrun): every rank decodes its own image (independent inputs, the
+same weights); there is no data-path collective, only a barrier and a max of the
+timings.  Scaling is weak.
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "unique tokens/sec per shared layer on 1 B200; % of bf16 tensor/HBM roofline"
+UNIT = "unique tokens/s per shared layer"
+BIG = ("w_qkv", "w_o", "w_1", "w_2")
+SCALE = {"w_qkv": "s_qkv", "w_o": "s_o", "w_1": "s_1", "w_2": "s_2"}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="tileshare", choices=["tileshare", "reference"])
+    ap.add_argument("--config", default="stack48_bf16")
+    ap.add_argument("--no-graph", action="store_true", help="launch the calls eagerly instead of CUDA graphs")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU oracle baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--trace-steps", type=int, default=20)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def flops_layer(rows, T, N, d, f):
+    return rows * 2.0 * (4 * d * d + 2 * d * f) + 4.0 * T * N * N * d
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples of one GPU while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.samples = []
+        self.proc = None
+        self.gpu_id = gpu_id
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        inside = [p for t, p in self.samples if t0 - 0.15 <= t <= t1 + 0.15]
+        if len(inside) < 3:
+            inside = [p for t, p in self.samples if t0 - 1.0 <= t <= t1 + 1.0]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        mhz, mx = [], []
+        for p in inside:
+            try:
+                mhz.append(float(p[1]))
+                mx.append(float(p[2]))
+            except ValueError:
+                pass
+            for n, v in zip(names, p[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(inside)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (the cpu_baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def oracle_shared_layer_timing(cfg, budget_s, max_steps, warmup=1):
+    """Time the float64 oracle's shared layer on the configuration's seeded input."""
+    from oracle import layers as OL
+    from oracle import plan as OP
+    from shared_token_transformer_b200 import workloads as W
+    op = OP.make_plan(cfg.grid, cfg.win, cfg.stride)
+    dr = W.Draw(cfg, op.T, seed=0)
+    S0, G0 = dr.states()
+    S = np.concatenate([S0, G0])
+    layer = dr.layer()
+    om = OL.Model(cfg.d, cfg.heads, cfg.mlp, cfg.rope_dims, fp8=(cfg.dtype == "fp8"))
+    for _ in range(warmup):
+        OL.block_shared(S, layer, om, op)
+    times = []
+    t_all = time.perf_counter()
+    while len(times) < max(1, max_steps):
+        t0 = time.perf_counter()
+        OL.block_shared(S, layer, om, op)
+        times.append(time.perf_counter() - t0)
+        if time.perf_counter() - t_all > budget_s:
+            break
+    return op.U, times
+
+
+# ---------------------------------------------------------------------------
+# tileshare arm
+# ---------------------------------------------------------------------------
+def run_tileshare(args, rank, world, local):
+    import torch
+    import torch.distributed as dist
+
+    from shared_token_transformer_b200 import binding as B
+    from shared_token_transformer_b200 import build as Bd
+    from shared_token_transformer_b200 import workloads as W
+
+    Bd.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    cfg = W.CONFIGS[args.config]
+    L, k = cfg.L, cfg.k
+    dt = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.bfloat16}[cfg.dtype]
+    plan = B.Plan(cfg.grid, cfg.win, cfg.stride)
+    U, T, N, d, f = plan.U, plan.T, plan.N, cfg.d, cfg.mlp
+    m = B.model_desc(d, cfg.heads, f, cfg.dtype, cfg.rope_dims)
+
+    # seeded inputs: weights from seed 0 (same on every rank); each rank its own image
+    dr = W.Draw(cfg, T, seed=0)
+    S0, G0 = dr.states()
+    if rank > 0:
+        S0, G0 = W.Draw(cfg, T, seed=rank).states()
+
+    def todev(a, dtype):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev, dtype)
+
+    dlayers = []
+    for _ in range(L):
+        p = dr.layer()
+        t = {}
+        for key, v in p.items():
+            if key in BIG:
+                x = todev(v, dt)
+                if cfg.dtype == "fp8":
+                    q = torch.empty(x.shape, dtype=torch.uint8, device=dev)
+                    s = torch.empty(x.shape[0], dtype=torch.float32, device=dev)
+                    B.quantize_rows_e4m3(x, q, s)
+                    t[key], t[SCALE[key]] = q, s
+                else:
+                    t[key] = x
+            else:
+                t[key] = todev(v, torch.float32)
+        dlayers.append(t)
+    wl = [B.layer_weights(t) for t in dlayers]
+    S0d, G0d = todev(S0, dt), todev(G0, dt)
+    X = torch.empty((T * N, d), dtype=dt, device=dev)
+    S = torch.empty((U + T, d), dtype=dt, device=dev)
+    out = torch.empty((U, d), dtype=dt, device=dev)
+    ws = torch.empty(B.workspace_size(plan, m, 0, 0), dtype=torch.uint8, device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    def part_tiled(kk=k):
+        if kk > 0:
+            B.gather_tiles(plan, m, S0d, G0d, X)
+            for li in range(kk):
+                B.block_tiled(plan, m, wl[li], X, ws)
+            if kk < L:
+                B.op_merge(plan, m, X, U + T, S)
+            else:
+                B.op_merge(plan, m, X, U, out)
+        else:
+            S[:U].copy_(S0d)
+            S[U:].copy_(G0d)
+
+    def part_shared():
+        for li in range(k, L):
+            B.block_shared(plan, m, wl[li], S, ws)
+
+    def part_out():
+        if k < L:
+            out.copy_(S[:U])
+
+    # warm-up (eager: configures every kernel), then capture
+    for _ in range(max(1, args.warmup)):
+        part_tiled()
+        part_shared()
+        part_out()
+    torch.cuda.synchronize()
+    use_graph = not args.no_graph
+    launches_per_step = None
+    if use_graph:
+        n0 = B.launch_count()
+        g1, g2, g3 = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g1, stream=side):
+                part_tiled()
+            with torch.cuda.graph(g2, stream=side):
+                part_shared()
+            with torch.cuda.graph(g3, stream=side):
+                part_out()
+        torch.cuda.current_stream().wait_stream(side)
+        launches_per_step = B.launch_count() - n0
+        run1, run2, run3 = g1.replay, g2.replay, g3.replay
+        for _ in range(max(3, args.warmup)):
+            run1(); run2(); run3()
+    else:
+        run1, run2, run3 = part_tiled, part_shared, part_out
+    torch.cuda.synchronize()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    gpu_id = local
+    try:
+        props = torch.cuda.get_device_properties(dev)
+        if getattr(props, "uuid", None) is not None:
+            gpu_id = "GPU-" + str(props.uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.6)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n_before = B.launch_count()
+    t_wall0 = time.time()
+    for i in range(K):
+        flush.zero_()
+        e = evs[i]
+        e[0].record()
+        run1()
+        e[1].record()
+        run2()
+        e[2].record()
+        run3()
+        e[3].record()
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    eager_launches = B.launch_count() - n_before
+    t_step = np.array([e[0].elapsed_time(e[3]) for e in evs])
+    t_tiled = np.array([e[0].elapsed_time(e[1]) for e in evs])
+    t_shared = np.array([e[1].elapsed_time(e[2]) for e in evs])
+    sums = torch.tensor([t_shared.sum(), t_step.mean(), t_tiled.mean()], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(sums, op=dist.ReduceOp.MAX)
+    shared_total_ms, step_ms, tiled_ms = (float(x) for x in sums.cpu())
+    value = (U * (L - k) * K * world) / (shared_total_ms / 1e3) if L > k else 0.0
+    gpu_launches = launches_per_step * K if use_graph else eager_launches
+
+    # own batched per-tile path on the same input: k = L (all layers per tile, blended at the end)
+    Kt = min(K, 100)
+    if use_graph:
+        gt = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            part_tiled(L)
+            with torch.cuda.graph(gt, stream=side):
+                part_tiled(L)
+        torch.cuda.current_stream().wait_stream(side)
+        run_t = gt.replay
+    else:
+        def run_t():
+            part_tiled(L)
+    run_t()
+    torch.cuda.synchronize()
+    tev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Kt)]
+    for i in range(Kt):
+        flush.zero_()
+        tev[i][0].record()
+        run_t()
+        tev[i][1].record()
+    torch.cuda.synchronize()
+    tiled_stack_ms = float(np.mean([a.elapsed_time(b) for a, b in tev]))
+
+    # e2e: one shared layer through the public call with pinned host buffers
+    Ke = min(K, 200)
+    S_host = torch.cat([S0d, G0d]).cpu().pin_memory()
+    S_back = torch.empty_like(S_host).pin_memory()
+    Sd = torch.empty((U + T, d), dtype=dt, device=dev)
+    eev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Ke)]
+    for i in range(Ke + 3):
+        flush.zero_()
+        if i >= 3:
+            eev[i - 3][0].record()
+        Sd.copy_(S_host, non_blocking=True)
+        B.block_shared(plan, m, wl[min(k, L - 1)], Sd, ws)
+        S_back.copy_(Sd, non_blocking=True)
+        if i >= 3:
+            eev[i - 3][1].record()
+    torch.cuda.synchronize()
+    e2e_ms = float(np.mean([a.elapsed_time(b) for a, b in eev]))
+    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    e2e_value = U * world / (float(e2e_t.item()) / 1e3)
+    state_bytes = (U + T) * d * S_host.element_size()
+
+    # traced pass: per-kernel times of the same step, eagerly launched
+    B.trace_begin(100000)
+    for _ in range(args.trace_steps):
+        flush.zero_()
+        part_tiled()
+        part_shared()
+        part_out()
+    tr = B.trace_end()
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
+
+    pk, pk_src = peaks()
+    tensor_peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    if cfg.dtype == "fp8":
+        tensor_peak = 2.0 * tensor_peak          # nominal e4m3 : bf16 dense ratio
+    total_ms = sum(v["ms"] for v in tr.values()) or 1.0
+    kernels = {}
+    for name, v in tr.items():
+        if v["timed"] == 0:
+            continue
+        per = v["ms"] / v["timed"]
+        tensor = v["flops"] > 0 and name.startswith(("gemm", "attention", "linear"))
+        if tensor:
+            ach = v["flops"] / (v["ms"] / 1e3) / 1e12
+            frac = ach / tensor_peak
+            unit = "TFLOP/s"
+        else:
+            ach = v["bytes"] / (v["ms"] / 1e3) / 1e9
+            frac = ach / pk["hbm_gbs"]
+            unit = "GB/s"
+        kernels[name] = {"launches": v["launches"], "ms_per_launch": round(per, 5),
+                         "share": round(v["ms"] / total_ms, 4), "achieved": round(ach, 2), "unit": unit,
+                         "frac": round(frac, 4),
+                         "flops_per_launch": v["flops"] / v["timed"], "bytes_per_launch": v["bytes"] / v["timed"]}
+    dom = max(kernels, key=lambda n: kernels[n]["share"])
+    kd = kernels[dom]
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as fh:
+            tj = json.load(fh)
+        ent = tj.get(args.config, {}).get(dom)
+        if ent and ent.get("kernel_source_sha") == kernel_source_sha():
+            traffic = ent.get("traffic_bytes_per_launch")
+    roofline = {"bound": "tensor" if kd["unit"] == "TFLOP/s" else "hbm", "kernel": dom, "achieved": kd["achieved"],
+                "peak": round(tensor_peak if kd["unit"] == "TFLOP/s" else pk["hbm_gbs"], 1), "unit": kd["unit"],
+                "frac": kd["frac"], "traffic": traffic,
+                "peak_source": (f"{pk_src} " + ("bf16_tflops_sustained" + (" x2 (e4m3:bf16 nominal)" if cfg.dtype == "fp8" else "")
+                                                if kd["unit"] == "TFLOP/s" else "hbm_gbs"))}
+
+    ft = flops_layer(T * N, T, N, d, f)
+    fs = flops_layer(U + T, T, N, d, f)
+    flop_ratio = (k * ft + (L - k) * fs) / (L * ft)
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(step_ms, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": {"bf16": "bf16", "f32": "f32", "fp8": "e4m3"}[cfg.dtype],
+        "data": "synthetic (seeded N(0,1) states, N(0,0.02) weights, random init)",
+        "config": {"workload": f"{cfg.name}: {cfg.note}", "grid": list(cfg.grid), "window": list(cfg.win),
+                   "stride": list(cfg.stride), "L": L, "k": k, "unique_tokens": U, "tiles": T, "rows_per_tile": N,
+                   "l2": "flushed before every step (512 MiB write, outside the timed events)",
+                   "launch": "CUDA graphs of the public calls" if use_graph else "eager public calls",
+                   "parallelism": f"replicas x{world} (one image per GPU)"},
+        "shared_layer_ms": round(shared_total_ms / K / max(1, L - k), 5),
+        "per_tile_part_ms": round(tiled_ms, 5),
+        "tiled_stack_ms": round(tiled_stack_ms, 5),
+        "speedup_vs_tiled": round(tiled_stack_ms / step_ms, 4),
+        "flop_ratio": round(flop_ratio, 4),
+        "speedup_bar": round(0.85 / flop_ratio, 4),
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": state_bytes,
+                "d2h_bytes_per_step": state_bytes, "call": "ts_block_shared with pinned host state in/out"},
+        "gpu_launches": int(gpu_launches),
+        "roofline": roofline,
+        "kernels": kernels,
+        "clocks": clocks,
+    }
+    return res, cfg
+
+
+def kernel_source_sha():
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "shared_token_transformer_b200", "csrc")
+    for fn in sorted(os.listdir(d)):
+        with open(os.path.join(d, fn), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from shared_token_transformer_b200 import workloads as W
+    cfg = W.CONFIGS[args.config]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        budget = 150.0
+        U, times = oracle_shared_layer_timing(cfg, budget, args.steps, warmup=min(args.warmup, 1))
+        mean = float(np.mean(times))
+        v = U / mean
+        res = {"impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": UNIT, "n_gpus": world,
+               "steps": len(times), "warmup": min(args.warmup, 1), "ms_per_step": round(mean * 1e3, 3),
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+               "data": "synthetic (seeded, same draws as the tileshare arm)",
+               "config": {"workload": f"{cfg.name}: {cfg.note}", "grid": list(cfg.grid), "L": cfg.L, "k": cfg.k},
+               "cpu_baseline": {"value": round(v, 2), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"{len(times)} float64 oracle shared layers of {cfg.name} "
+                                          f"(steps capped at a {budget:.0f} s budget)"},
+               "e2e": {"value": round(v, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(res))
+        return
+
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        import torch
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    res, cfg = run_tileshare(args, rank, world, local)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        if flops_layer(cfg.U + 1, 1, 1, cfg.d, cfg.mlp) < 5e11:
+            U, times = oracle_shared_layer_timing(cfg, args.cpu_seconds, 1000)
+            mean = float(np.mean(times))
+            res["cpu_baseline"] = {"value": round(U / mean, 2), "unit": UNIT, "cores": blas_threads(),
+                                   "kind": "oracle",
+                                   "sample": f"{len(times)} float64 oracle shared layers of {cfg.name} "
+                                             f"(~{args.cpu_seconds:.0f} s budget)"}
+        else:
+            res["cpu_baseline"] = None
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res))
+
+
+if __name__ == "__main__":
+    main()

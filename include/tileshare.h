@@ -165,6 +165,12 @@ ts_status ts_decode_stack(ts_plan_t plan, const ts_model_desc* model, const ts_l
                           int L, int k, const void* S0, const void* G0, void* out,
                           void* workspace, size_t workspace_bytes, void* stream);
 
+/* Per-tile copies of the stack input, as ts_decode_stack makes before its first
+   per-tile layer: X[t*N] = G0[t], X[t*N + 1 + j] = S0[grid token of slot j of t].
+   S0 [U, d], G0 [T, d], X [T*N, d] (device, model dtype). */
+ts_status ts_gather_tiles(ts_plan_t plan, const ts_model_desc* model, const void* S0, const void* G0,
+                          void* X, void* stream);
+
 /* Per-row e4m3 quantisation used by TS_FP8_E4M3: scale[r] = max|x[r, :]| / 448
    (1 for an all-zero row), q[r, c] = e4m3(x[r, c] / scale[r]) rounded to nearest
    even and saturated at +-448.  x bf16 [rows, cols] (device), q e4m3 bytes
@@ -177,6 +183,29 @@ ts_status ts_quantize_rows_e4m3(const void* x, int rows, int cols, void* q, floa
    check or bounded wait has failed since the last call, else a TS_ERR_* code.
    Synchronises the device and clears the word. */
 ts_status ts_device_status(void);
+
+/* Kernel trace (tracing subsystem).  Between ts_trace_begin() and ts_trace_end()
+   every kernel the library enqueues is bracketed by two CUDA events on its own
+   stream and recorded with its algorithmic work (FLOPs of the contraction, bytes
+   that must cross HBM at least once).  ts_trace_end() synchronises those events
+   and returns one entry per kernel class, in first-seen order; at most
+   `capacity` entries are written and *count is the number of classes.  Events
+   are taken from a pool made by ts_trace_begin (max_launches events pairs);
+   launches beyond it are counted but not timed.  Process-wide, not for
+   concurrent use by several threads. */
+typedef struct {
+  char name[48];      /* kernel class, e.g. "gemm_up", "attention", "blend"      */
+  int launches;       /* launches recorded                                       */
+  int timed;          /* launches with event timing                              */
+  double ms;          /* summed event time of the timed launches                 */
+  double flops;       /* summed algorithmic FLOPs of the timed launches          */
+  double bytes;       /* summed algorithmic HBM bytes of the timed launches      */
+} ts_trace_entry;
+ts_status ts_trace_begin(int max_launches);
+ts_status ts_trace_end(ts_trace_entry* entries, int capacity, int* count);
+
+/* Kernels enqueued by the library since it was loaded (all devices, all threads). */
+long long ts_launch_count(void);
 
 const char* ts_status_string(ts_status s);
 const char* ts_last_error(void);

@@ -52,6 +52,11 @@ class LayerWeights(ctypes.Structure):
     _fields_ = [(n, _cp) for n in _WEIGHT_FIELDS]
 
 
+class TraceEntry(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 48), ("launches", ctypes.c_int), ("timed", ctypes.c_int),
+                ("ms", ctypes.c_double), ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
+
+
 class TileShareError(RuntimeError):
     def __init__(self, fn, status, msg):
         super().__init__(f"{fn} -> status {status}: {msg}")
@@ -74,6 +79,10 @@ _SIGS = {
     "ts_decode_stack": [_cp, ctypes.POINTER(ModelDesc), ctypes.POINTER(LayerWeights), ctypes.c_int, ctypes.c_int,
                         _cp, _cp, _cp, _cp, ctypes.c_size_t, _cp],
     "ts_quantize_rows_e4m3": [_cp, ctypes.c_int, ctypes.c_int, _cp, _cp, _cp],
+    "ts_gather_tiles": [_cp, ctypes.POINTER(ModelDesc), _cp, _cp, _cp, _cp],
+    "ts_trace_begin": [ctypes.c_int],
+    "ts_trace_end": [ctypes.POINTER(TraceEntry), ctypes.c_int, ctypes.POINTER(ctypes.c_int)],
+    "ts_launch_count": [],
     "ts_device_status": [],
     "ts_status_string": [ctypes.c_int],
     "ts_last_error": [],
@@ -97,6 +106,7 @@ def lib():
             f = getattr(L, name)
             f.argtypes = args
             f.restype = None if name == "ts_plan_destroy" else ctypes.c_int
+        L.ts_launch_count.restype = ctypes.c_longlong
         L.ts_status_string.restype = ctypes.c_char_p
         L.ts_last_error.restype = ctypes.c_char_p
         _lib = L
@@ -204,6 +214,29 @@ def decode_stack(plan, model, weights_list, k, S0, G0, out, ws, stream=None):
     _check("ts_decode_stack", lib().ts_decode_stack(plan.handle, ctypes.byref(model), arr, L, k, _ptr(S0), _ptr(G0),
                                                     _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
                                                     _stream(stream)))
+
+
+def gather_tiles(plan, model, S0, G0, X, stream=None):
+    _check("ts_gather_tiles", lib().ts_gather_tiles(plan.handle, ctypes.byref(model), _ptr(S0), _ptr(G0), _ptr(X),
+                                                    _stream(stream)))
+
+
+def trace_begin(max_launches=100000):
+    _check("ts_trace_begin", lib().ts_trace_begin(max_launches))
+
+
+def trace_end():
+    """Per kernel class: dict name -> {launches, timed, ms, flops, bytes} (synchronises)."""
+    cap = 64
+    arr = (TraceEntry * cap)()
+    n = ctypes.c_int()
+    _check("ts_trace_end", lib().ts_trace_end(arr, cap, ctypes.byref(n)))
+    return {arr[i].name.decode(): {"launches": arr[i].launches, "timed": arr[i].timed, "ms": arr[i].ms,
+                                   "flops": arr[i].flops, "bytes": arr[i].bytes} for i in range(min(n.value, cap))}
+
+
+def launch_count():
+    return int(lib().ts_launch_count())
 
 
 def quantize_rows_e4m3(x, q, scale, stream=None):

@@ -17,7 +17,9 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <string>
+#include <vector>
 
 #include "../../include/tileshare.h"
 #include "../../include/tileshare_ops.h"
@@ -62,6 +64,66 @@ static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t
 static ts_status launched(const char* what) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(TS_ERR_CUDA, "launch of %s failed: %s", what, cudaGetErrorString(e));
+  return TS_OK;
+}
+
+// ============================================================================
+// kernel trace and launch counter
+//   Each launcher calls trace_pre(stream) right before its kernel launch and
+//   trace_post(stream, what) right after; the caller describes the launch's
+//   algorithmic work in g_work (kernel class, FLOPs, HBM bytes).
+// ============================================================================
+struct Work {
+  const char* name;
+  double flops;
+  double bytes;
+};
+static thread_local Work g_work = {"kernel", 0.0, 0.0};
+static thread_local int g_slot = -1;
+static std::atomic<long long> g_launches{0};
+
+struct TraceRec {
+  int cls, slot;
+  double flops, bytes;
+};
+static struct {
+  bool on = false;
+  int cap = 0, used = 0;
+  std::vector<cudaEvent_t> ev;
+  std::vector<std::string> names;
+  std::vector<long long> count;
+  std::vector<TraceRec> recs;
+} g_trace;
+
+static void set_work(const char* name, double flops, double bytes) { g_work = {name, flops, bytes}; }
+
+static void trace_pre(cudaStream_t st) {
+  g_slot = -1;
+  if (g_trace.on && g_trace.used < g_trace.cap) {
+    g_slot = g_trace.used++;
+    cudaEventRecord(g_trace.ev[2 * g_slot], st);
+  }
+}
+
+static ts_status trace_post(cudaStream_t st, const char* what) {
+  ++g_launches;
+  TS_TRY(launched(what));
+  if (g_trace.on) {
+    int cls = -1;
+    for (size_t i = 0; i < g_trace.names.size(); ++i)
+      if (g_trace.names[i] == g_work.name) cls = static_cast<int>(i);
+    if (cls < 0) {
+      cls = static_cast<int>(g_trace.names.size());
+      g_trace.names.push_back(g_work.name);
+      g_trace.count.push_back(0);
+    }
+    g_trace.count[cls]++;
+    if (g_slot >= 0) {
+      cudaEventRecord(g_trace.ev[2 * g_slot + 1], st);
+      g_trace.recs.push_back({cls, g_slot, g_work.flops, g_work.bytes});
+    }
+  }
+  g_slot = -1;
   return TS_OK;
 }
 
@@ -233,6 +295,7 @@ static ts_status launch_layernorm_vec(const void* x, int rows, int d, const floa
   const int nv = d / (32 * E);
   const T* xx = static_cast<const T*>(x);
   T* yy = static_cast<T*>(y);
+  trace_pre(st);
 #define TS_LN_CASE(NV) \
   case NV: ts::layernorm_kernel<T, NV, Q8><<<rows_grid(rows), 256, 0, st>>>(xx, rows, d, g, b, eps, yy, q8, qs); break;
   switch (nv) {
@@ -240,7 +303,7 @@ static ts_status launch_layernorm_vec(const void* x, int rows, int d, const floa
     default: return fail(TS_ERR_UNSUPPORTED, "layernorm width %d", d);
   }
 #undef TS_LN_CASE
-  return launched("layernorm");
+  return trace_post(st, "layernorm");
 }
 
 // y = LN(x); for e4m3 writes q8/qs instead of y.
@@ -248,11 +311,14 @@ static ts_status run_layernorm(const ts_model_desc* m, const void* x, int rows, 
                                void* y, uint8_t* q8, float* qs, cudaStream_t st) {
   if (rows == 0) return TS_OK;
   const int d = m->d;
+  const double e = esize(m->dtype);
+  set_work("layernorm", 0.0, static_cast<double>(rows) * d * (e + (q8 ? 1.0 : e)) + (q8 ? 4.0 * rows : 0.0));
   if (m->dtype == TS_F32) {
     if (d % 128 == 0 && d <= 1024) return launch_layernorm_vec<float, false>(x, rows, d, g, b, m->eps_ln, y, nullptr, nullptr, st);
+    trace_pre(st);
     ts::layernorm_generic_kernel<float><<<rows_grid(rows), 256, 0, st>>>(static_cast<const float*>(x), rows, d, g, b,
                                                                         m->eps_ln, static_cast<float*>(y));
-    return launched("layernorm_generic");
+    return trace_post(st, "layernorm_generic");
   }
   if (q8) return launch_layernorm_vec<bf16, true>(x, rows, d, g, b, m->eps_ln, nullptr, q8, qs, st);
   return launch_layernorm_vec<bf16, false>(x, rows, d, g, b, m->eps_ln, y, nullptr, nullptr, st);
@@ -265,6 +331,7 @@ static ts_status launch_merge_vec(const ts_plan_s* p, const void* P, int rows, i
   const int nv = d / (32 * E);
   const T* pp = static_cast<const T*>(P);
   T* aa = static_cast<T*>(A);
+  trace_pre(st);
 #define TS_MG_CASE(NV)                                                                                    \
   case NV:                                                                                                \
     ts::merge_kernel<T, NV, Q8><<<rows_grid(rows), 256, 0, st>>>(pp, rows, p->U, p->N, d, p->d_tok_ptr,  \
@@ -275,19 +342,27 @@ static ts_status launch_merge_vec(const ts_plan_s* p, const void* P, int rows, i
     default: return fail(TS_ERR_UNSUPPORTED, "merge width %d", d);
   }
 #undef TS_MG_CASE
-  return launched("merge");
+  return trace_post(st, "merge");
 }
 
-static ts_status run_merge(const ts_plan_s* p, const ts_model_desc* m, const void* P, int rows, void* A, uint8_t* q8,
-                           float* qs, cudaStream_t st) {
+static ts_status run_merge(const char* name, const ts_plan_s* p, const ts_model_desc* m, const void* P, int rows,
+                           void* A, uint8_t* q8, float* qs, cudaStream_t st) {
   if (rows == 0) return TS_OK;
   const int d = m->d;
+  {
+    // reads every (tile, slot) entry of the rows written once, writes each row once
+    const double e = esize(m->dtype);
+    const double reads = static_cast<double>(p->nnz) * d * e + (rows > p->U ? static_cast<double>(rows - p->U) * d * e : 0.0);
+    const double writes = static_cast<double>(rows) * d * (q8 ? 1.0 : e) + (q8 ? 4.0 * rows : 0.0);
+    set_work(name, 0.0, reads + writes);
+  }
   if (m->dtype == TS_F32) {
     if (d % 128 == 0 && d <= 1024) return launch_merge_vec<float, false>(p, P, rows, d, A, nullptr, nullptr, st);
+    trace_pre(st);
     ts::merge_generic_kernel<float><<<rows_grid(rows), 256, 0, st>>>(static_cast<const float*>(P), rows, p->U, p->N, d,
                                                                     p->d_tok_ptr, p->d_tok_ent, p->d_wbar,
                                                                     static_cast<float*>(A));
-    return launched("merge_generic");
+    return trace_post(st, "merge_generic");
   }
   if (q8) return launch_merge_vec<bf16, true>(p, P, rows, d, nullptr, q8, qs, st);
   return launch_merge_vec<bf16, false>(p, P, rows, d, A, nullptr, nullptr, st);
@@ -295,8 +370,10 @@ static ts_status run_merge(const ts_plan_s* p, const ts_model_desc* m, const voi
 
 static ts_status run_quantize(const void* x, int rows, int cols, uint8_t* q, float* s, cudaStream_t st) {
   if (rows == 0) return TS_OK;
+  set_work("quantize_e4m3", 0.0, static_cast<double>(rows) * cols * 3.0 + 4.0 * rows);
+  trace_pre(st);
   ts::quantize_rows_kernel<<<rows_grid(rows), 256, 0, st>>>(static_cast<const bf16*>(x), rows, cols, q, s);
-  return launched("quantize_rows");
+  return trace_post(st, "quantize_rows");
 }
 
 // ---------------------------------------------------------------------------
@@ -327,8 +404,9 @@ static ts_status launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, co
     configured[dev] = 1;
   }
   dim3 grid((args.M + 127) / 128, args.N / BN);
+  trace_pre(st);
   kern<<<grid, 192, SM::LAUNCH_BYTES, st>>>(ta, tb, args);
-  return launched("gemm_tc");
+  return trace_post(st, "gemm_tc");
 }
 
 template <int EPI, bool FP8, int R0, int R1, int R2>
@@ -352,11 +430,17 @@ static int pick_bn(int M, int N) {
 }
 
 // Y[M, N] = A[M, K] W[N, K]^T with epilogue; A bf16 (or e4m3 + a_scale), W bf16 (or e4m3 + w_scale).
-static ts_status run_gemm_tc(const ts_model_desc* m, int epi, const void* A, const float* a_scale, const void* W,
-                             const float* w_scale, int M, int N, int K, const float* bias, bf16* out,
+static ts_status run_gemm_tc(const char* name, const ts_model_desc* m, int epi, const void* A, const float* a_scale,
+                             const void* W, const float* w_scale, int M, int N, int K, const float* bias, bf16* out,
                              const ts_layer_weights* qk, const int* pos, cudaStream_t st) {
   if (M == 0) return TS_OK;
   const bool fp8 = m->dtype == TS_FP8_E4M3;
+  {
+    const double ea = fp8 ? 1.0 : 2.0;
+    const double bytes = static_cast<double>(M) * K * ea + static_cast<double>(N) * K * ea +
+                         static_cast<double>(M) * N * 2.0 * (epi == ts::EPI_RESID ? 2.0 : 1.0);
+    set_work(name, 2.0 * M * static_cast<double>(N) * K, bytes);
+  }
   if (K % (fp8 ? 128 : 64) || N % 64) return fail(TS_ERR_UNSUPPORTED, "GEMM sizes K=%d N=%d not tiled", K, N);
   const int bn = pick_bn(M, N);
   CUtensorMap ta, tb;
@@ -393,16 +477,19 @@ static ts_status run_gemm_tc(const ts_model_desc* m, int epi, const void* A, con
 }
 
 // fp32 SIMT GEMM
-static ts_status run_gemm_f32(int epi, const float* A, const float* W, int M, int N, int K, const float* bias, float* Y,
-                              cudaStream_t st) {
+static ts_status run_gemm_f32(const char* name, int epi, const float* A, const float* W, int M, int N, int K,
+                              const float* bias, float* Y, cudaStream_t st) {
   if (M == 0) return TS_OK;
+  set_work(name, 2.0 * M * static_cast<double>(N) * K,
+           4.0 * (static_cast<double>(M) * K + static_cast<double>(N) * K + M * static_cast<double>(N) * (epi == ts::EPI_RESID ? 2 : 1)));
   dim3 grid((M + 63) / 64, (N + 63) / 64);
+  trace_pre(st);
   switch (epi) {
     case ts::EPI_GELU: ts::gemm_f32_kernel<1><<<grid, 256, 0, st>>>(A, W, bias, Y, M, N, K); break;
     case ts::EPI_RESID: ts::gemm_f32_kernel<2><<<grid, 256, 0, st>>>(A, W, bias, Y, M, N, K); break;
     default: ts::gemm_f32_kernel<0><<<grid, 256, 0, st>>>(A, W, bias, Y, M, N, K); break;
   }
-  return launched("gemm_f32");
+  return trace_post(st, "gemm_f32");
 }
 
 // ---------------------------------------------------------------------------
@@ -422,6 +509,11 @@ static ts_status run_attention(const ts_plan_s* p, const ts_model_desc* m, bool 
   a.T = p->T;
   a.scale = 1.0f / std::sqrt(static_cast<float>(hd));
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(hd)));
+  {
+    const double e = esize(m->dtype), rows = static_cast<double>(p->T) * p->N;
+    set_work("attention", 4.0 * p->T * static_cast<double>(p->N) * p->N * m->d, rows * 3.0 * m->d * e + rows * m->d * e);
+  }
+  trace_pre(st);
   if (m->dtype == TS_F32) {
     dim3 grid((p->N + 63) / 64, m->heads, p->T);
     switch (hd) {
@@ -429,12 +521,12 @@ static ts_status run_attention(const ts_plan_s* p, const ts_model_desc* m, bool 
       case 32: ts::attn_f32_kernel<32><<<grid, 64, 0, st>>>(a); break;
       default: ts::attn_f32_kernel<64><<<grid, 64, 0, st>>>(a); break;
     }
-    return launched("attn_f32");
+    return trace_post(st, "attn_f32");
   }
   const int nqb = (p->Nw + ts::kAttnBQ - 1) / ts::kAttnBQ;
   dim3 grid(nqb + 1, m->heads, p->T);
   ts::attn_bf16_kernel<<<grid, 128, ts::kAttnBf16SmemMax, st>>>(a);
-  return launched("attn_bf16");
+  return trace_post(st, "attn_bf16");
 }
 
 // ---------------------------------------------------------------------------
@@ -447,23 +539,25 @@ static ts_status run_qkv(const ts_plan_s* p, const ts_model_desc* m, const ts_la
   const int d = m->d;
   if (m->dtype == TS_F32) {
     TS_TRY(run_layernorm(m, state, rows, w->ln1_g, w->ln1_b, ws.xn, nullptr, nullptr, st));
-    TS_TRY(run_gemm_f32(ts::EPI_BIAS, static_cast<const float*>(ws.xn), static_cast<const float*>(w->w_qkv), rows,
+    TS_TRY(run_gemm_f32("gemm_qkv", ts::EPI_BIAS, static_cast<const float*>(ws.xn), static_cast<const float*>(w->w_qkv), rows,
                         3 * d, d, w->b_qkv, static_cast<float*>(qkv), st));
     ts::RopeF32 r{};
     for (int a = 0; a < 3; ++a) r.dims[a] = m->rope_dims[a];
     fill_theta(m, r.th_hi, r.th_lo);
     const size_t n = static_cast<size_t>(rows) * m->heads * 2;
+    set_work("qk_norm_rope", 0.0, 2.0 * rows * 2.0 * d * 4.0);
+    trace_pre(st);
     ts::qk_norm_rope_f32_kernel<<<static_cast<unsigned>((n + 127) / 128), 128, 0, st>>>(
         static_cast<float*>(qkv), rows, d, m->heads, w->q_g, w->k_g, m->eps_qk, reinterpret_cast<const int4*>(pos), r);
-    return launched("qk_norm_rope_f32");
+    return trace_post(st, "qk_norm_rope_f32");
   }
   if (m->dtype == TS_FP8_E4M3) {
     TS_TRY(run_layernorm(m, state, rows, w->ln1_g, w->ln1_b, nullptr, ws.q8, ws.qs, st));
-    return run_gemm_tc(m, ts::EPI_QKV, ws.q8, ws.qs, w->w_qkv, w->s_qkv, rows, 3 * d, d, w->b_qkv,
+    return run_gemm_tc("gemm_qkv", m, ts::EPI_QKV, ws.q8, ws.qs, w->w_qkv, w->s_qkv, rows, 3 * d, d, w->b_qkv,
                        static_cast<bf16*>(qkv), w, pos, st);
   }
   TS_TRY(run_layernorm(m, state, rows, w->ln1_g, w->ln1_b, ws.xn, nullptr, nullptr, st));
-  return run_gemm_tc(m, ts::EPI_QKV, ws.xn, nullptr, w->w_qkv, nullptr, rows, 3 * d, d, w->b_qkv,
+  return run_gemm_tc("gemm_qkv", m, ts::EPI_QKV, ws.xn, nullptr, w->w_qkv, nullptr, rows, 3 * d, d, w->b_qkv,
                      static_cast<bf16*>(qkv), w, pos, st);
 }
 
@@ -472,14 +566,14 @@ static ts_status run_out_proj(const ts_model_desc* m, const ts_layer_weights* w,
                               int rows, void* state, const Workspace& ws, cudaStream_t st) {
   const int d = m->d;
   if (m->dtype == TS_F32)
-    return run_gemm_f32(ts::EPI_RESID, static_cast<const float*>(att), static_cast<const float*>(w->w_o), rows, d, d,
+    return run_gemm_f32("gemm_out", ts::EPI_RESID, static_cast<const float*>(att), static_cast<const float*>(w->w_o), rows, d, d,
                         w->b_o, static_cast<float*>(state), st);
   if (m->dtype == TS_FP8_E4M3) {
     if (!att_quantised) TS_TRY(run_quantize(att, rows, d, ws.q8, ws.qs, st));
-    return run_gemm_tc(m, ts::EPI_RESID, ws.q8, ws.qs, w->w_o, w->s_o, rows, d, d, w->b_o, static_cast<bf16*>(state),
+    return run_gemm_tc("gemm_out", m, ts::EPI_RESID, ws.q8, ws.qs, w->w_o, w->s_o, rows, d, d, w->b_o, static_cast<bf16*>(state),
                        nullptr, nullptr, st);
   }
-  return run_gemm_tc(m, ts::EPI_RESID, att, nullptr, w->w_o, nullptr, rows, d, d, w->b_o, static_cast<bf16*>(state),
+  return run_gemm_tc("gemm_out", m, ts::EPI_RESID, att, nullptr, w->w_o, nullptr, rows, d, d, w->b_o, static_cast<bf16*>(state),
                      nullptr, nullptr, st);
 }
 
@@ -489,24 +583,37 @@ static ts_status run_mlp(const ts_model_desc* m, const ts_layer_weights* w, int 
   const int d = m->d, f = m->mlp;
   if (m->dtype == TS_F32) {
     TS_TRY(run_layernorm(m, state, rows, w->ln2_g, w->ln2_b, ws.xn, nullptr, nullptr, st));
-    TS_TRY(run_gemm_f32(ts::EPI_GELU, static_cast<const float*>(ws.xn), static_cast<const float*>(w->w_1), rows, f, d,
+    TS_TRY(run_gemm_f32("gemm_up", ts::EPI_GELU, static_cast<const float*>(ws.xn), static_cast<const float*>(w->w_1), rows, f, d,
                         w->b_1, static_cast<float*>(ws.h), st));
-    return run_gemm_f32(ts::EPI_RESID, static_cast<const float*>(ws.h), static_cast<const float*>(w->w_2), rows, d, f,
+    return run_gemm_f32("gemm_down", ts::EPI_RESID, static_cast<const float*>(ws.h), static_cast<const float*>(w->w_2), rows, d, f,
                         w->b_2, static_cast<float*>(state), st);
   }
   if (m->dtype == TS_FP8_E4M3) {
     TS_TRY(run_layernorm(m, state, rows, w->ln2_g, w->ln2_b, nullptr, ws.q8, ws.qs, st));
-    TS_TRY(run_gemm_tc(m, ts::EPI_GELU, ws.q8, ws.qs, w->w_1, w->s_1, rows, f, d, w->b_1, static_cast<bf16*>(ws.h),
+    TS_TRY(run_gemm_tc("gemm_up", m, ts::EPI_GELU, ws.q8, ws.qs, w->w_1, w->s_1, rows, f, d, w->b_1, static_cast<bf16*>(ws.h),
                        nullptr, nullptr, st));
     TS_TRY(run_quantize(ws.h, rows, f, ws.q8, ws.qs, st));
-    return run_gemm_tc(m, ts::EPI_RESID, ws.q8, ws.qs, w->w_2, w->s_2, rows, d, f, w->b_2, static_cast<bf16*>(state),
+    return run_gemm_tc("gemm_down", m, ts::EPI_RESID, ws.q8, ws.qs, w->w_2, w->s_2, rows, d, f, w->b_2, static_cast<bf16*>(state),
                        nullptr, nullptr, st);
   }
   TS_TRY(run_layernorm(m, state, rows, w->ln2_g, w->ln2_b, ws.xn, nullptr, nullptr, st));
-  TS_TRY(run_gemm_tc(m, ts::EPI_GELU, ws.xn, nullptr, w->w_1, nullptr, rows, f, d, w->b_1, static_cast<bf16*>(ws.h),
+  TS_TRY(run_gemm_tc("gemm_up", m, ts::EPI_GELU, ws.xn, nullptr, w->w_1, nullptr, rows, f, d, w->b_1, static_cast<bf16*>(ws.h),
                      nullptr, nullptr, st));
-  return run_gemm_tc(m, ts::EPI_RESID, ws.h, nullptr, w->w_2, nullptr, rows, d, f, w->b_2, static_cast<bf16*>(state),
+  return run_gemm_tc("gemm_down", m, ts::EPI_RESID, ws.h, nullptr, w->w_2, nullptr, rows, d, f, w->b_2, static_cast<bf16*>(state),
                      nullptr, nullptr, st);
+}
+
+// per-tile copies of the stack input (grid tokens S0, global tokens G0)
+static ts_status run_gather(const ts_plan_s* p, const ts_model_desc* m, const void* S0, const void* G0, void* X,
+                            cudaStream_t st) {
+  const int nrows = p->T * p->N;
+  const size_t rb = static_cast<size_t>(m->d) * esize(m->dtype);
+  set_work("gather", 0.0, 2.0 * nrows * static_cast<double>(rb));
+  trace_pre(st);
+  ts::gather_rows_kernel<<<rows_grid(nrows), 256, 0, st>>>(static_cast<const uint8_t*>(S0),
+                                                           static_cast<const uint8_t*>(G0), p->d_rowmap, nrows, p->U,
+                                                           rb, static_cast<uint8_t*>(X));
+  return trace_post(st, "gather_rows");
 }
 
 // ============================================================================
@@ -527,7 +634,7 @@ static ts_status layer_shared(const ts_plan_s* p, const ts_model_desc* m, const 
   TS_TRY(run_qkv(p, m, w, true, S, ws.qkv, ws, st));
   TS_TRY(run_attention(p, m, true, ws.qkv, ws.o, st));
   const bool q = m->dtype == TS_FP8_E4M3;
-  TS_TRY(run_merge(p, m, ws.o, rows, q ? nullptr : ws.a, q ? ws.q8 : nullptr, q ? ws.qs : nullptr, st));
+  TS_TRY(run_merge("blend", p, m, ws.o, rows, q ? nullptr : ws.a, q ? ws.q8 : nullptr, q ? ws.qs : nullptr, st));
   TS_TRY(run_out_proj(m, w, ws.a, q, rows, S, ws, st));
   return run_mlp(m, w, rows, S, ws, st);
 }
@@ -546,6 +653,58 @@ static ts_status check_ws(const ts_plan_s* p, const ts_model_desc* m, bool stack
 // C ABI
 // ============================================================================
 extern "C" {
+
+ts_status ts_gather_tiles(ts_plan_t p, const ts_model_desc* m, const void* S0, const void* G0, void* X,
+                          void* stream) {
+  TS_TRY(check_plan(p));
+  TS_TRY(check_model(m));
+  if (!S0 || !G0 || !X || !aligned16(S0) || !aligned16(G0) || !aligned16(X))
+    return fail(TS_ERR_INVALID_ARG, "S0, G0, X must be 16-byte aligned device pointers");
+  return run_gather(p, m, S0, G0, X, static_cast<cudaStream_t>(stream));
+}
+
+ts_status ts_trace_begin(int max_launches) {
+  if (max_launches < 0) return fail(TS_ERR_INVALID_ARG, "max_launches < 0");
+  if (g_trace.on) return fail(TS_ERR_INVALID_ARG, "trace already running");
+  for (cudaEvent_t e : g_trace.ev) cudaEventDestroy(e);
+  g_trace.ev.assign(2 * static_cast<size_t>(max_launches), nullptr);
+  for (auto& e : g_trace.ev) TS_CUDA_CHECK(cudaEventCreate(&e));
+  g_trace.cap = max_launches;
+  g_trace.used = 0;
+  g_trace.names.clear();
+  g_trace.count.clear();
+  g_trace.recs.clear();
+  g_trace.on = true;
+  return TS_OK;
+}
+
+ts_status ts_trace_end(ts_trace_entry* entries, int capacity, int* count) {
+  if (!g_trace.on) return fail(TS_ERR_INVALID_ARG, "no trace running");
+  g_trace.on = false;
+  const size_t n = g_trace.names.size();
+  std::vector<ts_trace_entry> out(n);
+  for (size_t i = 0; i < n; ++i) {
+    std::memset(&out[i], 0, sizeof(ts_trace_entry));
+    std::strncpy(out[i].name, g_trace.names[i].c_str(), sizeof(out[i].name) - 1);
+    out[i].launches = static_cast<int>(g_trace.count[i]);
+  }
+  for (const TraceRec& r : g_trace.recs) {
+    TS_CUDA_CHECK(cudaEventSynchronize(g_trace.ev[2 * r.slot + 1]));
+    float ms = 0.f;
+    TS_CUDA_CHECK(cudaEventElapsedTime(&ms, g_trace.ev[2 * r.slot], g_trace.ev[2 * r.slot + 1]));
+    ts_trace_entry& e = out[r.cls];
+    e.timed += 1;
+    e.ms += ms;
+    e.flops += r.flops;
+    e.bytes += r.bytes;
+  }
+  if (count) *count = static_cast<int>(n);
+  if (entries)
+    for (size_t i = 0; i < n && static_cast<int>(i) < capacity; ++i) entries[i] = out[i];
+  return TS_OK;
+}
+
+long long ts_launch_count(void) { return g_launches.load(); }
 
 const char* ts_status_string(ts_status s) {
   switch (s) {
@@ -712,14 +871,10 @@ ts_status ts_decode_stack(ts_plan_t p, const ts_model_desc* m, const ts_layer_we
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t rb = static_cast<size_t>(m->d) * esize(m->dtype);
   if (k > 0) {
-    const int nrows = p->T * p->N;
-    ts::gather_rows_kernel<<<rows_grid(nrows), 256, 0, st>>>(static_cast<const uint8_t*>(S0),
-                                                             static_cast<const uint8_t*>(G0), p->d_rowmap, nrows, p->U,
-                                                             rb, static_cast<uint8_t*>(W.X));
-    TS_TRY(launched("gather_rows"));
+    TS_TRY(run_gather(p, m, S0, G0, W.X, st));
     for (int l = 0; l < k; ++l) TS_TRY(layer_tiled(p, m, w + l, W.X, W, st));
-    if (k == L) return run_merge(p, m, W.X, p->U, out, nullptr, nullptr, st);
-    TS_TRY(run_merge(p, m, W.X, p->U + p->T, W.S, nullptr, nullptr, st));
+    if (k == L) return run_merge("merge", p, m, W.X, p->U, out, nullptr, nullptr, st);
+    TS_TRY(run_merge("merge", p, m, W.X, p->U + p->T, W.S, nullptr, nullptr, st));
   } else {
     TS_CUDA_CHECK(cudaMemcpyAsync(W.S, S0, rb * p->U, cudaMemcpyDeviceToDevice, st));
     TS_CUDA_CHECK(cudaMemcpyAsync(static_cast<char*>(W.S) + rb * p->U, G0, rb * p->T, cudaMemcpyDeviceToDevice, st));
@@ -767,16 +922,16 @@ ts_status ts_op_linear(const ts_model_desc* m, const void* x, int rows, int K, c
   const int e = epi == TS_EPI_BIAS ? ts::EPI_BIAS : epi == TS_EPI_BIAS_GELU ? ts::EPI_GELU : ts::EPI_RESID;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (m->dtype == TS_F32)
-    return run_gemm_f32(e, static_cast<const float*>(x), static_cast<const float*>(W), rows, N, K, bias,
+    return run_gemm_f32("linear", e, static_cast<const float*>(x), static_cast<const float*>(W), rows, N, K, bias,
                         static_cast<float*>(y), st);
   if (m->dtype == TS_FP8_E4M3) {
     if (!scratch || !aligned16(scratch) || !w_scale) return fail(TS_ERR_INVALID_ARG, "e4m3 linear needs scratch and w_scale");
     uint8_t* q8 = static_cast<uint8_t*>(scratch);
     float* qs = reinterpret_cast<float*>(q8 + align256(static_cast<size_t>(rows) * K));
     TS_TRY(run_quantize(x, rows, K, q8, qs, st));
-    return run_gemm_tc(m, e, q8, qs, W, w_scale, rows, N, K, bias, static_cast<bf16*>(y), nullptr, nullptr, st);
+    return run_gemm_tc("linear", m, e, q8, qs, W, w_scale, rows, N, K, bias, static_cast<bf16*>(y), nullptr, nullptr, st);
   }
-  return run_gemm_tc(m, e, x, nullptr, W, nullptr, rows, N, K, bias, static_cast<bf16*>(y), nullptr, nullptr, st);
+  return run_gemm_tc("linear", m, e, x, nullptr, W, nullptr, rows, N, K, bias, static_cast<bf16*>(y), nullptr, nullptr, st);
 }
 
 ts_status ts_op_qkv(ts_plan_t p, const ts_model_desc* m, const ts_layer_weights* w, ts_rows_mode mode,
@@ -808,7 +963,7 @@ ts_status ts_op_merge(ts_plan_t p, const ts_model_desc* m, const void* P, int ro
   TS_TRY(check_model(m));
   if (!P || !A || !aligned16(P) || !aligned16(A)) return fail(TS_ERR_INVALID_ARG, "bad argument");
   if (rows != p->U && rows != p->U + p->T) return fail(TS_ERR_INVALID_ARG, "rows must be U or U + T");
-  return run_merge(p, m, P, rows, A, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+  return run_merge("merge", p, m, P, rows, A, nullptr, nullptr, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

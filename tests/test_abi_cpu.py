@@ -25,7 +25,7 @@ def _declared():
     names = set()
     for h in os.listdir(os.path.join(ROOT, "include")):
         txt = open(os.path.join(ROOT, "include", h)).read()
-        names |= set(re.findall(r"^(?:ts_status|void|const char\*)\s+(ts_\w+)\s*\(", txt, re.M))
+        names |= set(re.findall(r"^(?:ts_status|void|long long|const char\*)\s+(ts_\w+)\s*\(", txt, re.M))
     return names
 
 

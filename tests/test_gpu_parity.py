@@ -278,7 +278,7 @@ def test_error_paths():
         B.block_shared(c.plan, c.m, c.wlist[0], S, ws[:-1024])
     assert e.value.status == 3
     with pytest.raises(B.TileShareError) as e:
-        B.block_shared(c.plan, c.m, c.wlist[0], S.view(torch.uint8)[2:], ws)
+        B.block_shared(c.plan, c.m, c.wlist[0], S.view(torch.uint8).flatten()[2:], ws)
     assert e.value.status == 1
     bad = dict(c.dlayers[0])
     bad["w_o"] = None
