@@ -154,6 +154,31 @@ ts_status ts_block_tiled(ts_plan_t plan, const ts_model_desc* model, const ts_la
 ts_status ts_block_shared(ts_plan_t plan, const ts_model_desc* model, const ts_layer_weights* w,
                           void* S, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Shared layer without a caller workspace.  The paper has no counterpart: this
+   entry point exists for callers that cannot allocate device memory, such as a
+   plugin running inside a host application that owns every device buffer
+   through its own pool and forbids the plugin from calling cudaMalloc, or code
+   working inside a fixed, pre-partitioned memory budget.  It computes exactly
+   what ts_block_shared computes, in place on S [U + T, d], but its scratch
+   (normalised rows, q/k/v, attention outputs, blend, MLP hidden) lives in one
+   static device array of TS_NOALLOC_SCRATCH_BYTES (32 MiB) that every GPU
+   loading the library holds until the process exits.
+   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+   - Plans and models needing more scratch than the array holds are refused with
+     TS_ERR_WORKSPACE before anything is launched (the 48x48-token, d = 512
+     workload needs about 26 MB; large grids do not fit and must use
+     ts_block_shared).
+   - The first call on a device looks up the array's device address
+     (cudaGetSymbolAddress) with that device current; make that first call
+     before any stream capture on the device.
+   - Every call shares the one array and leaves its contents behind.  No region
+     has to start at zero: each is written before it is read within a call.
+     Calls that overlap on the GPU (other streams, other threads) race on the
+     array and must be serialised by the caller. */
+#define TS_NOALLOC_SCRATCH_BYTES (32u << 20)
+ts_status ts_block_shared_noalloc(ts_plan_t plan, const ts_model_desc* model, const ts_layer_weights* w,
+                                  void* S, void* stream);
+
 /* TileShare-k stack ([TileShare] abstract, Tab. 1): layers 0..k-1 per tile on the
    copies of S0/G0 in every tile, then the per-tile states are merged with w-bar
    (Fig. 3b), then layers k..L-1 shared.  With k = L this is overlapping tiled

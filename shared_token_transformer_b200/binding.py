@@ -76,6 +76,7 @@ _SIGS = {
     "ts_workspace_size": [_cp, ctypes.POINTER(ModelDesc), ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)],
     "ts_block_tiled": [_cp, ctypes.POINTER(ModelDesc), ctypes.POINTER(LayerWeights), _cp, _cp, ctypes.c_size_t, _cp],
     "ts_block_shared": [_cp, ctypes.POINTER(ModelDesc), ctypes.POINTER(LayerWeights), _cp, _cp, ctypes.c_size_t, _cp],
+    "ts_block_shared_noalloc": [_cp, ctypes.POINTER(ModelDesc), ctypes.POINTER(LayerWeights), _cp, _cp],
     "ts_decode_stack": [_cp, ctypes.POINTER(ModelDesc), ctypes.POINTER(LayerWeights), ctypes.c_int, ctypes.c_int,
                         _cp, _cp, _cp, _cp, ctypes.c_size_t, _cp],
     "ts_quantize_rows_e4m3": [_cp, ctypes.c_int, ctypes.c_int, _cp, _cp, _cp],
@@ -206,6 +207,12 @@ def block_tiled(plan, model, weights, X, ws, stream=None):
 def block_shared(plan, model, weights, S, ws, stream=None):
     _check("ts_block_shared", lib().ts_block_shared(plan.handle, ctypes.byref(model), ctypes.byref(weights), _ptr(S),
                                                     _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def block_shared_noalloc(plan, model, weights, S, stream=None):
+    """ts_block_shared with the library's static scratch instead of a workspace (allocates nothing)."""
+    _check("ts_block_shared_noalloc", lib().ts_block_shared_noalloc(plan.handle, ctypes.byref(model),
+                                                                    ctypes.byref(weights), _ptr(S), _stream(stream)))
 
 
 def decode_stack(plan, model, weights_list, k, S0, G0, out, ws, stream=None):

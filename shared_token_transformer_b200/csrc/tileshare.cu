@@ -18,6 +18,7 @@
 #include <cstdio>
 #include <cstring>
 #include <atomic>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -854,6 +855,78 @@ ts_status ts_block_shared(ts_plan_t p, const ts_model_desc* m, const ts_layer_we
   if (!S || !aligned16(S)) return fail(TS_ERR_INVALID_ARG, "S must be a 16-byte aligned device pointer");
   Workspace W;
   TS_TRY(check_ws(p, m, false, ws, ws_bytes, &W));
+  return layer_shared(p, m, w, S, W, static_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------------------
+// Shared layer with its scratch in a static device array (no allocation).
+// ---------------------------------------------------------------------------
+}  // extern "C"
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[TS_NOALLOC_SCRATCH_BYTES];
+
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_ptr[64];
+
+// Device address of the static scratch on the current device, looked up once per
+// device (with that device current) and cached.
+static ts_status noalloc_scratch(void** out) {
+  int dev = -1;
+  TS_CUDA_CHECK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(TS_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(TS_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return TS_OK;
+}
+
+// Scratch regions of one shared layer only (rows U + T, attention outputs T * N).
+static Workspace layout_shared_scratch(const ts_plan_s* p, const ts_model_desc* m, char* base) {
+  const size_t Mt = static_cast<size_t>(p->T) * p->N, Ms = static_cast<size_t>(p->U) + p->T;
+  const size_t e = esize(m->dtype), d = m->d, f = m->mlp;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* r = base ? base + off : nullptr;
+    off += align256(bytes);
+    return r;
+  };
+  Workspace w{};
+  w.xn = take(Ms * d * e);
+  w.qkv = take(Ms * 3 * d * e);
+  w.o = take(Mt * d * e);
+  w.a = take(Ms * d * e);
+  w.h = take(Ms * f * e);
+  if (m->dtype == TS_FP8_E4M3) {
+    w.q8 = reinterpret_cast<uint8_t*>(take(Ms * std::max(d, f)));
+    w.qs = reinterpret_cast<float*>(take(Ms * 4));
+  }
+  w.bytes = off;
+  return w;
+}
+
+extern "C" {
+
+ts_status ts_block_shared_noalloc(ts_plan_t p, const ts_model_desc* m, const ts_layer_weights* w, void* S,
+                                  void* stream) {
+  TS_TRY(check_plan(p));
+  TS_TRY(check_model(m));
+  TS_TRY(check_weights(m, w));
+  if (!S || !aligned16(S)) return fail(TS_ERR_INVALID_ARG, "S must be a 16-byte aligned device pointer");
+  const size_t need = layout_shared_scratch(p, m, nullptr).bytes;
+  if (need > TS_NOALLOC_SCRATCH_BYTES)
+    return fail(TS_ERR_WORKSPACE,
+                "ts_block_shared_noalloc: this plan and model need %zu bytes of scratch, the static array holds %u; "
+                "use ts_block_shared with a workspace",
+                need, TS_NOALLOC_SCRATCH_BYTES);
+  void* base = nullptr;
+  TS_TRY(noalloc_scratch(&base));
+  const Workspace W = layout_shared_scratch(p, m, static_cast<char*>(base));
   return layer_shared(p, m, w, S, W, static_cast<cudaStream_t>(stream));
 }
 
