@@ -11,15 +11,19 @@
 // For e4m3 operands acc is first multiplied by the row scale of A and the column
 // scale of W.
 //
-// Kernel design (one 128 x BN output tile per CTA, 192 threads):
-//   warp 0   TMA producer: A and W tiles of 128-byte K slices (64 bf16 / 128 e4m3)
-//            into a STAGES-deep ring of 128-byte-swizzled shared buffers;
-//   warp 1   allocates BN TMEM columns and, from one lane, issues tcgen05.mma
-//            (M = 128, N = BN, K = 16 bf16 / 32 e4m3 per instruction) into the fp32
-//            accumulator in TMEM; tcgen05.commit frees each ring slot and finally
-//            signals the epilogue;
-//   warps 2-5  epilogue: tcgen05.ld of their 32 TMEM lanes (one output row per
-//            thread), fused math, bf16 stores.
+// Kernel design: persistent, warp-specialised, 320 threads, CTAs walk the
+// 128 x BN output tiles in a static round-robin order.
+//   warp 8   TMA producer: A and W tiles of 128-byte K slices (64 bf16 / 128 e4m3)
+//            into a STAGES-deep ring of 128-byte-swizzled shared buffers
+//            (no multicast);
+//   warp 9   allocates 2 x BN TMEM columns (two accumulators) and, from one lane,
+//            issues tcgen05.mma (M = 128, N = BN, K = 16 bf16 / 32 e4m3 per
+//            instruction); tcgen05.commit frees ring slots and hands a finished
+//            accumulator to the epilogue;
+//   warps 0-7  epilogue in two warpgroups: warp w reads TMEM lane quarter w % 4
+//            (one output row per thread), warpgroup w / 4 takes every other
+//            64-column chunk; the fused math runs while the MMA warp already
+//            accumulates the next tile into the other TMEM buffer.
 // Every mbarrier wait is bounded (mbar_wait).
 #pragma once
 
@@ -50,14 +54,19 @@ struct GemmArgs {
   RopeTheta theta;
 };
 
+constexpr int kGemmThreads = 320;   // 8 epilogue warps + TMA warp + MMA warp
+constexpr int kGemmTmaWarp = 8;
+constexpr int kGemmMmaWarp = 9;
+
 template <int BN, int STAGES>
 struct GemmSmem {
   static constexpr int A_BYTES = 128 * 128;
   static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
-  static constexpr int BYTES = BAR_OFFSET + (2 * STAGES + 1) * 8 + 16;
-  static constexpr int LAUNCH_BYTES = BYTES + 1024;  // slack for 1024-byte alignment
+  static constexpr int NBARS = 2 * STAGES + 4;          // full, empty, tmem full x2, tmem empty x2
+  static constexpr int BYTES = BAR_OFFSET + NBARS * 8 + 16;
+  static constexpr int LAUNCH_BYTES = BYTES + 1024;     // slack for 1024-byte alignment
 };
 
 // QK-RMSNorm (gain g) then RoPE over one head of 64 channels held by this thread.
@@ -72,61 +81,113 @@ __device__ __forceinline__ void qk_norm_rope64(float* v, const float* __restrict
   for (int c = 0; c < 64; ++c) ss = fmaf(v[c], v[c], ss);
   const float r = rsqrtf(ss * (1.0f / 64.0f) + eps);
 #pragma unroll
-  for (int c = 0; c < 64; ++c) v[c] = v[c] * r * __ldg(g + c);
-  const float p[3] = {static_cast<float>(pos.x), static_cast<float>(pos.y), static_cast<float>(pos.z)};
-  constexpr int R[3] = {R0, R1, R2};
-  int off = 0, pair = 0;
+  for (int c = 0; c < 64; c += 4) {
+    const float4 gg = __ldg(reinterpret_cast<const float4*>(g + c));
+    v[c] *= r * gg.x;
+    v[c + 1] *= r * gg.y;
+    v[c + 2] *= r * gg.z;
+    v[c + 3] *= r * gg.w;
+  }
 #pragma unroll
   for (int a = 0; a < 3; ++a) {
-    const int half = R[a] / 2;
+    const int D = a == 0 ? R0 : (a == 1 ? R1 : R2);
+    const int off = a == 0 ? 0 : (a == 1 ? R0 : R0 + R1);
+    const int pair0 = off / 2;
+    const float p = static_cast<float>(a == 0 ? pos.x : (a == 1 ? pos.y : pos.z));
 #pragma unroll
-    for (int j = 0; j < half; ++j) {
+    for (int j = 0; j < D / 2; ++j) {
       float c, s;
-      rope_cos_sin(p[a], th.hi[pair + j], th.lo[pair + j], c, s);
-      const float x = v[off + j], y = v[off + j + half];
+      rope_cos_sin(p, th.hi[pair0 + j], th.lo[pair0 + j], c, s);
+      const float x = v[off + j], y = v[off + j + D / 2];
       v[off + j] = x * c - y * s;
-      v[off + j + half] = x * s + y * c;
+      v[off + j + D / 2] = x * s + y * c;
     }
-    off += R[a];
-    pair += half;
   }
 }
 
+template <int EPI, bool FP8, int R0, int R1, int R2>
+__device__ __forceinline__ void gemm_epilogue64(float* v, int row, int col, float rs, const int4 pos,
+                                                const GemmArgs& args) {
+  if (FP8) {
+#pragma unroll
+    for (int i = 0; i < 64; i += 4) {
+      const float4 ws = __ldg(reinterpret_cast<const float4*>(args.w_scale + col + i));
+      v[i] *= rs * ws.x;
+      v[i + 1] *= rs * ws.y;
+      v[i + 2] *= rs * ws.z;
+      v[i + 3] *= rs * ws.w;
+    }
+  }
+  if (args.bias) {
+#pragma unroll
+    for (int i = 0; i < 64; i += 4) {
+      const float4 b = __ldg(reinterpret_cast<const float4*>(args.bias + col + i));
+      v[i] += b.x;
+      v[i + 1] += b.y;
+      v[i + 2] += b.z;
+      v[i + 3] += b.w;
+    }
+  }
+  bf16* dst = args.out + static_cast<size_t>(row) * args.ldo + col;
+  if (EPI == EPI_GELU) {
+#pragma unroll
+    for (int i = 0; i < 64; ++i) v[i] = gelu_erf(v[i]);
+  } else if (EPI == EPI_RESID) {
+#pragma unroll
+    for (int i = 0; i < 64; i += 8) {
+      float r[8];
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(dst + i), r);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[i + e] += r[e];
+    }
+  } else if (EPI == EPI_QKV) {
+    if (col < 2 * args.d)
+      qk_norm_rope64<R0, R1, R2>(v, col < args.d ? args.q_g : args.k_g, args.eps_qk, pos, args.theta);
+  }
+#pragma unroll
+  for (int i = 0; i < 64; i += 8) *reinterpret_cast<uint4*>(dst + i) = f32_to_bf16x8(v + i);
+}
+
 template <int BN, int STAGES, int EPI, bool FP8, int R0, int R1, int R2>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmArgs args) {
   using SM = GemmSmem<BN, STAGES>;
-  constexpr int MMA_K_BYTES = 32;                 // 16 bf16 or 32 e4m3 per MMA
-  constexpr int NMMA = 128 / MMA_K_BYTES;         // MMAs per 128-byte K slice
-  constexpr uint32_t TMEM_COLS = BN;              // 64, 128 or 256 (power of two >= 32)
+  constexpr int NMMA = 128 / 32;                  // MMAs per 128-byte K slice (32 bytes each)
+  constexpr uint32_t TMEM_COLS = 2 * BN;          // two accumulators: 128, 256 or 512 columns
   constexpr uint32_t IDESC = idesc_make(FP8 ? 0u : 1u, BN);
+  constexpr int KE = FP8 ? 128 : 64;              // K elements per slice
+  constexpr int NCHUNK = BN / 64;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar_full = sbase + SM::BAR_OFFSET;      // STAGES barriers
-  const uint32_t bar_empty = bar_full + 8 * STAGES;      // STAGES barriers
-  const uint32_t bar_tmem = bar_empty + 8 * STAGES;      // 1 barrier
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::BAR_OFFSET + (2 * STAGES + 1) * 8);
+  const uint32_t bar_full = sbase + SM::BAR_OFFSET;       // STAGES
+  const uint32_t bar_empty = bar_full + 8 * STAGES;       // STAGES
+  const uint32_t bar_tfull = bar_empty + 8 * STAGES;      // 2
+  const uint32_t bar_tempty = bar_tfull + 16;             // 2
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::BAR_OFFSET + SM::NBARS * 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * 128;
-  const int n0 = blockIdx.y * BN;
-  const int KB = args.K / (FP8 ? 128 : 64);
+  const int mt = (args.M + 127) / 128;
+  const int ntiles = mt * (args.N / BN);
+  const int KB = args.K / KE;
 
-  if (warp == 0 && lane == 0) {
+  if (warp == kGemmTmaWarp && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
     }
-    mbar_init(bar_tmem, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_tfull + 8 * b, 1);
+      mbar_init(bar_tempty + 8 * b, 8);           // one arrival per epilogue warp
+    }
     fence_barrier_init();
   }
-  if (warp == 1) {
+  if (warp == kGemmMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
@@ -134,97 +195,96 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();        // A and the output/residual belong to the previous kernel
+  pdl_trigger();
 
-  if (warp == 0) {
+  if (warp == kGemmTmaWarp) {
     if (lane == 0) {
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % STAGES;
-        if (kb >= STAGES && !mbar_wait(bar_empty + 8 * s, ((kb / STAGES) - 1) & 1)) break;
-        const uint32_t sa = sbase + s * SM::STAGE_BYTES;
-        mbar_expect_tx(bar_full + 8 * s, SM::STAGE_BYTES);
-        tma_load_2d(sa, &tmA, bar_full + 8 * s, kb * (FP8 ? 128 : 64), m0);
-        tma_load_2d(sa + SM::A_BYTES, &tmB, bar_full + 8 * s, kb * (FP8 ? 128 : 64), n0);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const int m0 = (tile % mt) * 128, n0 = (tile / mt) * BN;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const uint32_t s = it % STAGES;
+          if (it >= STAGES && !mbar_wait(bar_empty + 8 * s, ((it / STAGES) - 1) & 1)) { ok = false; break; }
+          const uint32_t sa = sbase + s * SM::STAGE_BYTES;
+          mbar_expect_tx(bar_full + 8 * s, SM::STAGE_BYTES);
+          tma_load_2d(sa, &tmA, bar_full + 8 * s, kb * KE, m0);
+          tma_load_2d(sa + SM::A_BYTES, &tmB, bar_full + 8 * s, kb * KE, n0);
+        }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == kGemmMmaWarp) {
     if (lane == 0) {
+      uint32_t it = 0, j = 0;
       bool ok = true;
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % STAGES;
-        if (!mbar_wait(bar_full + 8 * s, (kb / STAGES) & 1)) { ok = false; break; }
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++j) {
+        const uint32_t acc = j & 1, use = j >> 1;
+        if (j >= 2 && !mbar_wait(bar_tempty + 8 * acc, (use - 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t sa = sbase + s * SM::STAGE_BYTES;
-        const uint64_t da = sdesc_sw128(sa);
-        const uint64_t db = sdesc_sw128(sa + SM::A_BYTES);
+        const uint32_t dt = tmem + acc * BN;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const uint32_t s = it % STAGES;
+          if (!mbar_wait(bar_full + 8 * s, (it / STAGES) & 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = sbase + s * SM::STAGE_BYTES;
+          const uint64_t da = sdesc_sw128(sa);
+          const uint64_t db = sdesc_sw128(sa + SM::A_BYTES);
 #pragma unroll
-        for (int k = 0; k < NMMA; ++k) {
-          // +32 bytes of K = +2 in the descriptor's (address >> 4) field
-          if (FP8)
-            tc_mma_f8(tmem, da + 2 * k, db + 2 * k, IDESC, (kb | k) != 0);
-          else
-            tc_mma_f16(tmem, da + 2 * k, db + 2 * k, IDESC, (kb | k) != 0);
+          for (int k = 0; k < NMMA; ++k) {
+            // +32 bytes of K = +2 in the descriptor's (address >> 4) field
+            if (FP8)
+              tc_mma_f8(dt, da + 2 * k, db + 2 * k, IDESC, (kb | k) != 0);
+            else
+              tc_mma_f16(dt, da + 2 * k, db + 2 * k, IDESC, (kb | k) != 0);
+          }
+          tc_commit(bar_empty + 8 * s);
         }
-        tc_commit(bar_empty + 8 * s);
+        tc_commit(bar_tfull + 8 * acc);
       }
-      (void)ok;
-      tc_commit(bar_tmem);
     }
   } else {
-    // epilogue: warps 2..5 own TMEM lane quarters (warp % 4)
+    // epilogue warps 0..7: lane quarter warp % 4, column half warp / 4
     const int quarter = warp & 3;
-    const int row = m0 + quarter * 32 + lane;
-    const bool waited = mbar_wait(bar_tmem, 0);
-    tc_fence_after();
-    if (waited) {
-      const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const int half = warp >> 2;
+    uint32_t j = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++j) {
+      const uint32_t acc = j & 1, use = j >> 1;
+      const int m0 = (tile % mt) * 128, n0 = (tile / mt) * BN;
+      const int row = m0 + quarter * 32 + lane;
+      if (!mbar_wait(bar_tfull + 8 * acc, use & 1)) break;
+      tc_fence_after();
+      const uint32_t trow = tmem + acc * BN + (static_cast<uint32_t>(quarter * 32) << 16);
       float rs = 1.f;
       if (FP8 && row < args.M) rs = __ldg(args.a_scale + row);
       int4 pos = make_int4(0, 0, 0, 0);
       if (EPI == EPI_QKV && row < args.M) pos = __ldg(args.pos + row);
+      int mine = 0;
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 64) {
+      for (int c = half; c < NCHUNK; c += 2) ++mine;
+      if (mine == 0) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_tempty + 8 * acc);
+      }
+#pragma unroll 1
+      for (int c = half, k = 0; c < NCHUNK; c += 2, ++k) {
         float v[64];
-        tmem_ld32(trow + c, v);
-        tmem_ld32(trow + c + 32, v + 32);
+        tmem_ld32(trow + c * 64, v);
+        tmem_ld32(trow + c * 64 + 32, v + 32);
         tmem_wait_ld();
-        if (row < args.M) {
-          const int col = n0 + c;
-          if (FP8) {
-#pragma unroll
-            for (int i = 0; i < 64; ++i) v[i] *= rs * __ldg(args.w_scale + col + i);
-          }
-          if (args.bias) {
-#pragma unroll
-            for (int i = 0; i < 64; i += 4) {
-              const float4 b = __ldg(reinterpret_cast<const float4*>(args.bias + col + i));
-              v[i] += b.x; v[i + 1] += b.y; v[i + 2] += b.z; v[i + 3] += b.w;
-            }
-          }
-          bf16* dst = args.out + static_cast<size_t>(row) * args.ldo + col;
-          if (EPI == EPI_GELU) {
-#pragma unroll
-            for (int i = 0; i < 64; ++i) v[i] = gelu_erf(v[i]);
-          } else if (EPI == EPI_RESID) {
-#pragma unroll
-            for (int i = 0; i < 64; i += 8) {
-              float r[8];
-              bf16x8_to_f32(*reinterpret_cast<const uint4*>(dst + i), r);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) v[i + e] += r[e];
-            }
-          } else if (EPI == EPI_QKV) {
-            if (col < 2 * args.d) qk_norm_rope64<R0, R1, R2>(v, col < args.d ? args.q_g : args.k_g, args.eps_qk, pos,
-                                                          args.theta);
-          }
-#pragma unroll
-          for (int i = 0; i < 64; i += 8) *reinterpret_cast<uint4*>(dst + i) = f32_to_bf16x8(v + i);
+        if (k == mine - 1) {           // last TMEM read of this warp for this tile
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_tempty + 8 * acc);
         }
+        if (row < args.M) gemm_epilogue64<EPI, FP8, R0, R1, R2>(v, row, n0 + c * 64, rs, pos, args);
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kGemmMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }

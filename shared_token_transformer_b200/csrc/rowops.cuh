@@ -69,6 +69,8 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const T* __restrict__ x,
                                                         const float* __restrict__ g, const float* __restrict__ b,
                                                         float eps, T* __restrict__ y, uint8_t* __restrict__ q8,
                                                         float* __restrict__ qscale) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int E = Vec<T>::E;
   const int lane = threadIdx.x & 31;
   const size_t row = static_cast<size_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -133,6 +135,8 @@ __global__ void __launch_bounds__(256) merge_kernel(const T* __restrict__ P, int
                                                     const int* __restrict__ tok_ptr, const int* __restrict__ tok_ent,
                                                     const float* __restrict__ wbar, T* __restrict__ A,
                                                     uint8_t* __restrict__ q8, float* __restrict__ qscale) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int E = Vec<T>::E;
   const int lane = threadIdx.x & 31;
   const size_t row = static_cast<size_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -192,6 +196,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint8_t* __restr
                                                           const uint8_t* __restrict__ G0,
                                                           const int* __restrict__ rowmap, int nrows, int U,
                                                           size_t row_bytes, uint8_t* __restrict__ X) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const size_t r = static_cast<size_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (r >= static_cast<size_t>(nrows)) return;
@@ -207,6 +213,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint8_t* __restr
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) quantize_rows_kernel(const bf16* __restrict__ x, int rows, int cols,
                                                             uint8_t* __restrict__ q, float* __restrict__ scale) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const size_t row = static_cast<size_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= static_cast<size_t>(rows)) return;

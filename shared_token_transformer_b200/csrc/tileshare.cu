@@ -16,10 +16,12 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <atomic>
 #include <mutex>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "../../include/tileshare.h"
@@ -167,6 +169,28 @@ static ts_status make_tmap(CUtensorMap* map, const void* base, int rows, int K, 
 }
 
 // ============================================================================
+// launches with programmatic dependent launch (PDL)
+//   Kernels launched this way call pdl_wait() before touching activations, so
+//   their prologue (barrier init, TMEM allocation, descriptor prefetch) overlaps
+//   the tail of the previous kernel in the stream.
+// ============================================================================
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// ============================================================================
 // model checks and RoPE tables
 // ============================================================================
 static int esize(ts_dtype dt) { return dt == TS_F32 ? 4 : 2; }
@@ -298,7 +322,10 @@ static ts_status launch_layernorm_vec(const void* x, int rows, int d, const floa
   T* yy = static_cast<T*>(y);
   trace_pre(st);
 #define TS_LN_CASE(NV) \
-  case NV: ts::layernorm_kernel<T, NV, Q8><<<rows_grid(rows), 256, 0, st>>>(xx, rows, d, g, b, eps, yy, q8, qs); break;
+  case NV:                                                                                                  \
+    launch_pdl(ts::layernorm_kernel<T, NV, Q8>, dim3(rows_grid(rows)), dim3(256), 0, st, xx, rows, d, g, b, eps, yy, \
+               q8, qs);                                                                                       \
+    break;
   switch (nv) {
     TS_LN_CASE(1) TS_LN_CASE(2) TS_LN_CASE(3) TS_LN_CASE(4) TS_LN_CASE(5) TS_LN_CASE(6) TS_LN_CASE(7) TS_LN_CASE(8)
     default: return fail(TS_ERR_UNSUPPORTED, "layernorm width %d", d);
@@ -335,8 +362,9 @@ static ts_status launch_merge_vec(const ts_plan_s* p, const void* P, int rows, i
   trace_pre(st);
 #define TS_MG_CASE(NV)                                                                                    \
   case NV:                                                                                                \
-    ts::merge_kernel<T, NV, Q8><<<rows_grid(rows), 256, 0, st>>>(pp, rows, p->U, p->N, d, p->d_tok_ptr,  \
-                                                                 p->d_tok_ent, p->d_wbar, aa, q8, qs);    \
+    launch_pdl(ts::merge_kernel<T, NV, Q8>, dim3(rows_grid(rows)), dim3(256), 0, st, pp, rows, p->U, p->N, d, \
+               static_cast<const int*>(p->d_tok_ptr), static_cast<const int*>(p->d_tok_ent),               \
+               static_cast<const float*>(p->d_wbar), aa, q8, qs);                                           \
     break;
   switch (nv) {
     TS_MG_CASE(1) TS_MG_CASE(2) TS_MG_CASE(3) TS_MG_CASE(4) TS_MG_CASE(5) TS_MG_CASE(6) TS_MG_CASE(7) TS_MG_CASE(8)
@@ -373,7 +401,8 @@ static ts_status run_quantize(const void* x, int rows, int cols, uint8_t* q, flo
   if (rows == 0) return TS_OK;
   set_work("quantize_e4m3", 0.0, static_cast<double>(rows) * cols * 3.0 + 4.0 * rows);
   trace_pre(st);
-  ts::quantize_rows_kernel<<<rows_grid(rows), 256, 0, st>>>(static_cast<const bf16*>(x), rows, cols, q, s);
+  launch_pdl(ts::quantize_rows_kernel, dim3(rows_grid(rows)), dim3(256), 0, st, static_cast<const bf16*>(x), rows, cols,
+             q, s);
   return trace_post(st, "quantize_rows");
 }
 
@@ -404,9 +433,10 @@ static ts_status launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, co
     TS_CUDA_CHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::LAUNCH_BYTES));
     configured[dev] = 1;
   }
-  dim3 grid((args.M + 127) / 128, args.N / BN);
+  const int tiles = ((args.M + 127) / 128) * (args.N / BN);
+  dim3 grid(std::min(tiles, num_sms()));
   trace_pre(st);
-  kern<<<grid, 192, SM::LAUNCH_BYTES, st>>>(ta, tb, args);
+  launch_pdl(kern, grid, dim3(ts::kGemmThreads), SM::LAUNCH_BYTES, st, ta, tb, args);
   return trace_post(st, "gemm_tc");
 }
 
@@ -420,14 +450,31 @@ static ts_status dispatch_gemm_bn(int bn, const CUtensorMap& ta, const CUtensorM
   }
 }
 
-// Output tile width: the widest of 256/128/64 dividing N that still gives at
-// least one CTA per SM; else the narrowest (most CTAs).
+// Output tile width for the persistent GEMM: the persistent CTAs walk the tiles
+// round-robin, so the busiest CTA handles ceil(tiles / SMs) tiles.  Cost model:
+// that count times (BN + 48), 48 columns standing for the fixed per-tile work
+// (pipeline fill, epilogue tail); ties go to the wider tile.
 static int pick_bn(int M, int N) {
+  // tuning override: TS_GEMM_BN=64|128|256 forces the tile width where it divides N
+  static const int forced = [] {
+    const char* e = std::getenv("TS_GEMM_BN");
+    return e ? std::atoi(e) : 0;
+  }();
+  if ((forced == 64 || forced == 128 || forced == 256) && N % forced == 0) return forced;
   const int mt = (M + 127) / 128;
   const int sms = num_sms();
-  for (int bn : {256, 128, 64})
-    if (N % bn == 0 && mt * (N / bn) >= sms) return bn;
-  return 64;
+  int best = 64;
+  long best_cost = -1;
+  for (int bn : {256, 128, 64}) {
+    if (N % bn) continue;
+    const long tiles = static_cast<long>(mt) * (N / bn);
+    const long cost = ((tiles + sms - 1) / sms) * (bn + 48);
+    if (best_cost < 0 || cost < best_cost) {
+      best = bn;
+      best_cost = cost;
+    }
+  }
+  return best;
 }
 
 // Y[M, N] = A[M, K] W[N, K]^T with epilogue; A bf16 (or e4m3 + a_scale), W bf16 (or e4m3 + w_scale).
@@ -525,8 +572,16 @@ static ts_status run_attention(const ts_plan_s* p, const ts_model_desc* m, bool 
     return trace_post(st, "attn_f32");
   }
   const int nqb = (p->Nw + ts::kAttnBQ - 1) / ts::kAttnBQ;
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    TS_CUDA_CHECK(cudaFuncSetAttribute(ts::attn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       ts::AttnSmem::LAUNCH_BYTES));
+    configured[dev] = 1;
+  }
   dim3 grid(nqb + 1, m->heads, p->T);
-  ts::attn_bf16_kernel<<<grid, 128, ts::kAttnBf16SmemMax, st>>>(a);
+  launch_pdl(ts::attn_bf16_kernel, grid, dim3(ts::kAttnThreads), ts::AttnSmem::LAUNCH_BYTES, st, a);
   return trace_post(st, "attn_bf16");
 }
 
@@ -611,9 +666,9 @@ static ts_status run_gather(const ts_plan_s* p, const ts_model_desc* m, const vo
   const size_t rb = static_cast<size_t>(m->d) * esize(m->dtype);
   set_work("gather", 0.0, 2.0 * nrows * static_cast<double>(rb));
   trace_pre(st);
-  ts::gather_rows_kernel<<<rows_grid(nrows), 256, 0, st>>>(static_cast<const uint8_t*>(S0),
-                                                           static_cast<const uint8_t*>(G0), p->d_rowmap, nrows, p->U,
-                                                           rb, static_cast<uint8_t*>(X));
+  launch_pdl(ts::gather_rows_kernel, dim3(rows_grid(nrows)), dim3(256), 0, st, static_cast<const uint8_t*>(S0),
+             static_cast<const uint8_t*>(G0), static_cast<const int*>(p->d_rowmap), nrows, p->U, rb,
+             static_cast<uint8_t*>(X));
   return trace_post(st, "gather_rows");
 }
 
