@@ -9,20 +9,23 @@
 // attention.
 //
 // bf16 kernel (hd = 64), grid (nqb + 1, heads, T), 288 threads, 2 CTAs per SM:
-//   blocks qb < nqb: 128 window queries.
-//     warps 4-7  loaders: cp.async gathers of Q (once) and of 128-key K/V blocks
-//                through the row map into 128-byte-swizzled shared rows; two
-//                warp pairs fill the two buffers independently and publish each
-//                block with fence.proxy.async and an mbarrier;
+//   blocks qb < nqb: 128 window queries, keys in blocks of 64.
+//     warps 4-7  loaders: cp.async gathers of Q (once) and of K/V blocks through
+//                the row map into 128-byte-swizzled shared rows; loader warp w
+//                owns K/V buffer w (blocks w, w+4, ...), so three blocks are in
+//                flight ahead of the math; each block is published with
+//                fence.proxy.async and an mbarrier;
 //     warp 8     MMA issuer (one lane): S = Q K^T (tcgen05 kind::f16, M = 128,
-//                N = 128 keys) into TMEM, then O += P V (M = 128, N = 64, V read
-//                as an MN-major operand) into TMEM; S of block j+1 is issued while
-//                the softmax of block j runs;
-//     warps 0-3  softmax, one query row per thread (TMEM lane = row): tcgen05.ld
-//                of S, online softmax in the exp2 domain, P as bf16 into swizzled
-//                shared memory, rescale of the O row in TMEM when the max moves;
-//                the global key (slot 0) seeds the running max and sum and is
-//                added back at the end with its running coefficient.
+//                N = 64) into one of two TMEM S buffers, then O += P V (M = 128,
+//                N = 64, V read as an MN-major operand) into TMEM; S of block j+1
+//                is issued as soon as the softmax has read block j-1's buffer;
+//     warps 0-3  softmax, one query row per thread (TMEM lane = row): one tcgen05
+//                round trip brings the row's 64 scores into registers; online
+//                softmax in the exp2 domain with a lazily moved reference maximum
+//                (O rescaled in TMEM only when a score exceeds it by 2^8); P as
+//                bf16 into one of two swizzled shared buffers; the global key
+//                (slot 0) seeds the running max and sum and is added back at the
+//                end with its running coefficient.
 //   block qb == nqb: the global token's own query row (one row attends to N keys):
 //     warps split the keys, lanes own channel pairs, partial states merged at the end.
 // fp32 kernel (any hd <= 64, multiple of 4): one thread per query row, keys in
@@ -51,16 +54,18 @@ __device__ __forceinline__ uint32_t swz(int r, int ch) { return r * 128 + ((ch ^
 
 constexpr int kAttnThreads = 288;        // 4 softmax + 4 loader + 1 MMA warps
 constexpr int kAttnBQ = 128;             // queries per CTA
-constexpr int kAttnBK = 128;             // keys per block
+constexpr int kAttnBK = 64;              // keys per block
+constexpr int kAttnKV = 4;               // K/V buffers (one loader warp each)
+constexpr float kAttnRescale = 8.0f;     // lazy rescale threshold (log2 units)
 
 struct AttnSmem {
-  static constexpr int Q = 0;                 // 16 KB
-  static constexpr int K = 16384;             // 2 x 16 KB
-  static constexpr int V = 16384 * 3;         // 2 x 16 KB
-  static constexpr int P = 16384 * 5;         // 2 x 16 KB (keys 0-63, keys 64-127)
-  static constexpr int KG = 16384 * 7;        // 64 floats k_g, 64 floats v_g
+  static constexpr int Q = 0;                 // 16 KB: 128 rows x 128 B
+  static constexpr int K = 16384;             // 4 x 8 KB: 64 rows x 128 B
+  static constexpr int V = 16384 + 32768;     // 4 x 8 KB
+  static constexpr int P = 16384 + 65536;     // 2 x 16 KB: 128 rows x 64 keys
+  static constexpr int KG = P + 32768;        // 64 floats k_g, 64 floats v_g
   static constexpr int BAR = KG + 512;        // barriers
-  static constexpr int NBAR = 8;
+  static constexpr int NBAR = 16;
   static constexpr int BYTES = BAR + NBAR * 8 + 16;
   static constexpr int LAUNCH_BYTES = BYTES;  // base must be 1024-aligned (checked): two CTAs per SM
 };
@@ -96,7 +101,34 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
       "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
 }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
+      : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// 2^x by the PTX approximate base-2 exponential (2 ulp; -inf gives 0)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
@@ -107,12 +139,12 @@ __device__ __forceinline__ void attn_window_block_tc(const AttnArgs& a, int qb, 
   const int ld = 3 * a.d;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sb = smem_u32(smem);
-  const uint32_t bar_kvfull = sb + AttnSmem::BAR;        // 2, count 64 (one loader pair each)
-  const uint32_t bar_kvempty = bar_kvfull + 16;          // 2, count 1 (commit)
-  const uint32_t bar_sfull = bar_kvempty + 16;           // 1, count 1 (commit)
-  const uint32_t bar_sfree = bar_sfull + 8;              // 1, count 4 (softmax warps)
-  const uint32_t bar_pfull = bar_sfree + 8;              // 1, count 4 (softmax warps)
-  const uint32_t bar_odone = bar_pfull + 8;              // 1, count 1 (commit)
+  const uint32_t bar_kvfull = sb + AttnSmem::BAR;        // 4, count 32 (one loader warp each)
+  const uint32_t bar_kvempty = bar_kvfull + 32;          // 4, count 1 (commit after P V)
+  const uint32_t bar_sfull = bar_kvempty + 32;           // 2, count 1 (commit after Q K^T)
+  const uint32_t bar_sfree = bar_sfull + 16;             // 2, count 4 (softmax warps read S)
+  const uint32_t bar_pfull = bar_sfree + 16;             // 2, count 4 (softmax warps wrote P)
+  const uint32_t bar_odone = bar_pfull + 16;             // 2, count 1 (commit after P V)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + AttnSmem::BAR + AttnSmem::NBAR * 8);
   float* sKg = reinterpret_cast<float*>(smem + AttnSmem::KG);
   float* sVg = sKg + 64;
@@ -120,18 +152,20 @@ __device__ __forceinline__ void attn_window_block_tc(const AttnArgs& a, int qb, 
   const int q0 = 1 + qb * kAttnBQ;  // first slot of this query block
 
   if (warp == 8 && lane == 0) {
-    mbar_init(bar_kvfull, 64);
-    mbar_init(bar_kvfull + 8, 64);
-    mbar_init(bar_kvempty, 1);
-    mbar_init(bar_kvempty + 8, 1);
-    mbar_init(bar_sfull, 1);
-    mbar_init(bar_sfree, 4);
-    mbar_init(bar_pfull, 4);
-    mbar_init(bar_odone, 1);
+    for (int i = 0; i < kAttnKV; ++i) {
+      mbar_init(bar_kvfull + 8 * i, 32);
+      mbar_init(bar_kvempty + 8 * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_sfull + 8 * i, 1);
+      mbar_init(bar_sfree + 8 * i, 4);
+      mbar_init(bar_pfull + 8 * i, 4);
+      mbar_init(bar_odone + 8 * i, 1);
+    }
     fence_barrier_init();
   }
   if (warp == 8) {
-    tmem_alloc(smem_u32(tmem_slot), 256);    // S: columns 0-127, O: columns 128-191
+    tmem_alloc(smem_u32(tmem_slot), 256);    // S0: cols 0-63, S1: 64-127, O: 128-191
     tmem_relinquish();
   }
   pdl_wait();
@@ -145,91 +179,82 @@ __device__ __forceinline__ void attn_window_block_tc(const AttnArgs& a, int qb, 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + 128;
+  const uint32_t tO = tmem + 128;
 
   if (warp >= 4 && warp < 8) {
-    // ---------------- loaders ----------------
-    // Two independent pairs of warps, one per K/V buffer: pair b loads the blocks
-    // j = b, b + 2, ... so that publishing one buffer never waits on the other.
-    const int grp = (warp - 4) >> 1;
-    const int lt = tid - 128 - grp * 64;       // 0..63
-    // thread lt copies 16-byte chunk (lt & 7) of rows (lt >> 3) + 8 i, i = 0..15; the
-    // row indices are read up front so that their loads overlap
-    const int ch = lt & 7, r0 = lt >> 3;
-    if (grp == 0) {
-      // Q rows travel with the first K/V block
-      int rows[16];
+    // ---------------- loaders: warp wl owns K/V buffer wl, blocks wl, wl + 4, ... ----------------
+    // The row indices of a block are read with one coalesced load (lane l holds
+    // rows l and 32 + l) and handed to the lanes that copy them by shuffles; the
+    // indices of a warp's next block are fetched before it waits for its buffer.
+    const int wl = warp - 4;
+    const int ch = lane & 7, r0 = lane >> 3;       // chunk ch of rows r0 + 4 i
+    auto row_of = [&](int slot) { return slot < a.N ? attn_row(a, t, slot) : -1; };
+    if (wl == 0) {
+      // Q rows (128 x 8 chunks) travel with block 0
+      int vq[4];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int slot = q0 + r0 + 8 * i;
-        rows[i] = slot < a.N ? attn_row(a, t, slot) : -1;
-      }
+      for (int k = 0; k < 4; ++k) vq[k] = row_of(q0 + 32 * k + lane);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int r = r0 + 8 * i;
-        const bool ok = rows[i] >= 0;
-        const bf16* src = qkv + (ok ? static_cast<size_t>(rows[i]) * ld + h * 64 + ch * 8 : 0);
+      for (int i = 0; i < 32; ++i) {
+        const int r = r0 + 4 * i;
+        const int row = __shfl_sync(0xffffffffu, vq[i >> 3], r & 31);
+        const bool ok = row >= 0;
+        const bf16* src = qkv + (ok ? static_cast<size_t>(row) * ld + h * 64 + ch * 8 : 0);
         cp_async16(sb + AttnSmem::Q + swz(r, ch), src, ok);
       }
     }
-    for (int j = grp; j < nkb; j += 2) {
-      const int b = grp;
-      if (j >= 2 && !mbar_wait(bar_kvempty + 8 * b, ((j >> 1) - 1) & 1)) break;
-      int rows[16];
+    int v0 = wl < nkb ? row_of(1 + wl * kAttnBK + lane) : -1;
+    int v1 = wl < nkb ? row_of(1 + wl * kAttnBK + 32 + lane) : -1;
+    for (int j = wl; j < nkb; j += kAttnKV) {
+      if (j >= kAttnKV && !mbar_wait(bar_kvempty + 8 * wl, ((j / kAttnKV) - 1) & 1)) break;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const int slot = 1 + j * kAttnBK + r0 + 8 * i;
-        rows[i] = slot < a.N ? attn_row(a, t, slot) : -1;
-      }
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int r = r0 + 8 * i;
-        const bool ok = rows[i] >= 0;
-        const size_t base = ok ? static_cast<size_t>(rows[i]) * ld + h * 64 + ch * 8 : 0;
-        cp_async16(sb + AttnSmem::K + b * 16384 + swz(r, ch), qkv + base + (ok ? a.d : 0), ok);
-        cp_async16(sb + AttnSmem::V + b * 16384 + swz(r, ch), qkv + base + (ok ? 2 * a.d : 0), ok);
+        const int r = r0 + 4 * i;
+        const int row = __shfl_sync(0xffffffffu, i < 8 ? v0 : v1, r & 31);
+        const bool ok = row >= 0;
+        const size_t base = ok ? static_cast<size_t>(row) * ld + h * 64 + ch * 8 : 0;
+        cp_async16(sb + AttnSmem::K + wl * 8192 + swz(r, ch), qkv + base + (ok ? a.d : 0), ok);
+        cp_async16(sb + AttnSmem::V + wl * 8192 + swz(r, ch), qkv + base + (ok ? 2 * a.d : 0), ok);
       }
       cp_async_commit();
+      const int jn = j + kAttnKV;
+      v0 = jn < nkb ? row_of(1 + jn * kAttnBK + lane) : -1;
+      v1 = jn < nkb ? row_of(1 + jn * kAttnBK + 32 + lane) : -1;
       cp_async_wait<0>();
       fence_proxy_async_smem();
-      mbar_arrive(bar_kvfull + 8 * b);
+      mbar_arrive(bar_kvfull + 8 * wl);
     }
     cp_async_wait<0>();
   } else if (warp == 8) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_make(1u, 128);                 // Q K^T: M 128, N 128
+      constexpr uint32_t IDESC_S = idesc_make(1u, kAttnBK);             // Q K^T: M 128, N 64
       constexpr uint32_t IDESC_O = idesc_make(1u, 64) | (1u << 16);     // P V: M 128, N 64, B MN-major
       const uint64_t dq = sdesc_sw128(sb + AttnSmem::Q);
-      bool ok = mbar_wait(bar_kvfull, 0);
-      if (ok) {
+      auto issue_s = [&](int j) -> bool {
+        const int b = j % kAttnKV, sbuf = j & 1;
+        if (!mbar_wait(bar_kvfull + 8 * b, (j / kAttnKV) & 1)) return false;
+        if (j >= 2 && !mbar_wait(bar_sfree + 8 * sbuf, ((j >> 1) - 1) & 1)) return false;
         tc_fence_after();
-        const uint64_t dk = sdesc_sw128(sb + AttnSmem::K);
+        const uint64_t dk = sdesc_sw128(sb + AttnSmem::K + b * 8192);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) tc_mma_f16(tS, dq + 2 * k, dk + 2 * k, IDESC_S, k != 0);
-        tc_commit(bar_sfull);
-      }
+        for (int k = 0; k < 4; ++k) tc_mma_f16(tmem + sbuf * 64, dq + 2 * k, dk + 2 * k, IDESC_S, k != 0);
+        tc_commit(bar_sfull + 8 * sbuf);
+        return true;
+      };
+      bool ok = issue_s(0);
       for (int j = 0; j < nkb && ok; ++j) {
-        const int b = j & 1;
-        if (j + 1 < nkb) {
-          const int b1 = (j + 1) & 1;
-          ok = mbar_wait(bar_kvfull + 8 * b1, ((j + 1) >> 1) & 1) && mbar_wait(bar_sfree, j & 1);
-          if (!ok) break;
-          tc_fence_after();
-          const uint64_t dk = sdesc_sw128(sb + AttnSmem::K + b1 * 16384);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) tc_mma_f16(tS, dq + 2 * k, dk + 2 * k, IDESC_S, k != 0);
-          tc_commit(bar_sfull);
-        }
-        if (!mbar_wait(bar_pfull, j & 1)) { ok = false; break; }
+        if (j + 1 < nkb && !(ok = issue_s(j + 1))) break;
+        const int pb = j & 1, b = j % kAttnKV;
+        if (!mbar_wait(bar_pfull + 8 * pb, (j >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
+        const uint64_t dp = sdesc_sw128(sb + AttnSmem::P + pb * 16384);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t dp = sdesc_sw128(sb + AttnSmem::P + (kk >> 2) * 16384) + 2 * (kk & 3);
-          const uint64_t dv = sdesc_sw128_mn(sb + AttnSmem::V + b * 16384 + kk * 2048);
-          tc_mma_f16(tO, dp, dv, IDESC_O, (j | kk) != 0);
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t dv = sdesc_sw128_mn(sb + AttnSmem::V + b * 8192 + kk * 2048);
+          tc_mma_f16(tO, dp + 2 * kk, dv, IDESC_O, (j | kk) != 0);
         }
-        tc_commit(bar_odone);
+        tc_commit(bar_odone + 8 * pb);
         tc_commit(bar_kvempty + 8 * b);
       }
     }
@@ -240,89 +265,93 @@ __device__ __forceinline__ void attn_window_block_tc(const AttnArgs& a, int qb, 
     bool ok = mbar_wait(bar_kvfull, 0);      // Q rows are in shared memory
     float m = -INFINITY, l = 0.f, gcoef = 0.f;
     if (ok) {
-      // score of the global key
+      // score of the global key seeds the running maximum and sum
       float sg = 0.f;
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
+      for (int c = 0; c < 8; ++c) {
         float f[8];
-        bf16x8_to_f32(*reinterpret_cast<const uint4*>(smem + AttnSmem::Q + swz(row, ch)), f);
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(smem + AttnSmem::Q + swz(row, c)), f);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) sg = fmaf(f[e], sKg[ch * 8 + e], sg);
+        for (int e = 0; e < 8; ++e) sg = fmaf(f[e], sKg[c * 8 + e], sg);
       }
       m = sg * a.scale_log2;
       l = 1.f;
       gcoef = 1.f;
     }
     for (int j = 0; j < nkb && ok; ++j) {
-      if (!mbar_wait(bar_sfull, j & 1)) { ok = false; break; }
+      const int sbuf = j & 1;
+      if (!mbar_wait(bar_sfull + 8 * sbuf, (j >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
-      const int kbase = j * kAttnBK;
-      // pass 1: row maximum of the block (32-column chunks of S read from TMEM)
-      float mx = m;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float sv[32];
-        tmem_ld32(tS + lane_off + c * 32, sv);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (kbase + c * 32 + i < a.Nw) mx = fmaxf(mx, sv[i] * a.scale_log2);
-      }
-      const float alpha = exp2f(m - mx);
-      // P_{j-1} and O are in use by the previous P V until it completes
-      if (j >= 1) {
-        if (!mbar_wait(bar_odone, (j - 1) & 1)) { ok = false; break; }
-        tc_fence_after();
-      }
-      // pass 2: probabilities as bf16 into P (keys 0-63 low block, 64-127 high block)
-      float sum = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float sv[32];
-        tmem_ld32(tS + lane_off + c * 32, sv);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p = (kbase + c * 32 + i < a.Nw) ? exp2f(sv[i] * a.scale_log2 - mx) : 0.f;
-          sv[i] = p;
-          sum += p;
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int ch = c * 4 + q;     // 16-byte chunk of the 256-byte P row
-          uint4 u;
-          u.x = pack_bf16(sv[q * 8 + 0], sv[q * 8 + 1]);
-          u.y = pack_bf16(sv[q * 8 + 2], sv[q * 8 + 3]);
-          u.z = pack_bf16(sv[q * 8 + 4], sv[q * 8 + 5]);
-          u.w = pack_bf16(sv[q * 8 + 6], sv[q * 8 + 7]);
-          *reinterpret_cast<uint4*>(smem + AttnSmem::P + (ch >> 3) * 16384 + swz(row, ch & 7)) = u;
-        }
-      }
+      float sv[kAttnBK];
+      tmem_ld32(tmem + sbuf * 64 + lane_off, sv);
+      tmem_ld32(tmem + sbuf * 64 + lane_off + 32, sv + 32);
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_sfree);   // S fully read: the next Q K^T may overwrite it
-      l = l * alpha + sum;
+      if (lane == 0) mbar_arrive(bar_sfree + 8 * sbuf);   // S buffer may be overwritten
+      const int kbase = j * kAttnBK;
+      // row maximum of the raw scores (the scale is positive); keys beyond the
+      // window exist only in the last block
+      float mr = -INFINITY;
+      if (kbase + kAttnBK <= a.Nw) {
+#pragma unroll
+        for (int i = 0; i < kAttnBK; ++i) mr = fmaxf(mr, sv[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < kAttnBK; ++i) {
+          if (kbase + i >= a.Nw) sv[i] = -INFINITY;
+          mr = fmaxf(mr, sv[i]);
+        }
+      }
+      const float mx = mr * a.scale_log2;
+      // lazy rescale: the reference maximum moves only when a score exceeds it by
+      // more than 2^8, so probabilities stay below 256 and O is rarely touched
+      const bool grow = mx > m + kAttnRescale;
+      const float mnew = grow ? mx : m;
+      const float alpha = exp2f(m - mnew);
+      const bool warp_grow = __any_sync(0xffffffffu, grow);
+      l *= alpha;
       gcoef *= alpha;
-      m = mx;
-      // rescale the running output when this warp's maxima moved
-      if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      m = mnew;
+      float sum = 0.f;
+#pragma unroll
+      for (int i = 0; i < kAttnBK; ++i) {
+        sv[i] = ex2_approx(fmaf(sv[i], a.scale_log2, -m));
+        sum += sv[i];
+      }
+      l += sum;
+      // P buffer sbuf was last read by P V of block j-2
+      if (j >= 2 && !mbar_wait(bar_odone + 8 * sbuf, ((j - 2) >> 1) & 1)) { ok = false; break; }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 u;
+        u.x = pack_bf16(sv[c * 8 + 0], sv[c * 8 + 1]);
+        u.y = pack_bf16(sv[c * 8 + 2], sv[c * 8 + 3]);
+        u.z = pack_bf16(sv[c * 8 + 4], sv[c * 8 + 5]);
+        u.w = pack_bf16(sv[c * 8 + 6], sv[c * 8 + 7]);
+        *reinterpret_cast<uint4*>(smem + AttnSmem::P + sbuf * 16384 + swz(row, c)) = u;
+      }
+      if (warp_grow && j >= 1) {
+        // O holds the sum up to block j-1: wait for that P V, then rescale the row
+        if (!mbar_wait(bar_odone + 8 * ((j - 1) & 1), ((j - 1) >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {
-          float o[32];
-          tmem_ld32(tO + lane_off + hh * 32, o);
+        for (int hh = 0; hh < 4; ++hh) {
+          float o[16];
+          tmem_ld16(tO + lane_off + hh * 16, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] *= alpha;
-          tmem_st32(tO + lane_off + hh * 32, o);
+          for (int c = 0; c < 16; ++c) o[c] *= alpha;
+          tmem_st16(tO + lane_off + hh * 16, o);
         }
         tmem_wait_st();
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_pfull);
+      if (lane == 0) mbar_arrive(bar_pfull + 8 * sbuf);
     }
-    if (ok && mbar_wait(bar_odone, (nkb - 1) & 1)) {
+    if (ok && mbar_wait(bar_odone + 8 * ((nkb - 1) & 1), ((nkb - 1) >> 1) & 1)) {
       tc_fence_after();
       const int slot = q0 + row;
       const float inv = 1.f / l;
@@ -368,17 +397,36 @@ __device__ __forceinline__ void attn_global_row(const AttnArgs& a, int h, int t,
       *reinterpret_cast<const __nv_bfloat162*>(qkv + static_cast<size_t>(attn_row(a, t, 0)) * ld + h * 64 + 2 * lane);
   const float2 q = __bfloat1622float2(q2);
   float m = -INFINITY, l = 0.f, acc0 = 0.f, acc1 = 0.f;
-  for (int s = warp; s < a.N; s += nw) {
-    const bf16* kr = qkv + static_cast<size_t>(attn_row(a, t, s)) * ld + a.d + h * 64 + 2 * lane;
-    const float2 k = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kr));
-    const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kr + a.d));
-    const float sc = warp_sum(q.x * k.x + q.y * k.y) * a.scale_log2;
-    const float mn = fmaxf(m, sc);
-    const float al = exp2f(m - mn), p = exp2f(sc - mn);
-    l = l * al + p;
-    acc0 = acc0 * al + p * v.x;
-    acc1 = acc1 * al + p * v.y;
-    m = mn;
+  // keys in batches of 8 per warp: all row indices, then all K/V loads, are issued
+  // before their first use so that their latencies overlap
+  constexpr int KB = 4;
+  for (int s0 = warp * KB; s0 < a.N; s0 += nw * KB) {
+    int rows[KB];
+#pragma unroll
+    for (int i = 0; i < KB; ++i) rows[i] = s0 + i < a.N ? attn_row(a, t, s0 + i) : -1;
+    float2 k[KB], v[KB];
+#pragma unroll
+    for (int i = 0; i < KB; ++i) {
+      if (rows[i] >= 0) {
+        const bf16* kr = qkv + static_cast<size_t>(rows[i]) * ld + a.d + h * 64 + 2 * lane;
+        k[i] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kr));
+        v[i] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kr + a.d));
+      } else {
+        k[i] = make_float2(0.f, 0.f);
+        v[i] = make_float2(0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < KB; ++i) {
+      if (rows[i] < 0) break;
+      const float sc = warp_sum(q.x * k[i].x + q.y * k[i].y) * a.scale_log2;
+      const float mn = fmaxf(m, sc);
+      const float al = exp2f(m - mn), p = exp2f(sc - mn);
+      l = l * al + p;
+      acc0 = acc0 * al + p * v[i].x;
+      acc1 = acc1 * al + p * v[i].y;
+      m = mn;
+    }
   }
   if (lane == 0) {
     sm[warp] = m;

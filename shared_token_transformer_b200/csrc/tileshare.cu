@@ -187,6 +187,17 @@ static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // one shared-memory carve-out for every hot kernel, so that consecutive kernels
+  // never wait for the SM to re-partition L1 and shared memory
+  static thread_local const void* seen[64];
+  static thread_local int nseen = 0;
+  const void* key = reinterpret_cast<const void*>(kern);
+  bool known = false;
+  for (int i = 0; i < nseen; ++i) known |= seen[i] == key;
+  if (!known) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    if (nseen < 64) seen[nseen++] = key;
+  }
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
