@@ -50,9 +50,10 @@ ts_status ts_op_linear(const ts_model_desc* model, const void* x, int rows, int 
    rotates grid token u by its grid coordinates and the global token of tile t by
    the tile's origin: attention scores then equal those of tile-local rotation
    exactly (RoPE scores depend on coordinate differences only), so the rotation
-   can run once per token.  `scratch` holds the normalised rows
-   (rows * d elements of the model dtype, plus rows * d + 4 * rows bytes for
-   TS_FP8_E4M3). */
+   can run once per token.  `scratch` holds, each region 256-byte aligned, the
+   normalised rows (rows * d elements of the model dtype), an e4m3 copy
+   (rows * d bytes) with per-row scales (4 * rows bytes), and the RoPE cos/sin
+   table (8 * (F * D_f + H * D_y + W * D_x) / 2 bytes). */
 ts_status ts_op_qkv(ts_plan_t plan, const ts_model_desc* model, const ts_layer_weights* w,
                     ts_rows_mode mode, const void* state, void* qkv, void* scratch, void* stream);
 

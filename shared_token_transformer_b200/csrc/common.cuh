@@ -268,6 +268,29 @@ __device__ __forceinline__ uint4 f32_to_bf16x8(const float* f) {
   return u;
 }
 
+// Cosine / sine table of the RoPE angles of one plan and model: for axis a,
+// coordinate p < G[a] and pair j < half[a], entry off[a] + p * half[a] + j holds
+// (cos, sin) of p * base^(-j / half[a]), computed in double and rounded to float.
+struct RopeTable {
+  float2* cs;
+  int G[3];
+  int half[3];
+  int off[3];
+  int total;
+  float base;
+};
+
+__device__ __forceinline__ void rope_table_fill(const RopeTable& rt, int e) {
+  if (e >= rt.total) return;
+  const int a = e >= rt.off[2] ? 2 : (e >= rt.off[1] ? 1 : 0);
+  const int r = e - rt.off[a];
+  const int p = r / rt.half[a], j = r % rt.half[a];
+  const double theta = exp(-log(static_cast<double>(rt.base)) * j / rt.half[a]);
+  double sn, cs;
+  sincos(static_cast<double>(p) * theta, &sn, &cs);
+  rt.cs[e] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+}
+
 // two floats -> two e4m3 bytes, nearest-even, saturating at +-448
 __device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float a, float b) {
   return static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));

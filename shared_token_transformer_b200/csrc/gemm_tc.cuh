@@ -33,10 +33,6 @@ namespace ts {
 
 enum GemmEpi : int { EPI_BIAS = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_QKV = 3 };
 
-struct RopeTheta {
-  float hi[32];  // per rotation pair p of a 64-channel head: theta as hi + lo floats
-  float lo[32];
-};
 
 struct GemmArgs {
   int M, N, K;
@@ -51,7 +47,8 @@ struct GemmArgs {
   const float* k_g;       // [64]
   float eps_qk;
   const int4* pos;        // [M] (f, y, x, unused) coordinates of each row
-  RopeTheta theta;
+  const float2* rope_cs;  // RoPE table (see RopeTable), filled by the preceding LayerNorm
+  int rope_off[3];        // first entry of each axis in rope_cs
 };
 
 constexpr int kGemmThreads = 320;   // 8 epilogue warps + TMA warp + MMA warp
@@ -71,10 +68,10 @@ struct GemmSmem {
 
 // QK-RMSNorm (gain g) then RoPE over one head of 64 channels held by this thread.
 // Channels of axis a form a block of R_a channels; channel j of a block pairs with
-// j + R_a / 2.  Pair index p runs over the blocks in order (the theta table order).
+// j + R_a / 2 and turns by the table's angle for (axis a, coordinate, pair j).
 template <int R0, int R1, int R2>
 __device__ __forceinline__ void qk_norm_rope64(float* v, const float* __restrict__ g, float eps, const int4 pos,
-                                               const RopeTheta& th) {
+                                               const GemmArgs& args) {
   static_assert(R0 + R1 + R2 == 64, "rope split must cover the 64-channel head");
   float ss = 0.f;
 #pragma unroll
@@ -91,16 +88,19 @@ __device__ __forceinline__ void qk_norm_rope64(float* v, const float* __restrict
 #pragma unroll
   for (int a = 0; a < 3; ++a) {
     const int D = a == 0 ? R0 : (a == 1 ? R1 : R2);
+    if (D == 0) continue;
     const int off = a == 0 ? 0 : (a == 1 ? R0 : R0 + R1);
-    const int pair0 = off / 2;
-    const float p = static_cast<float>(a == 0 ? pos.x : (a == 1 ? pos.y : pos.z));
+    const int p = a == 0 ? pos.x : (a == 1 ? pos.y : pos.z);
+    const float4* tab = reinterpret_cast<const float4*>(args.rope_cs + args.rope_off[a] + p * (D / 2));
 #pragma unroll
-    for (int j = 0; j < D / 2; ++j) {
-      float c, s;
-      rope_cos_sin(p, th.hi[pair0 + j], th.lo[pair0 + j], c, s);
-      const float x = v[off + j], y = v[off + j + D / 2];
-      v[off + j] = x * c - y * s;
-      v[off + j + D / 2] = x * s + y * c;
+    for (int j = 0; j < D / 2; j += 2) {
+      const float4 cs = __ldg(tab + j / 2);      // (cos, sin) of pairs j and j + 1
+      const float x0 = v[off + j], y0 = v[off + j + D / 2];
+      const float x1 = v[off + j + 1], y1 = v[off + j + 1 + D / 2];
+      v[off + j] = x0 * cs.x - y0 * cs.y;
+      v[off + j + D / 2] = x0 * cs.y + y0 * cs.x;
+      v[off + j + 1] = x1 * cs.z - y1 * cs.w;
+      v[off + j + 1 + D / 2] = x1 * cs.w + y1 * cs.z;
     }
   }
 }
@@ -142,7 +142,7 @@ __device__ __forceinline__ void gemm_epilogue64(float* v, int row, int col, floa
     }
   } else if (EPI == EPI_QKV) {
     if (col < 2 * args.d)
-      qk_norm_rope64<R0, R1, R2>(v, col < args.d ? args.q_g : args.k_g, args.eps_qk, pos, args.theta);
+      qk_norm_rope64<R0, R1, R2>(v, col < args.d ? args.q_g : args.k_g, args.eps_qk, pos, args);
   }
 #pragma unroll
   for (int i = 0; i < 64; i += 8) *reinterpret_cast<uint4*>(dst + i) = f32_to_bf16x8(v + i);

@@ -64,15 +64,22 @@ __device__ __forceinline__ void store_row(const float (&v)[NV][Vec<T>::E], int l
 // LayerNorm (pre-LN block, [TileShare] Tab. S1 Norm1 / Norm2): population variance,
 // two passes over the row held in registers.  NV = d / (32 * E) vectors per lane.
 // ---------------------------------------------------------------------------
+// Blocks past the rows (when rt.cs is set) fill the RoPE table that the next
+// QKV GEMM reads.
 template <typename T, int NV, bool Q8>
 __global__ void __launch_bounds__(256) layernorm_kernel(const T* __restrict__ x, int rows, int d,
                                                         const float* __restrict__ g, const float* __restrict__ b,
                                                         float eps, T* __restrict__ y, uint8_t* __restrict__ q8,
-                                                        float* __restrict__ qscale) {
+                                                        float* __restrict__ qscale, const RopeTable rt) {
   pdl_wait();
   pdl_trigger();
   constexpr int E = Vec<T>::E;
   const int lane = threadIdx.x & 31;
+  const unsigned row_blocks = (static_cast<unsigned>(rows) + 7) / 8;
+  if (blockIdx.x >= row_blocks) {
+    rope_table_fill(rt, static_cast<int>((blockIdx.x - row_blocks) * blockDim.x + threadIdx.x));
+    return;
+  }
   const size_t row = static_cast<size_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= static_cast<size_t>(rows)) return;
   float v[NV][E];

@@ -286,10 +286,33 @@ struct Workspace {
   float* qs;     // [Mx]      its per-row scales
   void* X;       // [T*N, d]  per-tile state (stack)
   void* S;       // [U+T, d]  shared state (stack)
+  float2* rope;  // RoPE cos/sin table (rope_table_entries)
   size_t bytes;
 };
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// entries of the RoPE table of a plan and model: per axis, grid extent x pairs
+static size_t rope_table_entries(const ts_plan_s* p, const ts_model_desc* m) {
+  size_t n = 0;
+  for (int a = 0; a < 3; ++a) n += static_cast<size_t>(p->grid[a]) * (m->rope_dims[a] / 2);
+  return n;
+}
+
+static ts::RopeTable make_rope_table(const ts_plan_s* p, const ts_model_desc* m, float2* cs) {
+  ts::RopeTable rt{};
+  rt.cs = cs;
+  int off = 0;
+  for (int a = 0; a < 3; ++a) {
+    rt.G[a] = p->grid[a];
+    rt.half[a] = m->rope_dims[a] / 2;
+    rt.off[a] = off;
+    off += rt.G[a] * rt.half[a];
+  }
+  rt.total = off;
+  rt.base = m->rope_base;
+  return rt;
+}
 
 static Workspace layout(const ts_plan_s* p, const ts_model_desc* m, bool stack, char* base) {
   const size_t Mt = static_cast<size_t>(p->T) * p->N, Ms = static_cast<size_t>(p->U) + p->T;
@@ -315,6 +338,7 @@ static Workspace layout(const ts_plan_s* p, const ts_model_desc* m, bool stack, 
     w.X = take(Mt * d * e);
     w.S = take(Ms * d * e);
   }
+  w.rope = reinterpret_cast<float2*>(take(rope_table_entries(p, m) * sizeof(float2)));
   w.bytes = off;
   return w;
 }
@@ -326,7 +350,8 @@ static inline unsigned rows_grid(size_t rows) { return static_cast<unsigned>((ro
 
 template <typename T, bool Q8>
 static ts_status launch_layernorm_vec(const void* x, int rows, int d, const float* g, const float* b, float eps,
-                                      void* y, uint8_t* q8, float* qs, cudaStream_t st) {
+                                      void* y, uint8_t* q8, float* qs, const ts::RopeTable& rt, cudaStream_t st) {
+  const unsigned fill_blocks = rt.cs ? static_cast<unsigned>((rt.total + 255) / 256) : 0u;
   constexpr int E = ts::Vec<T>::E;
   const int nv = d / (32 * E);
   const T* xx = static_cast<const T*>(x);
@@ -334,8 +359,8 @@ static ts_status launch_layernorm_vec(const void* x, int rows, int d, const floa
   trace_pre(st);
 #define TS_LN_CASE(NV) \
   case NV:                                                                                                  \
-    launch_pdl(ts::layernorm_kernel<T, NV, Q8>, dim3(rows_grid(rows)), dim3(256), 0, st, xx, rows, d, g, b, eps, yy, \
-               q8, qs);                                                                                       \
+    launch_pdl(ts::layernorm_kernel<T, NV, Q8>, dim3(rows_grid(rows) + fill_blocks), dim3(256), 0, st, xx, rows, d, \
+               g, b, eps, yy, q8, qs, rt);                                                                    \
     break;
   switch (nv) {
     TS_LN_CASE(1) TS_LN_CASE(2) TS_LN_CASE(3) TS_LN_CASE(4) TS_LN_CASE(5) TS_LN_CASE(6) TS_LN_CASE(7) TS_LN_CASE(8)
@@ -347,20 +372,22 @@ static ts_status launch_layernorm_vec(const void* x, int rows, int d, const floa
 
 // y = LN(x); for e4m3 writes q8/qs instead of y.
 static ts_status run_layernorm(const ts_model_desc* m, const void* x, int rows, const float* g, const float* b,
-                               void* y, uint8_t* q8, float* qs, cudaStream_t st) {
+                               void* y, uint8_t* q8, float* qs, cudaStream_t st,
+                               const ts::RopeTable& rt = ts::RopeTable{}) {
   if (rows == 0) return TS_OK;
   const int d = m->d;
   const double e = esize(m->dtype);
   set_work("layernorm", 0.0, static_cast<double>(rows) * d * (e + (q8 ? 1.0 : e)) + (q8 ? 4.0 * rows : 0.0));
   if (m->dtype == TS_F32) {
-    if (d % 128 == 0 && d <= 1024) return launch_layernorm_vec<float, false>(x, rows, d, g, b, m->eps_ln, y, nullptr, nullptr, st);
+    if (d % 128 == 0 && d <= 1024)
+      return launch_layernorm_vec<float, false>(x, rows, d, g, b, m->eps_ln, y, nullptr, nullptr, ts::RopeTable{}, st);
     trace_pre(st);
     ts::layernorm_generic_kernel<float><<<rows_grid(rows), 256, 0, st>>>(static_cast<const float*>(x), rows, d, g, b,
                                                                         m->eps_ln, static_cast<float*>(y));
     return trace_post(st, "layernorm_generic");
   }
-  if (q8) return launch_layernorm_vec<bf16, true>(x, rows, d, g, b, m->eps_ln, nullptr, q8, qs, st);
-  return launch_layernorm_vec<bf16, false>(x, rows, d, g, b, m->eps_ln, y, nullptr, nullptr, st);
+  if (q8) return launch_layernorm_vec<bf16, true>(x, rows, d, g, b, m->eps_ln, nullptr, q8, qs, rt, st);
+  return launch_layernorm_vec<bf16, false>(x, rows, d, g, b, m->eps_ln, y, nullptr, nullptr, rt, st);
 }
 
 template <typename T, bool Q8>
@@ -491,7 +518,8 @@ static int pick_bn(int M, int N) {
 // Y[M, N] = A[M, K] W[N, K]^T with epilogue; A bf16 (or e4m3 + a_scale), W bf16 (or e4m3 + w_scale).
 static ts_status run_gemm_tc(const char* name, const ts_model_desc* m, int epi, const void* A, const float* a_scale,
                              const void* W, const float* w_scale, int M, int N, int K, const float* bias, bf16* out,
-                             const ts_layer_weights* qk, const int* pos, cudaStream_t st) {
+                             const ts_layer_weights* qk, const int* pos, cudaStream_t st,
+                             const ts::RopeTable& rt = ts::RopeTable{}) {
   if (M == 0) return TS_OK;
   const bool fp8 = m->dtype == TS_FP8_E4M3;
   {
@@ -520,7 +548,8 @@ static ts_status run_gemm_tc(const char* name, const ts_model_desc* m, int epi, 
     g.q_g = qk->q_g;
     g.k_g = qk->k_g;
     g.pos = reinterpret_cast<const int4*>(pos);
-    fill_theta(m, g.theta.hi, g.theta.lo);
+    g.rope_cs = rt.cs;
+    for (int a = 0; a < 3; ++a) g.rope_off[a] = rt.off[a];
   }
   const bool r3 = m->rope_dims[0] == 16;
 #define TS_GEMM_EPI(E, R0, R1, R2) \
@@ -618,14 +647,16 @@ static ts_status run_qkv(const ts_plan_s* p, const ts_model_desc* m, const ts_la
         static_cast<float*>(qkv), rows, d, m->heads, w->q_g, w->k_g, m->eps_qk, reinterpret_cast<const int4*>(pos), r);
     return trace_post(st, "qk_norm_rope_f32");
   }
+  // LN1 also fills the RoPE table that the QKV epilogue reads
+  const ts::RopeTable rt = make_rope_table(p, m, ws.rope);
   if (m->dtype == TS_FP8_E4M3) {
-    TS_TRY(run_layernorm(m, state, rows, w->ln1_g, w->ln1_b, nullptr, ws.q8, ws.qs, st));
+    TS_TRY(run_layernorm(m, state, rows, w->ln1_g, w->ln1_b, nullptr, ws.q8, ws.qs, st, rt));
     return run_gemm_tc("gemm_qkv", m, ts::EPI_QKV, ws.q8, ws.qs, w->w_qkv, w->s_qkv, rows, 3 * d, d, w->b_qkv,
-                       static_cast<bf16*>(qkv), w, pos, st);
+                       static_cast<bf16*>(qkv), w, pos, st, rt);
   }
-  TS_TRY(run_layernorm(m, state, rows, w->ln1_g, w->ln1_b, ws.xn, nullptr, nullptr, st));
+  TS_TRY(run_layernorm(m, state, rows, w->ln1_g, w->ln1_b, ws.xn, nullptr, nullptr, st, rt));
   return run_gemm_tc("gemm_qkv", m, ts::EPI_QKV, ws.xn, nullptr, w->w_qkv, nullptr, rows, 3 * d, d, w->b_qkv,
-                     static_cast<bf16*>(qkv), w, pos, st);
+                     static_cast<bf16*>(qkv), w, pos, st, rt);
 }
 
 // out-proj (+= state) from attention/blend output `att` [rows, d]
@@ -972,6 +1003,7 @@ static Workspace layout_shared_scratch(const ts_plan_s* p, const ts_model_desc* 
     w.q8 = reinterpret_cast<uint8_t*>(take(Ms * std::max(d, f)));
     w.qs = reinterpret_cast<float*>(take(Ms * 4));
   }
+  w.rope = reinterpret_cast<float2*>(take(rope_table_entries(p, m) * sizeof(float2)));
   w.bytes = off;
   return w;
 }
@@ -1086,6 +1118,7 @@ ts_status ts_op_qkv(ts_plan_t p, const ts_model_desc* m, const ts_layer_weights*
   ws.xn = scratch;
   ws.q8 = static_cast<uint8_t*>(scratch) + align256(rows * m->d * esize(m->dtype));
   ws.qs = reinterpret_cast<float*>(ws.q8 + align256(rows * m->d));
+  ws.rope = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(ws.qs) + align256(rows * 4));
   return run_qkv(p, m, w, shared, state, qkv, ws, static_cast<cudaStream_t>(stream));
 }
 
