@@ -182,11 +182,15 @@ def model_desc(d, heads, mlp, dtype, rope_dims, eps_ln=1e-6, eps_qk=1e-6, rope_b
 
 
 def layer_weights(tensors):
-    """ts_layer_weights from a dict of device tensors (missing names -> NULL)."""
+    """ts_layer_weights from a dict of device tensors (missing names -> NULL).
+
+    The struct keeps a reference to the tensors: their device memory stays
+    allocated for as long as the struct is alive."""
     w = LayerWeights()
     for n in _WEIGHT_FIELDS:
         t = tensors.get(n)
         setattr(w, n, None if t is None else t.data_ptr())
+    w._tensors = dict(tensors)
     return w
 
 
@@ -217,7 +221,7 @@ def block_shared_noalloc(plan, model, weights, S, stream=None):
 
 def decode_stack(plan, model, weights_list, k, S0, G0, out, ws, stream=None):
     L = len(weights_list)
-    arr = (LayerWeights * L)(*weights_list)
+    arr = (LayerWeights * L)(*weights_list)      # copies of the structs; the originals keep the tensors alive
     _check("ts_decode_stack", lib().ts_decode_stack(plan.handle, ctypes.byref(model), arr, L, k, _ptr(S0), _ptr(G0),
                                                     _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
                                                     _stream(stream)))

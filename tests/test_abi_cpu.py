@@ -118,3 +118,20 @@ def test_compute_calls_refuse_host_plan():
     st = B.lib().ts_block_shared(p.handle, ctypes.byref(m), ctypes.byref(w), None, None, 0, None)
     assert st in (1, 4)     # invalid argument (or CUDA unavailable when querying the device)
     p.close()
+
+
+def test_layer_weights_keep_their_tensors_alive():
+    # the struct holds raw pointers; it must also hold the tensors behind them
+    import gc
+    import weakref
+
+    import torch
+    t = torch.zeros(16)
+    ref = weakref.ref(t)
+    w = B.layer_weights({"w_o": t})
+    del t
+    gc.collect()
+    assert ref() is not None and w.w_o == ref().data_ptr()
+    del w
+    gc.collect()
+    assert ref() is None
