@@ -8,7 +8,7 @@
 // (RoPE runs once per row in the QKV epilogue), so this is a plain gathered
 // attention.
 //
-// bf16 kernel (hd = 64), grid (nqb + 1, heads, T), 288 threads, 2 CTAs per SM:
+// bf16 kernel (hd = 64), grid (nqb, heads, T), 288 threads, 2 CTAs per SM:
 //   blocks qb < nqb: 128 window queries, keys in blocks of 64.
 //     warps 4-7  loaders: cp.async gathers of Q (once) and of K/V blocks through
 //                the row map into 128-byte-swizzled shared rows; loader warp w
@@ -26,8 +26,9 @@
 //                bf16 into one of two swizzled shared buffers; the global key
 //                (slot 0) seeds the running max and sum and is added back at the
 //                end with its running coefficient.
-//   block qb == nqb: the global token's own query row (one row attends to N keys):
-//     warps split the keys, lanes own channel pairs, partial states merged at the end.
+//   The global token's own query row (slot 0) rides along in query block 0: its
+//     loader warps update an online softmax for it on every K/V block they load
+//     (lanes own channel pairs) and merge their partial states at the end.
 // fp32 kernel (any hd <= 64, multiple of 4): one thread per query row, keys in
 //   shared memory, online softmax; for the fp32 reference-precision path.
 #pragma once
@@ -65,13 +66,10 @@ struct AttnSmem {
   static constexpr int P = 16384 + 65536;     // 2 x 16 KB: 128 rows x 64 keys
   static constexpr int KG = P + 32768;        // 64 floats k_g, 64 floats v_g
   static constexpr int BAR = KG + 512;        // barriers
-  static constexpr int NBAR = 16;
+  static constexpr int NBAR = 17;
   static constexpr int BYTES = BAR + NBAR * 8 + 16;
   static constexpr int LAUNCH_BYTES = BYTES;  // base must be 1024-aligned (checked): two CTAs per SM
 };
-// global-row blocks reuse the same dynamic shared memory
-constexpr int kAttnGlobalBytes = (32 + 32 + 32 * 64) * 4;
-static_assert(kAttnGlobalBytes <= AttnSmem::LAUNCH_BYTES, "global-row scratch must fit");
 
 // Shared-memory descriptor of an MN-major operand with the 128-byte swizzle: rows
 // of 128 bytes along K (here: keys), 64 elements along N contiguous in a row,
@@ -159,6 +157,7 @@ __device__ __forceinline__ void attn_window_block_tc(const AttnArgs& a, int qb, 
   const uint32_t bar_sfree = bar_sfull + 16;             // 2, count 4 (softmax warps read S)
   const uint32_t bar_pfull = bar_sfree + 16;             // 2, count 4 (softmax warps wrote P)
   const uint32_t bar_odone = bar_pfull + 16;             // 2, count 1 (commit after P V)
+  const uint32_t bar_ofinal = bar_odone + 16;            // 1, count 1 (commit after the last P V)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + AttnSmem::BAR + AttnSmem::NBAR * 8);
   float* sKg = reinterpret_cast<float*>(smem + AttnSmem::KG);
   float* sVg = sKg + 64;
@@ -176,6 +175,7 @@ __device__ __forceinline__ void attn_window_block_tc(const AttnArgs& a, int qb, 
       mbar_init(bar_pfull + 8 * i, 4);
       mbar_init(bar_odone + 8 * i, 1);
     }
+    mbar_init(bar_ofinal, 1);
     fence_barrier_init();
   }
   if (warp == 8) {
@@ -219,6 +219,22 @@ __device__ __forceinline__ void attn_window_block_tc(const AttnArgs& a, int qb, 
     }
     int v0 = wl < nkb ? row_of(1 + wl * kAttnBK + lane) : -1;
     int v1 = wl < nkb ? row_of(1 + wl * kAttnBK + 32 + lane) : -1;
+    // The CTA of query block 0 also computes the global token's own query row
+    // (slot 0): every loader warp runs an online softmax for it over the K/V
+    // blocks it has just loaded, its lanes owning channels 2 lane and 2 lane + 1.
+    const bool grow_row = qb == 0;
+    float gm = -INFINITY, gl = 0.f, ga0 = 0.f, ga1 = 0.f;
+    float2 gq = make_float2(0.f, 0.f);
+    if (grow_row) {
+      const size_t r = static_cast<size_t>(attn_row(a, t, 0));
+      gq = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(qkv + r * ld + h * 64 + 2 * lane));
+      if (wl == 0) {   // the global key itself
+        gm = warp_sum(gq.x * sKg[2 * lane] + gq.y * sKg[2 * lane + 1]) * a.scale_log2;
+        gl = 1.f;
+        ga0 = sVg[2 * lane];
+        ga1 = sVg[2 * lane + 1];
+      }
+    }
     for (int j = wl; j < nkb; j += kAttnKV) {
       if (j >= kAttnKV && !mbar_wait(bar_kvempty + 8 * wl, ((j / kAttnKV) - 1) & 1)) break;
 #pragma unroll
@@ -237,8 +253,78 @@ __device__ __forceinline__ void attn_window_block_tc(const AttnArgs& a, int qb, 
       cp_async_wait<0>();
       fence_proxy_async_smem();
       mbar_arrive(bar_kvfull + 8 * wl);
+      if (grow_row) {
+        __syncwarp();                    // the block's rows were copied by all lanes of this warp
+        const uint8_t* kbuf = smem + AttnSmem::K + wl * 8192;
+        const uint8_t* vbuf = smem + AttnSmem::V + wl * 8192;
+        const int nvalid = min(kAttnBK, a.Nw - j * kAttnBK);
+#pragma unroll 1
+        for (int rb = 0; rb < nvalid; rb += 8) {
+          float sc[8];
+          float2 vv[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t off = swz(rb + i, lane >> 2) + (lane & 3) * 4;
+            const float2 kk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kbuf + off));
+            vv[i] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vbuf + off));
+            sc[i] = gq.x * kk.x + gq.y * kk.y;
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) sc[i] += __shfl_xor_sync(0xffffffffu, sc[i], o);
+          float mx = gm;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            sc[i] = rb + i < nvalid ? sc[i] * a.scale_log2 : -INFINITY;
+            mx = fmaxf(mx, sc[i]);
+          }
+          const float al = exp2f(gm - mx);
+          gl *= al;
+          ga0 *= al;
+          ga1 *= al;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float pr = exp2f(sc[i] - mx);
+            gl += pr;
+            ga0 = fmaf(pr, vv[i].x, ga0);
+            ga1 = fmaf(pr, vv[i].y, ga1);
+          }
+          gm = mx;
+        }
+      }
     }
     cp_async_wait<0>();
+    if (grow_row) {
+      // merge the four loader warps' states through the P buffer, idle once the
+      // last P V has completed; the named barrier spans the loader warps only
+      const bool ok_g = mbar_wait(bar_ofinal, 0);
+      float* gbuf = reinterpret_cast<float*>(smem + AttnSmem::P);
+      if (ok_g) {
+        if (lane == 0) {
+          gbuf[wl * 66] = gm;
+          gbuf[wl * 66 + 1] = gl;
+        }
+        gbuf[wl * 66 + 2 + 2 * lane] = ga0;
+        gbuf[wl * 66 + 3 + 2 * lane] = ga1;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (ok_g && wl == 0) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kAttnKV; ++w) M = fmaxf(M, gbuf[w * 66]);
+        float L = 0.f, o0 = 0.f, o1 = 0.f;
+#pragma unroll
+        for (int w = 0; w < kAttnKV; ++w) {
+          const float f = gbuf[w * 66] == -INFINITY ? 0.f : exp2f(gbuf[w * 66] - M);
+          L += f * gbuf[w * 66 + 1];
+          o0 += f * gbuf[w * 66 + 2 + 2 * lane];
+          o1 += f * gbuf[w * 66 + 3 + 2 * lane];
+        }
+        bf16* O = reinterpret_cast<bf16*>(a.O) + static_cast<size_t>(t) * a.N * a.d + h * 64 + 2 * lane;
+        *reinterpret_cast<__nv_bfloat162*>(O) = __floats2bfloat162_rn(o0 / L, o1 / L);
+      }
+    }
   } else if (warp == 8) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
@@ -271,6 +357,8 @@ __device__ __forceinline__ void attn_window_block_tc(const AttnArgs& a, int qb, 
         tc_commit(bar_odone + 8 * pb);
         tc_commit(bar_kvempty + 8 * b);
       }
+      // single-phase barrier: waiters may arrive any number of phases early
+      if (ok) tc_commit(bar_ofinal);
     }
   } else {
     // ---------------- softmax: one query row per thread ----------------
@@ -368,7 +456,7 @@ __device__ __forceinline__ void attn_window_block_tc(const AttnArgs& a, int qb, 
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_pfull + 8 * sbuf);
     }
-    if (ok && mbar_wait(bar_odone + 8 * ((nkb - 1) & 1), ((nkb - 1) >> 1) & 1)) {
+    if (ok && mbar_wait(bar_ofinal, 0)) {
       tc_fence_after();
       const int slot = q0 + row;
       const float inv = 1.f / l;
@@ -398,75 +486,6 @@ __device__ __forceinline__ void attn_window_block_tc(const AttnArgs& a, int qb, 
   }
 }
 
-// the global token's query (slot 0): each warp takes every nw-th key, its lanes
-// own two of the 64 channels; the warps' partial softmax states are merged at the
-// end by warp 0.
-__device__ __forceinline__ void attn_global_row(const AttnArgs& a, int h, int t, uint8_t* smem) {
-  const bf16* qkv = reinterpret_cast<const bf16*>(a.qkv);
-  const int ld = 3 * a.d;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  float* sm = reinterpret_cast<float*>(smem);     // nw maxima
-  float* sl = sm + 32;                            // nw sums
-  float* sacc = sl + 32;                          // nw x 64
-  pdl_wait();
-  pdl_trigger();
-  const __nv_bfloat162 q2 =
-      *reinterpret_cast<const __nv_bfloat162*>(qkv + static_cast<size_t>(attn_row(a, t, 0)) * ld + h * 64 + 2 * lane);
-  const float2 q = __bfloat1622float2(q2);
-  float m = -INFINITY, l = 0.f, acc0 = 0.f, acc1 = 0.f;
-  // keys in batches of 8 per warp: all row indices, then all K/V loads, are issued
-  // before their first use so that their latencies overlap
-  constexpr int KB = 4;
-  for (int s0 = warp * KB; s0 < a.N; s0 += nw * KB) {
-    int rows[KB];
-#pragma unroll
-    for (int i = 0; i < KB; ++i) rows[i] = s0 + i < a.N ? attn_row(a, t, s0 + i) : -1;
-    float2 k[KB], v[KB];
-#pragma unroll
-    for (int i = 0; i < KB; ++i) {
-      if (rows[i] >= 0) {
-        const bf16* kr = qkv + static_cast<size_t>(rows[i]) * ld + a.d + h * 64 + 2 * lane;
-        k[i] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kr));
-        v[i] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kr + a.d));
-      } else {
-        k[i] = make_float2(0.f, 0.f);
-        v[i] = make_float2(0.f, 0.f);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < KB; ++i) {
-      if (rows[i] < 0) break;
-      const float sc = warp_sum(q.x * k[i].x + q.y * k[i].y) * a.scale_log2;
-      const float mn = fmaxf(m, sc);
-      const float al = exp2f(m - mn), p = exp2f(sc - mn);
-      l = l * al + p;
-      acc0 = acc0 * al + p * v[i].x;
-      acc1 = acc1 * al + p * v[i].y;
-      m = mn;
-    }
-  }
-  if (lane == 0) {
-    sm[warp] = m;
-    sl[warp] = l;
-  }
-  sacc[warp * 64 + 2 * lane] = acc0;
-  sacc[warp * 64 + 2 * lane + 1] = acc1;
-  __syncthreads();
-  if (warp == 0) {
-    float M = -INFINITY;
-    for (int w = 0; w < nw; ++w) M = fmaxf(M, sm[w]);
-    float L = 0.f, o0 = 0.f, o1 = 0.f;
-    for (int w = 0; w < nw; ++w) {
-      const float f = sm[w] == -INFINITY ? 0.f : exp2f(sm[w] - M);
-      L += f * sl[w];
-      o0 += f * sacc[w * 64 + 2 * lane];
-      o1 += f * sacc[w * 64 + 2 * lane + 1];
-    }
-    bf16* O = reinterpret_cast<bf16*>(a.O) + static_cast<size_t>(t) * a.N * a.d + h * 64 + 2 * lane;
-    *reinterpret_cast<__nv_bfloat162*>(O) = __floats2bfloat162_rn(o0 / L, o1 / L);
-  }
-}
-
 __global__ void __launch_bounds__(kAttnThreads, 2) attn_bf16_kernel(const AttnArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
@@ -474,12 +493,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_bf16_kernel(const AttnAr
     if (threadIdx.x == 0) set_status(kStatusDeviceCheck);
     return;
   }
-  const int nqb = gridDim.x - 1;
-  const int qb = blockIdx.x, h = blockIdx.y, t = blockIdx.z;
-  if (qb < nqb)
-    attn_window_block_tc(a, qb, h, t, smem);
-  else
-    attn_global_row(a, h, t, smem);
+  attn_window_block_tc(a, blockIdx.x, blockIdx.y, blockIdx.z, smem);
 }
 
 // ---------------------------------------------------------------------------

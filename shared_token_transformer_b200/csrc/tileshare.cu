@@ -620,7 +620,7 @@ static ts_status run_attention(const ts_plan_s* p, const ts_model_desc* m, bool 
                                        ts::AttnSmem::LAUNCH_BYTES));
     configured[dev] = 1;
   }
-  dim3 grid(nqb + 1, m->heads, p->T);
+  dim3 grid(nqb, m->heads, p->T);
   launch_pdl(ts::attn_bf16_kernel, grid, dim3(ts::kAttnThreads), ts::AttnSmem::LAUNCH_BYTES, st, a);
   return trace_post(st, "attn_bf16");
 }
