@@ -127,19 +127,31 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-// 2^x on the FMA pipe for x <= 9: x = n + f with n = floor(x) and f in [0, 1];
-// 2^f by a cubic fitted here to relative error (max 7.6e-5 on [0, 1], weighted
-// least squares on Chebyshev nodes), 2^n added to the exponent bits.  Arguments
-// below -125 give at most 2^-125 (treated as zero by the caller's sums).
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -125.0f);
-  const float t = (x - 0.5f) + 12582912.0f;              // 1.5 * 2^23: rounds x - 0.5 to an integer
-  const float n = t - 12582912.0f;                       // floor(x) (x itself at exact integers)
-  const int ni = __float_as_int(t) - 0x4B400000;
-  const float f = x - n;
-  const float p = fmaf(fmaf(fmaf(0.07809658348560333f, f, 0.22596493363380432f), f, 0.6958684325218201f), f,
-                       0.999923586845398f);
-  return __int_as_float(__float_as_int(p) + (ni << 23));
+// packed pairs of floats (low = first) and the sm_100 f32x2 arithmetic on them
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float lo_f32(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return lo;
+}
+__device__ __forceinline__ float hi_f32(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return hi;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
 }
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
@@ -416,15 +428,20 @@ __device__ __forceinline__ void attn_window_block_tc(const AttnArgs& a, int qb, 
       l *= alpha;
       gcoef *= alpha;
       m = mnew;
-      // every fourth exponential on the FMA pipe, the rest on the SFU; eight partial sums
-      float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      // pairs of scores through packed f32x2 arithmetic: one FMA per pair forms the
+      // exponents, the SFU takes each exponential, four packed partial sums
+      const uint64_t sc2 = pack_f32x2(a.scale_log2, a.scale_log2), nm2 = pack_f32x2(-m, -m);
+      uint64_t sp2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int i = 0; i < kAttnBK; ++i) {
-        const float xs = fmaf(sv[i], a.scale_log2, -m);
-        sv[i] = (i & 3) == 3 ? ex2_poly(xs) : ex2_approx(xs);
-        sp[i & 7] += sv[i];
+      for (int i = 0; i < kAttnBK; i += 2) {
+        const uint64_t x2 = fma_f32x2(pack_f32x2(sv[i], sv[i + 1]), sc2, nm2);
+        sv[i] = ex2_approx(lo_f32(x2));
+        sv[i + 1] = ex2_approx(hi_f32(x2));
+        sp2[(i >> 1) & 3] = add_f32x2(sp2[(i >> 1) & 3], pack_f32x2(sv[i], sv[i + 1]));
       }
-      l += ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+      const uint64_t s01 = add_f32x2(sp2[0], sp2[1]), s23 = add_f32x2(sp2[2], sp2[3]);
+      const uint64_t s0123 = add_f32x2(s01, s23);
+      l += lo_f32(s0123) + hi_f32(s0123);
       // P buffer sbuf was last read by P V of block j-2
       if (j >= 2 && !mbar_wait(bar_odone + 8 * sbuf, ((j - 2) >> 1) & 1)) { ok = false; break; }
 #pragma unroll
