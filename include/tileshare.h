@@ -75,6 +75,9 @@ typedef struct {
   int nnz;                         /* (tile, slot) entries = T * Nw                   */
   int max_cover;                   /* most tiles covering one token                   */
   int device;                      /* CUDA device holding the plan's device arrays    */
+  int run;                         /* attention loads: every aligned group of `run`    */
+                                   /* slots (1 + k*run ...) is a run of consecutive    */
+                                   /* grid tokens (64, 32, 16 or 8; 0: no such run)    */
   const int* origins;              /* host [T][3] tile origin (f, y, x)               */
   const int* tile_tok;             /* host [T][Nw] grid token of slot j of tile t      */
   const int* slot_pos;             /* host [Nw][3] tile-local (f, y, x) of slot j      */

@@ -33,6 +33,7 @@ class PlanDesc(ctypes.Structure):
     _fields_ = [("grid", _int3), ("win", _int3), ("stride", _int3),
                 ("T", ctypes.c_int), ("U", ctypes.c_int), ("Nw", ctypes.c_int), ("N", ctypes.c_int),
                 ("nnz", ctypes.c_int), ("max_cover", ctypes.c_int), ("device", ctypes.c_int),
+                ("run", ctypes.c_int),
                 ("origins", ctypes.POINTER(ctypes.c_int)), ("tile_tok", ctypes.POINTER(ctypes.c_int)),
                 ("slot_pos", ctypes.POINTER(ctypes.c_int)), ("tok_ptr", ctypes.POINTER(ctypes.c_int)),
                 ("tok_ent", ctypes.POINTER(ctypes.c_int)), ("wbar", ctypes.POINTER(ctypes.c_float))]
@@ -149,7 +150,7 @@ class Plan:
         _check("ts_plan_info", lib().ts_plan_info(h, ctypes.byref(d)))
         self.desc = d
         self.T, self.U, self.Nw, self.N, self.nnz = d.T, d.U, d.Nw, d.N, d.nnz
-        self.max_cover, self.device = d.max_cover, d.device
+        self.max_cover, self.device, self.run = d.max_cover, d.device, d.run
 
         def arr(p, n, dt):
             return np.ctypeslib.as_array(p, shape=(n,)).astype(dt).copy()

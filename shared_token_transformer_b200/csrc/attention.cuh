@@ -8,27 +8,28 @@
 // (RoPE runs once per row in the QKV epilogue), so this is a plain gathered
 // attention.
 //
-// bf16 kernel (hd = 64), grid (nqb, heads, T), 288 threads, 2 CTAs per SM:
+// bf16 kernel (hd = 64), grid (nqb, heads, T), 256 threads, 2 CTAs per SM:
 //   blocks qb < nqb: 128 window queries, keys in blocks of 64.
-//     warps 4-7  loaders: cp.async gathers of Q (once) and of K/V blocks through
-//                the row map into 128-byte-swizzled shared rows; loader warp w
-//                owns K/V buffer w (blocks w, w+4, ...), so three blocks are in
-//                flight ahead of the math; each block is published with
-//                fence.proxy.async and an mbarrier;
-//     warp 8     MMA issuer (one lane): S = Q K^T (tcgen05 kind::f16, M = 128,
-//                N = 64) into one of two TMEM S buffers, then O += P V (M = 128,
-//                N = 64, V read as an MN-major operand) into TMEM; S of block j+1
-//                is issued as soon as the softmax has read block j-1's buffer;
+//     warp 4     TMA producer: tile::gather4 loads (four rows per instruction)
+//                through the row map of Q (once) and of K/V blocks into
+//                128-byte-swizzled shared rows; four K/V buffers, completion by
+//                transaction bytes on one mbarrier per buffer;
+//     warp 5     MMA issuer (one lane): S = Q K^T (tcgen05 kind::f16, M = 128,
+//                N = 64) into one of two TMEM S buffers, then O += P V with P
+//                read from TMEM (A operand) and V from shared memory as an
+//                MN-major operand; S of block j+2 reuses the columns of P of
+//                block j and is issued after P V of block j (tcgen05.mma runs
+//                in issue order);
 //     warps 0-3  softmax, one query row per thread (TMEM lane = row): one tcgen05
 //                round trip brings the row's 64 scores into registers; online
 //                softmax in the exp2 domain with a lazily moved reference maximum
-//                (O rescaled in TMEM only when a score exceeds it by 2^8); P as
-//                bf16 into one of two swizzled shared buffers; the global key
-//                (slot 0) seeds the running max and sum and is added back at the
-//                end with its running coefficient.
-//   The global token's own query row (slot 0) rides along in query block 0: its
-//     loader warps update an online softmax for it on every K/V block they load
-//     (lanes own channel pairs) and merge their partial states at the end.
+//                (O rescaled in TMEM only when a score exceeds it by 2^8); P goes
+//                back over the scores as packed bf16; the global key (slot 0)
+//                seeds the running max and sum and is added back at the end with
+//                its running coefficient;
+//     warps 6-7  in query block 0 only: the global token's own query row (slot 0),
+//                an online softmax over the K/V blocks in shared memory (each
+//                warp every other block), merged at the end.
 // fp32 kernel (any hd <= 64, multiple of 4): one thread per query row, keys in
 //   shared memory, online softmax; for the fp32 reference-precision path.
 #pragma once
@@ -42,6 +43,7 @@ struct AttnArgs {
   const int* rowmap;  // [T * N]: qkv row of slot s of tile t (null: row = t*N + s)
   void* O;            // [T * N, d]
   int N, Nw, d, heads, T;
+  int run;            // > 0: slots come in runs of `run` consecutive rows (tiled boxes); 0: gathered rows
   float scale_log2;   // log2(e) / sqrt(hd)
   float scale;        // 1 / sqrt(hd)
 };
@@ -53,21 +55,21 @@ __device__ __forceinline__ int attn_row(const AttnArgs& a, int t, int s) {
 // byte offset of 16-byte chunk `ch` of row `r` in a 128-byte-swizzled tile
 __device__ __forceinline__ uint32_t swz(int r, int ch) { return r * 128 + ((ch ^ (r & 7)) << 4); }
 
-constexpr int kAttnThreads = 288;        // 4 softmax + 4 loader + 1 MMA warps
+constexpr int kAttnThreads = 256;        // 4 softmax, TMA producer, MMA issuer, 2 global-row warps
 constexpr int kAttnBQ = 128;             // queries per CTA
 constexpr int kAttnBK = 64;              // keys per block
-constexpr int kAttnKV = 4;               // K/V buffers (one loader warp each)
+constexpr int kAttnKV = 4;               // K/V buffers
 constexpr float kAttnRescale = 8.0f;     // lazy rescale threshold (log2 units)
 
 struct AttnSmem {
   static constexpr int Q = 0;                 // 16 KB: 128 rows x 128 B
   static constexpr int K = 16384;             // 4 x 8 KB: 64 rows x 128 B
   static constexpr int V = 16384 + 32768;     // 4 x 8 KB
-  static constexpr int P = 16384 + 65536;     // 2 x 16 KB: 128 rows x 64 keys
-  static constexpr int KG = P + 32768;        // 64 floats k_g, 64 floats v_g
-  static constexpr int BAR = KG + 512;        // barriers
-  static constexpr int NBAR = 17;
-  static constexpr int BYTES = BAR + NBAR * 8 + 16;
+  static constexpr int KG = 16384 + 65536;    // 64 floats k_g, 64 floats v_g
+  static constexpr int GR = KG + 512;         // 2 x 66 floats: partial states of the global query row
+  static constexpr int BAR = GR + 1024;       // barriers
+  static constexpr int NBAR = 15;
+  static constexpr int BYTES = BAR + NBAR * 8 + 8;
   static constexpr int LAUNCH_BYTES = BYTES;  // base must be 1024-aligned (checked): two CTAs per SM
 };
 
@@ -84,19 +86,15 @@ __device__ __forceinline__ uint64_t sdesc_sw128_mn(uint32_t saddr) {
   return d;
 }
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* v) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
       "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
       "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
-      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
-      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])),
-      "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
-      "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
-      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])),
-      "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+      "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
 }
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
@@ -154,20 +152,48 @@ __device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
   return d;
 }
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// Four rows (r0..r3) of one 128-byte column box (x = first element) gathered by
+// TMA into 512 consecutive bytes of shared memory, 128-byte swizzled like a
+// tiled load; completion is signalled on `bar` as transaction bytes.  The tensor
+// map's box is one row high.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const void* map, uint32_t bar, int x, int r0, int r1, int r2,
+                                            int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+      : "memory");
+}
+// D(tmem) (+)= A(tmem) * B(smem desc): A is read from tensor memory (row i in lane
+// i, two bf16 K elements per 32-bit column, the lower K index in the low half).
+__device__ __forceinline__ void tc_mma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 
 // ---------------------------------------------------------------------------
 // window-query block (tcgen05)
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void attn_window_block_tc(const AttnArgs& a, int qb, int h, int t, uint8_t* smem) {
+__device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, const AttnArgs& a, int qb, int h, int t,
+                                                     uint8_t* smem) {
   const bf16* qkv = reinterpret_cast<const bf16*>(a.qkv);
   const int ld = 3 * a.d;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sb = smem_u32(smem);
-  const uint32_t bar_kvfull = sb + AttnSmem::BAR;        // 4, count 32 (one loader warp each)
-  const uint32_t bar_kvempty = bar_kvfull + 32;          // 4, count 1 (commit after P V)
+  const uint32_t bar_kvfull = sb + AttnSmem::BAR;        // 4, count 1 (producer's expect_tx) + TMA bytes
+  const uint32_t bar_kvempty = bar_kvfull + 32;          // 4, count 1 (commit after P V) [+1 global-row warp]
   const uint32_t bar_sfull = bar_kvempty + 32;           // 2, count 1 (commit after Q K^T)
-  const uint32_t bar_sfree = bar_sfull + 16;             // 2, count 4 (softmax warps read S)
-  const uint32_t bar_pfull = bar_sfree + 16;             // 2, count 4 (softmax warps wrote P)
+  const uint32_t bar_pfull = bar_sfull + 16;             // 2, count 4 (softmax warps wrote P into TMEM)
   const uint32_t bar_odone = bar_pfull + 16;             // 2, count 1 (commit after P V)
   const uint32_t bar_ofinal = bar_odone + 16;            // 1, count 1 (commit after the last P V)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + AttnSmem::BAR + AttnSmem::NBAR * 8);
@@ -175,23 +201,26 @@ __device__ __forceinline__ void attn_window_block_tc(const AttnArgs& a, int qb, 
   float* sVg = sKg + 64;
   const int nkb = (a.Nw + kAttnBK - 1) / kAttnBK;
   const int q0 = 1 + qb * kAttnBQ;  // first slot of this query block
+  // The CTA of query block 0 also computes the global token's own query row
+  // (slot 0) in warps 6 and 7, which then co-own the K/V buffers they read.
+  const bool grow_row = qb == 0;
 
-  if (warp == 8 && lane == 0) {
+  if (warp == 4 && lane == 0) {
     for (int i = 0; i < kAttnKV; ++i) {
-      mbar_init(bar_kvfull + 8 * i, 32);
-      mbar_init(bar_kvempty + 8 * i, 1);
+      mbar_init(bar_kvfull + 8 * i, 1);
+      mbar_init(bar_kvempty + 8 * i, grow_row ? 2 : 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_sfull + 8 * i, 1);
-      mbar_init(bar_sfree + 8 * i, 4);
       mbar_init(bar_pfull + 8 * i, 4);
       mbar_init(bar_odone + 8 * i, 1);
     }
     mbar_init(bar_ofinal, 1);
     fence_barrier_init();
+    tma_prefetch_desc(tm);
   }
-  if (warp == 8) {
-    tmem_alloc(smem_u32(tmem_slot), 256);    // S0: cols 0-63, S1: 64-127, O: 128-191
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), 256);    // S0 / P0: cols 0-63, S1 / P1: 64-127, O: 128-191
     tmem_relinquish();
   }
   pdl_wait();
@@ -207,128 +236,192 @@ __device__ __forceinline__ void attn_window_block_tc(const AttnArgs& a, int qb, 
   const uint32_t tmem = *tmem_slot;
   const uint32_t tO = tmem + 128;
 
-  if (warp >= 4 && warp < 8) {
-    // ---------------- loaders: warp wl owns K/V buffer wl, blocks wl, wl + 4, ... ----------------
-    // The row indices of a block are read with one coalesced load (lane l holds
-    // rows l and 32 + l) and handed to the lanes that copy them by shuffles; the
-    // indices of a warp's next block are fetched before it waits for its buffer.
-    const int wl = warp - 4;
-    const int ch = lane & 7, r0 = lane >> 3;       // chunk ch of rows r0 + 4 i
-    auto row_of = [&](int slot) { return slot < a.N ? attn_row(a, t, slot) : -1; };
-    if (wl == 0) {
-      // Q rows (128 x 8 chunks) travel with block 0
-      int vq[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) vq[k] = row_of(q0 + 32 * k + lane);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int r = r0 + 4 * i;
-        const int row = __shfl_sync(0xffffffffu, vq[i >> 3], r & 31);
-        const bool ok = row >= 0;
-        const bf16* src = qkv + (ok ? static_cast<size_t>(row) * ld + h * 64 + ch * 8 : 0);
-        cp_async16(sb + AttnSmem::Q + swz(r, ch), src, ok);
+  if (warp == 4 && a.run > 0) {
+    // ---------------- TMA producer, runs of consecutive rows ----------------
+    // Each run of `run` slots is one tiled box (128 bytes x run rows) of the q/k/v
+    // columns of head h.  Runs past the tile's last slot (padding of the last key
+    // or query block) load the first run again: their scores are masked and their
+    // outputs are not stored.
+    if (lane == 0) {
+      const int L = a.run;
+      auto run_row = [&](int slot) { return attn_row(a, t, slot < a.N ? slot : 1); };
+      const int xq = h * 64, xk = a.d + h * 64, xv = 2 * a.d + h * 64;
+      mbar_expect_tx(bar_kvfull, 2 * 16384);   // Q rows travel with K/V block 0
+      for (int s = 0; s < kAttnBQ; s += L) tma_load_2d(sb + AttnSmem::Q + s * 128, tm, bar_kvfull, xq, run_row(q0 + s));
+      int armed = 0;
+      for (int j = 0; j < nkb; ++j) {
+        const int b = j % kAttnKV;
+        if (j > 0) {
+          if (j >= kAttnKV && !mbar_wait(bar_kvempty + 8 * b, ((j / kAttnKV) - 1) & 1)) break;
+          mbar_expect_tx(bar_kvfull + 8 * b, 16384);
+        }
+        for (int s = 0; s < kAttnBK; s += L) {
+          const int r = run_row(1 + j * kAttnBK + s);
+          tma_load_2d(sb + AttnSmem::K + b * 8192 + s * 128, tm, bar_kvfull + 8 * b, xk, r);
+          tma_load_2d(sb + AttnSmem::V + b * 8192 + s * 128, tm, bar_kvfull + 8 * b, xv, r);
+        }
+        armed = j + 1;
       }
+      // no copy may still be landing when the CTA exits (matters only after a timeout)
+      for (int j = max(0, armed - kAttnKV); j < armed; ++j) mbar_wait(bar_kvfull + 8 * (j % kAttnKV), (j / kAttnKV) & 1);
     }
-    int v0 = wl < nkb ? row_of(1 + wl * kAttnBK + lane) : -1;
-    int v1 = wl < nkb ? row_of(1 + wl * kAttnBK + 32 + lane) : -1;
-    // The CTA of query block 0 also computes the global token's own query row
-    // (slot 0): every loader warp runs an online softmax for it over the K/V
-    // blocks it has just loaded, its lanes owning channels 2 lane and 2 lane + 1.
-    const bool grow_row = qb == 0;
-    float gm = -INFINITY, gl = 0.f, ga0 = 0.f, ga1 = 0.f;
-    float2 gq = make_float2(0.f, 0.f);
+  } else if (warp == 4) {
+    // ---------------- TMA producer, gathered rows ----------------
+    // Rows are gathered four at a time (tile::gather4) from the q/k/v columns of
+    // head h.  Slots past the tile's last one (padding of the last key or query
+    // block) repeat the last slot's row, so every coordinate is in range; their
+    // scores are masked and their outputs are not stored.
+    auto row_of = [&](int slot) { return attn_row(a, t, min(slot, a.N - 1)); };
+    const int xq = h * 64, xk = a.d + h * 64, xv = 2 * a.d + h * 64;
+    int vq[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) vq[k] = row_of(q0 + 32 * k + lane);
+    int v0 = row_of(1 + lane), v1 = row_of(33 + lane);
+    if (lane == 0) mbar_expect_tx(bar_kvfull, 2 * 16384);   // Q rows travel with K/V block 0
+#pragma unroll
+    for (int g = 0; g < 32; ++g) {
+      int r[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) r[i] = __shfl_sync(0xffffffffu, vq[g >> 3], (4 * g + i) & 31);
+      if (lane == 0) tma_gather4(sb + AttnSmem::Q + g * 512, tm, bar_kvfull, xq, r[0], r[1], r[2], r[3]);
+    }
+    int armed = 0;
+    for (int j = 0; j < nkb; ++j) {
+      const int b = j % kAttnKV;
+      if (j > 0) {
+        v0 = row_of(1 + j * kAttnBK + lane);
+        v1 = row_of(1 + j * kAttnBK + 32 + lane);
+        int ok = 1;
+        if (lane == 0 && j >= kAttnKV) ok = mbar_wait(bar_kvempty + 8 * b, ((j / kAttnKV) - 1) & 1);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        if (lane == 0) mbar_expect_tx(bar_kvfull + 8 * b, 16384);
+      }
+#pragma unroll
+      for (int g = 0; g < 16; ++g) {
+        int r[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) r[i] = __shfl_sync(0xffffffffu, g < 8 ? v0 : v1, (4 * g + i) & 31);
+        if (lane == 0) {
+          tma_gather4(sb + AttnSmem::K + b * 8192 + g * 512, tm, bar_kvfull + 8 * b, xk, r[0], r[1], r[2], r[3]);
+          tma_gather4(sb + AttnSmem::V + b * 8192 + g * 512, tm, bar_kvfull + 8 * b, xv, r[0], r[1], r[2], r[3]);
+        }
+      }
+      armed = j + 1;
+    }
+    // no copy may still be landing when the CTA exits (matters only after a timeout)
+    if (lane == 0)
+      for (int j = max(0, armed - kAttnKV); j < armed; ++j) mbar_wait(bar_kvfull + 8 * (j % kAttnKV), (j / kAttnKV) & 1);
+  } else if (warp == 5) {
+    // ---------------- MMA issuer ----------------
+    // S of block j+2 goes into the TMEM columns that hold P of block j; it is
+    // issued after P V of block j, and tcgen05.mma runs in issue order.
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_make(1u, kAttnBK);             // Q K^T: M 128, N 64
+      constexpr uint32_t IDESC_O = idesc_make(1u, 64) | (1u << 16);     // P V: M 128, N 64, B MN-major
+      const uint64_t dq = sdesc_sw128(sb + AttnSmem::Q);
+      auto issue_s = [&](int j) -> bool {
+        const int b = j % kAttnKV, sbuf = j & 1;
+        if (!mbar_wait(bar_kvfull + 8 * b, (j / kAttnKV) & 1)) return false;
+        tc_fence_after();
+        const uint64_t dk = sdesc_sw128(sb + AttnSmem::K + b * 8192);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) tc_mma_f16(tmem + sbuf * 64, dq + 2 * k, dk + 2 * k, IDESC_S, k != 0);
+        tc_commit(bar_sfull + 8 * sbuf);
+        return true;
+      };
+      bool ok = issue_s(0) && (nkb < 2 || issue_s(1));
+      for (int j = 0; j < nkb && ok; ++j) {
+        const int pb = j & 1, b = j % kAttnKV;
+        if (!mbar_wait(bar_pfull + 8 * pb, (j >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t dv = sdesc_sw128_mn(sb + AttnSmem::V + b * 8192 + kk * 2048);
+          tc_mma_f16_tmem_a(tO, tmem + pb * 64 + kk * 8, dv, IDESC_O, (j | kk) != 0);
+        }
+        tc_commit(bar_odone + 8 * pb);
+        tc_commit(bar_kvempty + 8 * b);
+        if (j + 2 < nkb) ok = issue_s(j + 2);
+      }
+      // single-phase barrier: waiters may arrive any number of phases early
+      if (ok) tc_commit(bar_ofinal);
+    }
+  } else if (warp >= 6) {
+    // ---------------- global token's query row (query block 0 only) ----------------
+    // Warp 6 + g takes blocks g, g + 2, ...: lane l scores keys l and l + 32 with
+    // the full query in registers, then accumulates channels 2l, 2l + 1 of P V.
+    // The two warps' online-softmax states are merged at the end.
     if (grow_row) {
-      const size_t r = static_cast<size_t>(attn_row(a, t, 0));
-      gq = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(qkv + r * ld + h * 64 + 2 * lane));
-      if (wl == 0) {   // the global key itself
-        gm = warp_sum(gq.x * sKg[2 * lane] + gq.y * sKg[2 * lane + 1]) * a.scale_log2;
-        gl = 1.f;
+      const int g = warp - 6;
+      float qf[64];
+      {
+        const uint4* qr = reinterpret_cast<const uint4*>(qkv + static_cast<size_t>(attn_row(a, t, 0)) * ld + h * 64);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) bf16x8_to_f32(qr[c], qf + 8 * c);
+      }
+      float gm = -INFINITY, gl = 0.f, ga0 = 0.f, ga1 = 0.f;
+      if (g == 0) {   // the global key itself
+        float sg = 0.f;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) sg = fmaf(qf[c], sKg[c], sg);
+        gm = sg * a.scale_log2;
+        gl = lane == 0 ? 1.f : 0.f;
         ga0 = sVg[2 * lane];
         ga1 = sVg[2 * lane + 1];
       }
-    }
-    for (int j = wl; j < nkb; j += kAttnKV) {
-      if (j >= kAttnKV && !mbar_wait(bar_kvempty + 8 * wl, ((j / kAttnKV) - 1) & 1)) break;
+      for (int j = g; j < nkb; j += 2) {
+        const int b = j % kAttnKV;
+        if (!mbar_wait(bar_kvfull + 8 * b, (j / kAttnKV) & 1)) break;
+        const uint8_t* kbuf = smem + AttnSmem::K + b * 8192;
+        const uint8_t* vbuf = smem + AttnSmem::V + b * 8192;
+        float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int r = r0 + 4 * i;
-        const int row = __shfl_sync(0xffffffffu, i < 8 ? v0 : v1, r & 31);
-        const bool ok = row >= 0;
-        const size_t base = ok ? static_cast<size_t>(row) * ld + h * 64 + ch * 8 : 0;
-        cp_async16(sb + AttnSmem::K + wl * 8192 + swz(r, ch), qkv + base + (ok ? a.d : 0), ok);
-        cp_async16(sb + AttnSmem::V + wl * 8192 + swz(r, ch), qkv + base + (ok ? 2 * a.d : 0), ok);
-      }
-      cp_async_commit();
-      const int jn = j + kAttnKV;
-      v0 = jn < nkb ? row_of(1 + jn * kAttnBK + lane) : -1;
-      v1 = jn < nkb ? row_of(1 + jn * kAttnBK + 32 + lane) : -1;
-      cp_async_wait<0>();
-      fence_proxy_async_smem();
-      mbar_arrive(bar_kvfull + 8 * wl);
-      if (grow_row) {
-        __syncwarp();                    // the block's rows were copied by all lanes of this warp
-        const uint8_t* kbuf = smem + AttnSmem::K + wl * 8192;
-        const uint8_t* vbuf = smem + AttnSmem::V + wl * 8192;
+        for (int c = 0; c < 8; ++c) {
+          float f0[8], f1[8];
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(kbuf + swz(lane, c)), f0);
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(kbuf + swz(lane + 32, c)), f1);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            s0 = fmaf(qf[8 * c + e], f0[e], s0);
+            s1 = fmaf(qf[8 * c + e], f1[e], s1);
+          }
+        }
         const int nvalid = min(kAttnBK, a.Nw - j * kAttnBK);
-#pragma unroll 1
-        for (int rb = 0; rb < nvalid; rb += 8) {
-          float sc[8];
-          float2 vv[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint32_t off = swz(rb + i, lane >> 2) + (lane & 3) * 4;
-            const float2 kk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kbuf + off));
-            vv[i] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vbuf + off));
-            sc[i] = gq.x * kk.x + gq.y * kk.y;
-          }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-            for (int i = 0; i < 8; ++i) sc[i] += __shfl_xor_sync(0xffffffffu, sc[i], o);
-          float mx = gm;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            sc[i] = rb + i < nvalid ? sc[i] * a.scale_log2 : -INFINITY;
-            mx = fmaxf(mx, sc[i]);
-          }
-          const float al = exp2f(gm - mx);
-          gl *= al;
-          ga0 *= al;
-          ga1 *= al;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float pr = exp2f(sc[i] - mx);
-            gl += pr;
-            ga0 = fmaf(pr, vv[i].x, ga0);
-            ga1 = fmaf(pr, vv[i].y, ga1);
-          }
-          gm = mx;
+        const float x0 = lane < nvalid ? s0 * a.scale_log2 : -INFINITY;
+        const float x1 = lane + 32 < nvalid ? s1 * a.scale_log2 : -INFINITY;
+        const float mnew = fmaxf(gm, warp_max(fmaxf(x0, x1)));
+        const float al = ex2_approx(gm - mnew);
+        const float p0 = ex2_approx(x0 - mnew), p1 = ex2_approx(x1 - mnew);
+        gl = fmaf(gl, al, p0 + p1);
+        ga0 *= al;
+        ga1 *= al;
+#pragma unroll 8
+        for (int k = 0; k < kAttnBK; ++k) {
+          const float pk = __shfl_sync(0xffffffffu, k < 32 ? p0 : p1, k & 31);
+          const uint32_t off = swz(k, lane >> 2) + (lane & 3) * 4;
+          const float2 vv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vbuf + off));
+          ga0 = fmaf(pk, vv.x, ga0);
+          ga1 = fmaf(pk, vv.y, ga1);
         }
+        gm = mnew;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_kvempty + 8 * b);
       }
-    }
-    cp_async_wait<0>();
-    if (grow_row) {
-      // merge the four loader warps' states through the P buffer, idle once the
-      // last P V has completed; the named barrier spans the loader warps only
-      const bool ok_g = mbar_wait(bar_ofinal, 0);
-      float* gbuf = reinterpret_cast<float*>(smem + AttnSmem::P);
-      if (ok_g) {
-        if (lane == 0) {
-          gbuf[wl * 66] = gm;
-          gbuf[wl * 66 + 1] = gl;
-        }
-        gbuf[wl * 66 + 2 + 2 * lane] = ga0;
-        gbuf[wl * 66 + 3 + 2 * lane] = ga1;
+      gl = warp_sum(gl);
+      float* gbuf = reinterpret_cast<float*>(smem + AttnSmem::GR);
+      if (lane == 0) {
+        gbuf[g * 66] = gm;
+        gbuf[g * 66 + 1] = gl;
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (ok_g && wl == 0) {
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kAttnKV; ++w) M = fmaxf(M, gbuf[w * 66]);
+      gbuf[g * 66 + 2 + 2 * lane] = ga0;
+      gbuf[g * 66 + 3 + 2 * lane] = ga1;
+      asm volatile("bar.sync 1, 64;" ::: "memory");
+      if (g == 0) {
+        const float M = fmaxf(gbuf[0], gbuf[66]);
         float L = 0.f, o0 = 0.f, o1 = 0.f;
 #pragma unroll
-        for (int w = 0; w < kAttnKV; ++w) {
-          const float f = gbuf[w * 66] == -INFINITY ? 0.f : exp2f(gbuf[w * 66] - M);
+        for (int w = 0; w < 2; ++w) {
+          const float f = gbuf[w * 66] == -INFINITY ? 0.f : ex2_approx(gbuf[w * 66] - M);
           L += f * gbuf[w * 66 + 1];
           o0 += f * gbuf[w * 66 + 2 + 2 * lane];
           o1 += f * gbuf[w * 66 + 3 + 2 * lane];
@@ -337,42 +430,7 @@ __device__ __forceinline__ void attn_window_block_tc(const AttnArgs& a, int qb, 
         *reinterpret_cast<__nv_bfloat162*>(O) = __floats2bfloat162_rn(o0 / L, o1 / L);
       }
     }
-  } else if (warp == 8) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_make(1u, kAttnBK);             // Q K^T: M 128, N 64
-      constexpr uint32_t IDESC_O = idesc_make(1u, 64) | (1u << 16);     // P V: M 128, N 64, B MN-major
-      const uint64_t dq = sdesc_sw128(sb + AttnSmem::Q);
-      auto issue_s = [&](int j) -> bool {
-        const int b = j % kAttnKV, sbuf = j & 1;
-        if (!mbar_wait(bar_kvfull + 8 * b, (j / kAttnKV) & 1)) return false;
-        if (j >= 2 && !mbar_wait(bar_sfree + 8 * sbuf, ((j >> 1) - 1) & 1)) return false;
-        tc_fence_after();
-        const uint64_t dk = sdesc_sw128(sb + AttnSmem::K + b * 8192);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) tc_mma_f16(tmem + sbuf * 64, dq + 2 * k, dk + 2 * k, IDESC_S, k != 0);
-        tc_commit(bar_sfull + 8 * sbuf);
-        return true;
-      };
-      bool ok = issue_s(0);
-      for (int j = 0; j < nkb && ok; ++j) {
-        if (j + 1 < nkb && !(ok = issue_s(j + 1))) break;
-        const int pb = j & 1, b = j % kAttnKV;
-        if (!mbar_wait(bar_pfull + 8 * pb, (j >> 1) & 1)) { ok = false; break; }
-        tc_fence_after();
-        const uint64_t dp = sdesc_sw128(sb + AttnSmem::P + pb * 16384);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t dv = sdesc_sw128_mn(sb + AttnSmem::V + b * 8192 + kk * 2048);
-          tc_mma_f16(tO, dp + 2 * kk, dv, IDESC_O, (j | kk) != 0);
-        }
-        tc_commit(bar_odone + 8 * pb);
-        tc_commit(bar_kvempty + 8 * b);
-      }
-      // single-phase barrier: waiters may arrive any number of phases early
-      if (ok) tc_commit(bar_ofinal);
-    }
-  } else {
+  } else if (warp < 4) {
     // ---------------- softmax: one query row per thread ----------------
     const int row = tid;                     // 0..127, TMEM lane = row
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
@@ -400,9 +458,6 @@ __device__ __forceinline__ void attn_window_block_tc(const AttnArgs& a, int qb, 
       tmem_ld32(tmem + sbuf * 64 + lane_off, sv);
       tmem_ld32(tmem + sbuf * 64 + lane_off + 32, sv + 32);
       tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_sfree + 8 * sbuf);   // S buffer may be overwritten
       const int kbase = j * kAttnBK;
       // row maximum of the raw scores (the scale is positive); keys beyond the
       // window exist only in the last block
@@ -414,45 +469,39 @@ __device__ __forceinline__ void attn_window_block_tc(const AttnArgs& a, int qb, 
       // eight independent partial maxima keep the dependency chains short
       float mp[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) mp[q] = sv[q];
-#pragma unroll
-      for (int i = 8; i < kAttnBK; ++i) mp[i & 7] = fmaxf(mp[i & 7], sv[i]);
-      const float mr = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-      const float mx = mr * a.scale_log2;
+      for (int q = 0; q < 8; ++q) {
+        mp[q] = fmax3(sv[q], sv[8 + q], sv[16 + q]);
+        mp[q] = fmax3(mp[q], sv[24 + q], sv[32 + q]);
+        mp[q] = fmax3(mp[q], sv[40 + q], sv[48 + q]);
+        mp[q] = fmaxf(mp[q], sv[56 + q]);
+      }
+      const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7])) * a.scale_log2;
       // lazy rescale: the reference maximum moves only when a score exceeds it by
       // more than 2^8, so probabilities stay below 256 and O is rarely touched
       const bool grow = mx > m + kAttnRescale;
       const float mnew = grow ? mx : m;
-      const float alpha = exp2f(m - mnew);
+      const float alpha = grow ? ex2_approx(m - mnew) : 1.f;
       const bool warp_grow = __any_sync(0xffffffffu, grow);
       l *= alpha;
       gcoef *= alpha;
       m = mnew;
       // pairs of scores through packed f32x2 arithmetic: one FMA per pair forms the
-      // exponents, the SFU takes each exponential, four packed partial sums
+      // exponents, the SFU takes each exponential, four packed partial sums; P goes
+      // back into the S columns as packed bf16 pairs (the A operand of P V)
       const uint64_t sc2 = pack_f32x2(a.scale_log2, a.scale_log2), nm2 = pack_f32x2(-m, -m);
       uint64_t sp2[4] = {0ull, 0ull, 0ull, 0ull};
+      uint32_t pw[kAttnBK / 2];
 #pragma unroll
       for (int i = 0; i < kAttnBK; i += 2) {
         const uint64_t x2 = fma_f32x2(pack_f32x2(sv[i], sv[i + 1]), sc2, nm2);
-        sv[i] = ex2_approx(lo_f32(x2));
-        sv[i + 1] = ex2_approx(hi_f32(x2));
-        sp2[(i >> 1) & 3] = add_f32x2(sp2[(i >> 1) & 3], pack_f32x2(sv[i], sv[i + 1]));
+        const float e0 = ex2_approx(lo_f32(x2)), e1 = ex2_approx(hi_f32(x2));
+        sp2[(i >> 1) & 3] = add_f32x2(sp2[(i >> 1) & 3], pack_f32x2(e0, e1));
+        pw[i >> 1] = pack_bf16(e0, e1);
       }
       const uint64_t s01 = add_f32x2(sp2[0], sp2[1]), s23 = add_f32x2(sp2[2], sp2[3]);
       const uint64_t s0123 = add_f32x2(s01, s23);
       l += lo_f32(s0123) + hi_f32(s0123);
-      // P buffer sbuf was last read by P V of block j-2
-      if (j >= 2 && !mbar_wait(bar_odone + 8 * sbuf, ((j - 2) >> 1) & 1)) { ok = false; break; }
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 u;
-        u.x = pack_bf16(sv[c * 8 + 0], sv[c * 8 + 1]);
-        u.y = pack_bf16(sv[c * 8 + 2], sv[c * 8 + 3]);
-        u.z = pack_bf16(sv[c * 8 + 4], sv[c * 8 + 5]);
-        u.w = pack_bf16(sv[c * 8 + 6], sv[c * 8 + 7]);
-        *reinterpret_cast<uint4*>(smem + AttnSmem::P + sbuf * 16384 + swz(row, c)) = u;
-      }
+      tmem_st32u(tmem + sbuf * 64 + lane_off, pw);
       if (warp_grow && j >= 1) {
         // O holds the sum up to block j-1: wait for that P V, then rescale the row
         if (!mbar_wait(bar_odone + 8 * ((j - 1) & 1), ((j - 1) >> 1) & 1)) { ok = false; break; }
@@ -466,9 +515,8 @@ __device__ __forceinline__ void attn_window_block_tc(const AttnArgs& a, int qb, 
           for (int c = 0; c < 16; ++c) o[c] *= alpha;
           tmem_st16(tO + lane_off + hh * 16, o);
         }
-        tmem_wait_st();
       }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_pfull + 8 * sbuf);
@@ -497,20 +545,21 @@ __device__ __forceinline__ void attn_window_block_tc(const AttnArgs& a, int qb, 
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 5) {
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }
 }
 
-__global__ void __launch_bounds__(kAttnThreads, 2) attn_bf16_kernel(const AttnArgs a) {
+__global__ void __launch_bounds__(kAttnThreads, 2)
+    attn_bf16_kernel(const __grid_constant__ CUtensorMap tm, const AttnArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
   if (smem_u32(smem) & 1023u) {          // swizzled tiles need a 1024-byte aligned base
     if (threadIdx.x == 0) set_status(kStatusDeviceCheck);
     return;
   }
-  attn_window_block_tc(a, blockIdx.x, blockIdx.y, blockIdx.z, smem);
+  attn_window_block_tc(&tm, a, blockIdx.x, blockIdx.y, blockIdx.z, smem);
 }
 
 // ---------------------------------------------------------------------------

@@ -24,6 +24,7 @@
 struct ts_plan_s {
   int grid[3], win[3], stride[3];
   int T, U, Nw, N, nnz, max_cover, device;
+  int run;                       // window slots 1 + k*run .. are runs of consecutive shared rows (0: none)
   std::vector<int> origins, tile_tok, slot_pos, tok_ptr, tok_ent;
   std::vector<float> wbar;
   std::vector<int> rowmap;       // [T*N] shared-layout row of slot s of tile t (s = 0: U + t)
@@ -143,6 +144,16 @@ inline bool build(ts_plan_s& P) {
       P.rowmap[r] = P.tile_tok[static_cast<size_t>(t) * P.Nw + j];
       for (int a = 0; a < 3; ++a) P.pos_tiled[4 * r + a] = P.slot_pos[3 * j + a];
     }
+  }
+  // longest run length (64, 32, 16 or 8) such that every aligned group of slots
+  // 1 + k*run, ..., run + k*run of every tile maps to consecutive shared rows
+  P.run = 0;
+  for (int L = 64; L >= 8 && !P.run; L >>= 1) {
+    bool ok = true;
+    for (int t = 0; t < P.T && ok; ++t)
+      for (int j = 1; j < P.Nw && ok; ++j)
+        if (j % L) ok = P.rowmap[static_cast<size_t>(t) * P.N + 1 + j] == P.rowmap[static_cast<size_t>(t) * P.N + j] + 1;
+    if (ok) P.run = L;
   }
   P.pos_shared.assign(static_cast<size_t>(P.U + P.T) * 4, 0);
   for (int f = 0, u = 0; f < F; ++f)

@@ -620,8 +620,14 @@ static ts_status run_attention(const ts_plan_s* p, const ts_model_desc* m, bool 
                                        ts::AttnSmem::LAUNCH_BYTES));
     configured[dev] = 1;
   }
+  // map over the q/k/v rows: a 128-byte column box, `run` rows high for runs of
+  // consecutive rows (the per-tile layout is one run per tile), one row high for
+  // four-row gathers
+  a.run = shared ? p->run : 64;
+  CUtensorMap tm;
+  TS_TRY(make_tmap(&tm, qkv, shared ? p->U + p->T : p->T * p->N, 3 * m->d, 2, a.run > 0 ? a.run : 1));
   dim3 grid(nqb, m->heads, p->T);
-  launch_pdl(ts::attn_bf16_kernel, grid, dim3(ts::kAttnThreads), ts::AttnSmem::LAUNCH_BYTES, st, a);
+  launch_pdl(ts::attn_bf16_kernel, grid, dim3(ts::kAttnThreads), ts::AttnSmem::LAUNCH_BYTES, st, tm, a);
   return trace_post(st, "attn_bf16");
 }
 
@@ -897,6 +903,7 @@ ts_status ts_plan_info(ts_plan_t p, ts_plan_desc* out) {
   out->nnz = p->nnz;
   out->max_cover = p->max_cover;
   out->device = p->device;
+  out->run = p->run;
   out->origins = p->origins.data();
   out->tile_tok = p->tile_tok.data();
   out->slot_pos = p->slot_pos.data();

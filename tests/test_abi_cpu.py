@@ -70,6 +70,33 @@ def test_host_planner_bit_exact_against_oracle(grid, win, stride):
         p.close()
 
 
+RUNS = {(1, 48, 48): 16, (4, 44, 80): 32, (1, 128, 128): 32, (1, 11, 13): 8, (3, 7, 9): 0, (1, 20, 9): 0,
+        (1, 5, 5): 64}
+
+
+@pytest.mark.parametrize("grid,win,stride", GEOMS)
+def test_plan_run_length(grid, win, stride):
+    """Attention loads fetch each run of consecutive grid tokens as one box: the
+    planner's run length is the longest of 64, 32, 16, 8 whose aligned slot groups
+    are consecutive tokens in every tile (brute force over the oracle's map)."""
+    o = OP.make_plan(grid, win, stride)
+    want = 0
+    for L in (64, 32, 16, 8):
+        tt = np.asarray(o.tile_tok)
+        j = np.arange(1, o.Nw)
+        j = j[j % L != 0]
+        if np.all(tt[:, j] == tt[:, j - 1] + 1):
+            want = L
+            break
+    if grid in RUNS:
+        assert want == RUNS[grid]
+    p = B.Plan(grid, win, stride, host_only=True)
+    try:
+        assert p.run == want
+    finally:
+        p.close()
+
+
 def test_image4k_plan_counts():
     p = B.Plan((1, 256, 256), (1, 32, 32), (1, 24, 24), host_only=True)
     assert (p.T, p.U, p.N, p.nnz, p.max_cover) == (121, 65536, 1025, 123904, 4)
