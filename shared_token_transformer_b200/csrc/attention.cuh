@@ -241,30 +241,43 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
     // Each run of `run` slots is one tiled box (128 bytes x run rows) of the q/k/v
     // columns of head h.  Runs past the tile's last slot (padding of the last key
     // or query block) load the first run again: their scores are masked and their
-    // outputs are not stored.
-    if (lane == 0) {
-      const int L = a.run;
-      auto run_row = [&](int slot) { return attn_row(a, t, slot < a.N ? slot : 1); };
-      const int xq = h * 64, xk = a.d + h * 64, xv = 2 * a.d + h * 64;
-      mbar_expect_tx(bar_kvfull, 2 * 16384);   // Q rows travel with K/V block 0
-      for (int s = 0; s < kAttnBQ; s += L) tma_load_2d(sb + AttnSmem::Q + s * 128, tm, bar_kvfull, xq, run_row(q0 + s));
-      int armed = 0;
-      for (int j = 0; j < nkb; ++j) {
-        const int b = j % kAttnKV;
-        if (j > 0) {
-          if (j >= kAttnKV && !mbar_wait(bar_kvempty + 8 * b, ((j / kAttnKV) - 1) & 1)) break;
-          mbar_expect_tx(bar_kvfull + 8 * b, 16384);
-        }
-        for (int s = 0; s < kAttnBK; s += L) {
-          const int r = run_row(1 + j * kAttnBK + s);
-          tma_load_2d(sb + AttnSmem::K + b * 8192 + s * 128, tm, bar_kvfull + 8 * b, xk, r);
-          tma_load_2d(sb + AttnSmem::V + b * 8192 + s * 128, tm, bar_kvfull + 8 * b, xv, r);
-        }
-        armed = j + 1;
+    // outputs are not stored.  Lane i looks up the row of run i one block ahead;
+    // lane 0 issues the copies.
+    const int L = a.run, nrun = kAttnBK / L;
+    auto run_row = [&](int slot) { return attn_row(a, t, slot < a.N ? slot : 1); };
+    const int xq = h * 64, xk = a.d + h * 64, xv = 2 * a.d + h * 64;
+    {
+      const int rq = lane < kAttnBQ / L ? run_row(q0 + lane * L) : 0;
+      if (lane == 0) mbar_expect_tx(bar_kvfull, 2 * 16384);   // Q rows travel with K/V block 0
+      for (int i = 0; i < kAttnBQ / L; ++i) {
+        const int r = __shfl_sync(0xffffffffu, rq, i);
+        if (lane == 0) tma_load_2d(sb + AttnSmem::Q + i * L * 128, tm, bar_kvfull, xq, r);
       }
-      // no copy may still be landing when the CTA exits (matters only after a timeout)
-      for (int j = max(0, armed - kAttnKV); j < armed; ++j) mbar_wait(bar_kvfull + 8 * (j % kAttnKV), (j / kAttnKV) & 1);
     }
+    int rnext = lane < nrun ? run_row(1 + lane * L) : 0;
+    int armed = 0;
+    for (int j = 0; j < nkb; ++j) {
+      const int b = j % kAttnKV;
+      const int rcur = rnext;
+      if (j + 1 < nkb && lane < nrun) rnext = run_row(1 + (j + 1) * kAttnBK + lane * L);
+      if (j > 0) {
+        int ok = 1;
+        if (lane == 0 && j >= kAttnKV) ok = mbar_wait(bar_kvempty + 8 * b, ((j / kAttnKV) - 1) & 1);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        if (lane == 0) mbar_expect_tx(bar_kvfull + 8 * b, 16384);
+      }
+      for (int i = 0; i < nrun; ++i) {
+        const int r = __shfl_sync(0xffffffffu, rcur, i);
+        if (lane == 0) {
+          tma_load_2d(sb + AttnSmem::K + b * 8192 + i * L * 128, tm, bar_kvfull + 8 * b, xk, r);
+          tma_load_2d(sb + AttnSmem::V + b * 8192 + i * L * 128, tm, bar_kvfull + 8 * b, xv, r);
+        }
+      }
+      armed = j + 1;
+    }
+    // no copy may still be landing when the CTA exits (matters only after a timeout)
+    if (lane == 0)
+      for (int j = max(0, armed - kAttnKV); j < armed; ++j) mbar_wait(bar_kvfull + 8 * (j % kAttnKV), (j / kAttnKV) & 1);
   } else if (warp == 4) {
     // ---------------- TMA producer, gathered rows ----------------
     // Rows are gathered four at a time (tile::gather4) from the q/k/v columns of
