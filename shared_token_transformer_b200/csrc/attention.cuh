@@ -152,6 +152,14 @@ __device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
   return d;
 }
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// true in exactly one lane of the (fully active) warp
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(pred));
+  return pred != 0;
+}
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -327,26 +335,32 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
   } else if (warp == 5) {
     // ---------------- MMA issuer ----------------
     // S of block j+2 goes into the TMEM columns that hold P of block j; it is
-    // issued after P V of block j, and tcgen05.mma runs in issue order.
-    if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_make(1u, kAttnBK);             // Q K^T: M 128, N 64
-      constexpr uint32_t IDESC_O = idesc_make(1u, 64) | (1u << 16);     // P V: M 128, N 64, B MN-major
-      const uint64_t dq = sdesc_sw128(sb + AttnSmem::Q);
-      auto issue_s = [&](int j) -> bool {
-        const int b = j % kAttnKV, sbuf = j & 1;
-        if (!mbar_wait(bar_kvfull + 8 * b, (j / kAttnKV) & 1)) return false;
-        tc_fence_after();
+    // issued after P V of block j, and tcgen05.mma runs in issue order.  The whole
+    // warp waits on the barriers (lane 0's outcome decides for all); one elected
+    // lane issues the MMAs and commits.
+    constexpr uint32_t IDESC_S = idesc_make(1u, kAttnBK);             // Q K^T: M 128, N 64
+    constexpr uint32_t IDESC_O = idesc_make(1u, 64) | (1u << 16);     // P V: M 128, N 64, B MN-major
+    const uint64_t dq = sdesc_sw128(sb + AttnSmem::Q);
+    const bool leader = elect_one();
+    auto issue_s = [&](int j) -> bool {
+      const int b = j % kAttnKV, sbuf = j & 1;
+      if (!__shfl_sync(0xffffffffu, mbar_wait(bar_kvfull + 8 * b, (j / kAttnKV) & 1) ? 1 : 0, 0)) return false;
+      tc_fence_after();
+      if (leader) {
         const uint64_t dk = sdesc_sw128(sb + AttnSmem::K + b * 8192);
 #pragma unroll
         for (int k = 0; k < 4; ++k) tc_mma_f16(tmem + sbuf * 64, dq + 2 * k, dk + 2 * k, IDESC_S, k != 0);
         tc_commit(bar_sfull + 8 * sbuf);
-        return true;
-      };
-      bool ok = issue_s(0) && (nkb < 2 || issue_s(1));
-      for (int j = 0; j < nkb && ok; ++j) {
-        const int pb = j & 1, b = j % kAttnKV;
-        if (!mbar_wait(bar_pfull + 8 * pb, (j >> 1) & 1)) { ok = false; break; }
-        tc_fence_after();
+      }
+      __syncwarp();
+      return true;
+    };
+    bool ok = issue_s(0) && (nkb < 2 || issue_s(1));
+    for (int j = 0; j < nkb && ok; ++j) {
+      const int pb = j & 1, b = j % kAttnKV;
+      if (!__shfl_sync(0xffffffffu, mbar_wait(bar_pfull + 8 * pb, (j >> 1) & 1) ? 1 : 0, 0)) { ok = false; break; }
+      tc_fence_after();
+      if (leader) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t dv = sdesc_sw128_mn(sb + AttnSmem::V + b * 8192 + kk * 2048);
@@ -354,11 +368,12 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
         }
         tc_commit(bar_odone + 8 * pb);
         tc_commit(bar_kvempty + 8 * b);
-        if (j + 2 < nkb) ok = issue_s(j + 2);
       }
-      // single-phase barrier: waiters may arrive any number of phases early
-      if (ok) tc_commit(bar_ofinal);
+      __syncwarp();
+      if (j + 2 < nkb) ok = issue_s(j + 2);
     }
+    // single-phase barrier: waiters may arrive any number of phases early
+    if (ok && leader) tc_commit(bar_ofinal);
   } else if (warp >= 6) {
     // ---------------- global token's query row (query block 0 only) ----------------
     // Warp 6 + g takes blocks g, g + 2, ...: lane l scores keys l and l + 32 with
