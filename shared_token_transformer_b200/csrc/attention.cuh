@@ -63,12 +63,12 @@ constexpr float kAttnRescale = 8.0f;     // lazy rescale threshold (log2 units)
 
 struct AttnSmem {
   static constexpr int Q = 0;                 // 16 KB: 128 rows x 128 B
-  static constexpr int K = 16384;             // 4 x 8 KB: 64 rows x 128 B
-  static constexpr int V = 16384 + 32768;     // 4 x 8 KB
-  static constexpr int KG = 16384 + 65536;    // 64 floats k_g, 64 floats v_g
+  static constexpr int K = 16384;                       // kAttnKV x 8 KB: 64 rows x 128 B
+  static constexpr int V = K + kAttnKV * 8192;          // kAttnKV x 8 KB
+  static constexpr int KG = V + kAttnKV * 8192;         // 64 floats k_g, 64 floats v_g
   static constexpr int GR = KG + 512;         // 2 x 66 floats: partial states of the global query row
   static constexpr int BAR = GR + 1024;       // barriers
-  static constexpr int NBAR = 15;
+  static constexpr int NBAR = 2 * kAttnKV + 7;
   static constexpr int BYTES = BAR + NBAR * 8 + 8;
   static constexpr int LAUNCH_BYTES = BYTES;  // base must be 1024-aligned (checked): two CTAs per SM
 };
@@ -198,9 +198,9 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
   const int ld = 3 * a.d;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sb = smem_u32(smem);
-  const uint32_t bar_kvfull = sb + AttnSmem::BAR;        // 4, count 1 (producer's expect_tx) + TMA bytes
-  const uint32_t bar_kvempty = bar_kvfull + 32;          // 4, count 1 (commit after P V) [+1 global-row warp]
-  const uint32_t bar_sfull = bar_kvempty + 32;           // 2, count 1 (commit after Q K^T)
+  const uint32_t bar_kvfull = sb + AttnSmem::BAR;        // kAttnKV, count 1 (producer's expect_tx) + TMA bytes
+  const uint32_t bar_kvempty = bar_kvfull + 8 * kAttnKV; // kAttnKV, count 1 (commit after P V) [+1 global-row warp]
+  const uint32_t bar_sfull = bar_kvempty + 8 * kAttnKV;  // 2, count 1 (commit after Q K^T)
   const uint32_t bar_pfull = bar_sfull + 16;             // 2, count 4 (softmax warps wrote P into TMEM)
   const uint32_t bar_odone = bar_pfull + 16;             // 2, count 1 (commit after P V)
   const uint32_t bar_ofinal = bar_odone + 16;            // 1, count 1 (commit after the last P V)
