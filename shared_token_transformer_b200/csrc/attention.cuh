@@ -10,14 +10,16 @@
 //
 // bf16 kernel (hd = 64), grid (nqb, heads, T), 256 threads, 2 CTAs per SM:
 //   blocks qb < nqb: 128 window queries, keys in blocks of 64.
-//     warp 4     TMA producer: tile::gather4 loads (four rows per instruction)
-//                through the row map of Q (once) and of K/V blocks into
-//                128-byte-swizzled shared rows; four K/V buffers, completion by
-//                transaction bytes on one mbarrier per buffer;
+//     warp 4     TMA producer of Q (once) and of K/V blocks into 128-byte-
+//                swizzled shared rows: one box of a 3-D map over the grid per
+//                block when a block is whole window rows of one frame, else one
+//                2-D box per run of consecutive rows, else tile::gather4 loads
+//                through the row map (four rows per instruction); four K/V
+//                buffers, completion by transaction bytes on one mbarrier each;
 //     warp 5     MMA issuer (one lane): S = Q K^T (tcgen05 kind::f16, M = 128,
-//                N = 64) into one of two TMEM S buffers, then O += P V with P
+//                N = 64) into one of three TMEM S buffers, then O += P V with P
 //                read from TMEM (A operand) and V from shared memory as an
-//                MN-major operand; S of block j+2 reuses the columns of P of
+//                MN-major operand; S of block j+3 reuses the columns of P of
 //                block j and is issued after P V of block j (tcgen05.mma runs
 //                in issue order);
 //     warps 0-3  softmax, one query row per thread (TMEM lane = row): one tcgen05
@@ -43,7 +45,9 @@ struct AttnArgs {
   const int* rowmap;  // [T * N]: qkv row of slot s of tile t (null: row = t*N + s)
   void* O;            // [T * N, d]
   int N, Nw, d, heads, T;
-  int run;            // > 0: slots come in runs of `run` consecutive rows (tiled boxes); 0: gathered rows
+  int load;           // K/V/Q loads: 0 four-row gathers, 1 runs of `run` rows (2-D boxes), 2 grid boxes
+  int run;            // load 1: slots 1 + k*run ... come in runs of `run` consecutive rows
+  int gw;             // load 2: grid width; shared row u is grid row u / gw, column u % gw
   float scale_log2;   // log2(e) / sqrt(hd)
   float scale;        // 1 / sqrt(hd)
 };
@@ -59,6 +63,7 @@ constexpr int kAttnThreads = 256;        // 4 softmax, TMA producer, MMA issuer,
 constexpr int kAttnBQ = 128;             // queries per CTA
 constexpr int kAttnBK = 64;              // keys per block
 constexpr int kAttnKV = 4;               // K/V buffers
+constexpr int kAttnS = 3;                // S / P buffers in TMEM
 constexpr float kAttnRescale = 8.0f;     // lazy rescale threshold (log2 units)
 
 struct AttnSmem {
@@ -68,7 +73,7 @@ struct AttnSmem {
   static constexpr int KG = V + kAttnKV * 8192;         // 64 floats k_g, 64 floats v_g
   static constexpr int GR = KG + 512;         // 2 x 66 floats: partial states of the global query row
   static constexpr int BAR = GR + 1024;       // barriers
-  static constexpr int NBAR = 2 * kAttnKV + 7;
+  static constexpr int NBAR = 2 * kAttnKV + 2 * kAttnS + 3;
   static constexpr int BYTES = BAR + NBAR * 8 + 8;
   static constexpr int LAUNCH_BYTES = BYTES;  // base must be 1024-aligned (checked): two CTAs per SM
 };
@@ -200,9 +205,9 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
   const uint32_t sb = smem_u32(smem);
   const uint32_t bar_kvfull = sb + AttnSmem::BAR;        // kAttnKV, count 1 (producer's expect_tx) + TMA bytes
   const uint32_t bar_kvempty = bar_kvfull + 8 * kAttnKV; // kAttnKV, count 1 (commit after P V) [+1 global-row warp]
-  const uint32_t bar_sfull = bar_kvempty + 8 * kAttnKV;  // 2, count 1 (commit after Q K^T)
-  const uint32_t bar_pfull = bar_sfull + 16;             // 2, count 4 (softmax warps wrote P into TMEM)
-  const uint32_t bar_odone = bar_pfull + 16;             // 2, count 1 (commit after P V)
+  const uint32_t bar_sfull = bar_kvempty + 8 * kAttnKV;  // kAttnS, count 1 (commit after Q K^T)
+  const uint32_t bar_pfull = bar_sfull + 8 * kAttnS;     // kAttnS, count 4 (softmax warps wrote P into TMEM)
+  const uint32_t bar_odone = bar_pfull + 8 * kAttnS;     // 2, count 1 (commit after P V)
   const uint32_t bar_ofinal = bar_odone + 16;            // 1, count 1 (commit after the last P V)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + AttnSmem::BAR + AttnSmem::NBAR * 8);
   float* sKg = reinterpret_cast<float*>(smem + AttnSmem::KG);
@@ -218,17 +223,17 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
       mbar_init(bar_kvfull + 8 * i, 1);
       mbar_init(bar_kvempty + 8 * i, grow_row ? 2 : 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kAttnS; ++i) {
       mbar_init(bar_sfull + 8 * i, 1);
       mbar_init(bar_pfull + 8 * i, 4);
-      mbar_init(bar_odone + 8 * i, 1);
     }
+    for (int i = 0; i < 2; ++i) mbar_init(bar_odone + 8 * i, 1);
     mbar_init(bar_ofinal, 1);
     fence_barrier_init();
     tma_prefetch_desc(tm);
   }
   if (warp == 5) {
-    tmem_alloc(smem_u32(tmem_slot), 256);    // S0 / P0: cols 0-63, S1 / P1: 64-127, O: 128-191
+    tmem_alloc(smem_u32(tmem_slot), 256);    // S / P buffer k: cols 64k .. 64k + 63 (k < 3), O: 192-255
     tmem_relinquish();
   }
   pdl_wait();
@@ -242,9 +247,45 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tO = tmem + 128;
+  const uint32_t tO = tmem + 64 * kAttnS;
 
-  if (warp == 4 && a.run > 0) {
+  if (warp == 4 && a.load == 2) {
+    // ---------------- TMA producer, one grid box per 64 slots ----------------
+    // A block of 64 window slots is 64 / bx whole window rows of one frame: one
+    // box of the 3-D map (channels, grid column, grid row) starting at the row
+    // of its first slot.  Blocks past the tile's last slot load block 0 again.
+    auto box_at = [&](int slot, int& x, int& y) {
+      const int u = attn_row(a, t, slot < a.N ? slot : 1);
+      x = u % a.gw;
+      y = u / a.gw;
+    };
+    if (lane == 0) {
+      const int xq = h * 64, xk = a.d + h * 64, xv = 2 * a.d + h * 64;
+      int x, y;
+      mbar_expect_tx(bar_kvfull, 2 * 16384);   // Q rows travel with K/V block 0
+      box_at(q0, x, y);
+      tma_load_3d(sb + AttnSmem::Q, tm, bar_kvfull, xq, x, y);
+      box_at(q0 + 64, x, y);
+      tma_load_3d(sb + AttnSmem::Q + 8192, tm, bar_kvfull, xq, x, y);
+      int xn, yn;
+      box_at(1, xn, yn);
+      int armed = 0;
+      for (int j = 0; j < nkb; ++j) {
+        const int b = j % kAttnKV;
+        const int xc = xn, yc = yn;
+        if (j + 1 < nkb) box_at(1 + (j + 1) * kAttnBK, xn, yn);
+        if (j > 0) {
+          if (j >= kAttnKV && !mbar_wait(bar_kvempty + 8 * b, ((j / kAttnKV) - 1) & 1)) break;
+          mbar_expect_tx(bar_kvfull + 8 * b, 16384);
+        }
+        tma_load_3d(sb + AttnSmem::K + b * 8192, tm, bar_kvfull + 8 * b, xk, xc, yc);
+        tma_load_3d(sb + AttnSmem::V + b * 8192, tm, bar_kvfull + 8 * b, xv, xc, yc);
+        armed = j + 1;
+      }
+      // no copy may still be landing when the CTA exits (matters only after a timeout)
+      for (int j = max(0, armed - kAttnKV); j < armed; ++j) mbar_wait(bar_kvfull + 8 * (j % kAttnKV), (j / kAttnKV) & 1);
+    }
+  } else if (warp == 4 && a.load == 1) {
     // ---------------- TMA producer, runs of consecutive rows ----------------
     // Each run of `run` slots is one tiled box (128 bytes x run rows) of the q/k/v
     // columns of head h.  Runs past the tile's last slot (padding of the last key
@@ -334,7 +375,7 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
       for (int j = max(0, armed - kAttnKV); j < armed; ++j) mbar_wait(bar_kvfull + 8 * (j % kAttnKV), (j / kAttnKV) & 1);
   } else if (warp == 5) {
     // ---------------- MMA issuer ----------------
-    // S of block j+2 goes into the TMEM columns that hold P of block j; it is
+    // S of block j+3 goes into the TMEM columns that hold P of block j; it is
     // issued after P V of block j, and tcgen05.mma runs in issue order.  The whole
     // warp waits on the barriers (lane 0's outcome decides for all); one elected
     // lane issues the MMAs and commits.
@@ -343,7 +384,7 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
     const uint64_t dq = sdesc_sw128(sb + AttnSmem::Q);
     const bool leader = elect_one();
     auto issue_s = [&](int j) -> bool {
-      const int b = j % kAttnKV, sbuf = j & 1;
+      const int b = j % kAttnKV, sbuf = j % kAttnS;
       if (!__shfl_sync(0xffffffffu, mbar_wait(bar_kvfull + 8 * b, (j / kAttnKV) & 1) ? 1 : 0, 0)) return false;
       tc_fence_after();
       if (leader) {
@@ -355,10 +396,11 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
       __syncwarp();
       return true;
     };
-    bool ok = issue_s(0) && (nkb < 2 || issue_s(1));
+    bool ok = true;
+    for (int j = 0; j < kAttnS && j < nkb && ok; ++j) ok = issue_s(j);
     for (int j = 0; j < nkb && ok; ++j) {
-      const int pb = j & 1, b = j % kAttnKV;
-      if (!__shfl_sync(0xffffffffu, mbar_wait(bar_pfull + 8 * pb, (j >> 1) & 1) ? 1 : 0, 0)) { ok = false; break; }
+      const int pb = j % kAttnS, b = j % kAttnKV;
+      if (!__shfl_sync(0xffffffffu, mbar_wait(bar_pfull + 8 * pb, (j / kAttnS) & 1) ? 1 : 0, 0)) { ok = false; break; }
       tc_fence_after();
       if (leader) {
 #pragma unroll
@@ -366,11 +408,11 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
           const uint64_t dv = sdesc_sw128_mn(sb + AttnSmem::V + b * 8192 + kk * 2048);
           tc_mma_f16_tmem_a(tO, tmem + pb * 64 + kk * 8, dv, IDESC_O, (j | kk) != 0);
         }
-        tc_commit(bar_odone + 8 * pb);
+        tc_commit(bar_odone + 8 * (j & 1));
         tc_commit(bar_kvempty + 8 * b);
       }
       __syncwarp();
-      if (j + 2 < nkb) ok = issue_s(j + 2);
+      if (j + kAttnS < nkb) ok = issue_s(j + kAttnS);
     }
     // single-phase barrier: waiters may arrive any number of phases early
     if (ok && leader) tc_commit(bar_ofinal);
@@ -479,8 +521,8 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
       gcoef = 1.f;
     }
     for (int j = 0; j < nkb && ok; ++j) {
-      const int sbuf = j & 1;
-      if (!mbar_wait(bar_sfull + 8 * sbuf, (j >> 1) & 1)) { ok = false; break; }
+      const int sbuf = j % kAttnS;
+      if (!mbar_wait(bar_sfull + 8 * sbuf, (j / kAttnS) & 1)) { ok = false; break; }
       tc_fence_after();
       float sv[kAttnBK];
       tmem_ld32(tmem + sbuf * 64 + lane_off, sv);

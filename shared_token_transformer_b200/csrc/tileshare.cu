@@ -168,6 +168,22 @@ static ts_status make_tmap(CUtensorMap* map, const void* base, int rows, int K, 
   return TS_OK;
 }
 
+// 3-D bf16 map over the grid rows of a [F*H*W, cols] matrix: (column, grid x,
+// grid row f*H + y), box of 128 bytes x bx x by, 128-byte swizzle.
+static ts_status make_tmap_grid(CUtensorMap* map, const void* base, int cols, int W, int R, int bx, int by) {
+  EncodeTiledFn enc;
+  TS_TRY(encode_fn(&enc));
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(W), static_cast<cuuint64_t>(R)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 2, static_cast<cuuint64_t>(cols) * 2 * W};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(bx), static_cast<cuuint32_t>(by)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TS_ERR_CUDA, "cuTensorMapEncodeTiled (3-D) failed (%d)", static_cast<int>(r));
+  return TS_OK;
+}
+
 // ============================================================================
 // launches with programmatic dependent launch (PDL)
 //   Kernels launched this way call pdl_wait() before touching activations, so
@@ -623,9 +639,22 @@ static ts_status run_attention(const ts_plan_s* p, const ts_model_desc* m, bool 
   // map over the q/k/v rows: a 128-byte column box, `run` rows high for runs of
   // consecutive rows (the per-tile layout is one run per tile), one row high for
   // four-row gathers
-  a.run = shared ? p->run : 64;
+  // Loads: a block of 64 window slots that is whole window rows of one frame is
+  // one box of a 3-D map over the grid; otherwise runs of consecutive rows are
+  // 2-D boxes (the per-tile layout is one run per tile), else four-row gathers.
+  const int wx = p->win[2], wy = p->win[1];
+  const bool grid_box = wx <= 64 ? (64 % wx == 0 && (wy * wx) % 64 == 0) : wx % 64 == 0;
   CUtensorMap tm;
-  TS_TRY(make_tmap(&tm, qkv, shared ? p->U + p->T : p->T * p->N, 3 * m->d, 2, a.run > 0 ? a.run : 1));
+  if (shared && grid_box) {
+    a.load = 2;
+    a.gw = p->grid[2];
+    const int bx = std::min(wx, 64);
+    TS_TRY(make_tmap_grid(&tm, qkv, 3 * m->d, p->grid[2], p->grid[0] * p->grid[1], bx, 64 / bx));
+  } else {
+    a.run = shared ? p->run : 64;
+    a.load = a.run > 0 ? 1 : 0;
+    TS_TRY(make_tmap(&tm, qkv, shared ? p->U + p->T : p->T * p->N, 3 * m->d, 2, a.run > 0 ? a.run : 1));
+  }
   dim3 grid(nqb, m->heads, p->T);
   launch_pdl(ts::attn_bf16_kernel, grid, dim3(ts::kAttnThreads), ts::AttnSmem::LAUNCH_BYTES, st, tm, a);
   return trace_post(st, "attn_bf16");

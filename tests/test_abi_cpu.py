@@ -48,6 +48,8 @@ GEOMS = [
     ((3, 7, 9), (2, 4, 5), (1, 1, 2)),
     ((1, 20, 9), (1, 8, 3), (1, 3, 1)),
     ((1, 5, 5), (1, 5, 5), (1, 2, 2)),
+    ((1, 9, 40), (1, 3, 16), (1, 2, 12)),
+    ((1, 5, 200), (1, 2, 128), (1, 1, 72)),
 ]
 
 
@@ -71,7 +73,7 @@ def test_host_planner_bit_exact_against_oracle(grid, win, stride):
 
 
 RUNS = {(1, 48, 48): 16, (4, 44, 80): 32, (1, 128, 128): 32, (1, 11, 13): 8, (3, 7, 9): 0, (1, 20, 9): 0,
-        (1, 5, 5): 64}
+        (1, 5, 5): 64, (1, 9, 40): 16, (1, 5, 200): 64}
 
 
 @pytest.mark.parametrize("grid,win,stride", GEOMS)

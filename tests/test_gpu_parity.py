@@ -31,6 +31,13 @@ VOL = W.small_config("vol_bf16", grid=(3, 12, 14), win=(2, 8, 8), stride=(1, 4, 
 SMALL_FP8 = W.small_config("small_fp8", grid=(1, 11, 13), win=(1, 8, 8), stride=(1, 5, 6), d=256, heads=4,
                            mlp=512, dtype="fp8", L=2, k=1)
 VIT14 = W.CONFIGS["vit14_fp32"]
+# attention load paths: SMALL, VOL and the benchmark windows fetch a 64-slot block as one
+# grid box; RUNS16 (48-slot window rows of 16) as 2-D boxes of 16-row runs; WIDE (window
+# rows of 128) as grid boxes one row high; RAGGED (rows of 21) through four-row gathers
+RUNS16 = W.small_config("runs16_bf16", grid=(1, 9, 40), win=(1, 3, 16), stride=(1, 2, 12), d=256, heads=4,
+                        mlp=512, dtype="bf16", L=2, k=1)
+WIDE = W.small_config("wide_bf16", grid=(1, 5, 200), win=(1, 2, 128), stride=(1, 1, 72), d=256, heads=4,
+                      mlp=512, dtype="bf16", L=2, k=1)
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -152,7 +159,7 @@ def test_qkv_norm_rope(cfg, mode):
         assert rel_l2(got[:, sl], want[:, sl]) < tol, part
 
 
-@pytest.mark.parametrize("cfg", [SMALL, RAGGED, VOL, VIT14], ids=lambda c: c.name)
+@pytest.mark.parametrize("cfg", [SMALL, RAGGED, VOL, RUNS16, WIDE, VIT14], ids=lambda c: c.name)
 @pytest.mark.parametrize("mode", [B.TS_ROWS_SHARED, B.TS_ROWS_TILED])
 def test_attention(cfg, mode):
     c = case(cfg)
