@@ -384,9 +384,12 @@ def run_tileshare(args, rank, world, local):
     clocks = sampler.summary(t_wall0, t_wall1)
 
     pk, pk_src = peaks()
-    tensor_peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
-    if cfg.dtype == "fp8":
-        tensor_peak = 2.0 * tensor_peak          # nominal e4m3 : bf16 dense ratio
+    bf16_peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+
+    def tensor_peak_of(name):
+        # e4m3 GEMMs against the bf16 peak x the nominal e4m3 : bf16 dense ratio;
+        # attention computes in bf16 in every configuration
+        return 2.0 * bf16_peak if cfg.dtype == "fp8" and not name.startswith("attention") else bf16_peak
     total_ms = sum(v["ms"] for v in tr.values()) or 1.0
     kernels = {}
     for name, v in tr.items():
@@ -396,7 +399,7 @@ def run_tileshare(args, rank, world, local):
         tensor = v["flops"] > 0 and name.startswith(("gemm", "attention", "linear"))
         if tensor:
             ach = v["flops"] / (v["ms"] / 1e3) / 1e12
-            frac = ach / tensor_peak
+            frac = ach / tensor_peak_of(name)
             unit = "TFLOP/s"
         else:
             ach = v["bytes"] / (v["ms"] / 1e3) / 1e9
@@ -417,9 +420,10 @@ def run_tileshare(args, rank, world, local):
         if ent and ent.get("kernel_source_sha") == kernel_source_sha():
             traffic = ent.get("traffic_bytes_per_launch")
     roofline = {"bound": "tensor" if kd["unit"] == "TFLOP/s" else "hbm", "kernel": dom, "achieved": kd["achieved"],
-                "peak": round(tensor_peak if kd["unit"] == "TFLOP/s" else pk["hbm_gbs"], 1), "unit": kd["unit"],
+                "peak": round(tensor_peak_of(dom) if kd["unit"] == "TFLOP/s" else pk["hbm_gbs"], 1), "unit": kd["unit"],
                 "frac": kd["frac"], "traffic": traffic,
-                "peak_source": (f"{pk_src} " + ("bf16_tflops_sustained" + (" x2 (e4m3:bf16 nominal)" if cfg.dtype == "fp8" else "")
+                "peak_source": (f"{pk_src} " + ("bf16_tflops_sustained" + (" x2 (e4m3:bf16 nominal)"
+                                                                           if tensor_peak_of(dom) > bf16_peak else "")
                                                 if kd["unit"] == "TFLOP/s" else "hbm_gbs"))}
 
     ft = flops_layer(T * N, T, N, d, f)

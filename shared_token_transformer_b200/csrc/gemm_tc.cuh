@@ -12,7 +12,7 @@
 // scale of W.
 //
 // Kernel design: persistent, warp-specialised, 320 threads, CTAs walk the
-// 128 x BN output tiles in a static round-robin order.
+// 128 x BN output tiles in a static round-robin order over banded tiles.
 //   warp 8   TMA producer: A and W tiles of 128-byte K slices (64 bf16 / 128 e4m3)
 //            into a STAGES-deep ring of 128-byte-swizzled shared buffers
 //            (no multicast);
@@ -148,6 +148,19 @@ __device__ __forceinline__ void gemm_epilogue64(float* v, int row, int col, floa
   for (int i = 0; i < 64; i += 8) *reinterpret_cast<uint4*>(dst + i) = f32_to_bf16x8(v + i);
 }
 
+// Output tile order: bands of kGemmBand row tiles, each band walked across all
+// column tiles with the row tile fastest.  The CTAs in flight then share one or
+// two bands of A and the whole of W, which stay in L2 even when A does not.
+constexpr int kGemmBand = 16;
+__device__ __forceinline__ void gemm_tile_origin(int tile, int mt, int nt, int bn, int& m0, int& n0) {
+  const int band = tile / (kGemmBand * nt);
+  const int first = band * kGemmBand;
+  const int rows = min(kGemmBand, mt - first);
+  const int r = tile - first * nt;
+  m0 = (first + r % rows) * 128;
+  n0 = (r / rows) * bn;
+}
+
 template <int BN, int STAGES, int EPI, bool FP8, int R0, int R1, int R2>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -203,7 +216,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-        const int m0 = (tile % mt) * 128, n0 = (tile / mt) * BN;
+        int m0, n0;
+        gemm_tile_origin(tile, mt, args.N / BN, BN, m0, n0);
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const uint32_t s = it % STAGES;
           if (it >= STAGES && !mbar_wait(bar_empty + 8 * s, ((it / STAGES) - 1) & 1)) { ok = false; break; }
@@ -250,7 +264,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t j = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++j) {
       const uint32_t acc = j & 1, use = j >> 1;
-      const int m0 = (tile % mt) * 128, n0 = (tile / mt) * BN;
+      int m0, n0;
+      gemm_tile_origin(tile, mt, args.N / BN, BN, m0, n0);
       const int row = m0 + quarter * 32 + lane;
       if (!mbar_wait(bar_tfull + 8 * acc, use & 1)) break;
       tc_fence_after();
