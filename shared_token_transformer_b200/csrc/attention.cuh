@@ -194,6 +194,152 @@ __device__ __forceinline__ void tc_mma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tm
       : "memory");
 }
 
+// What the three load variants of the producer warp share.
+struct AttnLoad {
+  const CUtensorMap* tm;
+  uint32_t sb, bar_kvfull, bar_kvempty;
+  int q0, nkb, t, h, lane;
+};
+
+__device__ __forceinline__ void attn_load_grid(const AttnArgs& a, const AttnLoad& c) {
+  const CUtensorMap* tm = c.tm;
+  const uint32_t sb = c.sb, bar_kvfull = c.bar_kvfull, bar_kvempty = c.bar_kvempty;
+  const int q0 = c.q0, nkb = c.nkb, t = c.t, h = c.h, lane = c.lane;
+  // ---------------- TMA producer, one grid box per 64 slots ----------------
+  // A block of 64 window slots is 64 / bx whole window rows of one frame: one
+  // box of the 3-D map (channels, grid column, grid row) starting at the row
+  // of its first slot.  Blocks past the tile's last slot load block 0 again.
+  auto box_at = [&](int slot, int& x, int& y) {
+    const int u = attn_row(a, t, slot < a.N ? slot : 1);
+    x = u % a.gw;
+    y = u / a.gw;
+  };
+  if (lane == 0) {
+    const int xq = h * 64, xk = a.d + h * 64, xv = 2 * a.d + h * 64;
+    int x, y;
+    mbar_expect_tx(bar_kvfull, 2 * 16384);   // Q rows travel with K/V block 0
+    box_at(q0, x, y);
+    tma_load_3d(sb + AttnSmem::Q, tm, bar_kvfull, xq, x, y);
+    box_at(q0 + 64, x, y);
+    tma_load_3d(sb + AttnSmem::Q + 8192, tm, bar_kvfull, xq, x, y);
+    int xn, yn;
+    box_at(1, xn, yn);
+    int armed = 0;
+    for (int j = 0; j < nkb; ++j) {
+      const int b = j % kAttnKV;
+      const int xc = xn, yc = yn;
+      if (j + 1 < nkb) box_at(1 + (j + 1) * kAttnBK, xn, yn);
+      if (j > 0) {
+        if (j >= kAttnKV && !mbar_wait(bar_kvempty + 8 * b, ((j / kAttnKV) - 1) & 1)) break;
+        mbar_expect_tx(bar_kvfull + 8 * b, 16384);
+      }
+      tma_load_3d(sb + AttnSmem::K + b * 8192, tm, bar_kvfull + 8 * b, xk, xc, yc);
+      tma_load_3d(sb + AttnSmem::V + b * 8192, tm, bar_kvfull + 8 * b, xv, xc, yc);
+      armed = j + 1;
+    }
+    // no copy may still be landing when the CTA exits (matters only after a timeout)
+    for (int j = max(0, armed - kAttnKV); j < armed; ++j) mbar_wait(bar_kvfull + 8 * (j % kAttnKV), (j / kAttnKV) & 1);
+  }
+}
+
+__device__ __forceinline__ void attn_load_runs(const AttnArgs& a, const AttnLoad& c) {
+  const CUtensorMap* tm = c.tm;
+  const uint32_t sb = c.sb, bar_kvfull = c.bar_kvfull, bar_kvempty = c.bar_kvempty;
+  const int q0 = c.q0, nkb = c.nkb, t = c.t, h = c.h, lane = c.lane;
+  // ---------------- TMA producer, runs of consecutive rows ----------------
+  // Each run of `run` slots is one tiled box (128 bytes x run rows) of the q/k/v
+  // columns of head h.  Runs past the tile's last slot (padding of the last key
+  // or query block) load the first run again: their scores are masked and their
+  // outputs are not stored.  Lane i looks up the row of run i one block ahead;
+  // lane 0 issues the copies.
+  const int L = a.run, nrun = kAttnBK / L;
+  auto run_row = [&](int slot) { return attn_row(a, t, slot < a.N ? slot : 1); };
+  const int xq = h * 64, xk = a.d + h * 64, xv = 2 * a.d + h * 64;
+  {
+    const int rq = lane < kAttnBQ / L ? run_row(q0 + lane * L) : 0;
+    if (lane == 0) mbar_expect_tx(bar_kvfull, 2 * 16384);   // Q rows travel with K/V block 0
+    for (int i = 0; i < kAttnBQ / L; ++i) {
+      const int r = __shfl_sync(0xffffffffu, rq, i);
+      if (lane == 0) tma_load_2d(sb + AttnSmem::Q + i * L * 128, tm, bar_kvfull, xq, r);
+    }
+  }
+  int rnext = lane < nrun ? run_row(1 + lane * L) : 0;
+  int armed = 0;
+  for (int j = 0; j < nkb; ++j) {
+    const int b = j % kAttnKV;
+    const int rcur = rnext;
+    if (j + 1 < nkb && lane < nrun) rnext = run_row(1 + (j + 1) * kAttnBK + lane * L);
+    if (j > 0) {
+      int ok = 1;
+      if (lane == 0 && j >= kAttnKV) ok = mbar_wait(bar_kvempty + 8 * b, ((j / kAttnKV) - 1) & 1);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      if (lane == 0) mbar_expect_tx(bar_kvfull + 8 * b, 16384);
+    }
+    for (int i = 0; i < nrun; ++i) {
+      const int r = __shfl_sync(0xffffffffu, rcur, i);
+      if (lane == 0) {
+        tma_load_2d(sb + AttnSmem::K + b * 8192 + i * L * 128, tm, bar_kvfull + 8 * b, xk, r);
+        tma_load_2d(sb + AttnSmem::V + b * 8192 + i * L * 128, tm, bar_kvfull + 8 * b, xv, r);
+      }
+    }
+    armed = j + 1;
+  }
+  // no copy may still be landing when the CTA exits (matters only after a timeout)
+  if (lane == 0)
+    for (int j = max(0, armed - kAttnKV); j < armed; ++j) mbar_wait(bar_kvfull + 8 * (j % kAttnKV), (j / kAttnKV) & 1);
+}
+
+__device__ __forceinline__ void attn_load_gather(const AttnArgs& a, const AttnLoad& c) {
+  const CUtensorMap* tm = c.tm;
+  const uint32_t sb = c.sb, bar_kvfull = c.bar_kvfull, bar_kvempty = c.bar_kvempty;
+  const int q0 = c.q0, nkb = c.nkb, t = c.t, h = c.h, lane = c.lane;
+  // ---------------- TMA producer, gathered rows ----------------
+  // Rows are gathered four at a time (tile::gather4) from the q/k/v columns of
+  // head h.  Slots past the tile's last one (padding of the last key or query
+  // block) repeat the last slot's row, so every coordinate is in range; their
+  // scores are masked and their outputs are not stored.
+  auto row_of = [&](int slot) { return attn_row(a, t, min(slot, a.N - 1)); };
+  const int xq = h * 64, xk = a.d + h * 64, xv = 2 * a.d + h * 64;
+  int vq[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) vq[k] = row_of(q0 + 32 * k + lane);
+  int v0 = row_of(1 + lane), v1 = row_of(33 + lane);
+  if (lane == 0) mbar_expect_tx(bar_kvfull, 2 * 16384);   // Q rows travel with K/V block 0
+#pragma unroll
+  for (int g = 0; g < 32; ++g) {
+    int r[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) r[i] = __shfl_sync(0xffffffffu, vq[g >> 3], (4 * g + i) & 31);
+    if (lane == 0) tma_gather4(sb + AttnSmem::Q + g * 512, tm, bar_kvfull, xq, r[0], r[1], r[2], r[3]);
+  }
+  int armed = 0;
+  for (int j = 0; j < nkb; ++j) {
+    const int b = j % kAttnKV;
+    if (j > 0) {
+      v0 = row_of(1 + j * kAttnBK + lane);
+      v1 = row_of(1 + j * kAttnBK + 32 + lane);
+      int ok = 1;
+      if (lane == 0 && j >= kAttnKV) ok = mbar_wait(bar_kvempty + 8 * b, ((j / kAttnKV) - 1) & 1);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      if (lane == 0) mbar_expect_tx(bar_kvfull + 8 * b, 16384);
+    }
+#pragma unroll
+    for (int g = 0; g < 16; ++g) {
+      int r[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) r[i] = __shfl_sync(0xffffffffu, g < 8 ? v0 : v1, (4 * g + i) & 31);
+      if (lane == 0) {
+        tma_gather4(sb + AttnSmem::K + b * 8192 + g * 512, tm, bar_kvfull + 8 * b, xk, r[0], r[1], r[2], r[3]);
+        tma_gather4(sb + AttnSmem::V + b * 8192 + g * 512, tm, bar_kvfull + 8 * b, xv, r[0], r[1], r[2], r[3]);
+      }
+    }
+    armed = j + 1;
+  }
+  // no copy may still be landing when the CTA exits (matters only after a timeout)
+  if (lane == 0)
+    for (int j = max(0, armed - kAttnKV); j < armed; ++j) mbar_wait(bar_kvfull + 8 * (j % kAttnKV), (j / kAttnKV) & 1);
+}
+
 // ---------------------------------------------------------------------------
 // window-query block (tcgen05)
 // ---------------------------------------------------------------------------
@@ -218,396 +364,289 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
   // (slot 0) in warps 6 and 7, which then co-own the K/V buffers they read.
   const bool grow_row = qb == 0;
 
-  if (warp == 4 && lane == 0) {
-    for (int i = 0; i < kAttnKV; ++i) {
-      mbar_init(bar_kvfull + 8 * i, 1);
-      mbar_init(bar_kvempty + 8 * i, grow_row ? 2 : 1);
+  uint32_t tmem = 0;
+  if (warp == 4) {
+    // ---------------- TMA producer ----------------
+    // Its copies start as soon as the barriers exist; the other warps learn of
+    // the initialisation through a named barrier that this warp only arrives at.
+    if (warp == 4 && lane == 0) {
+      for (int i = 0; i < kAttnKV; ++i) {
+        mbar_init(bar_kvfull + 8 * i, 1);
+        mbar_init(bar_kvempty + 8 * i, grow_row ? 2 : 1);
+      }
+      for (int i = 0; i < kAttnS; ++i) {
+        mbar_init(bar_sfull + 8 * i, 1);
+        mbar_init(bar_pfull + 8 * i, 4);
+      }
+      for (int i = 0; i < 2; ++i) mbar_init(bar_odone + 8 * i, 1);
+      mbar_init(bar_ofinal, 1);
+      fence_barrier_init();
+      tma_prefetch_desc(tm);
     }
-    for (int i = 0; i < kAttnS; ++i) {
-      mbar_init(bar_sfull + 8 * i, 1);
-      mbar_init(bar_pfull + 8 * i, 4);
+    __syncwarp();
+    asm volatile("bar.arrive 2, %0;" ::"n"(kAttnThreads) : "memory");
+    pdl_wait();
+    pdl_trigger();
+    const AttnLoad c{tm, sb, bar_kvfull, bar_kvempty, q0, nkb, t, h, lane};
+    if (a.load == 2)
+      attn_load_grid(a, c);
+    else if (a.load == 1)
+      attn_load_runs(a, c);
+    else
+      attn_load_gather(a, c);
+  } else {
+    if (warp == 5) {
+      tmem_alloc(smem_u32(tmem_slot), 256);    // S / P buffer k: cols 64k .. 64k + 63 (k < 3), O: 192-255
+      tmem_relinquish();
     }
-    for (int i = 0; i < 2; ++i) mbar_init(bar_odone + 8 * i, 1);
-    mbar_init(bar_ofinal, 1);
-    fence_barrier_init();
-    tma_prefetch_desc(tm);
-  }
-  if (warp == 5) {
-    tmem_alloc(smem_u32(tmem_slot), 256);    // S / P buffer k: cols 64k .. 64k + 63 (k < 3), O: 192-255
-    tmem_relinquish();
-  }
-  pdl_wait();
-  pdl_trigger();
-  if (tid < 64) {
-    const size_t grow = static_cast<size_t>(attn_row(a, t, 0)) * ld + h * 64 + tid;
-    sKg[tid] = __bfloat162float(qkv[grow + a.d]);
-    sVg[tid] = __bfloat162float(qkv[grow + 2 * a.d]);
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t tO = tmem + 64 * kAttnS;
-
-  if (warp == 4 && a.load == 2) {
-    // ---------------- TMA producer, one grid box per 64 slots ----------------
-    // A block of 64 window slots is 64 / bx whole window rows of one frame: one
-    // box of the 3-D map (channels, grid column, grid row) starting at the row
-    // of its first slot.  Blocks past the tile's last slot load block 0 again.
-    auto box_at = [&](int slot, int& x, int& y) {
-      const int u = attn_row(a, t, slot < a.N ? slot : 1);
-      x = u % a.gw;
-      y = u / a.gw;
-    };
-    if (lane == 0) {
-      const int xq = h * 64, xk = a.d + h * 64, xv = 2 * a.d + h * 64;
-      int x, y;
-      mbar_expect_tx(bar_kvfull, 2 * 16384);   // Q rows travel with K/V block 0
-      box_at(q0, x, y);
-      tma_load_3d(sb + AttnSmem::Q, tm, bar_kvfull, xq, x, y);
-      box_at(q0 + 64, x, y);
-      tma_load_3d(sb + AttnSmem::Q + 8192, tm, bar_kvfull, xq, x, y);
-      int xn, yn;
-      box_at(1, xn, yn);
-      int armed = 0;
-      for (int j = 0; j < nkb; ++j) {
-        const int b = j % kAttnKV;
-        const int xc = xn, yc = yn;
-        if (j + 1 < nkb) box_at(1 + (j + 1) * kAttnBK, xn, yn);
-        if (j > 0) {
-          if (j >= kAttnKV && !mbar_wait(bar_kvempty + 8 * b, ((j / kAttnKV) - 1) & 1)) break;
-          mbar_expect_tx(bar_kvfull + 8 * b, 16384);
+    pdl_wait();
+    pdl_trigger();
+    if (tid < 64) {
+      const size_t grow = static_cast<size_t>(attn_row(a, t, 0)) * ld + h * 64 + tid;
+      sKg[tid] = __bfloat162float(qkv[grow + a.d]);
+      sVg[tid] = __bfloat162float(qkv[grow + 2 * a.d]);
+    }
+    tc_fence_before();
+    asm volatile("bar.sync 2, %0;" ::"n"(kAttnThreads) : "memory");
+    tc_fence_after();
+    tmem = *tmem_slot;
+    const uint32_t tO = tmem + 64 * kAttnS;
+    if (warp == 5) {
+      // ---------------- MMA issuer ----------------
+      // S of block j+3 goes into the TMEM columns that hold P of block j; it is
+      // issued after P V of block j, and tcgen05.mma runs in issue order.  The whole
+      // warp waits on the barriers (lane 0's outcome decides for all); one elected
+      // lane issues the MMAs and commits.
+      constexpr uint32_t IDESC_S = idesc_make(1u, kAttnBK);             // Q K^T: M 128, N 64
+      constexpr uint32_t IDESC_O = idesc_make(1u, 64) | (1u << 16);     // P V: M 128, N 64, B MN-major
+      const uint64_t dq = sdesc_sw128(sb + AttnSmem::Q);
+      const bool leader = elect_one();
+      auto issue_s = [&](int j) -> bool {
+        const int b = j % kAttnKV, sbuf = j % kAttnS;
+        if (!__shfl_sync(0xffffffffu, mbar_wait(bar_kvfull + 8 * b, (j / kAttnKV) & 1) ? 1 : 0, 0)) return false;
+        tc_fence_after();
+        if (leader) {
+          const uint64_t dk = sdesc_sw128(sb + AttnSmem::K + b * 8192);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) tc_mma_f16(tmem + sbuf * 64, dq + 2 * k, dk + 2 * k, IDESC_S, k != 0);
+          tc_commit(bar_sfull + 8 * sbuf);
         }
-        tma_load_3d(sb + AttnSmem::K + b * 8192, tm, bar_kvfull + 8 * b, xk, xc, yc);
-        tma_load_3d(sb + AttnSmem::V + b * 8192, tm, bar_kvfull + 8 * b, xv, xc, yc);
-        armed = j + 1;
+        __syncwarp();
+        return true;
+      };
+      bool ok = true;
+      for (int j = 0; j < kAttnS && j < nkb && ok; ++j) ok = issue_s(j);
+      for (int j = 0; j < nkb && ok; ++j) {
+        const int pb = j % kAttnS, b = j % kAttnKV;
+        if (!__shfl_sync(0xffffffffu, mbar_wait(bar_pfull + 8 * pb, (j / kAttnS) & 1) ? 1 : 0, 0)) { ok = false; break; }
+        tc_fence_after();
+        if (leader) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t dv = sdesc_sw128_mn(sb + AttnSmem::V + b * 8192 + kk * 2048);
+            tc_mma_f16_tmem_a(tO, tmem + pb * 64 + kk * 8, dv, IDESC_O, (j | kk) != 0);
+          }
+          tc_commit(bar_odone + 8 * (j & 1));
+          tc_commit(bar_kvempty + 8 * b);
+        }
+        __syncwarp();
+        if (j + kAttnS < nkb) ok = issue_s(j + kAttnS);
       }
-      // no copy may still be landing when the CTA exits (matters only after a timeout)
-      for (int j = max(0, armed - kAttnKV); j < armed; ++j) mbar_wait(bar_kvfull + 8 * (j % kAttnKV), (j / kAttnKV) & 1);
-    }
-  } else if (warp == 4 && a.load == 1) {
-    // ---------------- TMA producer, runs of consecutive rows ----------------
-    // Each run of `run` slots is one tiled box (128 bytes x run rows) of the q/k/v
-    // columns of head h.  Runs past the tile's last slot (padding of the last key
-    // or query block) load the first run again: their scores are masked and their
-    // outputs are not stored.  Lane i looks up the row of run i one block ahead;
-    // lane 0 issues the copies.
-    const int L = a.run, nrun = kAttnBK / L;
-    auto run_row = [&](int slot) { return attn_row(a, t, slot < a.N ? slot : 1); };
-    const int xq = h * 64, xk = a.d + h * 64, xv = 2 * a.d + h * 64;
-    {
-      const int rq = lane < kAttnBQ / L ? run_row(q0 + lane * L) : 0;
-      if (lane == 0) mbar_expect_tx(bar_kvfull, 2 * 16384);   // Q rows travel with K/V block 0
-      for (int i = 0; i < kAttnBQ / L; ++i) {
-        const int r = __shfl_sync(0xffffffffu, rq, i);
-        if (lane == 0) tma_load_2d(sb + AttnSmem::Q + i * L * 128, tm, bar_kvfull, xq, r);
-      }
-    }
-    int rnext = lane < nrun ? run_row(1 + lane * L) : 0;
-    int armed = 0;
-    for (int j = 0; j < nkb; ++j) {
-      const int b = j % kAttnKV;
-      const int rcur = rnext;
-      if (j + 1 < nkb && lane < nrun) rnext = run_row(1 + (j + 1) * kAttnBK + lane * L);
-      if (j > 0) {
-        int ok = 1;
-        if (lane == 0 && j >= kAttnKV) ok = mbar_wait(bar_kvempty + 8 * b, ((j / kAttnKV) - 1) & 1);
-        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-        if (lane == 0) mbar_expect_tx(bar_kvfull + 8 * b, 16384);
-      }
-      for (int i = 0; i < nrun; ++i) {
-        const int r = __shfl_sync(0xffffffffu, rcur, i);
+      // single-phase barrier: waiters may arrive any number of phases early
+      if (ok && leader) tc_commit(bar_ofinal);
+    } else if (warp >= 6) {
+      // ---------------- global token's query row (query block 0 only) ----------------
+      // Warp 6 + g takes blocks g, g + 2, ...: lane l scores keys l and l + 32 with
+      // the full query in registers, then accumulates channels 2l, 2l + 1 of P V.
+      // The two warps' online-softmax states are merged at the end.
+      if (grow_row) {
+        const int g = warp - 6;
+        float qf[64];
+        {
+          const uint4* qr = reinterpret_cast<const uint4*>(qkv + static_cast<size_t>(attn_row(a, t, 0)) * ld + h * 64);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) bf16x8_to_f32(qr[c], qf + 8 * c);
+        }
+        float gm = -INFINITY, gl = 0.f, ga0 = 0.f, ga1 = 0.f;
+        if (g == 0) {   // the global key itself
+          float sg = 0.f;
+#pragma unroll
+          for (int c = 0; c < 64; ++c) sg = fmaf(qf[c], sKg[c], sg);
+          gm = sg * a.scale_log2;
+          gl = lane == 0 ? 1.f : 0.f;
+          ga0 = sVg[2 * lane];
+          ga1 = sVg[2 * lane + 1];
+        }
+        for (int j = g; j < nkb; j += 2) {
+          const int b = j % kAttnKV;
+          if (!mbar_wait(bar_kvfull + 8 * b, (j / kAttnKV) & 1)) break;
+          const uint8_t* kbuf = smem + AttnSmem::K + b * 8192;
+          const uint8_t* vbuf = smem + AttnSmem::V + b * 8192;
+          float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            float f0[8], f1[8];
+            bf16x8_to_f32(*reinterpret_cast<const uint4*>(kbuf + swz(lane, c)), f0);
+            bf16x8_to_f32(*reinterpret_cast<const uint4*>(kbuf + swz(lane + 32, c)), f1);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              s0 = fmaf(qf[8 * c + e], f0[e], s0);
+              s1 = fmaf(qf[8 * c + e], f1[e], s1);
+            }
+          }
+          const int nvalid = min(kAttnBK, a.Nw - j * kAttnBK);
+          const float x0 = lane < nvalid ? s0 * a.scale_log2 : -INFINITY;
+          const float x1 = lane + 32 < nvalid ? s1 * a.scale_log2 : -INFINITY;
+          const float mnew = fmaxf(gm, warp_max(fmaxf(x0, x1)));
+          const float al = ex2_approx(gm - mnew);
+          const float p0 = ex2_approx(x0 - mnew), p1 = ex2_approx(x1 - mnew);
+          gl = fmaf(gl, al, p0 + p1);
+          ga0 *= al;
+          ga1 *= al;
+#pragma unroll 8
+          for (int k = 0; k < kAttnBK; ++k) {
+            const float pk = __shfl_sync(0xffffffffu, k < 32 ? p0 : p1, k & 31);
+            const uint32_t off = swz(k, lane >> 2) + (lane & 3) * 4;
+            const float2 vv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vbuf + off));
+            ga0 = fmaf(pk, vv.x, ga0);
+            ga1 = fmaf(pk, vv.y, ga1);
+          }
+          gm = mnew;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_kvempty + 8 * b);
+        }
+        gl = warp_sum(gl);
+        float* gbuf = reinterpret_cast<float*>(smem + AttnSmem::GR);
         if (lane == 0) {
-          tma_load_2d(sb + AttnSmem::K + b * 8192 + i * L * 128, tm, bar_kvfull + 8 * b, xk, r);
-          tma_load_2d(sb + AttnSmem::V + b * 8192 + i * L * 128, tm, bar_kvfull + 8 * b, xv, r);
+          gbuf[g * 66] = gm;
+          gbuf[g * 66 + 1] = gl;
+        }
+        gbuf[g * 66 + 2 + 2 * lane] = ga0;
+        gbuf[g * 66 + 3 + 2 * lane] = ga1;
+        asm volatile("bar.sync 1, 64;" ::: "memory");
+        if (g == 0) {
+          const float M = fmaxf(gbuf[0], gbuf[66]);
+          float L = 0.f, o0 = 0.f, o1 = 0.f;
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            const float f = gbuf[w * 66] == -INFINITY ? 0.f : ex2_approx(gbuf[w * 66] - M);
+            L += f * gbuf[w * 66 + 1];
+            o0 += f * gbuf[w * 66 + 2 + 2 * lane];
+            o1 += f * gbuf[w * 66 + 3 + 2 * lane];
+          }
+          bf16* O = reinterpret_cast<bf16*>(a.O) + static_cast<size_t>(t) * a.N * a.d + h * 64 + 2 * lane;
+          *reinterpret_cast<__nv_bfloat162*>(O) = __floats2bfloat162_rn(o0 / L, o1 / L);
         }
       }
-      armed = j + 1;
-    }
-    // no copy may still be landing when the CTA exits (matters only after a timeout)
-    if (lane == 0)
-      for (int j = max(0, armed - kAttnKV); j < armed; ++j) mbar_wait(bar_kvfull + 8 * (j % kAttnKV), (j / kAttnKV) & 1);
-  } else if (warp == 4) {
-    // ---------------- TMA producer, gathered rows ----------------
-    // Rows are gathered four at a time (tile::gather4) from the q/k/v columns of
-    // head h.  Slots past the tile's last one (padding of the last key or query
-    // block) repeat the last slot's row, so every coordinate is in range; their
-    // scores are masked and their outputs are not stored.
-    auto row_of = [&](int slot) { return attn_row(a, t, min(slot, a.N - 1)); };
-    const int xq = h * 64, xk = a.d + h * 64, xv = 2 * a.d + h * 64;
-    int vq[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) vq[k] = row_of(q0 + 32 * k + lane);
-    int v0 = row_of(1 + lane), v1 = row_of(33 + lane);
-    if (lane == 0) mbar_expect_tx(bar_kvfull, 2 * 16384);   // Q rows travel with K/V block 0
-#pragma unroll
-    for (int g = 0; g < 32; ++g) {
-      int r[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) r[i] = __shfl_sync(0xffffffffu, vq[g >> 3], (4 * g + i) & 31);
-      if (lane == 0) tma_gather4(sb + AttnSmem::Q + g * 512, tm, bar_kvfull, xq, r[0], r[1], r[2], r[3]);
-    }
-    int armed = 0;
-    for (int j = 0; j < nkb; ++j) {
-      const int b = j % kAttnKV;
-      if (j > 0) {
-        v0 = row_of(1 + j * kAttnBK + lane);
-        v1 = row_of(1 + j * kAttnBK + 32 + lane);
-        int ok = 1;
-        if (lane == 0 && j >= kAttnKV) ok = mbar_wait(bar_kvempty + 8 * b, ((j / kAttnKV) - 1) & 1);
-        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-        if (lane == 0) mbar_expect_tx(bar_kvfull + 8 * b, 16384);
-      }
-#pragma unroll
-      for (int g = 0; g < 16; ++g) {
-        int r[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) r[i] = __shfl_sync(0xffffffffu, g < 8 ? v0 : v1, (4 * g + i) & 31);
-        if (lane == 0) {
-          tma_gather4(sb + AttnSmem::K + b * 8192 + g * 512, tm, bar_kvfull + 8 * b, xk, r[0], r[1], r[2], r[3]);
-          tma_gather4(sb + AttnSmem::V + b * 8192 + g * 512, tm, bar_kvfull + 8 * b, xv, r[0], r[1], r[2], r[3]);
-        }
-      }
-      armed = j + 1;
-    }
-    // no copy may still be landing when the CTA exits (matters only after a timeout)
-    if (lane == 0)
-      for (int j = max(0, armed - kAttnKV); j < armed; ++j) mbar_wait(bar_kvfull + 8 * (j % kAttnKV), (j / kAttnKV) & 1);
-  } else if (warp == 5) {
-    // ---------------- MMA issuer ----------------
-    // S of block j+3 goes into the TMEM columns that hold P of block j; it is
-    // issued after P V of block j, and tcgen05.mma runs in issue order.  The whole
-    // warp waits on the barriers (lane 0's outcome decides for all); one elected
-    // lane issues the MMAs and commits.
-    constexpr uint32_t IDESC_S = idesc_make(1u, kAttnBK);             // Q K^T: M 128, N 64
-    constexpr uint32_t IDESC_O = idesc_make(1u, 64) | (1u << 16);     // P V: M 128, N 64, B MN-major
-    const uint64_t dq = sdesc_sw128(sb + AttnSmem::Q);
-    const bool leader = elect_one();
-    auto issue_s = [&](int j) -> bool {
-      const int b = j % kAttnKV, sbuf = j % kAttnS;
-      if (!__shfl_sync(0xffffffffu, mbar_wait(bar_kvfull + 8 * b, (j / kAttnKV) & 1) ? 1 : 0, 0)) return false;
-      tc_fence_after();
-      if (leader) {
-        const uint64_t dk = sdesc_sw128(sb + AttnSmem::K + b * 8192);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) tc_mma_f16(tmem + sbuf * 64, dq + 2 * k, dk + 2 * k, IDESC_S, k != 0);
-        tc_commit(bar_sfull + 8 * sbuf);
-      }
-      __syncwarp();
-      return true;
-    };
-    bool ok = true;
-    for (int j = 0; j < kAttnS && j < nkb && ok; ++j) ok = issue_s(j);
-    for (int j = 0; j < nkb && ok; ++j) {
-      const int pb = j % kAttnS, b = j % kAttnKV;
-      if (!__shfl_sync(0xffffffffu, mbar_wait(bar_pfull + 8 * pb, (j / kAttnS) & 1) ? 1 : 0, 0)) { ok = false; break; }
-      tc_fence_after();
-      if (leader) {
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t dv = sdesc_sw128_mn(sb + AttnSmem::V + b * 8192 + kk * 2048);
-          tc_mma_f16_tmem_a(tO, tmem + pb * 64 + kk * 8, dv, IDESC_O, (j | kk) != 0);
-        }
-        tc_commit(bar_odone + 8 * (j & 1));
-        tc_commit(bar_kvempty + 8 * b);
-      }
-      __syncwarp();
-      if (j + kAttnS < nkb) ok = issue_s(j + kAttnS);
-    }
-    // single-phase barrier: waiters may arrive any number of phases early
-    if (ok && leader) tc_commit(bar_ofinal);
-  } else if (warp >= 6) {
-    // ---------------- global token's query row (query block 0 only) ----------------
-    // Warp 6 + g takes blocks g, g + 2, ...: lane l scores keys l and l + 32 with
-    // the full query in registers, then accumulates channels 2l, 2l + 1 of P V.
-    // The two warps' online-softmax states are merged at the end.
-    if (grow_row) {
-      const int g = warp - 6;
-      float qf[64];
-      {
-        const uint4* qr = reinterpret_cast<const uint4*>(qkv + static_cast<size_t>(attn_row(a, t, 0)) * ld + h * 64);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) bf16x8_to_f32(qr[c], qf + 8 * c);
-      }
-      float gm = -INFINITY, gl = 0.f, ga0 = 0.f, ga1 = 0.f;
-      if (g == 0) {   // the global key itself
+    } else if (warp < 4) {
+      // ---------------- softmax: one query row per thread ----------------
+      const int row = tid;                     // 0..127, TMEM lane = row
+      const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+      bool ok = mbar_wait(bar_kvfull, 0);      // Q rows are in shared memory
+      float m = -INFINITY, l = 0.f, gcoef = 0.f;
+      if (ok) {
+        // score of the global key seeds the running maximum and sum
         float sg = 0.f;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) sg = fmaf(qf[c], sKg[c], sg);
-        gm = sg * a.scale_log2;
-        gl = lane == 0 ? 1.f : 0.f;
-        ga0 = sVg[2 * lane];
-        ga1 = sVg[2 * lane + 1];
-      }
-      for (int j = g; j < nkb; j += 2) {
-        const int b = j % kAttnKV;
-        if (!mbar_wait(bar_kvfull + 8 * b, (j / kAttnKV) & 1)) break;
-        const uint8_t* kbuf = smem + AttnSmem::K + b * 8192;
-        const uint8_t* vbuf = smem + AttnSmem::V + b * 8192;
-        float s0 = 0.f, s1 = 0.f;
-#pragma unroll
         for (int c = 0; c < 8; ++c) {
-          float f0[8], f1[8];
-          bf16x8_to_f32(*reinterpret_cast<const uint4*>(kbuf + swz(lane, c)), f0);
-          bf16x8_to_f32(*reinterpret_cast<const uint4*>(kbuf + swz(lane + 32, c)), f1);
+          float f[8];
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(smem + AttnSmem::Q + swz(row, c)), f);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            s0 = fmaf(qf[8 * c + e], f0[e], s0);
-            s1 = fmaf(qf[8 * c + e], f1[e], s1);
+          for (int e = 0; e < 8; ++e) sg = fmaf(f[e], sKg[c * 8 + e], sg);
+        }
+        m = sg * a.scale_log2;
+        l = 1.f;
+        gcoef = 1.f;
+      }
+      for (int j = 0; j < nkb && ok; ++j) {
+        const int sbuf = j % kAttnS;
+        if (!mbar_wait(bar_sfull + 8 * sbuf, (j / kAttnS) & 1)) { ok = false; break; }
+        tc_fence_after();
+        float sv[kAttnBK];
+        tmem_ld32(tmem + sbuf * 64 + lane_off, sv);
+        tmem_ld32(tmem + sbuf * 64 + lane_off + 32, sv + 32);
+        tmem_wait_ld();
+        const int kbase = j * kAttnBK;
+        // row maximum of the raw scores (the scale is positive); keys beyond the
+        // window exist only in the last block
+        if (kbase + kAttnBK > a.Nw) {
+#pragma unroll
+          for (int i = 0; i < kAttnBK; ++i)
+            if (kbase + i >= a.Nw) sv[i] = -INFINITY;
+        }
+        // eight independent partial maxima keep the dependency chains short
+        float mp[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          mp[q] = fmax3(sv[q], sv[8 + q], sv[16 + q]);
+          mp[q] = fmax3(mp[q], sv[24 + q], sv[32 + q]);
+          mp[q] = fmax3(mp[q], sv[40 + q], sv[48 + q]);
+          mp[q] = fmaxf(mp[q], sv[56 + q]);
+        }
+        const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7])) * a.scale_log2;
+        // lazy rescale: the reference maximum moves only when a score exceeds it by
+        // more than 2^8, so probabilities stay below 256 and O is rarely touched
+        const bool grow = mx > m + kAttnRescale;
+        const float mnew = grow ? mx : m;
+        const float alpha = grow ? ex2_approx(m - mnew) : 1.f;
+        const bool warp_grow = __any_sync(0xffffffffu, grow);
+        l *= alpha;
+        gcoef *= alpha;
+        m = mnew;
+        // pairs of scores through packed f32x2 arithmetic: one FMA per pair forms the
+        // exponents, the SFU takes each exponential, four packed partial sums; P goes
+        // back into the S columns as packed bf16 pairs (the A operand of P V)
+        const uint64_t sc2 = pack_f32x2(a.scale_log2, a.scale_log2), nm2 = pack_f32x2(-m, -m);
+        uint64_t sp2[4] = {0ull, 0ull, 0ull, 0ull};
+        uint32_t pw[kAttnBK / 2];
+#pragma unroll
+        for (int i = 0; i < kAttnBK; i += 2) {
+          const uint64_t x2 = fma_f32x2(pack_f32x2(sv[i], sv[i + 1]), sc2, nm2);
+          const float e0 = ex2_approx(lo_f32(x2)), e1 = ex2_approx(hi_f32(x2));
+          sp2[(i >> 1) & 3] = add_f32x2(sp2[(i >> 1) & 3], pack_f32x2(e0, e1));
+          pw[i >> 1] = pack_bf16(e0, e1);
+        }
+        const uint64_t s01 = add_f32x2(sp2[0], sp2[1]), s23 = add_f32x2(sp2[2], sp2[3]);
+        const uint64_t s0123 = add_f32x2(s01, s23);
+        l += lo_f32(s0123) + hi_f32(s0123);
+        tmem_st32u(tmem + sbuf * 64 + lane_off, pw);
+        if (warp_grow && j >= 1) {
+          // O holds the sum up to block j-1: wait for that P V, then rescale the row
+          if (!mbar_wait(bar_odone + 8 * ((j - 1) & 1), ((j - 1) >> 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int hh = 0; hh < 4; ++hh) {
+            float o[16];
+            tmem_ld16(tO + lane_off + hh * 16, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 16; ++c) o[c] *= alpha;
+            tmem_st16(tO + lane_off + hh * 16, o);
           }
         }
-        const int nvalid = min(kAttnBK, a.Nw - j * kAttnBK);
-        const float x0 = lane < nvalid ? s0 * a.scale_log2 : -INFINITY;
-        const float x1 = lane + 32 < nvalid ? s1 * a.scale_log2 : -INFINITY;
-        const float mnew = fmaxf(gm, warp_max(fmaxf(x0, x1)));
-        const float al = ex2_approx(gm - mnew);
-        const float p0 = ex2_approx(x0 - mnew), p1 = ex2_approx(x1 - mnew);
-        gl = fmaf(gl, al, p0 + p1);
-        ga0 *= al;
-        ga1 *= al;
-#pragma unroll 8
-        for (int k = 0; k < kAttnBK; ++k) {
-          const float pk = __shfl_sync(0xffffffffu, k < 32 ? p0 : p1, k & 31);
-          const uint32_t off = swz(k, lane >> 2) + (lane & 3) * 4;
-          const float2 vv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vbuf + off));
-          ga0 = fmaf(pk, vv.x, ga0);
-          ga1 = fmaf(pk, vv.y, ga1);
-        }
-        gm = mnew;
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_kvempty + 8 * b);
+        if (lane == 0) mbar_arrive(bar_pfull + 8 * sbuf);
       }
-      gl = warp_sum(gl);
-      float* gbuf = reinterpret_cast<float*>(smem + AttnSmem::GR);
-      if (lane == 0) {
-        gbuf[g * 66] = gm;
-        gbuf[g * 66 + 1] = gl;
-      }
-      gbuf[g * 66 + 2 + 2 * lane] = ga0;
-      gbuf[g * 66 + 3 + 2 * lane] = ga1;
-      asm volatile("bar.sync 1, 64;" ::: "memory");
-      if (g == 0) {
-        const float M = fmaxf(gbuf[0], gbuf[66]);
-        float L = 0.f, o0 = 0.f, o1 = 0.f;
-#pragma unroll
-        for (int w = 0; w < 2; ++w) {
-          const float f = gbuf[w * 66] == -INFINITY ? 0.f : ex2_approx(gbuf[w * 66] - M);
-          L += f * gbuf[w * 66 + 1];
-          o0 += f * gbuf[w * 66 + 2 + 2 * lane];
-          o1 += f * gbuf[w * 66 + 3 + 2 * lane];
-        }
-        bf16* O = reinterpret_cast<bf16*>(a.O) + static_cast<size_t>(t) * a.N * a.d + h * 64 + 2 * lane;
-        *reinterpret_cast<__nv_bfloat162*>(O) = __floats2bfloat162_rn(o0 / L, o1 / L);
-      }
-    }
-  } else if (warp < 4) {
-    // ---------------- softmax: one query row per thread ----------------
-    const int row = tid;                     // 0..127, TMEM lane = row
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    bool ok = mbar_wait(bar_kvfull, 0);      // Q rows are in shared memory
-    float m = -INFINITY, l = 0.f, gcoef = 0.f;
-    if (ok) {
-      // score of the global key seeds the running maximum and sum
-      float sg = 0.f;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float f[8];
-        bf16x8_to_f32(*reinterpret_cast<const uint4*>(smem + AttnSmem::Q + swz(row, c)), f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sg = fmaf(f[e], sKg[c * 8 + e], sg);
-      }
-      m = sg * a.scale_log2;
-      l = 1.f;
-      gcoef = 1.f;
-    }
-    for (int j = 0; j < nkb && ok; ++j) {
-      const int sbuf = j % kAttnS;
-      if (!mbar_wait(bar_sfull + 8 * sbuf, (j / kAttnS) & 1)) { ok = false; break; }
-      tc_fence_after();
-      float sv[kAttnBK];
-      tmem_ld32(tmem + sbuf * 64 + lane_off, sv);
-      tmem_ld32(tmem + sbuf * 64 + lane_off + 32, sv + 32);
-      tmem_wait_ld();
-      const int kbase = j * kAttnBK;
-      // row maximum of the raw scores (the scale is positive); keys beyond the
-      // window exist only in the last block
-      if (kbase + kAttnBK > a.Nw) {
-#pragma unroll
-        for (int i = 0; i < kAttnBK; ++i)
-          if (kbase + i >= a.Nw) sv[i] = -INFINITY;
-      }
-      // eight independent partial maxima keep the dependency chains short
-      float mp[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        mp[q] = fmax3(sv[q], sv[8 + q], sv[16 + q]);
-        mp[q] = fmax3(mp[q], sv[24 + q], sv[32 + q]);
-        mp[q] = fmax3(mp[q], sv[40 + q], sv[48 + q]);
-        mp[q] = fmaxf(mp[q], sv[56 + q]);
-      }
-      const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7])) * a.scale_log2;
-      // lazy rescale: the reference maximum moves only when a score exceeds it by
-      // more than 2^8, so probabilities stay below 256 and O is rarely touched
-      const bool grow = mx > m + kAttnRescale;
-      const float mnew = grow ? mx : m;
-      const float alpha = grow ? ex2_approx(m - mnew) : 1.f;
-      const bool warp_grow = __any_sync(0xffffffffu, grow);
-      l *= alpha;
-      gcoef *= alpha;
-      m = mnew;
-      // pairs of scores through packed f32x2 arithmetic: one FMA per pair forms the
-      // exponents, the SFU takes each exponential, four packed partial sums; P goes
-      // back into the S columns as packed bf16 pairs (the A operand of P V)
-      const uint64_t sc2 = pack_f32x2(a.scale_log2, a.scale_log2), nm2 = pack_f32x2(-m, -m);
-      uint64_t sp2[4] = {0ull, 0ull, 0ull, 0ull};
-      uint32_t pw[kAttnBK / 2];
-#pragma unroll
-      for (int i = 0; i < kAttnBK; i += 2) {
-        const uint64_t x2 = fma_f32x2(pack_f32x2(sv[i], sv[i + 1]), sc2, nm2);
-        const float e0 = ex2_approx(lo_f32(x2)), e1 = ex2_approx(hi_f32(x2));
-        sp2[(i >> 1) & 3] = add_f32x2(sp2[(i >> 1) & 3], pack_f32x2(e0, e1));
-        pw[i >> 1] = pack_bf16(e0, e1);
-      }
-      const uint64_t s01 = add_f32x2(sp2[0], sp2[1]), s23 = add_f32x2(sp2[2], sp2[3]);
-      const uint64_t s0123 = add_f32x2(s01, s23);
-      l += lo_f32(s0123) + hi_f32(s0123);
-      tmem_st32u(tmem + sbuf * 64 + lane_off, pw);
-      if (warp_grow && j >= 1) {
-        // O holds the sum up to block j-1: wait for that P V, then rescale the row
-        if (!mbar_wait(bar_odone + 8 * ((j - 1) & 1), ((j - 1) >> 1) & 1)) { ok = false; break; }
+      if (ok && mbar_wait(bar_ofinal, 0)) {
         tc_fence_after();
+        const int slot = q0 + row;
+        const float inv = 1.f / l;
+        bf16* dst = reinterpret_cast<bf16*>(a.O) + (static_cast<size_t>(t) * a.N + slot) * a.d + h * 64;
 #pragma unroll 1
-        for (int hh = 0; hh < 4; ++hh) {
-          float o[16];
-          tmem_ld16(tO + lane_off + hh * 16, o);
+        for (int hh = 0; hh < 2; ++hh) {
+          float o[32];
+          tmem_ld32(tO + lane_off + hh * 32, o);
           tmem_wait_ld();
+          if (slot < a.N) {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) o[c] *= alpha;
-          tmem_st16(tO + lane_off + hh * 16, o);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_pfull + 8 * sbuf);
-    }
-    if (ok && mbar_wait(bar_ofinal, 0)) {
-      tc_fence_after();
-      const int slot = q0 + row;
-      const float inv = 1.f / l;
-      bf16* dst = reinterpret_cast<bf16*>(a.O) + (static_cast<size_t>(t) * a.N + slot) * a.d + h * 64;
-#pragma unroll 1
-      for (int hh = 0; hh < 2; ++hh) {
-        float o[32];
-        tmem_ld32(tO + lane_off + hh * 32, o);
-        tmem_wait_ld();
-        if (slot < a.N) {
+            for (int c = 0; c < 32; c += 8) {
+              float f[8];
 #pragma unroll
-          for (int c = 0; c < 32; c += 8) {
-            float f[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = (o[c + e] + gcoef * sVg[hh * 32 + c + e]) * inv;
-            *reinterpret_cast<uint4*>(dst + hh * 32 + c) = f32_to_bf16x8(f);
+              for (int e = 0; e < 8; ++e) f[e] = (o[c + e] + gcoef * sVg[hh * 32 + c + e]) * inv;
+              *reinterpret_cast<uint4*>(dst + hh * 32 + c) = f32_to_bf16x8(f);
+            }
           }
         }
       }
