@@ -174,6 +174,99 @@ __global__ void __launch_bounds__(256) merge_kernel(const T* __restrict__ P, int
   store_row<T, NV, Q8>(v, lane, A, q8, qscale, row, d);
 }
 
+// The same blend with the tile rows staged in shared memory: each warp owns two
+// buffers of `cover` rows (cover = most tiles on one token) and keeps two output
+// rows in flight; for each, the lanes read the token's entries (one per lane) and
+// issue one bulk copy per entry, so loads in flight hold no registers.  Row
+// U + t is the single entry t*N with weight 1.  Sums run in ascending entry order,
+// as in merge_kernel.
+constexpr int kMergeWarps = 4;
+template <typename T, int NV, bool Q8>
+__global__ void __launch_bounds__(kMergeWarps * 32) merge_bulk_kernel(
+    const T* __restrict__ P, int rows, int U, int N, int d, const int* __restrict__ tok_ptr,
+    const int* __restrict__ tok_ent, const float* __restrict__ wbar, int cover, T* __restrict__ A,
+    uint8_t* __restrict__ q8, float* __restrict__ qscale) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  constexpr int E = Vec<T>::E;
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const uint32_t rowbytes = static_cast<uint32_t>(d) * sizeof(T);
+  uint8_t* wbuf = smem + static_cast<size_t>(wib) * 2 * cover * rowbytes;
+  const uint32_t bar = smem_u32(smem + static_cast<size_t>(kMergeWarps) * 2 * cover * rowbytes) + 16 * wib;
+  if (lane == 0) {
+    mbar_init(bar, 1);
+    mbar_init(bar + 8, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  pdl_wait();
+  pdl_trigger();
+  // entries of row r (lane k < n holds entry k's weight) and their copies into buffer b
+  auto issue = [&](int r, int b, int& n, float& wl) {
+    int ent = 0;
+    wl = 0.f;
+    if (r < U) {
+      const int e0 = __ldg(tok_ptr + r);
+      n = __ldg(tok_ptr + r + 1) - e0;
+      if (lane < n) {
+        ent = __ldg(tok_ent + e0 + lane);
+        wl = __ldg(wbar + e0 + lane);
+      }
+    } else {
+      n = 1;
+      ent = (r - U) * N;
+      wl = 1.f;
+    }
+    fence_proxy_async_smem();   // this warp's reads of the buffer precede the copies that overwrite it
+    __syncwarp();
+    if (lane == 0) mbar_expect_tx(bar + 8 * b, n * rowbytes);
+    __syncwarp();
+    if (lane < n)
+      bulk_load(smem_u32(wbuf + (static_cast<size_t>(b) * cover + lane) * rowbytes), P + static_cast<size_t>(ent) * d,
+                rowbytes, bar + 8 * b);
+  };
+  const int stride = gridDim.x * kMergeWarps;
+  int row = blockIdx.x * kMergeWarps + wib;
+  int nc = 0, nn = 0;
+  float wc = 0.f, wn = 0.f;
+  bool pending_next = false;
+  int broke_at = -1;
+  if (row < rows) issue(row, 0, nc, wc);
+  for (int i = 0; row < rows; ++i, row += stride) {
+    pending_next = row + stride < rows;
+    if (pending_next) issue(row + stride, (i + 1) & 1, nn, wn);
+    if (!mbar_wait(bar + 8 * (i & 1), (i >> 1) & 1)) {
+      broke_at = i;
+      break;
+    }
+    pending_next = false;
+    const uint8_t* buf = wbuf + static_cast<size_t>(i & 1) * cover * rowbytes;
+    float v[NV][E];
+#pragma unroll
+    for (int k = 0; k < NV; ++k)
+#pragma unroll
+      for (int e = 0; e < E; ++e) v[k][e] = 0.f;
+    for (int k = 0; k < nc; ++k) {
+      const float w = __shfl_sync(0xffffffffu, wc, k);
+      const T* src = reinterpret_cast<const T*>(buf + static_cast<size_t>(k) * rowbytes);
+#pragma unroll
+      for (int q = 0; q < NV; ++q) {
+        float f[E];
+        Vec<T>::load(src + (q * 32 + lane) * E, f);
+#pragma unroll
+        for (int e = 0; e < E; ++e) v[q][e] = fmaf(w, f[e], v[q][e]);
+      }
+    }
+    store_row<T, NV, Q8>(v, lane, A, q8, qscale, row, d);
+    nc = nn;
+    wc = wn;
+  }
+  // no copy may still be landing when the CTA exits (matters only after a timeout)
+  if (broke_at >= 0) {
+    mbar_wait(bar + 8 * (broke_at & 1), (broke_at >> 1) & 1);
+    if (pending_next) mbar_wait(bar + 8 * ((broke_at + 1) & 1), ((broke_at + 1) >> 1) & 1);
+  }
+}
+
 // generic fallback of the blend for any d (scalar)
 template <typename T>
 __global__ void __launch_bounds__(256) merge_generic_kernel(const T* __restrict__ P, int rows, int U, int N, int d,

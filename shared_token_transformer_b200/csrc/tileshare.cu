@@ -362,6 +362,17 @@ static Workspace layout(const ts_plan_s* p, const ts_model_desc* m, bool stack, 
 // ============================================================================
 // launchers
 // ============================================================================
+static int g_num_sms = 0;
+static int num_sms() {
+  if (!g_num_sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_num_sms <= 0) g_num_sms = 148;
+  }
+  return g_num_sms;
+}
+
 static inline unsigned rows_grid(size_t rows) { return static_cast<unsigned>((rows + 7) / 8); }
 
 template <typename T, bool Q8>
@@ -413,6 +424,36 @@ static ts_status launch_merge_vec(const ts_plan_s* p, const void* P, int rows, i
   const int nv = d / (32 * E);
   const T* pp = static_cast<const T*>(P);
   T* aa = static_cast<T*>(A);
+  // Staged variant: every warp holds two buffers of max_cover rows in shared memory.
+  const size_t smem = static_cast<size_t>(ts::kMergeWarps) * 2 * p->max_cover * d * sizeof(T) + 16 * ts::kMergeWarps;
+  const int per_sm = static_cast<int>(std::min<size_t>(8, (227u * 1024u) / std::max<size_t>(smem, 1)));
+  if (per_sm >= 1) {
+    trace_pre(st);
+    const unsigned grid = static_cast<unsigned>(
+        std::min<size_t>((static_cast<size_t>(rows) + ts::kMergeWarps - 1) / ts::kMergeWarps,
+                         static_cast<size_t>(per_sm) * num_sms()));
+#define TS_MB_CASE(NV)                                                                                        \
+  case NV: {                                                                                                  \
+    auto kern = ts::merge_bulk_kernel<T, NV, Q8>;                                                             \
+    static int configured[64] = {0};                                                                          \
+    int dev = 0;                                                                                              \
+    cudaGetDevice(&dev);                                                                                      \
+    if (dev < 64 && !configured[dev]) {                                                                       \
+      TS_CUDA_CHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));     \
+      configured[dev] = 1;                                                                                    \
+    }                                                                                                         \
+    launch_pdl(kern, dim3(grid), dim3(32 * ts::kMergeWarps), smem, st, pp, rows, p->U, p->N, d,                \
+               static_cast<const int*>(p->d_tok_ptr), static_cast<const int*>(p->d_tok_ent),                   \
+               static_cast<const float*>(p->d_wbar), p->max_cover, aa, q8, qs);                              \
+    break;                                                                                                    \
+  }
+    switch (nv) {
+      TS_MB_CASE(1) TS_MB_CASE(2) TS_MB_CASE(3) TS_MB_CASE(4) TS_MB_CASE(5) TS_MB_CASE(6) TS_MB_CASE(7) TS_MB_CASE(8)
+      default: return fail(TS_ERR_UNSUPPORTED, "merge width %d", d);
+    }
+#undef TS_MB_CASE
+    return trace_post(st, "merge");
+  }
   trace_pre(st);
 #define TS_MG_CASE(NV)                                                                                    \
   case NV:                                                                                                \
@@ -463,17 +504,7 @@ static ts_status run_quantize(const void* x, int rows, int cols, uint8_t* q, flo
 // ---------------------------------------------------------------------------
 // tensor-core GEMM
 // ---------------------------------------------------------------------------
-static int g_num_sms = 0;
 
-static int num_sms() {
-  if (!g_num_sms) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (g_num_sms <= 0) g_num_sms = 148;
-  }
-  return g_num_sms;
-}
 
 template <int BN, int STAGES, int EPI, bool FP8, int R0, int R1, int R2>
 static ts_status launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, const ts::GemmArgs& args,
