@@ -76,6 +76,26 @@ def test_layernorm(cfg):
     assert rel_l2(host(y), want) < tol
 
 
+def test_gelu_epilogue_matches_exact_erf():
+    """The GELU epilogue evaluates erf by Abramowitz & Stegun 7.1.26 with the
+    approximate reciprocal and exponential: through an identity fp32 linear layer,
+    every output must be within 2e-6 of 0.5 x (1 + erf(x / sqrt 2)) (plus fp32
+    rounding), over x in [-10, 10] including 0, both signs and the tails."""
+    import math
+    m = B.model_desc(64, 1, 64, "f32", (0, 32, 32))
+    x = np.linspace(-10.0, 10.0, 64 * 64).reshape(64, 64)
+    x[0, 0] = 0.0
+    xd = torch.tensor(x, dtype=torch.float32, device="cuda")
+    W = torch.eye(64, dtype=torch.float32, device="cuda")
+    b = torch.zeros(64, dtype=torch.float32, device="cuda")
+    y = torch.empty(64, 64, dtype=torch.float32, device="cuda")
+    B.op_linear(m, xd, W, b, y, epi=B.TS_EPI_BIAS_GELU)
+    got = host(y).astype(np.float64)
+    xf = x.astype(np.float32).astype(np.float64)
+    want = np.vectorize(lambda v: 0.5 * v * (1.0 + math.erf(v / math.sqrt(2.0))))(xf)
+    assert np.max(np.abs(got - want) / np.maximum(1.0, np.abs(want))) < 2e-6
+
+
 @pytest.mark.parametrize("M,K,N", [(300, 256, 512), (128, 512, 768), (129, 256, 192), (1, 256, 64), (2320, 512, 1536),
                                    (777, 2048, 512)])
 @pytest.mark.parametrize("epi", [B.TS_EPI_BIAS, B.TS_EPI_BIAS_GELU, B.TS_EPI_BIAS_RESID])
