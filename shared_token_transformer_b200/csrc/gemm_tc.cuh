@@ -60,8 +60,9 @@ struct GemmSmem {
   static constexpr int A_BYTES = 128 * 128;
   static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
-  static constexpr int NBARS = 2 * STAGES + 4;          // full, empty, tmem full x2, tmem empty x2
+  static constexpr int EPI_OFFSET = STAGES * STAGE_BYTES;   // 8 x 4 KB: one 32 x 64 output chunk per epilogue warp
+  static constexpr int BAR_OFFSET = EPI_OFFSET + 8 * 4096;
+  static constexpr int NBARS = 2 * STAGES + 4 + 8;      // full, empty, tmem full x2, tmem empty x2, residual x8
   static constexpr int BYTES = BAR_OFFSET + NBARS * 8 + 16;
   static constexpr int LAUNCH_BYTES = BYTES + 1024;     // slack for 1024-byte alignment
 };
@@ -105,9 +106,10 @@ __device__ __forceinline__ void qk_norm_rope64(float* v, const float* __restrict
   }
 }
 
+// Epilogue arithmetic of one 64-column chunk of a row held by this thread: e4m3
+// scales, bias, then GELU or QK-RMSNorm + RoPE (the residual is added by the caller).
 template <int EPI, bool FP8, int R0, int R1, int R2>
-__device__ __forceinline__ void gemm_epilogue64(float* v, int row, int col, float rs, const int4 pos,
-                                                const GemmArgs& args) {
+__device__ __forceinline__ void gemm_epilogue64(float* v, int col, float rs, const int4 pos, const GemmArgs& args) {
   if (FP8) {
 #pragma unroll
     for (int i = 0; i < 64; i += 4) {
@@ -128,25 +130,25 @@ __device__ __forceinline__ void gemm_epilogue64(float* v, int row, int col, floa
       v[i + 3] += b.w;
     }
   }
-  bf16* dst = args.out + static_cast<size_t>(row) * args.ldo + col;
   if (EPI == EPI_GELU) {
 #pragma unroll
     for (int i = 0; i < 64; ++i) v[i] = gelu_erf(v[i]);
-  } else if (EPI == EPI_RESID) {
-#pragma unroll
-    for (int i = 0; i < 64; i += 8) {
-      float r[8];
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(dst + i), r);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[i + e] += r[e];
-    }
   } else if (EPI == EPI_QKV) {
     if (col < 2 * args.d)
       qk_norm_rope64<R0, R1, R2>(v, col < args.d ? args.q_g : args.k_g, args.eps_qk, pos, args);
   }
-#pragma unroll
-  for (int i = 0; i < 64; i += 8) *reinterpret_cast<uint4*>(dst + i) = f32_to_bf16x8(v + i);
 }
+
+// TMA tile store of a shared-memory box to global memory (bulk-group completion).
+__device__ __forceinline__ void tma_store_2d(const void* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Output tile order: bands of kGemmBand row tiles, each band walked across all
 // column tiles with the row tile fastest.  The CTAs in flight then share one or
@@ -164,7 +166,7 @@ __device__ __forceinline__ void gemm_tile_origin(int tile, int mt, int nt, int b
 template <int BN, int STAGES, int EPI, bool FP8, int R0, int R1, int R2>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmArgs args) {
+                   const __grid_constant__ CUtensorMap tmD, const GemmArgs args) {
   using SM = GemmSmem<BN, STAGES>;
   constexpr int NMMA = 128 / 32;                  // MMAs per 128-byte K slice (32 bytes each)
   constexpr uint32_t TMEM_COLS = 2 * BN;          // two accumulators: 128, 256 or 512 columns
@@ -179,6 +181,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t bar_empty = bar_full + 8 * STAGES;       // STAGES
   const uint32_t bar_tfull = bar_empty + 8 * STAGES;      // 2
   const uint32_t bar_tempty = bar_tfull + 16;             // 2
+  const uint32_t bar_resid = bar_tempty + 16;             // 8: residual chunk of each epilogue warp
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::BAR_OFFSET + SM::NBARS * 8);
 
   const int warp = threadIdx.x >> 5;
@@ -190,6 +193,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == kGemmTmaWarp && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmD);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
@@ -198,6 +202,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(bar_tfull + 8 * b, 1);
       mbar_init(bar_tempty + 8 * b, 8);           // one arrival per epilogue warp
     }
+    for (int w = 0; w < 8; ++w) mbar_init(bar_resid + 8 * w, 1);
     fence_barrier_init();
   }
   if (warp == kGemmMmaWarp) {
@@ -261,6 +266,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // epilogue warps 0..7: lane quarter warp % 4, column half warp / 4
     const int quarter = warp & 3;
     const int half = warp >> 2;
+    const uint32_t stg = sbase + SM::EPI_OFFSET + warp * 4096;
+    const uint32_t rbar = bar_resid + 8 * warp;
+    uint32_t nres = 0;                 // residual chunks this warp has loaded
+    bool store_pending = false;        // a tile store may still be reading the staging buffer
+    bool eok = true;
     uint32_t j = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++j) {
       const uint32_t acc = j & 1, use = j >> 1;
@@ -284,6 +294,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
 #pragma unroll 1
       for (int c = half, k = 0; c < NCHUNK; c += 2, ++k) {
+        // the chunk goes out through this warp's 4 KB staging buffer (32 rows x 128 B,
+        // 128-byte swizzle) as one TMA tile store; the residual comes in the same way
+        if (store_pending) {
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+          store_pending = false;
+        }
+        const int col = n0 + c * 64, row0 = m0 + quarter * 32;
+        if (EPI == EPI_RESID && lane == 0) {
+          mbar_expect_tx(rbar, 4096);
+          tma_load_2d(stg, &tmD, rbar, col, row0);
+        }
         float v[64];
         tmem_ld32(trow + c * 64, v);
         tmem_ld32(trow + c * 64 + 32, v + 32);
@@ -293,9 +315,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(bar_tempty + 8 * acc);
         }
-        if (row < args.M) gemm_epilogue64<EPI, FP8, R0, R1, R2>(v, row, n0 + c * 64, rs, pos, args);
+        gemm_epilogue64<EPI, FP8, R0, R1, R2>(v, col, rs, pos, args);
+        uint8_t* srow = smem + SM::EPI_OFFSET + warp * 4096 + lane * 128;
+        if (EPI == EPI_RESID) {
+          if (!mbar_wait(rbar, nres & 1)) {
+            eok = false;
+            break;
+          }
+          ++nres;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float r[8];
+            bf16x8_to_f32(*reinterpret_cast<const uint4*>(srow + ((q ^ (lane & 7)) << 4)), r);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[8 * q + e] += r[e];
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) *reinterpret_cast<uint4*>(srow + ((q ^ (lane & 7)) << 4)) = f32_to_bf16x8(v + 8 * q);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmD, stg, col, row0);     // rows past M are clipped by the copy
+          bulk_commit();
+        }
+        store_pending = true;
       }
+      if (!eok) break;
     }
+    if (lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();

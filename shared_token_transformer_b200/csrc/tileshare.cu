@@ -507,8 +507,8 @@ static ts_status run_quantize(const void* x, int rows, int cols, uint8_t* q, flo
 
 
 template <int BN, int STAGES, int EPI, bool FP8, int R0, int R1, int R2>
-static ts_status launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, const ts::GemmArgs& args,
-                                cudaStream_t st) {
+static ts_status launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
+                                const ts::GemmArgs& args, cudaStream_t st) {
   using SM = ts::GemmSmem<BN, STAGES>;
   auto kern = ts::gemm_tc_kernel<BN, STAGES, EPI, FP8, R0, R1, R2>;
   static int configured[64] = {0};
@@ -521,17 +521,17 @@ static ts_status launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, co
   const int tiles = ((args.M + 127) / 128) * (args.N / BN);
   dim3 grid(std::min(tiles, num_sms()));
   trace_pre(st);
-  launch_pdl(kern, grid, dim3(ts::kGemmThreads), SM::LAUNCH_BYTES, st, ta, tb, args);
+  launch_pdl(kern, grid, dim3(ts::kGemmThreads), SM::LAUNCH_BYTES, st, ta, tb, td, args);
   return trace_post(st, "gemm_tc");
 }
 
 template <int EPI, bool FP8, int R0, int R1, int R2>
-static ts_status dispatch_gemm_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const ts::GemmArgs& args,
-                                  cudaStream_t st) {
+static ts_status dispatch_gemm_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
+                                  const ts::GemmArgs& args, cudaStream_t st) {
   switch (bn) {
-    case 256: return launch_gemm_tc<256, 4, EPI, FP8, R0, R1, R2>(ta, tb, args, st);
-    case 128: return launch_gemm_tc<128, 6, EPI, FP8, R0, R1, R2>(ta, tb, args, st);
-    default: return launch_gemm_tc<64, 8, EPI, FP8, R0, R1, R2>(ta, tb, args, st);
+    case 256: return launch_gemm_tc<256, 4, EPI, FP8, R0, R1, R2>(ta, tb, td, args, st);
+    case 128: return launch_gemm_tc<128, 6, EPI, FP8, R0, R1, R2>(ta, tb, td, args, st);
+    default: return launch_gemm_tc<64, 8, EPI, FP8, R0, R1, R2>(ta, tb, td, args, st);
   }
 }
 
@@ -577,9 +577,10 @@ static ts_status run_gemm_tc(const char* name, const ts_model_desc* m, int epi, 
   }
   if (K % (fp8 ? 128 : 64) || N % 64) return fail(TS_ERR_UNSUPPORTED, "GEMM sizes K=%d N=%d not tiled", K, N);
   const int bn = pick_bn(M, N);
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, td;
   TS_TRY(make_tmap(&ta, A, M, K, fp8 ? 1 : 2, 128));
   TS_TRY(make_tmap(&tb, W, N, K, fp8 ? 1 : 2, bn));
+  TS_TRY(make_tmap(&td, out, M, N, 2, 32));   // output (and residual): 32 x 64 chunks of the epilogue warps
   ts::GemmArgs g{};
   g.M = M;
   g.N = N;
@@ -600,7 +601,8 @@ static ts_status run_gemm_tc(const char* name, const ts_model_desc* m, int epi, 
   }
   const bool r3 = m->rope_dims[0] == 16;
 #define TS_GEMM_EPI(E, R0, R1, R2) \
-  (fp8 ? dispatch_gemm_bn<E, true, R0, R1, R2>(bn, ta, tb, g, st) : dispatch_gemm_bn<E, false, R0, R1, R2>(bn, ta, tb, g, st))
+  (fp8 ? dispatch_gemm_bn<E, true, R0, R1, R2>(bn, ta, tb, td, g, st)     \
+       : dispatch_gemm_bn<E, false, R0, R1, R2>(bn, ta, tb, td, g, st))
   switch (epi) {
     case ts::EPI_BIAS: return TS_GEMM_EPI(ts::EPI_BIAS, 0, 32, 32);
     case ts::EPI_GELU: return TS_GEMM_EPI(ts::EPI_GELU, 0, 32, 32);
