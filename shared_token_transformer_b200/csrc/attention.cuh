@@ -567,8 +567,30 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
           for (int i = 0; i < kAttnBK; ++i)
             if (kbase + i >= a.Nw) sv[i] = -INFINITY;
         }
-        // eight independent partial maxima keep the dependency chains short
-        float mp[8];
+        // The exponentials are taken against the current reference maximum m right
+        // away; the block's maximum is formed alongside them (independent chains).
+        // The reference moves only when a score exceeds it by more than 2^8 (lazy
+        // rescale: probabilities stay below 256 and O is rarely touched); such a row
+        // takes its exponentials again against the new reference.
+        const uint64_t sc2 = pack_f32x2(a.scale_log2, a.scale_log2);
+        uint64_t sp2[4];
+        uint32_t pw[kAttnBK / 2];
+        // pairs of scores through packed f32x2 arithmetic: one FMA per pair forms the
+        // exponents, the SFU takes each exponential, four packed partial sums; P goes
+        // back into the S columns as packed bf16 pairs (the A operand of P V)
+        auto exps = [&](float mref) {
+          const uint64_t nm2 = pack_f32x2(-mref, -mref);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) sp2[q] = 0ull;
+#pragma unroll
+          for (int i = 0; i < kAttnBK; i += 2) {
+            const uint64_t x2 = fma_f32x2(pack_f32x2(sv[i], sv[i + 1]), sc2, nm2);
+            const float e0 = ex2_approx(lo_f32(x2)), e1 = ex2_approx(hi_f32(x2));
+            sp2[(i >> 1) & 3] = add_f32x2(sp2[(i >> 1) & 3], pack_f32x2(e0, e1));
+            pw[i >> 1] = pack_bf16(e0, e1);
+          }
+        };
+        float mp[8];   // eight independent partial maxima keep the dependency chains short
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           mp[q] = fmax3(sv[q], sv[8 + q], sv[16 + q]);
@@ -576,28 +598,17 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
           mp[q] = fmax3(mp[q], sv[40 + q], sv[48 + q]);
           mp[q] = fmaxf(mp[q], sv[56 + q]);
         }
+        exps(m);
         const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7])) * a.scale_log2;
-        // lazy rescale: the reference maximum moves only when a score exceeds it by
-        // more than 2^8, so probabilities stay below 256 and O is rarely touched
         const bool grow = mx > m + kAttnRescale;
-        const float mnew = grow ? mx : m;
-        const float alpha = grow ? ex2_approx(m - mnew) : 1.f;
         const bool warp_grow = __any_sync(0xffffffffu, grow);
-        l *= alpha;
-        gcoef *= alpha;
-        m = mnew;
-        // pairs of scores through packed f32x2 arithmetic: one FMA per pair forms the
-        // exponents, the SFU takes each exponential, four packed partial sums; P goes
-        // back into the S columns as packed bf16 pairs (the A operand of P V)
-        const uint64_t sc2 = pack_f32x2(a.scale_log2, a.scale_log2), nm2 = pack_f32x2(-m, -m);
-        uint64_t sp2[4] = {0ull, 0ull, 0ull, 0ull};
-        uint32_t pw[kAttnBK / 2];
-#pragma unroll
-        for (int i = 0; i < kAttnBK; i += 2) {
-          const uint64_t x2 = fma_f32x2(pack_f32x2(sv[i], sv[i + 1]), sc2, nm2);
-          const float e0 = ex2_approx(lo_f32(x2)), e1 = ex2_approx(hi_f32(x2));
-          sp2[(i >> 1) & 3] = add_f32x2(sp2[(i >> 1) & 3], pack_f32x2(e0, e1));
-          pw[i >> 1] = pack_bf16(e0, e1);
+        float alpha = 1.f;
+        if (grow) {
+          alpha = ex2_approx(m - mx);
+          l *= alpha;
+          gcoef *= alpha;
+          m = mx;
+          exps(m);
         }
         const uint64_t s01 = add_f32x2(sp2[0], sp2[1]), s23 = add_f32x2(sp2[2], sp2[3]);
         const uint64_t s0123 = add_f32x2(s01, s23);
