@@ -104,7 +104,14 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const T* __restrict__ x,
   for (int i = 0; i < NV; ++i) {
     const int c0 = (i * 32 + lane) * E;
 #pragma unroll
-    for (int e = 0; e < E; ++e) v[i][e] = (v[i][e] - mean) * rstd * __ldg(g + c0 + e) + __ldg(b + c0 + e);
+    for (int e = 0; e < E; e += 4) {   // gains and biases as 16-byte vectors
+      const float4 gg = __ldg(reinterpret_cast<const float4*>(g + c0 + e));
+      const float4 bb = __ldg(reinterpret_cast<const float4*>(b + c0 + e));
+      v[i][e] = (v[i][e] - mean) * rstd * gg.x + bb.x;
+      v[i][e + 1] = (v[i][e + 1] - mean) * rstd * gg.y + bb.y;
+      v[i][e + 2] = (v[i][e + 2] - mean) * rstd * gg.z + bb.z;
+      v[i][e + 3] = (v[i][e + 3] - mean) * rstd * gg.w + bb.w;
+    }
   }
   store_row<T, NV, Q8>(v, lane, y, q8, qscale, row, d);
 }
