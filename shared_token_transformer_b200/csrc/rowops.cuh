@@ -45,12 +45,13 @@ __device__ __forceinline__ void store_row(const float (&v)[NV][Vec<T>::E], int l
       for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(v[i][e]));
     amax = warp_max(amax);
     const float s = amax > 0.f ? amax / 448.0f : 1.0f;
+    const float inv = 1.0f / s;
     if (lane == 0) qscale[row] = s;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       uint16_t pk[E / 2];
 #pragma unroll
-      for (int e = 0; e < E; e += 2) pk[e / 2] = f32x2_to_e4m3x2(v[i][e] / s, v[i][e + 1] / s);
+      for (int e = 0; e < E; e += 2) pk[e / 2] = f32x2_to_e4m3x2(v[i][e] * inv, v[i][e + 1] * inv);
       uint8_t* dst = q8 + row * d + (i * 32 + lane) * E;
       if (E == 8)
         *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(pk);
@@ -335,13 +336,14 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const bf16* __restri
   }
   amax = warp_max(amax);
   const float s = amax > 0.f ? amax / 448.0f : 1.0f;
+  const float inv = 1.0f / s;   // one division per row; x / s becomes x * (1 / s) (within an fp32 ulp)
   if (lane == 0) scale[row] = s;
   for (int c = lane * 8; c < cols; c += 256) {
     float f[8];
     bf16x8_to_f32(*reinterpret_cast<const uint4*>(xr + c), f);
     uint16_t pk[4];
 #pragma unroll
-    for (int e = 0; e < 8; e += 2) pk[e / 2] = f32x2_to_e4m3x2(f[e] / s, f[e + 1] / s);
+    for (int e = 0; e < 8; e += 2) pk[e / 2] = f32x2_to_e4m3x2(f[e] * inv, f[e + 1] * inv);
     *reinterpret_cast<uint2*>(q + row * cols + c) = *reinterpret_cast<const uint2*>(pk);
   }
 }
