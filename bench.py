@@ -316,11 +316,8 @@ def run_tileshare(args, rank, world, local):
     t_step = np.array([e[0].elapsed_time(e[3]) for e in evs])
     t_tiled = np.array([e[0].elapsed_time(e[1]) for e in evs])
     t_shared = np.array([e[1].elapsed_time(e[2]) for e in evs])
-    sums = torch.tensor([t_shared.sum(), t_step.mean(), t_tiled.mean()], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(sums, op=dist.ReduceOp.MAX)
-    shared_total_ms, step_ms, tiled_ms = (float(x) for x in sums.cpu())
-    value = (U * (L - k) * K * world) / (shared_total_ms / 1e3) if L > k else 0.0
+    shared_total_ms, step_ms, tiled_ms = max_over_ranks([t_shared.sum(), t_step.mean(), t_tiled.mean()], world)
+    value = replica_rate(U * (L - k) * K, world, shared_total_ms)
     gpu_launches = launches_per_step * K if use_graph else eager_launches
 
     # own batched per-tile path on the same input: k = L (all layers per tile, blended at the end)
@@ -366,10 +363,8 @@ def run_tileshare(args, rank, world, local):
             eev[i - 3][1].record()
     torch.cuda.synchronize()
     e2e_ms = float(np.mean([a.elapsed_time(b) for a, b in eev]))
-    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-    e2e_value = U * world / (float(e2e_t.item()) / 1e3)
+    (e2e_max,) = max_over_ranks([e2e_ms], world)
+    e2e_value = replica_rate(U, world, e2e_max)
     state_bytes = (U + T) * d * S_host.element_size()
 
     # traced pass: per-kernel times of the same step, eagerly launched
@@ -453,6 +448,26 @@ def run_tileshare(args, rank, world, local):
         "clocks": clocks,
     }
     return res, cfg
+
+
+def max_over_ranks(vals, world):
+    """Element-wise maximum over the ranks of a list of floats (the slowest rank's
+    times; identity with one rank).  The tensor lives where the process group's
+    backend wants it: on the rank's GPU for NCCL, on the host for gloo."""
+    if world <= 1:
+        return [float(v) for v in vals]
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def replica_rate(units_per_rank, world, ms):
+    """Whole-job rate of `world` replicas, each processing `units_per_rank` units,
+    over the slowest rank's `ms` milliseconds."""
+    return units_per_rank * world / (ms / 1e3) if ms > 0 else 0.0
 
 
 def kernel_source_sha():
