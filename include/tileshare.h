@@ -212,6 +212,15 @@ ts_status ts_quantize_rows_e4m3(const void* x, int rows, int cols, void* q, floa
    Synchronises the device and clears the word. */
 ts_status ts_device_status(void);
 
+/* Self-test of the kernels' bounded waits (the pages have no counterpart; it checks
+   the library's failure reporting).  Launches one thread that waits on an mbarrier
+   nothing arrives at, with the kernels' own wait routine and a limit of limit_ns
+   (0 < limit_ns <= 1e9).  The wait gives up, the kernel writes done[0] = 1 and
+   done[1] = 0 (device int[2], caller-owned) and returns, and the next
+   ts_device_status() reports TS_ERR_TIMEOUT; the context stays usable.
+   Asynchronous on `stream`. */
+ts_status ts_selftest_bounded_wait(long long limit_ns, int* done, void* stream);
+
 /* Kernel trace (tracing subsystem).  Between ts_trace_begin() and ts_trace_end()
    every kernel the library enqueues is bracketed by two CUDA events on its own
    stream and recorded with its algorithmic work (FLOPs of the contraction, bytes

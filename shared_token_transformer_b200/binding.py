@@ -86,6 +86,7 @@ _SIGS = {
     "ts_trace_end": [ctypes.POINTER(TraceEntry), ctypes.c_int, ctypes.POINTER(ctypes.c_int)],
     "ts_launch_count": [],
     "ts_device_status": [],
+    "ts_selftest_bounded_wait": [ctypes.c_longlong, _cp, _cp],
     "ts_status_string": [ctypes.c_int],
     "ts_last_error": [],
     "ts_op_layernorm": [ctypes.POINTER(ModelDesc), _cp, ctypes.c_int, _cp, _cp, _cp, _cp],
@@ -259,6 +260,11 @@ def quantize_rows_e4m3(x, q, scale, stream=None):
 
 def device_status():
     _check("ts_device_status", lib().ts_device_status())
+
+
+def selftest_bounded_wait(limit_ns, done, stream=None):
+    """ts_selftest_bounded_wait: a wait that nothing satisfies must time out (device int32 done[2])."""
+    _check("ts_selftest_bounded_wait", lib().ts_selftest_bounded_wait(int(limit_ns), _ptr(done), _stream(stream)))
 
 
 def op_layernorm(model, x, g, b, y, stream=None):

@@ -78,19 +78,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete; gives up after
-// kWaitLimitNs, writes kStatusTimeout and returns false.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// limit_ns (kWaitLimitNs in the kernels), writes kStatusTimeout and returns false.
+__device__ __noinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 256; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       set_status(kStatusTimeout);
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) { return mbar_wait_for(bar, parity, kWaitLimitNs); }
+
+// Self-test of the bounded wait: one thread initialises an mbarrier that nothing
+// arrives at and waits for it with a short limit; the wait must give up, write
+// kStatusTimeout and let the kernel return.  `done` receives 1 (returned) and the
+// wait's result.
+__global__ void wait_selftest_kernel(uint64_t limit_ns, int* done) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  fence_barrier_init();
+  const bool ok = mbar_wait_for(b, 0, limit_ns);
+  done[0] = 1;
+  done[1] = ok ? 1 : 0;
 }
 
 // ----------------------------------------------------------------------------

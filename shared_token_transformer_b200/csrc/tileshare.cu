@@ -1141,6 +1141,15 @@ ts_status ts_device_status(void) {
   return fail(static_cast<ts_status>(v), "device status %d", v);
 }
 
+ts_status ts_selftest_bounded_wait(long long limit_ns, int* done, void* stream) {
+  if (!done || limit_ns <= 0 || limit_ns > 1000000000LL)
+    return fail(TS_ERR_INVALID_ARG, "need done != NULL and 0 < limit_ns <= 1e9");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ts::wait_selftest_kernel<<<1, 1, 0, st>>>(static_cast<uint64_t>(limit_ns), done);
+  TS_CUDA_CHECK(cudaGetLastError());
+  return TS_OK;
+}
+
 // ---------------------------------------------------------------------------
 // op-level entry points (include/tileshare_ops.h)
 // ---------------------------------------------------------------------------

@@ -316,6 +316,24 @@ def test_attention_bitwise_repeatable(name):
 # ---------------------------------------------------------------------------
 # error paths: refused on the host, nothing written
 # ---------------------------------------------------------------------------
+def test_bounded_wait_times_out_and_context_survives():
+    """A kernel wait that nothing satisfies gives up after its limit (here 2 ms),
+    reports TS_ERR_TIMEOUT through ts_device_status, and the context keeps working:
+    no trap, no fault, no hang."""
+    done = torch.zeros(2, dtype=torch.int32, device="cuda")
+    B.selftest_bounded_wait(2_000_000, done)
+    with pytest.raises(B.TileShareError) as e:
+        B.device_status()
+    assert e.value.status == 6
+    assert done.tolist() == [1, 0]
+    B.device_status()                      # the status word was cleared
+    c = case(SMALL)                        # and the library still computes
+    S = dev(c.S, c.dt)
+    B.block_shared(c.plan, c.m, c.wlist[0], S, c.workspace())
+    B.device_status()
+    assert torch.isfinite(S.float()).all()
+
+
 def test_error_paths():
     c = case(SMALL)
     S = dev(c.S, c.dt)
