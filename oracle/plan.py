@@ -27,6 +27,11 @@ Readings taken where the pages are silent (stated here and in the design doc)
        per-tile state of tile t has N = Nw + 1 rows: row 0 is the tile's global
        token, row 1 + j its window slot j.  A (tile, slot) entry is addressed as
        t*N + 1 + j.
+    R11 hard stitching (blend rule "hard", [TileShare] discussion of blending versus
+       stitching the tiles' outputs): each token takes its value from one tile, the
+       covering tile with the largest unnormalised R2 weight, the lowest tile index
+       on ties; w-bar is 1 for that tile and 0 for the others, and the token's CSR
+       row holds that single entry.
 """
 
 from dataclasses import dataclass, field
@@ -101,8 +106,13 @@ class Plan:
         return int(self.tok_ent.shape[0])
 
 
-def make_plan(grid, win, stride) -> Plan:
-    """Tile plan for a token grid (F, H, W); 2-D grids use F = wf = sf = 1."""
+def make_plan(grid, win, stride, rule: str = "ramp") -> Plan:
+    """Tile plan for a token grid (F, H, W); 2-D grids use F = wf = sf = 1.
+
+    rule "ramp": w-bar of R2 (normalised ramp weights); rule "hard": R11.
+    """
+    if rule not in ("ramp", "hard"):
+        raise ValueError(f"unknown blend rule {rule!r}")
     F, H, W = (int(v) for v in grid)
     wf, wh, ww = (int(v) for v in win)
     sf, sh, sw = (int(v) for v in stride)
@@ -137,12 +147,30 @@ def make_plan(grid, win, stride) -> Plan:
     if np.any(coverage == 0):
         raise ValueError("tiling leaves a token uncovered")
     wbar = wraw / total[tile_tok]
+    if rule == "hard":
+        # the covering tile with the largest raw weight; strict > keeps the first
+        # (lowest) tile on ties, tiles being visited in ascending order
+        best_t = np.full(U, -1, dtype=np.int64)
+        best_w = np.full(U, -1.0, dtype=np.float64)
+        for t in range(T):
+            for j in range(Nw):
+                u = tile_tok[t, j]
+                if wraw[t, j] > best_w[u]:
+                    best_w[u] = wraw[t, j]
+                    best_t[u] = t
+        wbar = np.zeros((T, Nw), dtype=np.float64)
+        for t in range(T):
+            for j in range(Nw):
+                if best_t[tile_tok[t, j]] == t:
+                    wbar[t, j] = 1.0
 
     # CSR over grid tokens; tiles are visited in ascending order, so each token's
     # entries come out in ascending tile index.
     lists = [[] for _ in range(U)]
     for t in range(T):
         for j in range(Nw):
+            if rule == "hard" and wbar[t, j] == 0.0:
+                continue
             lists[tile_tok[t, j]].append((t * N + 1 + j, wbar[t, j]))
     tok_ptr = np.zeros(U + 1, dtype=np.int64)
     for u in range(U):

@@ -135,3 +135,65 @@ def test_single_tile_and_no_overlap_degenerate():
     assert p.T == 1 and np.all(p.tok_w == 1.0) and p.nnz == 64
     p = P.make_plan((1, 16, 16), (1, 8, 8), (1, 8, 8))
     assert p.T == 4 and np.all(p.coverage == 1) and np.all(p.tok_w == 1.0)
+
+
+# ---------------------------------------------------------------------------
+# hard stitching (reading R11): one tile per token, the largest ramp weight,
+# lowest tile index on ties
+# ---------------------------------------------------------------------------
+def test_hard_stitch_one_entry_of_weight_one():
+    for grid, win, stride in _small_geometries():
+        p = P.make_plan(grid, win, stride, rule="hard")
+        assert np.all(np.diff(p.tok_ptr) == 1) and p.nnz == p.U
+        assert np.all(p.tok_w == 1.0)
+        # every entry is a (tile, slot) that contains its token
+        t = p.tok_ent // p.N
+        j = p.tok_ent % p.N - 1
+        np.testing.assert_array_equal(p.tile_tok[t, j], np.arange(p.U))
+
+
+def test_hard_stitch_choice_is_argmax_lowest_tile_on_ties():
+    """Recomputed here with a vectorised argmax over the ramp plan's raw weights:
+    for each token, the largest raw weight among its tiles, then the lowest tile."""
+    for grid, win, stride in _small_geometries()[::7]:
+        ramp = P.make_plan(grid, win, stride)
+        hard = P.make_plan(grid, win, stride, rule="hard")
+        t_all = np.repeat(np.arange(ramp.T), ramp.Nw)
+        u_all = ramp.tile_tok.reshape(-1)
+        w_all = ramp.wraw.reshape(-1)
+        order = np.lexsort((t_all, -w_all, u_all))      # by token, weight descending, tile ascending
+        first = order[np.r_[0, np.flatnonzero(np.diff(u_all[order])) + 1]]
+        want_t = np.empty(ramp.U, dtype=np.int64)
+        want_t[u_all[first]] = t_all[first]
+        np.testing.assert_array_equal(hard.tok_ent // hard.N, want_t)
+
+
+def test_hard_stitch_two_tile_split_point():
+    """Two tiles overlapping by o tokens on one axis: at band position i the weights
+    are (o - i)/(o + 1) and (i + 1)/(o + 1), so the first tile keeps the positions
+    i <= (o - 1)/2 (the tie at odd o goes to the lower tile) and the second the rest."""
+    for G, w, s in [(14, 8, 6), (10, 6, 4), (9, 5, 4), (12, 8, 4), (11, 7, 4), (13, 10, 3)]:
+        o_list = P.axis_origins(G, w, s)
+        assert len(o_list) == 2
+        lo, hi = o_list[1], o_list[0] + w
+        o = hi - lo
+        p = P.make_plan((1, 1, G), (1, 1, w), (1, 1, s), rule="hard")
+        chosen = p.tok_ent // p.N
+        for g in range(G):
+            if g < lo:
+                assert chosen[g] == 0
+            elif g >= hi:
+                assert chosen[g] == 1
+            else:
+                i = g - lo
+                assert chosen[g] == (0 if 2 * i <= o - 1 else 1), (G, w, s, g)
+
+
+def test_hard_stitch_equals_ramp_without_overlap():
+    for grid, win, stride in [((1, 16, 16), (1, 8, 8), (1, 8, 8)), ((2, 6, 9), (1, 3, 3), (1, 3, 3)),
+                              ((1, 8, 8), (1, 8, 8), (1, 2, 2))]:
+        a = P.make_plan(grid, win, stride)
+        b = P.make_plan(grid, win, stride, rule="hard")
+        np.testing.assert_array_equal(a.tok_ptr, b.tok_ptr)
+        np.testing.assert_array_equal(a.tok_ent, b.tok_ent)
+        np.testing.assert_array_equal(a.tok_w, b.tok_w)
