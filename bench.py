@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--trace-steps", type=int, default=20)
+    ap.add_argument("--blend", default="ramp", choices=["ramp", "hard"],
+                    help="blend rule of the plan: normalised linear ramp (default) or hard stitching")
     return ap.parse_args()
 
 
@@ -152,12 +154,12 @@ def blas_threads():
     return os.cpu_count()
 
 
-def oracle_shared_layer_timing(cfg, budget_s, max_steps, warmup=1):
+def oracle_shared_layer_timing(cfg, budget_s, max_steps, warmup=1, rule="ramp"):
     """Time the float64 oracle's shared layer on the configuration's seeded input."""
     from oracle import layers as OL
     from oracle import plan as OP
     from shared_token_transformer_b200 import workloads as W
-    op = OP.make_plan(cfg.grid, cfg.win, cfg.stride)
+    op = OP.make_plan(cfg.grid, cfg.win, cfg.stride, rule=rule)
     dr = W.Draw(cfg, op.T, seed=0)
     S0, G0 = dr.states()
     S = np.concatenate([S0, G0])
@@ -193,7 +195,8 @@ def run_tileshare(args, rank, world, local):
     cfg = W.CONFIGS[args.config]
     L, k = cfg.L, cfg.k
     dt = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.bfloat16}[cfg.dtype]
-    plan = B.Plan(cfg.grid, cfg.win, cfg.stride)
+    plan = B.Plan(cfg.grid, cfg.win, cfg.stride,
+                  rule=B.TS_BLEND_HARD_STITCH if args.blend == "hard" else B.TS_BLEND_LINEAR_RAMP)
     U, T, N, d, f = plan.U, plan.T, plan.N, cfg.d, cfg.mlp
     m = B.model_desc(d, cfg.heads, f, cfg.dtype, cfg.rope_dims)
 
@@ -430,7 +433,7 @@ def run_tileshare(args, rank, world, local):
         "vs_baseline": None, "dtype": {"bf16": "bf16", "f32": "f32", "fp8": "e4m3"}[cfg.dtype],
         "data": "synthetic (seeded N(0,1) states, N(0,0.02) weights, random init)",
         "config": {"workload": f"{cfg.name}: {cfg.note}", "grid": list(cfg.grid), "window": list(cfg.win),
-                   "stride": list(cfg.stride), "L": L, "k": k, "unique_tokens": U, "tiles": T, "rows_per_tile": N,
+                   "stride": list(cfg.stride), "blend": args.blend, "L": L, "k": k, "unique_tokens": U, "tiles": T, "rows_per_tile": N,
                    "l2": "flushed before every step (512 MiB write, outside the timed events)",
                    "launch": "CUDA graphs of the public calls" if use_graph else "eager public calls",
                    "parallelism": f"replicas x{world} (one image per GPU)"},
@@ -492,7 +495,7 @@ def main():
         if rank != 0:
             return
         budget = 150.0
-        U, times = oracle_shared_layer_timing(cfg, budget, args.steps, warmup=min(args.warmup, 1))
+        U, times = oracle_shared_layer_timing(cfg, budget, args.steps, warmup=min(args.warmup, 1), rule=args.blend)
         mean = float(np.mean(times))
         v = U / mean
         res = {"impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": UNIT, "n_gpus": world,
@@ -516,7 +519,7 @@ def main():
     res, cfg = run_tileshare(args, rank, world, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         if flops_layer(cfg.U + 1, 1, 1, cfg.d, cfg.mlp) < 5e11:
-            U, times = oracle_shared_layer_timing(cfg, args.cpu_seconds, 1000)
+            U, times = oracle_shared_layer_timing(cfg, args.cpu_seconds, 1000, rule=args.blend)
             mean = float(np.mean(times))
             res["cpu_baseline"] = {"value": round(U / mean, 2), "unit": UNIT, "cores": blas_threads(),
                                    "kind": "oracle",

@@ -55,7 +55,13 @@ typedef enum {
   /* [TileShare] Fig. 2 and abstract: overlap tokens are blended "with the released
      weights".  Read as a separable linear ramp across each overlap band, normalised
      to sum 1 per token. */
-  TS_BLEND_LINEAR_RAMP = 0
+  TS_BLEND_LINEAR_RAMP = 0,
+  /* Hard stitching ([TileShare] Tab. 2 / Tab. S2 "Hard stitching" baseline; Tab. S11:
+     each pixel from its dominant tile), applied to the blend of overlap tokens: each
+     token takes its value from one tile, the covering tile with the largest
+     linear-ramp weight, the lowest tile index on ties; its CSR row holds that single
+     entry with w-bar = 1 (nnz = U). */
+  TS_BLEND_HARD_STITCH = 1
 } ts_blend_rule;
 
 typedef enum {
@@ -72,7 +78,7 @@ typedef struct ts_plan_s* ts_plan_t;
 typedef struct {
   int grid[3], win[3], stride[3];  /* (F, H, W), (wf, wh, ww), (sf, sh, sw)          */
   int T, U, Nw, N;                 /* tiles, grid tokens, window slots, Nw + 1        */
-  int nnz;                         /* (tile, slot) entries = T * Nw                   */
+  int nnz;                         /* CSR entries: T * Nw (ramp), U (hard stitching)  */
   int max_cover;                   /* most tiles covering one token                   */
   int device;                      /* CUDA device holding the plan's device arrays    */
   int run;                         /* attention loads: every aligned group of `run`    */

@@ -27,11 +27,12 @@ Readings taken where the pages are silent (stated here and in the design doc)
        per-tile state of tile t has N = Nw + 1 rows: row 0 is the tile's global
        token, row 1 + j its window slot j.  A (tile, slot) entry is addressed as
        t*N + 1 + j.
-    R11 hard stitching (blend rule "hard", [TileShare] discussion of blending versus
-       stitching the tiles' outputs): each token takes its value from one tile, the
-       covering tile with the largest unnormalised R2 weight, the lowest tile index
-       on ties; w-bar is 1 for that tile and 0 for the others, and the token's CSR
-       row holds that single entry.
+    R11 hard stitching (blend rule "hard"; [TileShare] Tab. 2 and Tab. S2 list a
+       "Hard stitching" baseline, Tab. S11 describes it as each pixel taken from its
+       dominant tile): applied to the blend of overlap tokens, each token takes its
+       value from one tile, the covering tile with the largest unnormalised R2
+       weight (the dominant one), the lowest tile index on ties; w-bar is 1 for that
+       tile and 0 for the others, and the token's CSR row holds that single entry.
 """
 
 from dataclasses import dataclass, field

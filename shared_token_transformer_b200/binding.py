@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libtileshare.so")
 # ---------------------------------------------------------------------------
 TS_OK = 0
 TS_BLEND_LINEAR_RAMP = 0
+TS_BLEND_HARD_STITCH = 1
 TS_F32, TS_BF16, TS_FP8_E4M3 = 0, 1, 2
 TS_ROWS_SHARED, TS_ROWS_TILED = 0, 1
 TS_EPI_BIAS, TS_EPI_BIAS_GELU, TS_EPI_BIAS_RESID = 0, 1, 2
@@ -141,11 +142,11 @@ def _stream(stream=None):
 class Plan:
     """ts_plan_t with its host arrays as NumPy views (copied)."""
 
-    def __init__(self, grid, win, stride, host_only=False):
+    def __init__(self, grid, win, stride, host_only=False, rule=TS_BLEND_LINEAR_RAMP):
         g, w, s = _int3(*grid), _int3(*win), _int3(*stride)
         h = _cp()
         fn = "ts_plan_create_host" if host_only else "ts_plan_create"
-        _check(fn, getattr(lib(), fn)(g, w, s, TS_BLEND_LINEAR_RAMP, ctypes.byref(h)))
+        _check(fn, getattr(lib(), fn)(g, w, s, rule, ctypes.byref(h)))
         self.handle = h
         d = PlanDesc()
         _check("ts_plan_info", lib().ts_plan_info(h, ctypes.byref(d)))

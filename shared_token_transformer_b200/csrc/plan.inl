@@ -25,6 +25,7 @@ struct ts_plan_s {
   int grid[3], win[3], stride[3];
   int T, U, Nw, N, nnz, max_cover, device;
   int run;                       // window slots 1 + k*run .. are runs of consecutive shared rows (0: none)
+  int rule;                      // blend rule: 0 linear ramp (normalised), 1 hard stitching (one tile per token)
   std::vector<int> origins, tile_tok, slot_pos, tok_ptr, tok_ent;
   std::vector<float> wbar;
   std::vector<int> rowmap;       // [T*N] shared-layout row of slot s of tile t (s = 0: U + t)
@@ -120,9 +121,26 @@ inline bool build(ts_plan_s& P) {
     if (cover[u] == 0) return false;
     P.max_cover = std::max(P.max_cover, cover[u]);
   }
+  // hard stitching: the covering tile with the largest raw weight (first, i.e.
+  // lowest, tile on ties) is the token's only entry, with weight 1
+  std::vector<int> best_t;
+  if (P.rule == 1) {
+    best_t.assign(P.U, -1);
+    std::vector<double> best_w(P.U, -1.0);
+    for (int t = 0; t < P.T; ++t)
+      for (int j = 0; j < P.Nw; ++j) {
+        const size_t e = static_cast<size_t>(t) * P.Nw + j;
+        const int u = P.tile_tok[e];
+        if (wraw[e] > best_w[u]) {
+          best_w[u] = wraw[e];
+          best_t[u] = t;
+        }
+      }
+    P.nnz = P.U;
+  }
   // CSR over grid tokens; entries in ascending tile order
   P.tok_ptr.assign(P.U + 1, 0);
-  for (int u = 0; u < P.U; ++u) P.tok_ptr[u + 1] = P.tok_ptr[u] + cover[u];
+  for (int u = 0; u < P.U; ++u) P.tok_ptr[u + 1] = P.tok_ptr[u] + (P.rule == 1 ? 1 : cover[u]);
   P.tok_ent.assign(P.nnz, 0);
   P.wbar.assign(P.nnz, 0.f);
   std::vector<int> fill(P.tok_ptr.begin(), P.tok_ptr.end() - 1);
@@ -130,9 +148,10 @@ inline bool build(ts_plan_s& P) {
     for (int j = 0; j < P.Nw; ++j) {
       const size_t e = static_cast<size_t>(t) * P.Nw + j;
       const int u = P.tile_tok[e];
+      if (P.rule == 1 && best_t[u] != t) continue;
       const int k = fill[u]++;
       P.tok_ent[k] = t * P.N + 1 + j;
-      P.wbar[k] = static_cast<float>(wraw[e] / total[u]);
+      P.wbar[k] = P.rule == 1 ? 1.0f : static_cast<float>(wraw[e] / total[u]);
     }
   // attention row map of the shared layout and RoPE coordinates
   P.rowmap.assign(static_cast<size_t>(P.T) * P.N, 0);

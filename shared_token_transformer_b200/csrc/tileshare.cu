@@ -892,7 +892,8 @@ static ts_status plan_build_host(const int grid[3], const int win[3], const int 
                                  ts_plan_s** out) {
   if (!grid || !win || !stride || !out) return fail(TS_ERR_INVALID_ARG, "NULL argument");
   *out = nullptr;
-  if (rule != TS_BLEND_LINEAR_RAMP) return fail(TS_ERR_UNSUPPORTED, "unknown blend rule %d", static_cast<int>(rule));
+  if (rule != TS_BLEND_LINEAR_RAMP && rule != TS_BLEND_HARD_STITCH)
+    return fail(TS_ERR_INVALID_ARG, "unknown blend rule %d", static_cast<int>(rule));
   for (int a = 0; a < 3; ++a) {
     if (grid[a] < 1 || win[a] < 1 || win[a] > grid[a] || stride[a] < 1 || stride[a] > win[a])
       return fail(TS_ERR_INVALID_ARG, "axis %d: need 1 <= win <= grid and 1 <= stride <= win", a);
@@ -907,6 +908,7 @@ static ts_status plan_build_host(const int grid[3], const int win[3], const int 
     P->stride[a] = stride[a];
   }
   P->device = -1;
+  P->rule = rule == TS_BLEND_HARD_STITCH ? 1 : 0;
   if (!tsplan::build(*P)) {
     delete P;
     return fail(TS_ERR_INVALID_ARG, "tiling leaves a token uncovered");

@@ -57,10 +57,11 @@ def dev_layer(cfg, p):
 class Case:
     """Seeded inputs of a configuration, on both sides."""
 
-    def __init__(self, cfg, seed=0, affine=True, L=None):
+    def __init__(self, cfg, seed=0, affine=True, L=None, rule="ramp"):
         self.cfg = cfg
-        self.oplan = OP.make_plan(cfg.grid, cfg.win, cfg.stride)
-        self.plan = B.Plan(cfg.grid, cfg.win, cfg.stride)
+        self.oplan = OP.make_plan(cfg.grid, cfg.win, cfg.stride, rule=rule)
+        self.plan = B.Plan(cfg.grid, cfg.win, cfg.stride,
+                           rule=B.TS_BLEND_HARD_STITCH if rule == "hard" else B.TS_BLEND_LINEAR_RAMP)
         dr = W.Draw(cfg, self.oplan.T, seed=seed, affine=affine)
         self.S0, self.G0 = dr.states()
         self.layers = dr.layers(L)

@@ -99,6 +99,25 @@ def test_plan_run_length(grid, win, stride):
         p.close()
 
 
+@pytest.mark.parametrize("grid,win,stride", GEOMS)
+def test_host_planner_hard_stitch_bit_exact_against_oracle(grid, win, stride):
+    o = OP.make_plan(grid, win, stride, rule="hard")
+    p = B.Plan(grid, win, stride, host_only=True, rule=B.TS_BLEND_HARD_STITCH)
+    try:
+        assert (p.T, p.U, p.N, p.nnz) == (o.T, o.U, o.N, o.nnz) and p.nnz == p.U
+        np.testing.assert_array_equal(p.tok_ptr, o.tok_ptr)
+        np.testing.assert_array_equal(p.tok_ent, o.tok_ent)
+        np.testing.assert_array_equal(p.wbar, o.tok_w.astype(np.float32))
+    finally:
+        p.close()
+
+
+def test_unknown_blend_rule_rejected():
+    with pytest.raises(B.TileShareError) as e:
+        B.Plan((1, 8, 8), (1, 4, 4), (1, 2, 2), host_only=True, rule=7)
+    assert e.value.status == 1
+
+
 def test_image4k_plan_counts():
     p = B.Plan((1, 256, 256), (1, 32, 32), (1, 24, 24), host_only=True)
     assert (p.T, p.U, p.N, p.nnz, p.max_cover) == (121, 65536, 1025, 123904, 4)

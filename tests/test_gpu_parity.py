@@ -277,6 +277,23 @@ def test_decode_stack(cfg, ks):
         assert rel_l2(got, want) < _tol(cfg), k
 
 
+@pytest.mark.parametrize("cfg", [SMALL, VOL, SMALL_FP8], ids=lambda c: c.name)
+def test_hard_stitch_shared_layer_and_stack(cfg):
+    """Hard stitching: the plan's CSR has one entry of weight one per token, so the
+    blend and the transition copy each token's row from its chosen tile.  A shared
+    layer and a stack (k = 1) against the oracle with the same rule."""
+    c = case(cfg, rule="hard")
+    assert c.plan.nnz == c.plan.U
+    S_in = c.S
+    S = dev(S_in, c.dt)
+    B.block_shared(c.plan, c.m, c.wlist[0], S, c.workspace())
+    want = OL.block_shared(S_in, c.layers[0], c.om, c.oplan)
+    assert rel_l2(host(S), want) < _tol(cfg)
+    got = host(_run_stack(c, 1))
+    want = OL.decode_stack(c.S0, c.G0, c.layers, c.om, c.oplan, 1)
+    assert rel_l2(got, want) < _tol(cfg)
+
+
 def test_stack48_bf16_full():
     """The benchmark stack (48x48 tokens, d=512, L=8, k=2) against the full oracle."""
     cfg = W.CONFIGS["stack48_bf16"]
