@@ -35,6 +35,14 @@ Readings taken where the pages are silent (also listed in the design doc)
        blending before or after the out-projection and residual is the same map.
     R8 the transition at layer k merges the per-tile states with the same w-bar
        (Fig. 3b); each global token keeps its own tile's state.
+    R12 partial sharing (Tab. 1 top: from layer k on each tile keeps its own
+       residual stream and only the listed operations are shared; attention always
+       runs per tile): a shared operation takes, for each grid token, the w-bar
+       blend of its tiles' inputs (the merge of R8; a tile's global token keeps its
+       own row) and runs once per token.  Its result serves every tile covering
+       the token: shared q/k/v feed each tile's attention through the tile's rows;
+       the shared out-projection's and MLP's outputs are added to every tile's copy
+       of the token.
 """
 
 import math
@@ -149,11 +157,16 @@ def tile_attention(q, k, v, slot_pos, m: Model):
     return attention(q, k, v)
 
 
-def mlp_residual(x, p, m: Model):
-    """x + W_2 GELU(W_1 LN2(x) + b_1) + b_2, once per row."""
+def mlp_out(x, p, m: Model):
+    """W_2 GELU(W_1 LN2(x) + b_1) + b_2, once per row."""
     h = layer_norm(x, p["ln2_g"], p["ln2_b"], m.eps_ln)
     h = gelu(linear(h, p["w_1"], p["b_1"], m))
-    return x + linear(h, p["w_2"], p["b_2"], m)
+    return linear(h, p["w_2"], p["b_2"], m)
+
+
+def mlp_residual(x, p, m: Model):
+    """x + W_2 GELU(W_1 LN2(x) + b_1) + b_2, once per row."""
+    return x + mlp_out(x, p, m)
 
 
 # ---------------------------------------------------------------------------
@@ -225,6 +238,48 @@ def block_shared(S, p, m: Model, plan):
     A = merge(O, plan)
     S = S + linear(A, p["w_o"], p["b_o"], m)
     return mlp_residual(S, p, m)
+
+
+SHARED_OPS = ("qkv", "out", "mlp")
+
+
+def block_partial(X, p, m: Model, plan, shared):
+    """One layer on per-tile states X [T, N, d] in which only the operations named
+    in `shared` (of "qkv", "out", "mlp") run once per token (Tab. 1 top, R12).
+
+    "qkv": Norm1, QKV and QK-RMSNorm on the merge of X, then each tile attends over
+    its rows of the shared q/k/v (RoPE per tile, as released).  "out": the tiles'
+    attention outputs are blended and projected once per token, and the result is
+    added to every tile's copy.  "mlp": the MLP runs on the merge of X after the
+    attention sublayer, and its output is added to every tile's copy.  Everything
+    else runs per tile as in block_tiled.
+    """
+    shared = set(shared)
+    if not shared <= set(SHARED_OPS):
+        raise ValueError(f"unknown shared operations {shared - set(SHARED_OPS)}")
+    T, N, U = plan.T, plan.N, plan.U
+    X = np.asarray(X, np.float64).copy()
+    O = np.empty((T, N, m.d), dtype=np.float64)
+    if "qkv" in shared:
+        q, k, v = qkv_project(merge(X, plan), p, m)
+        for t in range(T):
+            rows = np.concatenate([[U + t], plan.tile_tok[t]])
+            O[t] = tile_attention(q[rows], k[rows], v[rows], plan.slot_pos, m)
+    else:
+        for t in range(T):
+            q, k, v = qkv_project(X[t], p, m)
+            O[t] = tile_attention(q, k, v, plan.slot_pos, m)
+    if "out" in shared:
+        X = X + gather(linear(merge(O, plan), p["w_o"], p["b_o"], m), plan)
+    else:
+        for t in range(T):
+            X[t] = X[t] + linear(O[t], p["w_o"], p["b_o"], m)
+    if "mlp" in shared:
+        X = X + gather(mlp_out(merge(X, plan), p, m), plan)
+    else:
+        for t in range(T):
+            X[t] = mlp_residual(X[t], p, m)
+    return X
 
 
 def decode_stack(S0, G0, layers, m: Model, plan, k: int):

@@ -288,3 +288,60 @@ def test_elementary_ops_against_library():
     np.testing.assert_allclose(Lo.rms_norm(x, g, 1e-6),
                                Fn.rms_norm(torch.from_numpy(x), (48,), torch.from_numpy(g), eps=1e-6).numpy(),
                                atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# partial sharing (Tab. 1 top, reading R12)
+# ---------------------------------------------------------------------------
+
+_PARTIAL_CFG = W.small_config(grid=(2, 9, 11), win=(2, 5, 6), stride=(1, 3, 4), d=32, heads=2, mlp=48,
+                              dtype="f32")
+
+
+def test_partial_sharing_nothing_shared_is_the_per_tile_layer():
+    m = _model(_PARTIAL_CFG)
+    p, S, layers = _setup(_PARTIAL_CFG, seed=11)
+    X = Lo.gather(S, p)
+    X = X + 0.1 * np.random.default_rng(1).standard_normal(X.shape)   # tiles disagree on overlap tokens
+    np.testing.assert_array_equal(Lo.block_partial(X, layers[0], m, p, ()), Lo.block_tiled(X, layers[0], m, p))
+
+
+@pytest.mark.parametrize("shared", [("out",), ("qkv", "out"), ("qkv", "out", "mlp"), ("out", "mlp")])
+def test_partial_sharing_on_identical_copies_is_the_shared_layer(shared):
+    """Tab. 1's footnote: with the out-projection shared, identical per-tile states stay
+    identical, so from gathered copies the layer equals the TileShare shared layer
+    (every tile holds the shared result for each of its tokens)."""
+    m = _model(_PARTIAL_CFG)
+    p, S, layers = _setup(_PARTIAL_CFG, seed=12)
+    got = Lo.block_partial(Lo.gather(S, p), layers[0], m, p, shared)
+    want = Lo.gather(Lo.block_shared(S, layers[0], m, p), p)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_partial_sharing_mlp_only_merges_to_the_shared_layer():
+    """MLP only, from identical copies: the tiles' attention outputs differ, but the
+    MLP input is their blend, which by linearity of the out-projection is the shared
+    layer's state after attention; merging the result gives the shared layer."""
+    m = _model(_PARTIAL_CFG)
+    p, S, layers = _setup(_PARTIAL_CFG, seed=13)
+    X = Lo.block_partial(Lo.gather(S, p), layers[0], m, p, ("mlp",))
+    np.testing.assert_allclose(Lo.merge(X, p), Lo.block_shared(S, layers[0], m, p), rtol=0, atol=1e-12)
+
+
+def test_partial_sharing_qkv_only_from_distinct_copies():
+    """QKV only, on per-tile states that disagree: q/k/v come from the merged state and
+    are identical for every copy of a token, while the out-projection and MLP stay
+    per tile.  Checked against a per-tile loop written out here."""
+    m = _model(_PARTIAL_CFG)
+    p, S, layers = _setup(_PARTIAL_CFG, seed=14)
+    prm = layers[0]
+    X = Lo.gather(S, p) + 0.1 * np.random.default_rng(2).standard_normal((p.T, p.N, m.d))
+    Sm = Lo.merge(X, p)
+    q, k, v = Lo.qkv_project(Sm, prm, m)
+    want = np.empty_like(X)
+    for t in range(p.T):
+        rows = np.concatenate([[p.U + t], p.tile_tok[t]])
+        o = Lo.tile_attention(q[rows], k[rows], v[rows], p.slot_pos, m)
+        x = X[t] + o @ prm["w_o"].T + prm["b_o"]
+        want[t] = Lo.mlp_residual(x, prm, m)
+    np.testing.assert_allclose(Lo.block_partial(X, prm, m, p, ("qkv",)), want, rtol=0, atol=1e-12)
