@@ -59,6 +59,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--trace-steps", type=int, default=20)
+    ap.add_argument("--shared-ops", default=None,
+                    help="partial sharing from layer k on: comma list of qkv,out,mlp ('none': nothing shared) run "
+                         "once per token on per-tile residual streams; default: the TileShare shared layer")
     ap.add_argument("--blend", default="ramp", choices=["ramp", "hard"],
                     help="blend rule of the plan: normalised linear ramp (default) or hard stitching")
     return ap.parse_args()
@@ -234,7 +237,21 @@ def run_tileshare(args, rank, world, local):
     ws = torch.empty(B.workspace_size(plan, m, 0, 0), dtype=torch.uint8, device=dev)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
 
+    share = None
+    if args.shared_ops is not None:
+        names = [x for x in args.shared_ops.split(",") if x and x != "none"]
+        bits = {"qkv": B.TS_SHARE_QKV, "out": B.TS_SHARE_OUT, "mlp": B.TS_SHARE_MLP}
+        share = 0
+        for x in names:
+            share |= bits[x]
+
     def part_tiled(kk=k):
+        if share is not None:
+            # partial sharing keeps per-tile states throughout; merged once at the end
+            B.gather_tiles(plan, m, S0d, G0d, X)
+            for li in range(kk):
+                B.block_tiled(plan, m, wl[li], X, ws)
+            return
         if kk > 0:
             B.gather_tiles(plan, m, S0d, G0d, X)
             for li in range(kk):
@@ -249,10 +266,15 @@ def run_tileshare(args, rank, world, local):
 
     def part_shared():
         for li in range(k, L):
-            B.block_shared(plan, m, wl[li], S, ws)
+            if share is not None:
+                B.block_partial(plan, m, wl[li], share, X, ws)
+            else:
+                B.block_shared(plan, m, wl[li], S, ws)
 
     def part_out():
-        if k < L:
+        if share is not None:
+            B.op_merge(plan, m, X, U, out)
+        elif k < L:
             out.copy_(S[:U])
 
     # warm-up (eager: configures every kernel), then capture
@@ -351,14 +373,22 @@ def run_tileshare(args, rank, world, local):
 
     # e2e: one shared layer through the public call with pinned host buffers
     Ke = min(K, 200)
-    S_host = torch.cat([S0d, G0d]).cpu().pin_memory()
+    if share is not None:
+        # partial sharing: the per-tile state [T * N, d] goes in and out
+        B.gather_tiles(plan, m, S0d, G0d, X)
+        S_host = X.cpu().pin_memory()
+    else:
+        S_host = torch.cat([S0d, G0d]).cpu().pin_memory()
     S_back = torch.empty_like(S_host).pin_memory()
-    Sd = torch.empty((U + T, d), dtype=dt, device=dev)
+    Sd = torch.empty(tuple(S_host.shape), dtype=dt, device=dev)
     eev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Ke)]
 
     def e2e_step():
         Sd.copy_(S_host, non_blocking=True)
-        B.block_shared(plan, m, wl[min(k, L - 1)], Sd, ws)
+        if share is not None:
+            B.block_partial(plan, m, wl[min(k, L - 1)], share, Sd, ws)
+        else:
+            B.block_shared(plan, m, wl[min(k, L - 1)], Sd, ws)
         S_back.copy_(Sd, non_blocking=True)
 
     run_e = e2e_step
@@ -384,7 +414,7 @@ def run_tileshare(args, rank, world, local):
     e2e_ms = float(np.mean([a.elapsed_time(b) for a, b in eev]))
     (e2e_max,) = max_over_ranks([e2e_ms], world)
     e2e_value = replica_rate(U, world, e2e_max)
-    state_bytes = (U + T) * d * S_host.element_size()
+    state_bytes = S_host.numel() * S_host.element_size()
 
     # traced pass: per-kernel times of the same step, eagerly launched
     B.trace_begin(100000)
@@ -442,6 +472,12 @@ def run_tileshare(args, rank, world, local):
 
     ft = flops_layer(T * N, T, N, d, f)
     fs = flops_layer(U + T, T, N, d, f)
+    if share is not None:
+        # partial sharing: each shared operation on U + T rows, the others on T * N rows
+        def rows(bit):
+            return U + T if share & bit else T * N
+        fs = (2.0 * 3 * d * d * rows(B.TS_SHARE_QKV) + 2.0 * d * d * rows(B.TS_SHARE_OUT) +
+              4.0 * d * f * rows(B.TS_SHARE_MLP) + 4.0 * T * N * N * d)
     flop_ratio = (k * ft + (L - k) * fs) / (L * ft)
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
@@ -449,7 +485,9 @@ def run_tileshare(args, rank, world, local):
         "vs_baseline": None, "dtype": {"bf16": "bf16", "f32": "f32", "fp8": "e4m3"}[cfg.dtype],
         "data": "synthetic (seeded N(0,1) states, N(0,0.02) weights, random init)",
         "config": {"workload": f"{cfg.name}: {cfg.note}", "grid": list(cfg.grid), "window": list(cfg.win),
-                   "stride": list(cfg.stride), "blend": args.blend, "L": L, "k": k, "unique_tokens": U, "tiles": T, "rows_per_tile": N,
+                   "stride": list(cfg.stride), "blend": args.blend,
+                   "shared_ops": (args.shared_ops or "none") if share is not None else "TileShare shared layer",
+                   "L": L, "k": k, "unique_tokens": U, "tiles": T, "rows_per_tile": N,
                    "l2": "flushed before every step (512 MiB write, outside the timed events)",
                    "launch": "CUDA graphs of the public calls" if use_graph else "eager public calls",
                    "parallelism": f"replicas x{world} (one image per GPU)"},
@@ -460,7 +498,7 @@ def run_tileshare(args, rank, world, local):
         "flop_ratio": round(flop_ratio, 4),
         "speedup_bar": round(0.85 / flop_ratio, 4),
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": state_bytes,
-                "d2h_bytes_per_step": state_bytes, "call": "ts_block_shared with pinned host state in/out" +
+                "d2h_bytes_per_step": state_bytes, "call": ("ts_block_partial" if share is not None else "ts_block_shared") + " with pinned host state in/out" +
                         (", copies and call replayed as one CUDA graph per step" if use_graph else "")},
         "gpu_launches": int(gpu_launches),
         "roofline": roofline,

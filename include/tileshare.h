@@ -213,6 +213,27 @@ ts_status ts_gather_tiles(ts_plan_t plan, const ts_model_desc* model, const void
 ts_status ts_quantize_rows_e4m3(const void* x, int rows, int cols, void* q, float* scale,
                                 void* stream);
 
+/* Operations a partially shared layer runs once per token (bit mask). */
+typedef enum {
+  TS_SHARE_QKV = 1,   /* Norm1, QKV projection, QK-RMSNorm                    */
+  TS_SHARE_OUT = 2,   /* out-projection (of the blended attention outputs)     */
+  TS_SHARE_MLP = 4    /* Norm2 and MLP                                         */
+} ts_shared_op;
+
+/* One layer with per-tile residual streams in which only the operations in
+   shared_ops run once per token ([TileShare] Tab. 1 top: from layer k on, each
+   tile keeps its own residual stream and only the listed operations are shared;
+   attention always runs per tile).  In place on X [T, N, d] as ts_block_tiled.
+   A shared operation takes, for each grid token, the w-bar blend of its tiles'
+   inputs (each tile's global token keeps its own row) and runs once per token;
+   shared q/k/v feed every tile's attention through the tile's rows, and the
+   shared out-projection's and MLP's outputs are added to every tile's copy of the
+   token.  shared_ops = 0 is ts_block_tiled; from identical per-tile copies, any set
+   with TS_SHARE_OUT gives the shared layer's result in every copy.  Workspace as
+   for ts_block_tiled. */
+ts_status ts_block_partial(ts_plan_t plan, const ts_model_desc* model, const ts_layer_weights* w,
+                           unsigned shared_ops, void* X, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Device-side status word of the library on the current device: 0 if no kernel
    check or bounded wait has failed since the last call, else a TS_ERR_* code.
    Synchronises the device and clears the word. */

@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libtileshare.so")
 TS_OK = 0
 TS_BLEND_LINEAR_RAMP = 0
 TS_BLEND_HARD_STITCH = 1
+TS_SHARE_QKV, TS_SHARE_OUT, TS_SHARE_MLP = 1, 2, 4
 TS_F32, TS_BF16, TS_FP8_E4M3 = 0, 1, 2
 TS_ROWS_SHARED, TS_ROWS_TILED = 0, 1
 TS_EPI_BIAS, TS_EPI_BIAS_GELU, TS_EPI_BIAS_RESID = 0, 1, 2
@@ -79,6 +80,8 @@ _SIGS = {
     "ts_block_tiled": [_cp, ctypes.POINTER(ModelDesc), ctypes.POINTER(LayerWeights), _cp, _cp, ctypes.c_size_t, _cp],
     "ts_block_shared": [_cp, ctypes.POINTER(ModelDesc), ctypes.POINTER(LayerWeights), _cp, _cp, ctypes.c_size_t, _cp],
     "ts_block_shared_noalloc": [_cp, ctypes.POINTER(ModelDesc), ctypes.POINTER(LayerWeights), _cp, _cp],
+    "ts_block_partial": [_cp, ctypes.POINTER(ModelDesc), ctypes.POINTER(LayerWeights), ctypes.c_uint, _cp, _cp,
+                         ctypes.c_size_t, _cp],
     "ts_decode_stack": [_cp, ctypes.POINTER(ModelDesc), ctypes.POINTER(LayerWeights), ctypes.c_int, ctypes.c_int,
                         _cp, _cp, _cp, _cp, ctypes.c_size_t, _cp],
     "ts_quantize_rows_e4m3": [_cp, ctypes.c_int, ctypes.c_int, _cp, _cp, _cp],
@@ -214,6 +217,13 @@ def block_tiled(plan, model, weights, X, ws, stream=None):
 def block_shared(plan, model, weights, S, ws, stream=None):
     _check("ts_block_shared", lib().ts_block_shared(plan.handle, ctypes.byref(model), ctypes.byref(weights), _ptr(S),
                                                     _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def block_partial(plan, model, weights, shared_ops, X, ws, stream=None):
+    """ts_block_partial: per-tile states X, the TS_SHARE_* operations in shared_ops once per token."""
+    _check("ts_block_partial", lib().ts_block_partial(plan.handle, ctypes.byref(model), ctypes.byref(weights),
+                                                      int(shared_ops), _ptr(X), _ptr(ws),
+                                                      ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def block_shared_noalloc(plan, model, weights, S, stream=None):

@@ -316,6 +316,33 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint8_t* __restr
 }
 
 // ---------------------------------------------------------------------------
+// Partial sharing ([TileShare] Tab. 1 top): a per-token result R [U + T, d] of a
+// shared operation is added to every tile's copy of the token, X[r] += R[rowmap[r]]
+// for the T * N per-tile rows (row t*N of tile t takes R[U + t]).  fp32 add, one
+// warp per row, 16-byte vectors; every X row is written by one warp.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) scatter_add_rows_kernel(const T* __restrict__ R, const int* __restrict__ rowmap,
+                                                               int nrows, int d, T* __restrict__ X) {
+  pdl_wait();
+  pdl_trigger();
+  constexpr int E = Vec<T>::E;
+  const int lane = threadIdx.x & 31;
+  const size_t r = static_cast<size_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= static_cast<size_t>(nrows)) return;
+  const T* src = R + static_cast<size_t>(__ldg(rowmap + r)) * d;
+  T* dst = X + r * d;
+  for (int c = lane * E; c < d; c += 32 * E) {
+    float a[E], b[E];
+    Vec<T>::load(dst + c, a);
+    Vec<T>::load(src + c, b);
+#pragma unroll
+    for (int e = 0; e < E; ++e) a[e] += b[e];
+    Vec<T>::store(dst + c, a);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Per-row e4m3 quantisation of a bf16 matrix: scale = absmax / 448 (1 if zero),
 // q = e4m3(x / scale), nearest-even, saturating.  cols % 8 == 0.
 // ---------------------------------------------------------------------------

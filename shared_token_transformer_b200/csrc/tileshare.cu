@@ -303,6 +303,7 @@ struct Workspace {
   void* X;       // [T*N, d]  per-tile state (stack)
   void* S;       // [U+T, d]  shared state (stack)
   float2* rope;  // RoPE cos/sin table (rope_table_entries)
+  void* sm;      // [U+T, d]  partial sharing: merged per-tile state, then a per-token result
   size_t bytes;
 };
 
@@ -355,6 +356,7 @@ static Workspace layout(const ts_plan_s* p, const ts_model_desc* m, bool stack, 
     w.S = take(Ms * d * e);
   }
   w.rope = reinterpret_cast<float2*>(take(rope_table_entries(p, m) * sizeof(float2)));
+  w.sm = take(Ms * d * e);
   w.bytes = off;
   return w;
 }
@@ -782,6 +784,64 @@ static ts_status run_gather(const ts_plan_s* p, const ts_model_desc* m, const vo
   return trace_post(st, "gather_rows");
 }
 
+// X[r] += R[rowmap[r]] over the T * N per-tile rows (partial sharing)
+static ts_status run_scatter_add(const ts_plan_s* p, const ts_model_desc* m, const void* R, void* X, cudaStream_t st) {
+  const int nrows = p->T * p->N;
+  const int d = m->d;
+  const double e = esize(m->dtype);
+  set_work("scatter_add", 0.0, 3.0 * nrows * static_cast<double>(d) * e);
+  trace_pre(st);
+  if (m->dtype == TS_F32)
+    launch_pdl(ts::scatter_add_rows_kernel<float>, dim3(rows_grid(nrows)), dim3(256), 0, st,
+               static_cast<const float*>(R), static_cast<const int*>(p->d_rowmap), nrows, d, static_cast<float*>(X));
+  else
+    launch_pdl(ts::scatter_add_rows_kernel<bf16>, dim3(rows_grid(nrows)), dim3(256), 0, st,
+               static_cast<const bf16*>(R), static_cast<const int*>(p->d_rowmap), nrows, d, static_cast<bf16*>(X));
+  return trace_post(st, "scatter_add");
+}
+
+// out = att W_o^T + b_o (no residual): the out-projection of a shared operation
+static ts_status run_out_bias(const ts_model_desc* m, const ts_layer_weights* w, const void* att, bool att_quantised,
+                              int rows, void* out, const Workspace& ws, cudaStream_t st) {
+  const int d = m->d;
+  if (m->dtype == TS_F32)
+    return run_gemm_f32("gemm_out", ts::EPI_BIAS, static_cast<const float*>(att), static_cast<const float*>(w->w_o), rows, d, d,
+                        w->b_o, static_cast<float*>(out), st);
+  if (m->dtype == TS_FP8_E4M3) {
+    if (!att_quantised) TS_TRY(run_quantize(att, rows, d, ws.q8, ws.qs, st));
+    return run_gemm_tc("gemm_out", m, ts::EPI_BIAS, ws.q8, ws.qs, w->w_o, w->s_o, rows, d, d, w->b_o, static_cast<bf16*>(out),
+                       nullptr, nullptr, st);
+  }
+  return run_gemm_tc("gemm_out", m, ts::EPI_BIAS, att, nullptr, w->w_o, nullptr, rows, d, d, w->b_o, static_cast<bf16*>(out),
+                     nullptr, nullptr, st);
+}
+
+// out = W2 GELU(W1 LN2(in) + b1) + b2 (no residual): the MLP of a shared operation
+static ts_status run_mlp_out(const ts_model_desc* m, const ts_layer_weights* w, int rows, const void* in, void* out,
+                             const Workspace& ws, cudaStream_t st) {
+  const int d = m->d, f = m->mlp;
+  if (m->dtype == TS_F32) {
+    TS_TRY(run_layernorm(m, in, rows, w->ln2_g, w->ln2_b, ws.xn, nullptr, nullptr, st));
+    TS_TRY(run_gemm_f32("gemm_up", ts::EPI_GELU, static_cast<const float*>(ws.xn), static_cast<const float*>(w->w_1), rows, f, d,
+                        w->b_1, static_cast<float*>(ws.h), st));
+    return run_gemm_f32("gemm_down", ts::EPI_BIAS, static_cast<const float*>(ws.h), static_cast<const float*>(w->w_2), rows, d, f,
+                        w->b_2, static_cast<float*>(out), st);
+  }
+  if (m->dtype == TS_FP8_E4M3) {
+    TS_TRY(run_layernorm(m, in, rows, w->ln2_g, w->ln2_b, nullptr, ws.q8, ws.qs, st));
+    TS_TRY(run_gemm_tc("gemm_up", m, ts::EPI_GELU, ws.q8, ws.qs, w->w_1, w->s_1, rows, f, d, w->b_1, static_cast<bf16*>(ws.h),
+                       nullptr, nullptr, st));
+    TS_TRY(run_quantize(ws.h, rows, f, ws.q8, ws.qs, st));
+    return run_gemm_tc("gemm_down", m, ts::EPI_BIAS, ws.q8, ws.qs, w->w_2, w->s_2, rows, d, f, w->b_2, static_cast<bf16*>(out),
+                       nullptr, nullptr, st);
+  }
+  TS_TRY(run_layernorm(m, in, rows, w->ln2_g, w->ln2_b, ws.xn, nullptr, nullptr, st));
+  TS_TRY(run_gemm_tc("gemm_up", m, ts::EPI_GELU, ws.xn, nullptr, w->w_1, nullptr, rows, f, d, w->b_1, static_cast<bf16*>(ws.h),
+                     nullptr, nullptr, st));
+  return run_gemm_tc("gemm_down", m, ts::EPI_BIAS, ws.h, nullptr, w->w_2, nullptr, rows, d, f, w->b_2, static_cast<bf16*>(out),
+                     nullptr, nullptr, st);
+}
+
 // ============================================================================
 // layers
 // ============================================================================
@@ -803,6 +863,36 @@ static ts_status layer_shared(const ts_plan_s* p, const ts_model_desc* m, const 
   TS_TRY(run_merge("blend", p, m, ws.o, rows, q ? nullptr : ws.a, q ? ws.q8 : nullptr, q ? ws.qs : nullptr, st));
   TS_TRY(run_out_proj(m, w, ws.a, q, rows, S, ws, st));
   return run_mlp(m, w, rows, S, ws, st);
+}
+
+// Partial sharing ([TileShare] Tab. 1 top): per-tile residual streams X, the
+// operations in `ops` once per token on the merged inputs, their results used by
+// (QKV) or added to (out-projection, MLP) every tile's copy of the token.
+static ts_status layer_partial(const ts_plan_s* p, const ts_model_desc* m, const ts_layer_weights* w, unsigned ops,
+                               void* X, const Workspace& ws, cudaStream_t st) {
+  const int rows_t = p->T * p->N, rows_s = p->U + p->T;
+  const bool q8 = m->dtype == TS_FP8_E4M3;
+  if (ops & TS_SHARE_QKV) {
+    TS_TRY(run_merge("merge", p, m, X, rows_s, ws.sm, nullptr, nullptr, st));
+    TS_TRY(run_qkv(p, m, w, true, ws.sm, ws.qkv, ws, st));
+    TS_TRY(run_attention(p, m, true, ws.qkv, ws.o, st));
+  } else {
+    TS_TRY(run_qkv(p, m, w, false, X, ws.qkv, ws, st));
+    TS_TRY(run_attention(p, m, false, ws.qkv, ws.o, st));
+  }
+  if (ops & TS_SHARE_OUT) {
+    TS_TRY(run_merge("blend", p, m, ws.o, rows_s, q8 ? nullptr : ws.a, q8 ? ws.q8 : nullptr, q8 ? ws.qs : nullptr, st));
+    TS_TRY(run_out_bias(m, w, ws.a, q8, rows_s, ws.sm, ws, st));
+    TS_TRY(run_scatter_add(p, m, ws.sm, X, st));
+  } else {
+    TS_TRY(run_out_proj(m, w, ws.o, false, rows_t, X, ws, st));
+  }
+  if (ops & TS_SHARE_MLP) {
+    TS_TRY(run_merge("merge", p, m, X, rows_s, ws.sm, nullptr, nullptr, st));
+    TS_TRY(run_mlp_out(m, w, rows_s, ws.sm, ws.a, ws, st));
+    return run_scatter_add(p, m, ws.a, X, st);
+  }
+  return run_mlp(m, w, rows_t, X, ws, st);
 }
 
 static ts_status check_ws(const ts_plan_s* p, const ts_model_desc* m, bool stack, void* ws, size_t ws_bytes,
@@ -1024,6 +1114,19 @@ ts_status ts_block_shared(ts_plan_t p, const ts_model_desc* m, const ts_layer_we
   Workspace W;
   TS_TRY(check_ws(p, m, false, ws, ws_bytes, &W));
   return layer_shared(p, m, w, S, W, static_cast<cudaStream_t>(stream));
+}
+
+ts_status ts_block_partial(ts_plan_t p, const ts_model_desc* m, const ts_layer_weights* w, unsigned shared_ops,
+                           void* X, void* ws, size_t ws_bytes, void* stream) {
+  TS_TRY(check_plan(p));
+  TS_TRY(check_model(m));
+  TS_TRY(check_weights(m, w));
+  if (shared_ops & ~static_cast<unsigned>(TS_SHARE_QKV | TS_SHARE_OUT | TS_SHARE_MLP))
+    return fail(TS_ERR_INVALID_ARG, "unknown shared operations 0x%x", shared_ops);
+  if (!X || !aligned16(X)) return fail(TS_ERR_INVALID_ARG, "X must be a 16-byte aligned device pointer");
+  Workspace W;
+  TS_TRY(check_ws(p, m, false, ws, ws_bytes, &W));
+  return layer_partial(p, m, w, shared_ops, X, W, static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------

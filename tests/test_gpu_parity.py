@@ -294,6 +294,38 @@ def test_hard_stitch_shared_layer_and_stack(cfg):
     assert rel_l2(got, want) < _tol(cfg)
 
 
+_SHARE = {"qkv": B.TS_SHARE_QKV, "out": B.TS_SHARE_OUT, "mlp": B.TS_SHARE_MLP}
+
+
+@pytest.mark.parametrize("cfg", [SMALL, VOL, VIT14, SMALL_FP8], ids=lambda c: c.name)
+@pytest.mark.parametrize("shared", [(), ("qkv",), ("out",), ("mlp",), ("qkv", "mlp"), ("qkv", "out", "mlp")],
+                         ids=lambda s: "+".join(s) or "none")
+def test_block_partial(cfg, shared):
+    """Partial sharing against the oracle, from per-tile states that disagree on
+    their overlap tokens (gathered copies plus seeded noise)."""
+    c = case(cfg)
+    op = c.oplan
+    X = OL.gather(c.S, op) + 0.1 * np.random.default_rng(21).standard_normal((op.T, op.N, cfg.d))
+    X = W.round_to(X, cfg.dtype if cfg.dtype != "fp8" else "bf16")
+    Xd = dev(X.reshape(op.T * op.N, cfg.d), c.dt)
+    ops = 0
+    for s in shared:
+        ops |= _SHARE[s]
+    B.block_partial(c.plan, c.m, c.wlist[0], ops, Xd, c.workspace())
+    want = OL.block_partial(X, c.layers[0], c.om, op, shared)
+    got = host(Xd).reshape(op.T, op.N, cfg.d)
+    assert rel_l2(got, want) < _tol(cfg)
+    assert rel_l2(got - X, want - X) < 3 * _tol(cfg)
+
+
+def test_block_partial_rejects_unknown_operations():
+    c = case(SMALL)
+    Xd = torch.zeros((c.oplan.T * c.oplan.N, SMALL.d), dtype=c.dt, device="cuda")
+    with pytest.raises(B.TileShareError) as e:
+        B.block_partial(c.plan, c.m, c.wlist[0], 8, Xd, c.workspace())
+    assert e.value.status == 1
+
+
 def test_stack48_bf16_full():
     """The benchmark stack (48x48 tokens, d=512, L=8, k=2) against the full oracle."""
     cfg = W.CONFIGS["stack48_bf16"]
