@@ -6,28 +6,29 @@ TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).
 layers relative to per-tile layers; Tab. S6 notes that per-token work shrinks
 with the token count while attention is unchanged.  Counted here: the four
 linear layers (2 FLOPs per multiply-add) and the two attention contractions;
-norms, softmax, GELU and the blend are not counted.
+norms, softmax, GELU / SiLU gating and the blend are not counted.
 """
 
 
-def linear_flops_per_row(d: int, f: int) -> int:
-    return 2 * (3 * d * d + d * d + 2 * d * f)
+def linear_flops_per_row(d: int, f: int, gated: bool = False) -> int:
+    """QKV, out-projection, MLP up (2f rows when gated: SwiGLU gate and up) and down."""
+    return 2 * (3 * d * d + d * d + (3 if gated else 2) * d * f)
 
 
 def attention_flops(T: int, N: int, d: int) -> int:
     return 4 * T * N * N * d
 
 
-def tiled_layer_flops(T: int, N: int, d: int, f: int) -> int:
-    return T * N * linear_flops_per_row(d, f) + attention_flops(T, N, d)
+def tiled_layer_flops(T: int, N: int, d: int, f: int, gated: bool = False) -> int:
+    return T * N * linear_flops_per_row(d, f, gated) + attention_flops(T, N, d)
 
 
-def shared_layer_flops(U: int, T: int, N: int, d: int, f: int) -> int:
-    return (U + T) * linear_flops_per_row(d, f) + attention_flops(T, N, d)
+def shared_layer_flops(U: int, T: int, N: int, d: int, f: int, gated: bool = False) -> int:
+    return (U + T) * linear_flops_per_row(d, f, gated) + attention_flops(T, N, d)
 
 
-def stack_flop_ratio(U: int, T: int, N: int, d: int, f: int, L: int, k: int) -> float:
+def stack_flop_ratio(U: int, T: int, N: int, d: int, f: int, L: int, k: int, gated: bool = False) -> float:
     """FLOPs of TileShare-k over FLOPs of L per-tile layers."""
-    tiled = tiled_layer_flops(T, N, d, f)
-    shared = shared_layer_flops(U, T, N, d, f)
+    tiled = tiled_layer_flops(T, N, d, f, gated)
+    shared = shared_layer_flops(U, T, N, d, f, gated)
     return (k * tiled + (L - k) * shared) / (L * tiled)

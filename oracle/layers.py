@@ -35,6 +35,11 @@ Readings taken where the pages are silent (also listed in the design doc)
        blending before or after the out-projection and residual is the same map.
     R8 the transition at layer k merges the per-tile states with the same w-bar
        (Fig. 3b); each global token keeps its own tile's state.
+    R13 block flavour "rms_swiglu" (Tab. S6 profiles a block with "RMSNorm +
+       residual" and a "SwiGLU gate"): Norm1 and Norm2 are RMSNorm with a gain and
+       no bias (eps_ln); the MLP is  W_2 (silu(W_g h + b_g) * (W_u h + b_u)) + b_2
+       with silu(z) = z / (1 + exp(-z)), where w_1 = [W_g; W_u] stacks the f gate
+       rows above the f up rows and b_1 = [b_g; b_u].  Everything else as in R4.
     R12 partial sharing (Tab. 1 top: from layer k on each tile keeps its own
        residual stream and only the listed operations are shared; attention always
        runs per tile): a shared operation takes, for each grid token, the w-bar
@@ -64,6 +69,7 @@ class Model:
     eps_qk: float = 1e-6
     rope_base: float = 10000.0
     fp8: bool = False         # e4m3 GEMMs with per-channel / per-token scales
+    block: str = "ln_gelu"    # "ln_gelu" (R4) or "rms_swiglu" (R13)
 
     @property
     def hd(self):
@@ -86,6 +92,19 @@ def rms_norm(x, g, eps):
 
 def gelu(x):
     return 0.5 * x * (1.0 + erf(x / math.sqrt(2.0)))
+
+
+def silu(x):
+    """z / (1 + exp(-z)); exp overflows to inf for z < -709, where the quotient is -0."""
+    with np.errstate(over="ignore"):
+        return x / (1.0 + np.exp(-x))
+
+
+def block_norm(x, g, b, m):
+    """Norm1 / Norm2 of the block: LayerNorm (R4) or RMSNorm without bias (R13)."""
+    if m.block == "rms_swiglu":
+        return rms_norm(x, g, m.eps_ln)
+    return layer_norm(x, g, b, m.eps_ln)
 
 
 def rope(x, pos, m: Model):
@@ -134,7 +153,7 @@ def attention(q, k, v):
 def qkv_project(x, p, m: Model):
     """Norm1, QKV projection and QK-RMSNorm of rows x [n, d] -> q, k, v [n, heads, hd]."""
     n = x.shape[0]
-    h = layer_norm(x, p["ln1_g"], p["ln1_b"], m.eps_ln)
+    h = block_norm(x, p["ln1_g"], p["ln1_b"], m)
     qkv = linear(h, p["w_qkv"], p["b_qkv"], m)
     q = qkv[:, 0 * m.d:1 * m.d].reshape(n, m.heads, m.hd)
     k = qkv[:, 1 * m.d:2 * m.d].reshape(n, m.heads, m.hd)
@@ -158,9 +177,13 @@ def tile_attention(q, k, v, slot_pos, m: Model):
 
 
 def mlp_out(x, p, m: Model):
-    """W_2 GELU(W_1 LN2(x) + b_1) + b_2, once per row."""
-    h = layer_norm(x, p["ln2_g"], p["ln2_b"], m.eps_ln)
-    h = gelu(linear(h, p["w_1"], p["b_1"], m))
+    """W_2 GELU(W_1 LN2(x) + b_1) + b_2 (R4), or the SwiGLU MLP of R13, once per row."""
+    h = block_norm(x, p["ln2_g"], p["ln2_b"], m)
+    a = linear(h, p["w_1"], p["b_1"], m)
+    if m.block == "rms_swiglu":
+        h = silu(a[:, :m.mlp]) * a[:, m.mlp:]
+    else:
+        h = gelu(a)
     return linear(h, p["w_2"], p["b_2"], m)
 
 

@@ -36,6 +36,7 @@ class Config:
     rope_dims: tuple      # channels of the head dimension given to the (f, y, x) axes
     note: str = ""
     ks: tuple = field(default=())   # further k values the configuration compares
+    block: str = "ln_gelu"          # "ln_gelu" or "rms_swiglu" (MLP up of 2 x mlp rows: gate, then up)
 
     @property
     def hd(self):
@@ -78,12 +79,13 @@ CONFIGS = {
 
 
 def small_config(name="tiny", grid=(1, 11, 13), win=(1, 8, 8), stride=(1, 5, 6), d=128, heads=2, mlp=256,
-                 dtype="bf16", L=3, k=1, rope_dims=None):
+                 dtype="bf16", L=3, k=1, rope_dims=None, block="ln_gelu"):
     """A reduced configuration for fast parity tests (ragged tiles, several GEMM tiles)."""
     hd = d // heads
     if rope_dims is None:
         rope_dims = (0, hd // 2, hd // 2) if grid[0] == 1 else (hd // 4, 3 * hd // 8, 3 * hd // 8)
-    return Config(name, tuple(grid), tuple(win), tuple(stride), d, heads, mlp, dtype, L, k, tuple(rope_dims))
+    return Config(name, tuple(grid), tuple(win), tuple(stride), d, heads, mlp, dtype, L, k, tuple(rope_dims),
+                  block=block)
 
 
 # ---------------------------------------------------------------------------
@@ -125,24 +127,25 @@ class Draw:
         """One layer's parameters (dict of float64 arrays rounded to the working dtype)."""
         c = self.cfg
         d, f, hd = c.d, c.mlp, c.hd
+        f1 = 2 * f if c.block == "rms_swiglu" else f     # rows of w_1
         r = self.rng
         p = {
             "w_qkv": 0.02 * r.standard_normal((3 * d, d)),
             "w_o": 0.02 * r.standard_normal((d, d)),
-            "w_1": 0.02 * r.standard_normal((f, d)),
+            "w_1": 0.02 * r.standard_normal((f1, d)),
             "w_2": 0.02 * r.standard_normal((d, f)),
         }
         if self.affine:
             p.update({
                 "b_qkv": 0.1 * r.standard_normal(3 * d), "b_o": 0.1 * r.standard_normal(d),
-                "b_1": 0.1 * r.standard_normal(f), "b_2": 0.1 * r.standard_normal(d),
+                "b_1": 0.1 * r.standard_normal(f1), "b_2": 0.1 * r.standard_normal(d),
                 "ln1_g": 1 + 0.2 * r.standard_normal(d), "ln1_b": 0.1 * r.standard_normal(d),
                 "ln2_g": 1 + 0.2 * r.standard_normal(d), "ln2_b": 0.1 * r.standard_normal(d),
                 "q_g": 1 + 0.2 * r.standard_normal(hd), "k_g": 1 + 0.2 * r.standard_normal(hd),
             })
         else:
             p.update({
-                "b_qkv": np.zeros(3 * d), "b_o": np.zeros(d), "b_1": np.zeros(f), "b_2": np.zeros(d),
+                "b_qkv": np.zeros(3 * d), "b_o": np.zeros(d), "b_1": np.zeros(f1), "b_2": np.zeros(d),
                 "ln1_g": np.ones(d), "ln1_b": np.zeros(d), "ln2_g": np.ones(d), "ln2_b": np.zeros(d),
                 "q_g": np.ones(hd), "k_g": np.ones(hd),
             })

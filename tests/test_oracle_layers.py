@@ -12,6 +12,7 @@ Each test ties the vectorised float64 oracle to something other than itself:
     * RoPE invariants (relative positions, norms).
 """
 
+import dataclasses
 import math
 
 import numpy as np
@@ -25,7 +26,7 @@ from shared_token_transformer_b200 import workloads as W
 
 
 def _model(cfg):
-    return Lo.Model(cfg.d, cfg.heads, cfg.mlp, cfg.rope_dims)
+    return Lo.Model(cfg.d, cfg.heads, cfg.mlp, cfg.rope_dims, block=cfg.block)
 
 
 def _setup(cfg, seed=0, affine=True):
@@ -44,7 +45,12 @@ def _torch_block(x, prm, m, pos):
     t = {k: torch.from_numpy(np.asarray(v)) for k, v in prm.items()}
     x = torch.from_numpy(x)
     n, d, h, hd = x.shape[0], m.d, m.heads, m.hd
-    a = Fn.layer_norm(x, (d,), t["ln1_g"], t["ln1_b"], eps=m.eps_ln)
+    swiglu = m.block == "rms_swiglu"
+
+    def norm(z, g, b):
+        return Fn.rms_norm(z, (d,), g, eps=m.eps_ln) if swiglu else Fn.layer_norm(z, (d,), g, b, eps=m.eps_ln)
+
+    a = norm(x, t["ln1_g"], t["ln1_b"])
     qkv = Fn.linear(a, t["w_qkv"], t["b_qkv"])
     q, k, v = (qkv[:, i * d:(i + 1) * d].reshape(n, h, hd) for i in range(3))
     q = Fn.rms_norm(q, (hd,), t["q_g"], eps=m.eps_qk)
@@ -69,14 +75,21 @@ def _torch_block(x, prm, m, pos):
     o = Fn.scaled_dot_product_attention(q.transpose(0, 1), k.transpose(0, 1), v.transpose(0, 1))
     o = o.transpose(0, 1).reshape(n, d)
     x = x + Fn.linear(o, t["w_o"], t["b_o"])
-    a = Fn.layer_norm(x, (d,), t["ln2_g"], t["ln2_b"], eps=m.eps_ln)
-    x = x + Fn.linear(Fn.gelu(Fn.linear(a, t["w_1"], t["b_1"])), t["w_2"], t["b_2"])
+    a = norm(x, t["ln2_g"], t["ln2_b"])
+    up = Fn.linear(a, t["w_1"], t["b_1"])
+    if swiglu:
+        gate, val = up.chunk(2, dim=-1)          # gate rows first
+        hid = Fn.silu(gate) * val
+    else:
+        hid = Fn.gelu(up)
+    x = x + Fn.linear(hid, t["w_2"], t["b_2"])
     return x.numpy()
 
 
+@pytest.mark.parametrize("block", ["ln_gelu", "rms_swiglu"])
 @pytest.mark.parametrize("grid,rope", [((1, 6, 7), (0, 8, 8)), ((2, 3, 4), (4, 6, 6))])
-def test_single_tile_equals_library_block(grid, rope):
-    cfg = W.Config("one_tile", grid, grid, grid, 64, 4, 96, "f32", 1, 0, rope)
+def test_single_tile_equals_library_block(grid, rope, block):
+    cfg = W.Config("one_tile", grid, grid, grid, 64, 4, 96, "f32", 1, 0, rope, block=block)
     m = _model(cfg)
     p, S, layers = _setup(cfg)
     assert p.T == 1
@@ -97,10 +110,21 @@ def _loop_layer_shared(S, prm, m, p):
     U, T, d, h, hd = p.U, p.T, m.d, m.heads, m.hd
     n = S.shape[0]
 
+    swiglu = m.block == "rms_swiglu"
+
     def ln(row, g, b):
+        if swiglu:                      # RMSNorm: no centring, no bias
+            r = math.sqrt(sum(v * v for v in row) / d + m.eps_ln)
+            return [row[c] / r * g[c] for c in range(d)]
         mu = sum(row) / d
         var = sum((v - mu) ** 2 for v in row) / d
         return [(row[c] - mu) / math.sqrt(var + m.eps_ln) * g[c] + b[c] for c in range(d)]
+
+    def act(up):
+        if swiglu:                      # first half gates the second
+            f = len(up) // 2
+            return [up[c] / (1 + math.exp(-up[c])) * up[f + c] for c in range(f)]
+        return [gelu(z) for z in up]
 
     def lin(row, w, b):
         return [sum(row[c] * w[o][c] for c in range(len(row))) + b[o] for o in range(len(w))]
@@ -163,17 +187,18 @@ def _loop_layer_shared(S, prm, m, p):
     out = np.empty_like(S)
     for r in range(n):
         x = [S[r][c] + y for c, y in enumerate(lin(A[r], prm["w_o"], prm["b_o"]))]
-        hid = [gelu(z) for z in lin(ln(x, prm["ln2_g"], prm["ln2_b"]), prm["w_1"], prm["b_1"])]
+        hid = act(lin(ln(x, prm["ln2_g"], prm["ln2_b"]), prm["w_1"], prm["b_1"]))
         out[r] = [x[c] + y for c, y in enumerate(lin(hid, prm["w_2"], prm["b_2"]))]
     return out
 
 
-@pytest.mark.parametrize("grid,win,stride,rope", [
-    ((1, 5, 5), (1, 3, 3), (1, 2, 2), (0, 2, 2)),
-    ((2, 4, 5), (2, 3, 3), (1, 1, 2), (2, 2, 4)),
+@pytest.mark.parametrize("grid,win,stride,rope,block", [
+    ((1, 5, 5), (1, 3, 3), (1, 2, 2), (0, 2, 2), "ln_gelu"),
+    ((2, 4, 5), (2, 3, 3), (1, 1, 2), (2, 2, 4), "ln_gelu"),
+    ((1, 5, 5), (1, 3, 3), (1, 2, 2), (0, 2, 2), "rms_swiglu"),
 ])
-def test_shared_layer_brute_force(grid, win, stride, rope):
-    cfg = W.Config("bf", grid, win, stride, 16, 2, 24, "f32", 1, 0, rope)
+def test_shared_layer_brute_force(grid, win, stride, rope, block):
+    cfg = W.Config("bf", grid, win, stride, 16, 2, 24, "f32", 1, 0, rope, block=block)
     m = _model(cfg)
     p, S, layers = _setup(cfg, seed=3)
     prm = {k: (v.tolist() if v.ndim == 2 else list(v)) for k, v in layers[0].items()}
@@ -186,8 +211,9 @@ def test_shared_layer_brute_force(grid, win, stride, rope):
 # exactness statements of the pages
 # ---------------------------------------------------------------------------
 
-def test_no_overlap_shared_equals_tiled():
-    cfg = W.CONFIGS["vit16_nooverlap_fp32"]
+@pytest.mark.parametrize("block", ["ln_gelu", "rms_swiglu"])
+def test_no_overlap_shared_equals_tiled(block):
+    cfg = dataclasses.replace(W.CONFIGS["vit16_nooverlap_fp32"], block=block)
     m = _model(cfg)
     p, S, layers = _setup(cfg)
     got = Lo.block_shared(S, layers[0], m, p)
@@ -227,9 +253,10 @@ def test_identical_per_tile_states_stay_identical():
     np.testing.assert_allclose(Lo.merge(X, p), S, rtol=0, atol=1e-14)
 
 
-def test_stack_k_equals_L_is_tiled_decoding_blended_at_the_end():
+@pytest.mark.parametrize("block", ["ln_gelu", "rms_swiglu"])
+def test_stack_k_equals_L_is_tiled_decoding_blended_at_the_end(block):
     cfg = W.small_config(grid=(1, 10, 9), win=(1, 6, 5), stride=(1, 4, 3), d=32, heads=2, mlp=48,
-                         dtype="f32", L=3, k=3)
+                         dtype="f32", L=3, k=3, block=block)
     m = _model(cfg)
     p, S, layers = _setup(cfg, seed=11)
     got = Lo.decode_stack(S[:p.U], S[p.U:], layers, m, p, k=3)
@@ -345,3 +372,76 @@ def test_partial_sharing_qkv_only_from_distinct_copies():
         x = X[t] + o @ prm["w_o"].T + prm["b_o"]
         want[t] = Lo.mlp_residual(x, prm, m)
     np.testing.assert_allclose(Lo.block_partial(X, prm, m, p, ("qkv",)), want, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# RMSNorm + SwiGLU block flavour (Tab. S6, reading R13)
+# ---------------------------------------------------------------------------
+
+def test_silu_against_library_and_identities():
+    from scipy.special import expit
+    z = np.concatenate([np.linspace(-40, 40, 801), [-800.0, -1e-300, 0.0, 1e-300, 800.0]])
+    np.testing.assert_allclose(Lo.silu(z), z * expit(z), rtol=1e-15, atol=1e-300)
+    assert Lo.silu(np.array([0.0]))[0] == 0.0
+    # silu(z) - silu(-z) = z (sigmoid(z) + sigmoid(-z) = 1)
+    np.testing.assert_allclose(Lo.silu(z[:801]) - Lo.silu(-z[:801]), z[:801], rtol=0, atol=1e-13)
+
+
+def _swiglu_setup(seed=4):
+    cfg = W.small_config(grid=(1, 4, 4), win=(1, 4, 4), stride=(1, 4, 4), d=32, heads=2, mlp=40, dtype="f32",
+                         block="rms_swiglu")
+    m = _model(cfg)
+    dr = W.Draw(cfg, 1, seed=seed, affine=True)
+    x = dr.rng.standard_normal((9, cfg.d))
+    return cfg, m, dr.layer(), x
+
+
+def _rms_rows(x, g, eps):
+    # RMSNorm through the Euclidean norm: x * sqrt(d) / sqrt(|x|^2 + d eps) * g
+    d = x.shape[1]
+    return x * math.sqrt(d) / np.sqrt(np.linalg.norm(x, axis=1, keepdims=True) ** 2 + d * eps) * g
+
+
+def test_swiglu_mlp_odd_part_is_the_gated_product():
+    # Negating the gate rows and gate bias: silu(z) - silu(-z) = z, so the difference
+    # of the two MLPs is W_2 ((W_g h + b_g) * (W_u h + b_u)); b_2 cancels.  A swapped
+    # gate/up split, a dropped bias or a LayerNorm in place of RMSNorm all break it.
+    cfg, m, prm, x = _swiglu_setup()
+    f = cfg.mlp
+    neg = dict(prm)
+    neg["w_1"] = prm["w_1"].copy()
+    neg["b_1"] = prm["b_1"].copy()
+    neg["w_1"][:f] *= -1
+    neg["b_1"][:f] *= -1
+    h = _rms_rows(x, prm["ln2_g"], m.eps_ln)
+    g = h @ prm["w_1"][:f].T + prm["b_1"][:f]
+    u = h @ prm["w_1"][f:].T + prm["b_1"][f:]
+    want = (g * u) @ prm["w_2"].T
+    np.testing.assert_allclose(Lo.mlp_out(x, prm, m) - Lo.mlp_out(x, neg, m), want, rtol=0, atol=1e-13)
+
+
+def test_swiglu_saturated_gate():
+    # W_g = 0: the gate is the constant b_g.  b_g = 60 -> silu = 60 (to 1e-24), the MLP is
+    # the linear map 60 W_2 (W_u h + b_u) + b_2;  b_g = -60 -> silu ~ 0, the MLP is b_2.
+    cfg, m, prm, x = _swiglu_setup(seed=8)
+    f = cfg.mlp
+    h = _rms_rows(x, prm["ln2_g"], m.eps_ln)
+    for bg, want in ((60.0, 60.0 * (h @ prm["w_1"][f:].T + prm["b_1"][f:]) @ prm["w_2"].T + prm["b_2"]),
+                     (-60.0, np.broadcast_to(prm["b_2"], (x.shape[0], cfg.d)))):
+        q = dict(prm)
+        q["w_1"] = prm["w_1"].copy()
+        q["b_1"] = prm["b_1"].copy()
+        q["w_1"][:f] = 0.0
+        q["b_1"][:f] = bg
+        np.testing.assert_allclose(Lo.mlp_out(x, q, m), want, rtol=1e-13, atol=1e-13)
+
+
+def test_rms_block_norm_is_layer_norm_of_centred_rows():
+    # On rows of zero mean, RMSNorm with gain g is LayerNorm with gain g and bias 0.
+    m = Lo.Model(48, 2, 64, (0, 12, 12), block="rms_swiglu")
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((5, 48))
+    x -= x.mean(axis=1, keepdims=True)
+    g = rng.standard_normal(48)
+    b = rng.standard_normal(48)          # ignored by RMSNorm
+    np.testing.assert_allclose(Lo.block_norm(x, g, b, m), Lo.layer_norm(x, g, np.zeros(48), 1e-6), atol=1e-14)
