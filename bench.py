@@ -64,7 +64,19 @@ def parse():
                          "once per token on per-tile residual streams; default: the TileShare shared layer")
     ap.add_argument("--blend", default="ramp", choices=["ramp", "hard"],
                     help="blend rule of the plan: normalised linear ramp (default) or hard stitching")
+    ap.add_argument("--block", default=None, choices=["ln_gelu", "rms_swiglu"],
+                    help="block flavour: the configuration's (pre-LN + GELU) or RMSNorm + SwiGLU (gate and up "
+                         "of the configuration's MLP width each)")
     return ap.parse_args()
+
+
+def config_of(args):
+    import dataclasses
+    from shared_token_transformer_b200 import workloads as W
+    cfg = W.CONFIGS[args.config]
+    if args.block is not None and args.block != cfg.block:
+        cfg = dataclasses.replace(cfg, block=args.block)
+    return cfg
 
 
 # ---------------------------------------------------------------------------
@@ -79,8 +91,9 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def flops_layer(rows, T, N, d, f):
-    return rows * 2.0 * (4 * d * d + 2 * d * f) + 4.0 * T * N * N * d
+def flops_layer(rows, T, N, d, f, gated=False):
+    # QKV + out-projection, MLP up (gate and up rows when gated) and down, attention
+    return rows * 2.0 * (4 * d * d + (3 if gated else 2) * d * f) + 4.0 * T * N * N * d
 
 
 class ClockSampler:
@@ -167,7 +180,7 @@ def oracle_shared_layer_timing(cfg, budget_s, max_steps, warmup=1, rule="ramp"):
     S0, G0 = dr.states()
     S = np.concatenate([S0, G0])
     layer = dr.layer()
-    om = OL.Model(cfg.d, cfg.heads, cfg.mlp, cfg.rope_dims, fp8=(cfg.dtype == "fp8"))
+    om = OL.Model(cfg.d, cfg.heads, cfg.mlp, cfg.rope_dims, fp8=(cfg.dtype == "fp8"), block=cfg.block)
     for _ in range(warmup):
         OL.block_shared(S, layer, om, op)
     times = []
@@ -195,13 +208,13 @@ def run_tileshare(args, rank, world, local):
     Bd.build()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    cfg = W.CONFIGS[args.config]
+    cfg = config_of(args)
     L, k = cfg.L, cfg.k
     dt = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.bfloat16}[cfg.dtype]
     plan = B.Plan(cfg.grid, cfg.win, cfg.stride,
                   rule=B.TS_BLEND_HARD_STITCH if args.blend == "hard" else B.TS_BLEND_LINEAR_RAMP)
     U, T, N, d, f = plan.U, plan.T, plan.N, cfg.d, cfg.mlp
-    m = B.model_desc(d, cfg.heads, f, cfg.dtype, cfg.rope_dims)
+    m = B.model_desc(d, cfg.heads, f, cfg.dtype, cfg.rope_dims, block=cfg.block)
 
     # seeded inputs: weights from seed 0 (same on every rank); each rank its own image
     dr = W.Draw(cfg, T, seed=0)
@@ -470,14 +483,15 @@ def run_tileshare(args, rank, world, local):
                                                                            if tensor_peak_of(dom) > bf16_peak else "")
                                                 if kd["unit"] == "TFLOP/s" else "hbm_gbs"))}
 
-    ft = flops_layer(T * N, T, N, d, f)
-    fs = flops_layer(U + T, T, N, d, f)
+    gated = cfg.block == "rms_swiglu"
+    ft = flops_layer(T * N, T, N, d, f, gated)
+    fs = flops_layer(U + T, T, N, d, f, gated)
     if share is not None:
         # partial sharing: each shared operation on U + T rows, the others on T * N rows
         def rows(bit):
             return U + T if share & bit else T * N
         fs = (2.0 * 3 * d * d * rows(B.TS_SHARE_QKV) + 2.0 * d * d * rows(B.TS_SHARE_OUT) +
-              4.0 * d * f * rows(B.TS_SHARE_MLP) + 4.0 * T * N * N * d)
+              (6.0 if gated else 4.0) * d * f * rows(B.TS_SHARE_MLP) + 4.0 * T * N * N * d)
     flop_ratio = (k * ft + (L - k) * fs) / (L * ft)
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
@@ -485,7 +499,7 @@ def run_tileshare(args, rank, world, local):
         "vs_baseline": None, "dtype": {"bf16": "bf16", "f32": "f32", "fp8": "e4m3"}[cfg.dtype],
         "data": "synthetic (seeded N(0,1) states, N(0,0.02) weights, random init)",
         "config": {"workload": f"{cfg.name}: {cfg.note}", "grid": list(cfg.grid), "window": list(cfg.win),
-                   "stride": list(cfg.stride), "blend": args.blend,
+                   "stride": list(cfg.stride), "blend": args.blend, "block": cfg.block,
                    "shared_ops": (args.shared_ops or "none") if share is not None else "TileShare shared layer",
                    "L": L, "k": k, "unique_tokens": U, "tiles": T, "rows_per_tile": N,
                    "l2": "flushed before every step (512 MiB write, outside the timed events)",
@@ -544,7 +558,7 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     from shared_token_transformer_b200 import workloads as W
-    cfg = W.CONFIGS[args.config]
+    cfg = config_of(args)
 
     if args.impl == "reference":
         if rank != 0:
@@ -557,7 +571,7 @@ def main():
                "steps": len(times), "warmup": min(args.warmup, 1), "ms_per_step": round(mean * 1e3, 3),
                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                "data": "synthetic (seeded, same draws as the tileshare arm)",
-               "config": {"workload": f"{cfg.name}: {cfg.note}", "grid": list(cfg.grid), "L": cfg.L, "k": cfg.k},
+               "config": {"workload": f"{cfg.name}: {cfg.note}", "grid": list(cfg.grid), "L": cfg.L, "k": cfg.k, "block": cfg.block},
                "cpu_baseline": {"value": round(v, 2), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"{len(times)} float64 oracle shared layers of {cfg.name} "
                                           f"(steps capped at a {budget:.0f} s budget)"},
@@ -573,7 +587,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     res, cfg = run_tileshare(args, rank, world, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        if flops_layer(cfg.U + 1, 1, 1, cfg.d, cfg.mlp) < 5e11:
+        if flops_layer(cfg.U + 1, 1, 1, cfg.d, cfg.mlp, cfg.block == "rms_swiglu") < 5e11:
             U, times = oracle_shared_layer_timing(cfg, args.cpu_seconds, 1000, rule=args.blend)
             mean = float(np.mean(times))
             res["cpu_baseline"] = {"value": round(U / mean, 2), "unit": UNIT, "cores": blas_threads(),

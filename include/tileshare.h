@@ -72,6 +72,19 @@ typedef enum {
                        per token ([TileShare] Tab. S2 "FP8")                          */
 } ts_dtype;
 
+/* Block flavour ([TileShare] Tab. S1 block; Tab. S6 profiles a block with "RMSNorm +
+   residual" and a "SwiGLU gate"). */
+typedef enum {
+  /* pre-LN ViT block: Norm1/Norm2 LayerNorm with gain and bias, MLP
+     W_2 GELU(W_1 h + b_1) + b_2 (exact erf GELU) */
+  TS_BLOCK_LN_GELU = 0,
+  /* Norm1/Norm2 RMSNorm with gain, no bias (ln*_b unused, may be NULL); MLP
+     W_2 (silu(W_g h + b_g) * (W_u h + b_u)) + b_2 with silu(z) = z / (1 + e^-z).
+     w_1 [2f, d] holds the f gate rows W_g above the f up rows W_u; b_1 [2f] and, for
+     e4m3, s_1 [2f] follow the same order. */
+  TS_BLOCK_RMS_SWIGLU = 1
+} ts_block_kind;
+
 typedef struct ts_plan_s* ts_plan_t;
 
 /* Read-only view of a plan.  Host arrays stay valid until ts_plan_destroy. */
@@ -102,6 +115,7 @@ typedef struct {
   int rope_dims[3];       /* head-dimension channels rotated by the f, y, x
                              coordinate; sum = hd, each even.  Inside an axis block
                              of D channels, channel j pairs with j + D/2.            */
+  ts_block_kind block;    /* block flavour (TS_BLOCK_LN_GELU unless set)              */
 } ts_model_desc;
 
 /* One layer's parameters, all device pointers.  Matrices are [out, in] row-major
@@ -114,10 +128,10 @@ typedef struct {
   const float* q_g;   const float* k_g;      /* [hd] QK-RMSNorm gains              */
   const void* w_o;    const float* b_o;      /* [d, d], [d]          */
   const float* ln2_g; const float* ln2_b;    /* [d]                 */
-  const void* w_1;    const float* b_1;      /* [f, d], [f]          */
+  const void* w_1;    const float* b_1;      /* [f, d], [f]; [2f, d], [2f] for TS_BLOCK_RMS_SWIGLU */
   const void* w_2;    const float* b_2;      /* [d, f], [d]          */
   const float* s_qkv; const float* s_o;      /* TS_FP8_E4M3 only: [3d], [d] */
-  const float* s_1;   const float* s_2;      /* TS_FP8_E4M3 only: [f], [d]  */
+  const float* s_1;   const float* s_2;      /* TS_FP8_E4M3 only: [f] ([2f] SwiGLU), [d] */
 } ts_layer_weights;
 
 /* ---------------------------------------------------------------------------

@@ -23,11 +23,16 @@ typedef enum { TS_ROWS_SHARED = 0, TS_ROWS_TILED = 1 } ts_rows_mode;
 typedef enum {
   TS_EPI_BIAS = 0,        /* y = x W^T + b                                  */
   TS_EPI_BIAS_GELU = 1,   /* y = GELU(x W^T + b), exact erf GELU            */
-  TS_EPI_BIAS_RESID = 2   /* y += x W^T + b  (y is the residual, in place)  */
+  TS_EPI_BIAS_RESID = 2,  /* y += x W^T + b  (y is the residual, in place)  */
+  TS_EPI_BIAS_SWIGLU = 3  /* y = silu(x W_g^T + b_g) * (x W_u^T + b_u): W [2N, K]
+                             holds the N gate rows above the N up rows, bias and
+                             w_scale [2N] likewise; y [rows, N]                   */
 } ts_epilogue;
 
-/* LayerNorm over the last dimension ([TileShare] Tab. S1 "Norm1"; pre-LN block):
-   y[r] = (x[r] - mean) / sqrt(var + eps) * g + b, population variance.
+/* Norm1 / Norm2 over the last dimension ([TileShare] Tab. S1 "Norm1"; pre-LN block):
+   y[r] = (x[r] - mean) / sqrt(var + eps) * g + b, population variance, eps = eps_ln.
+   For TS_BLOCK_RMS_SWIGLU models RMSNorm instead: y[r] = x[r] / sqrt(mean(x[r]^2) +
+   eps) * g, and b is unused (may be NULL).
    x, y [rows, d] in the model dtype (bf16 for TS_FP8_E4M3); g, b fp32 [d]. */
 ts_status ts_op_layernorm(const ts_model_desc* model, const void* x, int rows,
                           const float* g, const float* b, void* y, void* stream);
@@ -37,7 +42,7 @@ ts_status ts_op_layernorm(const ts_model_desc* model, const void* x, int rows,
    the model dtype (TS_FP8_E4M3: x bf16, W e4m3 with per-row scales w_scale [N];
    x is quantised per row inside the call using `scratch`, which must hold
    rows * K + 4 * rows bytes; scratch is unused otherwise and may be NULL).
-   bf16/e4m3 need K % 64 == 0 and N % 64 == 0. */
+   bf16/e4m3 need K % 64 == 0 and N % 64 == 0 (K % 128 for e4m3). */
 ts_status ts_op_linear(const ts_model_desc* model, const void* x, int rows, int K,
                        const void* W, const float* w_scale, int N, const float* bias,
                        ts_epilogue epi, void* y, void* scratch, void* stream);

@@ -24,7 +24,9 @@ TS_BLEND_HARD_STITCH = 1
 TS_SHARE_QKV, TS_SHARE_OUT, TS_SHARE_MLP = 1, 2, 4
 TS_F32, TS_BF16, TS_FP8_E4M3 = 0, 1, 2
 TS_ROWS_SHARED, TS_ROWS_TILED = 0, 1
-TS_EPI_BIAS, TS_EPI_BIAS_GELU, TS_EPI_BIAS_RESID = 0, 1, 2
+TS_EPI_BIAS, TS_EPI_BIAS_GELU, TS_EPI_BIAS_RESID, TS_EPI_BIAS_SWIGLU = 0, 1, 2, 3
+TS_BLOCK_LN_GELU, TS_BLOCK_RMS_SWIGLU = 0, 1
+BLOCKS = {"ln_gelu": TS_BLOCK_LN_GELU, "rms_swiglu": TS_BLOCK_RMS_SWIGLU}
 DTYPES = {"f32": TS_F32, "bf16": TS_BF16, "fp8": TS_FP8_E4M3}
 
 _int3 = ctypes.c_int * 3
@@ -44,7 +46,7 @@ class PlanDesc(ctypes.Structure):
 class ModelDesc(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int), ("heads", ctypes.c_int), ("mlp", ctypes.c_int), ("dtype", ctypes.c_int),
                 ("eps_ln", ctypes.c_float), ("eps_qk", ctypes.c_float), ("rope_base", ctypes.c_float),
-                ("rope_dims", _int3)]
+                ("rope_dims", _int3), ("block", ctypes.c_int)]
 
 
 _WEIGHT_FIELDS = ["ln1_g", "ln1_b", "w_qkv", "b_qkv", "q_g", "k_g", "w_o", "b_o", "ln2_g", "ln2_b",
@@ -182,9 +184,9 @@ class Plan:
 # ---------------------------------------------------------------------------
 # model / weights
 # ---------------------------------------------------------------------------
-def model_desc(d, heads, mlp, dtype, rope_dims, eps_ln=1e-6, eps_qk=1e-6, rope_base=10000.0):
+def model_desc(d, heads, mlp, dtype, rope_dims, eps_ln=1e-6, eps_qk=1e-6, rope_base=10000.0, block="ln_gelu"):
     return ModelDesc(d, heads, mlp, DTYPES[dtype] if isinstance(dtype, str) else dtype, eps_ln, eps_qk, rope_base,
-                     _int3(*rope_dims))
+                     _int3(*rope_dims), BLOCKS[block] if isinstance(block, str) else block)
 
 
 def layer_weights(tensors):
@@ -285,7 +287,7 @@ def op_layernorm(model, x, g, b, y, stream=None):
 
 def op_linear(model, x, W, bias, y, epi=TS_EPI_BIAS, w_scale=None, scratch=None, stream=None):
     rows, K = x.shape
-    N = W.shape[0]
+    N = W.shape[0] // 2 if epi == TS_EPI_BIAS_SWIGLU else W.shape[0]     # output width
     _check("ts_op_linear", lib().ts_op_linear(ctypes.byref(model), _ptr(x), rows, K, _ptr(W), _ptr(w_scale), N,
                                               _ptr(bias), epi, _ptr(y), _ptr(scratch), _stream(stream)))
 

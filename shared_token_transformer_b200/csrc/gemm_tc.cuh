@@ -8,6 +8,10 @@
 //   EPI_RESID  y = y + acc + b   (y is the residual stream)   (out-proj, MLP down)
 //   EPI_QKV    q, k: QK-RMSNorm over each head of 64 channels, gain, then RoPE at
 //              the row's coordinates; v: acc + b               (QKV projection)
+//   EPI_SWIGLU y = silu(acc_g + b_g) * (acc_u + b_u)          (SwiGLU MLP up, Tab. S6)
+//              W holds N/2 gate rows above N/2 up rows; a 128 x BN tile loads BN/2
+//              gate rows and the BN/2 matching up rows, so the two sums of an
+//              output sit in one accumulator, BN/2 columns apart; y is [M, N/2].
 // For e4m3 operands acc is first multiplied by the row scale of A and the column
 // scale of W.
 //
@@ -31,11 +35,11 @@
 
 namespace ts {
 
-enum GemmEpi : int { EPI_BIAS = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_QKV = 3 };
+enum GemmEpi : int { EPI_BIAS = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_QKV = 3, EPI_SWIGLU = 4 };
 
 
 struct GemmArgs {
-  int M, N, K;
+  int M, N, K;            // N: accumulator columns (2 x the output width for EPI_SWIGLU)
   const float* bias;      // [N] or null
   bf16* out;              // [M, ldo]
   int ldo;
@@ -139,6 +143,32 @@ __device__ __forceinline__ void gemm_epilogue64(float* v, int col, float rs, con
   }
 }
 
+// SwiGLU of 32 outputs held by this thread: g (gate sums) is overwritten with
+// silu(g * sg + b_g) * (u * su + b_u); col is the output column of g[0], F the
+// output width (gate row col + i, up row F + col + i of W, bias and w_scale).
+template <bool FP8>
+__device__ __forceinline__ void swiglu32(float* g, const float* u, int col, int F, float rs, const GemmArgs& args) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 4) {
+    float gg[4] = {g[i], g[i + 1], g[i + 2], g[i + 3]};
+    float uu[4] = {u[i], u[i + 1], u[i + 2], u[i + 3]};
+    if (FP8) {
+      const float4 wg = __ldg(reinterpret_cast<const float4*>(args.w_scale + col + i));
+      const float4 wu = __ldg(reinterpret_cast<const float4*>(args.w_scale + F + col + i));
+      gg[0] *= rs * wg.x; gg[1] *= rs * wg.y; gg[2] *= rs * wg.z; gg[3] *= rs * wg.w;
+      uu[0] *= rs * wu.x; uu[1] *= rs * wu.y; uu[2] *= rs * wu.z; uu[3] *= rs * wu.w;
+    }
+    if (args.bias) {
+      const float4 bg = __ldg(reinterpret_cast<const float4*>(args.bias + col + i));
+      const float4 bu = __ldg(reinterpret_cast<const float4*>(args.bias + F + col + i));
+      gg[0] += bg.x; gg[1] += bg.y; gg[2] += bg.z; gg[3] += bg.w;
+      uu[0] += bu.x; uu[1] += bu.y; uu[2] += bu.z; uu[3] += bu.w;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) g[i + e] = gg[e] / (1.0f + __expf(-gg[e])) * uu[e];
+  }
+}
+
 // TMA tile store of a shared-memory box to global memory (bulk-group completion).
 __device__ __forceinline__ void tma_store_2d(const void* map, uint32_t src, int x, int y) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
@@ -172,7 +202,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   constexpr uint32_t TMEM_COLS = 2 * BN;          // two accumulators: 128, 256 or 512 columns
   constexpr uint32_t IDESC = idesc_make(FP8 ? 0u : 1u, BN);
   constexpr int KE = FP8 ? 128 : 64;              // K elements per slice
-  constexpr int NCHUNK = BN / 64;
+  constexpr bool GLU = EPI == EPI_SWIGLU;
+  static_assert(!GLU || BN >= 128, "SwiGLU tiles need 64-column output chunks");
+  constexpr int NCHUNK = GLU ? BN / 128 : BN / 64;   // 64-column output chunks per tile
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -229,7 +261,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t sa = sbase + s * SM::STAGE_BYTES;
           mbar_expect_tx(bar_full + 8 * s, SM::STAGE_BYTES);
           tma_load_2d(sa, &tmA, bar_full + 8 * s, kb * KE, m0);
-          tma_load_2d(sa + SM::A_BYTES, &tmB, bar_full + 8 * s, kb * KE, n0);
+          if (GLU) {    // BN/2 gate rows, then the BN/2 up rows of the same outputs
+            tma_load_2d(sa + SM::A_BYTES, &tmB, bar_full + 8 * s, kb * KE, n0 / 2);
+            tma_load_2d(sa + SM::A_BYTES + (BN / 2) * 128, &tmB, bar_full + 8 * s, kb * KE, args.N / 2 + n0 / 2);
+          } else {
+            tma_load_2d(sa + SM::A_BYTES, &tmB, bar_full + 8 * s, kb * KE, n0);
+          }
         }
       }
     }
@@ -301,7 +338,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           __syncwarp();
           store_pending = false;
         }
-        const int col = n0 + c * 64, row0 = m0 + quarter * 32;
+        const int col = (GLU ? n0 / 2 : n0) + c * 64, row0 = m0 + quarter * 32;
         if (EPI == EPI_RESID && lane == 0) {
           mbar_expect_tx(rbar, 4096);
           tma_load_2d(stg, &tmD, rbar, col, row0);
@@ -310,12 +347,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_ld32(trow + c * 64, v);
         tmem_ld32(trow + c * 64 + 32, v + 32);
         tmem_wait_ld();
-        if (k == mine - 1) {           // last TMEM read of this warp for this tile
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar_tempty + 8 * acc);
+        if (GLU) {
+          float u[32];
+          tmem_ld32(trow + BN / 2 + c * 64, u);
+          tmem_wait_ld();
+          swiglu32<FP8>(v, u, col, args.N / 2, rs, args);
+          tmem_ld32(trow + BN / 2 + c * 64 + 32, u);
+          tmem_wait_ld();
+          if (k == mine - 1) {         // last TMEM read of this warp for this tile
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_tempty + 8 * acc);
+          }
+          swiglu32<FP8>(v + 32, u, col + 32, args.N / 2, rs, args);
+        } else {
+          if (k == mine - 1) {         // last TMEM read of this warp for this tile
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_tempty + 8 * acc);
+          }
+          gemm_epilogue64<EPI, FP8, R0, R1, R2>(v, col, rs, pos, args);
         }
-        gemm_epilogue64<EPI, FP8, R0, R1, R2>(v, col, rs, pos, args);
         uint8_t* srow = smem + SM::EPI_OFFSET + warp * 4096 + lane * 128;
         if (EPI == EPI_RESID) {
           if (!mbar_wait(rbar, nres & 1)) {

@@ -64,13 +64,14 @@ __device__ __forceinline__ void store_row(const float (&v)[NV][Vec<T>::E], int l
 // ---------------------------------------------------------------------------
 // LayerNorm (pre-LN block, [TileShare] Tab. S1 Norm1 / Norm2): population variance,
 // two passes over the row held in registers.  NV = d / (32 * E) vectors per lane.
+// With rms set it is RMSNorm (Tab. S6 "RMSNorm"): no centring and no bias.
 // ---------------------------------------------------------------------------
 // Blocks past the rows (when rt.cs is set) fill the RoPE table that the next
 // QKV GEMM reads.
 template <typename T, int NV, bool Q8>
 __global__ void __launch_bounds__(256) layernorm_kernel(const T* __restrict__ x, int rows, int d,
                                                         const float* __restrict__ g, const float* __restrict__ b,
-                                                        float eps, T* __restrict__ y, uint8_t* __restrict__ q8,
+                                                        float eps, int rms, T* __restrict__ y, uint8_t* __restrict__ q8,
                                                         float* __restrict__ qscale, const RopeTable rt) {
   pdl_wait();
   pdl_trigger();
@@ -91,7 +92,7 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const T* __restrict__ x,
 #pragma unroll
     for (int e = 0; e < E; ++e) s += v[i][e];
   }
-  const float mean = warp_sum(s) / d;
+  const float mean = rms ? 0.f : warp_sum(s) / d;
   float q = 0.f;
 #pragma unroll
   for (int i = 0; i < NV; ++i)
@@ -107,7 +108,7 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const T* __restrict__ x,
 #pragma unroll
     for (int e = 0; e < E; e += 4) {   // gains and biases as 16-byte vectors
       const float4 gg = __ldg(reinterpret_cast<const float4*>(g + c0 + e));
-      const float4 bb = __ldg(reinterpret_cast<const float4*>(b + c0 + e));
+      const float4 bb = rms ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldg(reinterpret_cast<const float4*>(b + c0 + e));
       v[i][e] = (v[i][e] - mean) * rstd * gg.x + bb.x;
       v[i][e + 1] = (v[i][e + 1] - mean) * rstd * gg.y + bb.y;
       v[i][e + 2] = (v[i][e + 2] - mean) * rstd * gg.z + bb.z;
@@ -121,7 +122,7 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const T* __restrict__ x,
 template <typename T>
 __global__ void __launch_bounds__(256) layernorm_generic_kernel(const T* __restrict__ x, int rows, int d,
                                                                 const float* __restrict__ g,
-                                                                const float* __restrict__ b, float eps,
+                                                                const float* __restrict__ b, float eps, int rms,
                                                                 T* __restrict__ y) {
   const int lane = threadIdx.x & 31;
   const size_t row = static_cast<size_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -129,14 +130,15 @@ __global__ void __launch_bounds__(256) layernorm_generic_kernel(const T* __restr
   const T* xr = x + row * d;
   float s = 0.f;
   for (int c = lane; c < d; c += 32) s += static_cast<float>(xr[c]);
-  const float mean = warp_sum(s) / d;
+  const float mean = rms ? 0.f : warp_sum(s) / d;
   float q = 0.f;
   for (int c = lane; c < d; c += 32) {
     const float t = static_cast<float>(xr[c]) - mean;
     q = fmaf(t, t, q);
   }
   const float rstd = rsqrtf(warp_sum(q) / d + eps);
-  for (int c = lane; c < d; c += 32) y[row * d + c] = static_cast<T>((static_cast<float>(xr[c]) - mean) * rstd * g[c] + b[c]);
+  for (int c = lane; c < d; c += 32)
+    y[row * d + c] = static_cast<T>((static_cast<float>(xr[c]) - mean) * rstd * g[c] + (rms ? 0.f : b[c]));
 }
 
 // ---------------------------------------------------------------------------
@@ -425,8 +427,13 @@ __global__ void __launch_bounds__(128) qk_norm_rope_f32_kernel(float* __restrict
 
 // ---------------------------------------------------------------------------
 // fp32 path: SIMT GEMM Y = A W^T (+ b) with the same epilogues as the tensor-core
-// kernel (bias, GELU, residual).  64 x 64 tiles, K slices of 16, 4 x 4 per thread.
+// kernel (bias, GELU, residual, SwiGLU).  64 x 64 tiles, K slices of 16, 4 x 4 per
+// thread.  EPI 3 (SwiGLU): N is the output width, W has 2N rows (gate rows, then
+// up rows); a tile loads 32 gate rows and the 32 matching up rows, so that lane l
+// (tx < 8) and lane l + 8 of a warp hold the gate and up sums of the same outputs.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+
 template <int EPI>
 __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__ A, const float* __restrict__ W,
                                                        const float* __restrict__ bias, float* __restrict__ Y, int M,
@@ -434,14 +441,21 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
   __shared__ float sA[16][64 + 4];
   __shared__ float sW[16][64 + 4];
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  const int m0 = blockIdx.x * 64, n0 = blockIdx.y * 64;
+  const int m0 = blockIdx.x * 64, n0 = blockIdx.y * (EPI == 3 ? 32 : 64);
   float acc[4][4] = {};
   for (int k0 = 0; k0 < K; k0 += 16) {
     for (int i = threadIdx.x; i < 64 * 16; i += 256) {
       const int r = i / 16, c = i % 16;
-      const int gm = m0 + r, gn = n0 + r, gk = k0 + c;
+      const int gm = m0 + r, gk = k0 + c;
+      int gn = n0 + r;
+      bool wok = gn < N;
+      if (EPI == 3) {
+        gn = n0 + (r & 31);
+        wok = gn < N;
+        gn += (r >> 5) * N;     // rows 32..63 of the tile: the up rows
+      }
       sA[c][r] = (gm < M && gk < K) ? A[static_cast<size_t>(gm) * K + gk] : 0.f;
-      sW[c][r] = (gn < N && gk < K) ? W[static_cast<size_t>(gn) * K + gk] : 0.f;
+      sW[c][r] = (wok && gk < K) ? W[static_cast<size_t>(gn) * K + gk] : 0.f;
     }
     __syncthreads();
 #pragma unroll
@@ -458,6 +472,22 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
         for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], w[j], acc[i][j]);
     }
     __syncthreads();
+  }
+  if (EPI == 3) {
+    // lanes tx < 8 hold gate columns tx*4 + j, lanes tx + 8 the up columns
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float u = __shfl_down_sync(0xffffffffu, acc[i][j], 8);
+        const int m = m0 + ty * 4 + i, n = n0 + tx * 4 + j;
+        if (tx < 8 && m < M && n < N) {
+          const float gv = acc[i][j] + (bias ? bias[n] : 0.f);
+          const float uv = u + (bias ? bias[N + n] : 0.f);
+          Y[static_cast<size_t>(m) * N + n] = silu_f(gv) * uv;
+        }
+      }
+    return;
   }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {

@@ -235,6 +235,8 @@ static ts_status check_model(const ts_model_desc* m) {
     sum += m->rope_dims[a];
   }
   if (sum != hd) return fail(TS_ERR_INVALID_ARG, "rope_dims sum %d != head dim %d", sum, hd);
+  if (m->block != TS_BLOCK_LN_GELU && m->block != TS_BLOCK_RMS_SWIGLU)
+    return fail(TS_ERR_INVALID_ARG, "unknown block flavour %d", static_cast<int>(m->block));
   if (!(m->eps_ln > 0.f) || !(m->eps_qk > 0.f) || !(m->rope_base > 0.f))
     return fail(TS_ERR_INVALID_ARG, "eps and rope_base must be positive");
   if (m->dtype == TS_F32) {
@@ -275,8 +277,9 @@ static ts_status check_plan(ts_plan_t p) {
 
 static ts_status check_weights(const ts_model_desc* m, const ts_layer_weights* w) {
   if (!w) return fail(TS_ERR_INVALID_ARG, "weights are NULL");
-  const void* ptrs[] = {w->ln1_g, w->ln1_b, w->w_qkv, w->b_qkv, w->q_g, w->k_g, w->w_o, w->b_o,
-                        w->ln2_g, w->ln2_b, w->w_1,   w->b_1,   w->w_2, w->b_2};
+  const bool rms = m->block == TS_BLOCK_RMS_SWIGLU;
+  const void* ptrs[] = {w->ln1_g, rms ? w->ln1_g : w->ln1_b, w->w_qkv, w->b_qkv, w->q_g, w->k_g, w->w_o, w->b_o,
+                        w->ln2_g, rms ? w->ln2_g : w->ln2_b, w->w_1,   w->b_1,   w->w_2, w->b_2};
   for (const void* p : ptrs) {
     if (!p) return fail(TS_ERR_INVALID_ARG, "a weight pointer is NULL");
     if (!aligned16(p)) return fail(TS_ERR_INVALID_ARG, "weight pointers must be 16-byte aligned");
@@ -378,7 +381,7 @@ static int num_sms() {
 static inline unsigned rows_grid(size_t rows) { return static_cast<unsigned>((rows + 7) / 8); }
 
 template <typename T, bool Q8>
-static ts_status launch_layernorm_vec(const void* x, int rows, int d, const float* g, const float* b, float eps,
+static ts_status launch_layernorm_vec(const void* x, int rows, int d, const float* g, const float* b, float eps, int rms,
                                       void* y, uint8_t* q8, float* qs, const ts::RopeTable& rt, cudaStream_t st) {
   const unsigned fill_blocks = rt.cs ? static_cast<unsigned>((rt.total + 255) / 256) : 0u;
   constexpr int E = ts::Vec<T>::E;
@@ -389,7 +392,7 @@ static ts_status launch_layernorm_vec(const void* x, int rows, int d, const floa
 #define TS_LN_CASE(NV) \
   case NV:                                                                                                  \
     launch_pdl(ts::layernorm_kernel<T, NV, Q8>, dim3(rows_grid(rows) + fill_blocks), dim3(256), 0, st, xx, rows, d, \
-               g, b, eps, yy, q8, qs, rt);                                                                    \
+               g, b, eps, rms, yy, q8, qs, rt);                                                               \
     break;
   switch (nv) {
     TS_LN_CASE(1) TS_LN_CASE(2) TS_LN_CASE(3) TS_LN_CASE(4) TS_LN_CASE(5) TS_LN_CASE(6) TS_LN_CASE(7) TS_LN_CASE(8)
@@ -399,24 +402,26 @@ static ts_status launch_layernorm_vec(const void* x, int rows, int d, const floa
   return trace_post(st, "layernorm");
 }
 
-// y = LN(x); for e4m3 writes q8/qs instead of y.
+// y = Norm(x): LayerNorm, or RMSNorm for TS_BLOCK_RMS_SWIGLU (b unused); for e4m3
+// writes q8/qs instead of y.
 static ts_status run_layernorm(const ts_model_desc* m, const void* x, int rows, const float* g, const float* b,
                                void* y, uint8_t* q8, float* qs, cudaStream_t st,
                                const ts::RopeTable& rt = ts::RopeTable{}) {
   if (rows == 0) return TS_OK;
   const int d = m->d;
+  const int rms = m->block == TS_BLOCK_RMS_SWIGLU;
   const double e = esize(m->dtype);
   set_work("layernorm", 0.0, static_cast<double>(rows) * d * (e + (q8 ? 1.0 : e)) + (q8 ? 4.0 * rows : 0.0));
   if (m->dtype == TS_F32) {
     if (d % 128 == 0 && d <= 1024)
-      return launch_layernorm_vec<float, false>(x, rows, d, g, b, m->eps_ln, y, nullptr, nullptr, ts::RopeTable{}, st);
+      return launch_layernorm_vec<float, false>(x, rows, d, g, b, m->eps_ln, rms, y, nullptr, nullptr, ts::RopeTable{}, st);
     trace_pre(st);
     ts::layernorm_generic_kernel<float><<<rows_grid(rows), 256, 0, st>>>(static_cast<const float*>(x), rows, d, g, b,
-                                                                        m->eps_ln, static_cast<float*>(y));
+                                                                        m->eps_ln, rms, static_cast<float*>(y));
     return trace_post(st, "layernorm_generic");
   }
-  if (q8) return launch_layernorm_vec<bf16, true>(x, rows, d, g, b, m->eps_ln, nullptr, q8, qs, rt, st);
-  return launch_layernorm_vec<bf16, false>(x, rows, d, g, b, m->eps_ln, y, nullptr, nullptr, rt, st);
+  if (q8) return launch_layernorm_vec<bf16, true>(x, rows, d, g, b, m->eps_ln, rms, nullptr, q8, qs, rt, st);
+  return launch_layernorm_vec<bf16, false>(x, rows, d, g, b, m->eps_ln, rms, y, nullptr, nullptr, rt, st);
 }
 
 template <typename T, bool Q8>
@@ -533,7 +538,11 @@ static ts_status dispatch_gemm_bn(int bn, const CUtensorMap& ta, const CUtensorM
   switch (bn) {
     case 256: return launch_gemm_tc<256, 4, EPI, FP8, R0, R1, R2>(ta, tb, td, args, st);
     case 128: return launch_gemm_tc<128, 6, EPI, FP8, R0, R1, R2>(ta, tb, td, args, st);
-    default: return launch_gemm_tc<64, 8, EPI, FP8, R0, R1, R2>(ta, tb, td, args, st);
+    default:
+      if constexpr (EPI == ts::EPI_SWIGLU)   // SwiGLU tiles are at least 128 wide
+        return launch_gemm_tc<128, 6, EPI, FP8, R0, R1, R2>(ta, tb, td, args, st);
+      else
+        return launch_gemm_tc<64, 8, EPI, FP8, R0, R1, R2>(ta, tb, td, args, st);
   }
 }
 
@@ -565,27 +574,31 @@ static int pick_bn(int M, int N) {
 }
 
 // Y[M, N] = A[M, K] W[N, K]^T with epilogue; A bf16 (or e4m3 + a_scale), W bf16 (or e4m3 + w_scale).
+// EPI_SWIGLU: N is the output width and W, bias, w_scale have 2N rows (gate, then up).
 static ts_status run_gemm_tc(const char* name, const ts_model_desc* m, int epi, const void* A, const float* a_scale,
                              const void* W, const float* w_scale, int M, int N, int K, const float* bias, bf16* out,
                              const ts_layer_weights* qk, const int* pos, cudaStream_t st,
                              const ts::RopeTable& rt = ts::RopeTable{}) {
   if (M == 0) return TS_OK;
   const bool fp8 = m->dtype == TS_FP8_E4M3;
+  const bool glu = epi == ts::EPI_SWIGLU;
+  const int NA = glu ? 2 * N : N;   // accumulator columns = rows of W
   {
     const double ea = fp8 ? 1.0 : 2.0;
-    const double bytes = static_cast<double>(M) * K * ea + static_cast<double>(N) * K * ea +
+    const double bytes = static_cast<double>(M) * K * ea + static_cast<double>(NA) * K * ea +
                          static_cast<double>(M) * N * 2.0 * (epi == ts::EPI_RESID ? 2.0 : 1.0);
-    set_work(name, 2.0 * M * static_cast<double>(N) * K, bytes);
+    set_work(name, 2.0 * M * static_cast<double>(NA) * K, bytes);
   }
   if (K % (fp8 ? 128 : 64) || N % 64) return fail(TS_ERR_UNSUPPORTED, "GEMM sizes K=%d N=%d not tiled", K, N);
-  const int bn = pick_bn(M, N);
+  int bn = pick_bn(M, NA);
+  if (glu && bn < 128) bn = 128;    // NA = 2N is a multiple of 128
   CUtensorMap ta, tb, td;
   TS_TRY(make_tmap(&ta, A, M, K, fp8 ? 1 : 2, 128));
-  TS_TRY(make_tmap(&tb, W, N, K, fp8 ? 1 : 2, bn));
+  TS_TRY(make_tmap(&tb, W, NA, K, fp8 ? 1 : 2, glu ? bn / 2 : bn));
   TS_TRY(make_tmap(&td, out, M, N, 2, 32));   // output (and residual): 32 x 64 chunks of the epilogue warps
   ts::GemmArgs g{};
   g.M = M;
-  g.N = N;
+  g.N = NA;
   g.K = K;
   g.bias = bias;
   g.out = out;
@@ -610,20 +623,26 @@ static ts_status run_gemm_tc(const char* name, const ts_model_desc* m, int epi, 
     case ts::EPI_GELU: return TS_GEMM_EPI(ts::EPI_GELU, 0, 32, 32);
     case ts::EPI_RESID: return TS_GEMM_EPI(ts::EPI_RESID, 0, 32, 32);
     case ts::EPI_QKV: return r3 ? TS_GEMM_EPI(ts::EPI_QKV, 16, 24, 24) : TS_GEMM_EPI(ts::EPI_QKV, 0, 32, 32);
+    case ts::EPI_SWIGLU: return TS_GEMM_EPI(ts::EPI_SWIGLU, 0, 32, 32);
   }
 #undef TS_GEMM_EPI
   return fail(TS_ERR_INVALID_ARG, "unknown epilogue");
 }
 
-// fp32 SIMT GEMM
+// fp32 SIMT GEMM (EPI_SWIGLU: N is the output width, W has 2N rows)
 static ts_status run_gemm_f32(const char* name, int epi, const float* A, const float* W, int M, int N, int K,
                               const float* bias, float* Y, cudaStream_t st) {
   if (M == 0) return TS_OK;
-  set_work(name, 2.0 * M * static_cast<double>(N) * K,
-           4.0 * (static_cast<double>(M) * K + static_cast<double>(N) * K + M * static_cast<double>(N) * (epi == ts::EPI_RESID ? 2 : 1)));
+  const int NA = epi == ts::EPI_SWIGLU ? 2 * N : N;
+  set_work(name, 2.0 * M * static_cast<double>(NA) * K,
+           4.0 * (static_cast<double>(M) * K + static_cast<double>(NA) * K + M * static_cast<double>(N) * (epi == ts::EPI_RESID ? 2 : 1)));
   dim3 grid((M + 63) / 64, (N + 63) / 64);
   trace_pre(st);
   switch (epi) {
+    case ts::EPI_SWIGLU:
+      grid.y = (N + 31) / 32;
+      ts::gemm_f32_kernel<3><<<grid, 256, 0, st>>>(A, W, bias, Y, M, N, K);
+      break;
     case ts::EPI_GELU: ts::gemm_f32_kernel<1><<<grid, 256, 0, st>>>(A, W, bias, Y, M, N, K); break;
     case ts::EPI_RESID: ts::gemm_f32_kernel<2><<<grid, 256, 0, st>>>(A, W, bias, Y, M, N, K); break;
     default: ts::gemm_f32_kernel<0><<<grid, 256, 0, st>>>(A, W, bias, Y, M, N, K); break;
@@ -745,30 +764,40 @@ static ts_status run_out_proj(const ts_model_desc* m, const ts_layer_weights* w,
                      nullptr, nullptr, st);
 }
 
-// state += W2 GELU(W1 LN2(state) + b1) + b2
-static ts_status run_mlp(const ts_model_desc* m, const ts_layer_weights* w, int rows, void* state, const Workspace& ws,
-                         cudaStream_t st) {
+// out (+)= W2 act(W1 Norm2(in) + b1) + b2 with act GELU, or SwiGLU for
+// TS_BLOCK_RMS_SWIGLU (W1 [2f, d]); resid: out is the residual stream (in place
+// when out == in), else out is written.
+static ts_status run_mlp_any(const ts_model_desc* m, const ts_layer_weights* w, int rows, const void* in, void* out,
+                             bool resid, const Workspace& ws, cudaStream_t st) {
   const int d = m->d, f = m->mlp;
+  const int up = m->block == TS_BLOCK_RMS_SWIGLU ? ts::EPI_SWIGLU : ts::EPI_GELU;
+  const int down = resid ? ts::EPI_RESID : ts::EPI_BIAS;
   if (m->dtype == TS_F32) {
-    TS_TRY(run_layernorm(m, state, rows, w->ln2_g, w->ln2_b, ws.xn, nullptr, nullptr, st));
-    TS_TRY(run_gemm_f32("gemm_up", ts::EPI_GELU, static_cast<const float*>(ws.xn), static_cast<const float*>(w->w_1), rows, f, d,
+    TS_TRY(run_layernorm(m, in, rows, w->ln2_g, w->ln2_b, ws.xn, nullptr, nullptr, st));
+    TS_TRY(run_gemm_f32("gemm_up", up, static_cast<const float*>(ws.xn), static_cast<const float*>(w->w_1), rows, f, d,
                         w->b_1, static_cast<float*>(ws.h), st));
-    return run_gemm_f32("gemm_down", ts::EPI_RESID, static_cast<const float*>(ws.h), static_cast<const float*>(w->w_2), rows, d, f,
-                        w->b_2, static_cast<float*>(state), st);
+    return run_gemm_f32("gemm_down", down, static_cast<const float*>(ws.h), static_cast<const float*>(w->w_2), rows, d, f,
+                        w->b_2, static_cast<float*>(out), st);
   }
   if (m->dtype == TS_FP8_E4M3) {
-    TS_TRY(run_layernorm(m, state, rows, w->ln2_g, w->ln2_b, nullptr, ws.q8, ws.qs, st));
-    TS_TRY(run_gemm_tc("gemm_up", m, ts::EPI_GELU, ws.q8, ws.qs, w->w_1, w->s_1, rows, f, d, w->b_1, static_cast<bf16*>(ws.h),
+    TS_TRY(run_layernorm(m, in, rows, w->ln2_g, w->ln2_b, nullptr, ws.q8, ws.qs, st));
+    TS_TRY(run_gemm_tc("gemm_up", m, up, ws.q8, ws.qs, w->w_1, w->s_1, rows, f, d, w->b_1, static_cast<bf16*>(ws.h),
                        nullptr, nullptr, st));
     TS_TRY(run_quantize(ws.h, rows, f, ws.q8, ws.qs, st));
-    return run_gemm_tc("gemm_down", m, ts::EPI_RESID, ws.q8, ws.qs, w->w_2, w->s_2, rows, d, f, w->b_2, static_cast<bf16*>(state),
+    return run_gemm_tc("gemm_down", m, down, ws.q8, ws.qs, w->w_2, w->s_2, rows, d, f, w->b_2, static_cast<bf16*>(out),
                        nullptr, nullptr, st);
   }
-  TS_TRY(run_layernorm(m, state, rows, w->ln2_g, w->ln2_b, ws.xn, nullptr, nullptr, st));
-  TS_TRY(run_gemm_tc("gemm_up", m, ts::EPI_GELU, ws.xn, nullptr, w->w_1, nullptr, rows, f, d, w->b_1, static_cast<bf16*>(ws.h),
+  TS_TRY(run_layernorm(m, in, rows, w->ln2_g, w->ln2_b, ws.xn, nullptr, nullptr, st));
+  TS_TRY(run_gemm_tc("gemm_up", m, up, ws.xn, nullptr, w->w_1, nullptr, rows, f, d, w->b_1, static_cast<bf16*>(ws.h),
                      nullptr, nullptr, st));
-  return run_gemm_tc("gemm_down", m, ts::EPI_RESID, ws.h, nullptr, w->w_2, nullptr, rows, d, f, w->b_2, static_cast<bf16*>(state),
+  return run_gemm_tc("gemm_down", m, down, ws.h, nullptr, w->w_2, nullptr, rows, d, f, w->b_2, static_cast<bf16*>(out),
                      nullptr, nullptr, st);
+}
+
+// state += MLP(state)
+static ts_status run_mlp(const ts_model_desc* m, const ts_layer_weights* w, int rows, void* state, const Workspace& ws,
+                         cudaStream_t st) {
+  return run_mlp_any(m, w, rows, state, state, true, ws, st);
 }
 
 // per-tile copies of the stack input (grid tokens S0, global tokens G0)
@@ -816,30 +845,10 @@ static ts_status run_out_bias(const ts_model_desc* m, const ts_layer_weights* w,
                      nullptr, nullptr, st);
 }
 
-// out = W2 GELU(W1 LN2(in) + b1) + b2 (no residual): the MLP of a shared operation
+// out = MLP(in) (no residual): the MLP of a shared operation
 static ts_status run_mlp_out(const ts_model_desc* m, const ts_layer_weights* w, int rows, const void* in, void* out,
                              const Workspace& ws, cudaStream_t st) {
-  const int d = m->d, f = m->mlp;
-  if (m->dtype == TS_F32) {
-    TS_TRY(run_layernorm(m, in, rows, w->ln2_g, w->ln2_b, ws.xn, nullptr, nullptr, st));
-    TS_TRY(run_gemm_f32("gemm_up", ts::EPI_GELU, static_cast<const float*>(ws.xn), static_cast<const float*>(w->w_1), rows, f, d,
-                        w->b_1, static_cast<float*>(ws.h), st));
-    return run_gemm_f32("gemm_down", ts::EPI_BIAS, static_cast<const float*>(ws.h), static_cast<const float*>(w->w_2), rows, d, f,
-                        w->b_2, static_cast<float*>(out), st);
-  }
-  if (m->dtype == TS_FP8_E4M3) {
-    TS_TRY(run_layernorm(m, in, rows, w->ln2_g, w->ln2_b, nullptr, ws.q8, ws.qs, st));
-    TS_TRY(run_gemm_tc("gemm_up", m, ts::EPI_GELU, ws.q8, ws.qs, w->w_1, w->s_1, rows, f, d, w->b_1, static_cast<bf16*>(ws.h),
-                       nullptr, nullptr, st));
-    TS_TRY(run_quantize(ws.h, rows, f, ws.q8, ws.qs, st));
-    return run_gemm_tc("gemm_down", m, ts::EPI_BIAS, ws.q8, ws.qs, w->w_2, w->s_2, rows, d, f, w->b_2, static_cast<bf16*>(out),
-                       nullptr, nullptr, st);
-  }
-  TS_TRY(run_layernorm(m, in, rows, w->ln2_g, w->ln2_b, ws.xn, nullptr, nullptr, st));
-  TS_TRY(run_gemm_tc("gemm_up", m, ts::EPI_GELU, ws.xn, nullptr, w->w_1, nullptr, rows, f, d, w->b_1, static_cast<bf16*>(ws.h),
-                     nullptr, nullptr, st));
-  return run_gemm_tc("gemm_down", m, ts::EPI_BIAS, ws.h, nullptr, w->w_2, nullptr, rows, d, f, w->b_2, static_cast<bf16*>(out),
-                     nullptr, nullptr, st);
+  return run_mlp_any(m, w, rows, in, out, false, ws, st);
 }
 
 // ============================================================================
@@ -1261,8 +1270,9 @@ ts_status ts_selftest_bounded_wait(long long limit_ns, int* done, void* stream) 
 ts_status ts_op_layernorm(const ts_model_desc* m, const void* x, int rows, const float* g, const float* b, void* y,
                           void* stream) {
   TS_TRY(check_model(m));
-  if (!x || !y || !g || !b || rows < 0) return fail(TS_ERR_INVALID_ARG, "bad argument");
-  if (!aligned16(x) || !aligned16(y) || !aligned16(g) || !aligned16(b)) return fail(TS_ERR_INVALID_ARG, "alignment");
+  const bool rms = m->block == TS_BLOCK_RMS_SWIGLU;
+  if (!x || !y || !g || (!b && !rms) || rows < 0) return fail(TS_ERR_INVALID_ARG, "bad argument");
+  if (!aligned16(x) || !aligned16(y) || !aligned16(g) || (b && !aligned16(b))) return fail(TS_ERR_INVALID_ARG, "alignment");
   return run_layernorm(m, x, rows, g, b, y, nullptr, nullptr, static_cast<cudaStream_t>(stream));
 }
 
@@ -1271,9 +1281,12 @@ ts_status ts_op_linear(const ts_model_desc* m, const void* x, int rows, int K, c
   TS_TRY(check_model(m));
   if (!x || !W || !y || !bias || rows < 0 || K <= 0 || N <= 0) return fail(TS_ERR_INVALID_ARG, "bad argument");
   if (!aligned16(x) || !aligned16(W) || !aligned16(y) || !aligned16(bias)) return fail(TS_ERR_INVALID_ARG, "alignment");
-  if (epi != TS_EPI_BIAS && epi != TS_EPI_BIAS_GELU && epi != TS_EPI_BIAS_RESID)
+  if (epi != TS_EPI_BIAS && epi != TS_EPI_BIAS_GELU && epi != TS_EPI_BIAS_RESID && epi != TS_EPI_BIAS_SWIGLU)
     return fail(TS_ERR_INVALID_ARG, "unknown epilogue");
-  const int e = epi == TS_EPI_BIAS ? ts::EPI_BIAS : epi == TS_EPI_BIAS_GELU ? ts::EPI_GELU : ts::EPI_RESID;
+  const int e = epi == TS_EPI_BIAS        ? ts::EPI_BIAS
+                : epi == TS_EPI_BIAS_GELU ? ts::EPI_GELU
+                : epi == TS_EPI_BIAS_RESID ? ts::EPI_RESID
+                                           : ts::EPI_SWIGLU;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (m->dtype == TS_F32)
     return run_gemm_f32("linear", e, static_cast<const float*>(x), static_cast<const float*>(W), rows, N, K, bias,

@@ -21,11 +21,11 @@ def rel_l2(got, want):
 
 
 def oracle_model(cfg):
-    return OL.Model(cfg.d, cfg.heads, cfg.mlp, cfg.rope_dims, fp8=(cfg.dtype == "fp8"))
+    return OL.Model(cfg.d, cfg.heads, cfg.mlp, cfg.rope_dims, fp8=(cfg.dtype == "fp8"), block=cfg.block)
 
 
 def model_desc(cfg):
-    return B.model_desc(cfg.d, cfg.heads, cfg.mlp, cfg.dtype, cfg.rope_dims)
+    return B.model_desc(cfg.d, cfg.heads, cfg.mlp, cfg.dtype, cfg.rope_dims, block=cfg.block)
 
 
 def dev(a, dtype):

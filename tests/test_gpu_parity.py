@@ -10,6 +10,8 @@ Tolerances (relative L2 against the oracle): fp32 path 1e-5 per layer; bf16 path
 the rounding of one bf16 store (2^-8 relative per element) as their scale.
 """
 
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -316,6 +318,139 @@ def test_block_partial(cfg, shared):
     got = host(Xd).reshape(op.T, op.N, cfg.d)
     assert rel_l2(got, want) < _tol(cfg)
     assert rel_l2(got - X, want - X) < 3 * _tol(cfg)
+
+
+# ---------------------------------------------------------------------------
+# RMSNorm + SwiGLU block flavour (Tab. S6)
+# ---------------------------------------------------------------------------
+SMALL_SW = dataclasses.replace(SMALL, name="small_swiglu_bf16", block="rms_swiglu")
+VOL_SW = dataclasses.replace(VOL, name="vol_swiglu_bf16", block="rms_swiglu")
+VIT14_SW = dataclasses.replace(VIT14, name="vit14_swiglu_fp32", block="rms_swiglu")
+SMALL_FP8_SW = dataclasses.replace(SMALL_FP8, name="small_swiglu_fp8", block="rms_swiglu")
+_SW = [SMALL_SW, VOL_SW, VIT14_SW, SMALL_FP8_SW]
+
+
+@pytest.mark.parametrize("cfg", [SMALL_SW, VIT14_SW], ids=lambda c: c.name)
+def test_rmsnorm(cfg):
+    c = case(cfg)
+    x = dev(c.S, c.dt)
+    y = torch.empty_like(x)
+    B.op_layernorm(c.m, x, c.dlayers[0]["ln1_g"], None, y)
+    want = OL.rms_norm(c.S, c.layers[0]["ln1_g"], 1e-6)
+    assert rel_l2(host(y), want) < (1e-6 if cfg.dtype == "f32" else 3e-3)
+
+
+def _swiglu_want(x, w, b):
+    n = w.shape[0] // 2
+    a = x @ w.T + b
+    return OL.silu(a[:, :n]) * a[:, n:]
+
+
+@pytest.mark.parametrize("M,K,N", [(300, 256, 256), (129, 512, 192), (1, 256, 64), (2320, 512, 2048),
+                                   (777, 1024, 320)])
+def test_linear_swiglu_bf16(M, K, N):
+    rng = np.random.default_rng(M * 3 + N)
+    x = W.round_to(rng.standard_normal((M, K)), "bf16")
+    w = W.round_to(0.05 * rng.standard_normal((2 * N, K)), "bf16")
+    b = W.round_to(0.5 * rng.standard_normal(2 * N), "f32")
+    m = B.model_desc(256, 4, 256, "bf16", (0, 32, 32), block="rms_swiglu")
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    B.op_linear(m, dev(x, torch.bfloat16), dev(w, torch.bfloat16), dev(b, torch.float32), y,
+                epi=B.TS_EPI_BIAS_SWIGLU)
+    assert rel_l2(host(y), _swiglu_want(x, w, b)) < 3e-3
+
+
+@pytest.mark.parametrize("M,K,N", [(70, 48, 40), (129, 64, 96)])
+def test_linear_swiglu_f32(M, K, N):
+    rng = np.random.default_rng(M + N)
+    x = W.round_to(rng.standard_normal((M, K)), "f32")
+    w = W.round_to(0.2 * rng.standard_normal((2 * N, K)), "f32")
+    b = W.round_to(0.5 * rng.standard_normal(2 * N), "f32")
+    m = B.model_desc(64, 1, 64, "f32", (0, 32, 32), block="rms_swiglu")
+    y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    B.op_linear(m, dev(x, torch.float32), dev(w, torch.float32), dev(b, torch.float32), y, epi=B.TS_EPI_BIAS_SWIGLU)
+    assert rel_l2(host(y), _swiglu_want(x, w, b)) < 1e-6
+
+
+def test_linear_swiglu_fp8():
+    from oracle import fp8 as F8
+    M, K, N = 300, 256, 256
+    rng = np.random.default_rng(5)
+    x = W.round_to(rng.standard_normal((M, K)), "bf16")
+    w = W.round_to(0.02 * rng.standard_normal((2 * N, K)), "bf16")
+    b = W.round_to(0.1 * rng.standard_normal(2 * N), "f32")
+    m = B.model_desc(256, 4, 256, "fp8", (0, 32, 32), block="rms_swiglu")
+    q = torch.empty((2 * N, K), dtype=torch.uint8, device="cuda")
+    s = torch.empty(2 * N, dtype=torch.float32, device="cuda")
+    B.quantize_rows_e4m3(dev(w, torch.bfloat16), q, s)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    scratch = torch.empty(M * K + 4 * M + 512, dtype=torch.uint8, device="cuda")
+    B.op_linear(m, dev(x, torch.bfloat16), q, dev(b, torch.float32), y, epi=B.TS_EPI_BIAS_SWIGLU, w_scale=s,
+                scratch=scratch)
+    a = F8.scaled_matmul(x, w) + b
+    want = OL.silu(a[:, :N]) * a[:, N:]
+    assert rel_l2(host(y), want) < 1e-2
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_silu_epilogue_values(dtype):
+    """Gate rows = identity, up rows = 0 with bias 1: the layer returns silu(x) itself,
+    over x in [-30, 30] with 0 and both tails; fp32 within 2e-6 (relative to
+    max(1, |silu|)), bf16 within its output rounding."""
+    n = 64
+    x = np.linspace(-30.0, 30.0, 128 * n).reshape(128, n)
+    x[0, 0] = 0.0
+    dt = torch.float32 if dtype == "f32" else torch.bfloat16
+    x = W.round_to(x, dtype)
+    w = np.concatenate([np.eye(n), np.zeros((n, n))])
+    b = np.concatenate([np.zeros(n), np.ones(n)])
+    m = B.model_desc(256, 4, 256, dtype, (0, 32, 32), block="rms_swiglu")
+    y = torch.empty((128, n), dtype=dt, device="cuda")
+    B.op_linear(m, dev(x, dt), dev(w, dt), dev(b, torch.float32), y, epi=B.TS_EPI_BIAS_SWIGLU)
+    want = x / (1.0 + np.exp(-x))
+    err = np.max(np.abs(host(y) - want) / np.maximum(1.0, np.abs(want)))
+    assert err < (2e-6 if dtype == "f32" else 2.0 ** -8)
+
+
+@pytest.mark.parametrize("cfg", _SW, ids=lambda c: c.name)
+def test_swiglu_block_shared_and_tiled(cfg):
+    c = case(cfg)
+    S_in = c.S
+    S = dev(S_in, c.dt)
+    B.block_shared(c.plan, c.m, c.wlist[0], S, c.workspace())
+    want = OL.block_shared(S_in, c.layers[0], c.om, c.oplan)
+    assert rel_l2(host(S), want) < _tol(cfg)
+    assert rel_l2(host(S) - S_in, want - S_in) < 3 * _tol(cfg)
+    X_in = OL.gather(S_in, c.oplan)
+    X = dev(X_in.reshape(c.oplan.T * c.oplan.N, -1), c.dt)
+    B.block_tiled(c.plan, c.m, c.wlist[0], X, c.workspace())
+    want = OL.block_tiled(X_in, c.layers[0], c.om, c.oplan).reshape(X.shape)
+    assert rel_l2(host(X), want) < _tol(cfg)
+
+
+@pytest.mark.parametrize("cfg", _SW, ids=lambda c: c.name)
+def test_swiglu_decode_stack(cfg):
+    c = case(cfg)
+    for k in (0, 1):
+        got = host(_run_stack(c, k))
+        want = OL.decode_stack(c.S0, c.G0, c.layers, c.om, c.oplan, k)
+        assert rel_l2(got, want) < _tol(cfg), k
+
+
+@pytest.mark.parametrize("cfg", [SMALL_SW, SMALL_FP8_SW], ids=lambda c: c.name)
+@pytest.mark.parametrize("shared", [("mlp",), ("qkv", "out", "mlp")], ids=lambda s: "+".join(s))
+def test_swiglu_block_partial(cfg, shared):
+    c = case(cfg)
+    op = c.oplan
+    X = OL.gather(c.S, op) + 0.1 * np.random.default_rng(22).standard_normal((op.T, op.N, cfg.d))
+    X = W.round_to(X, cfg.dtype if cfg.dtype != "fp8" else "bf16")
+    Xd = dev(X.reshape(op.T * op.N, cfg.d), c.dt)
+    ops = 0
+    for s_ in shared:
+        ops |= _SHARE[s_]
+    B.block_partial(c.plan, c.m, c.wlist[0], ops, Xd, c.workspace())
+    want = OL.block_partial(X, c.layers[0], c.om, op, shared)
+    assert rel_l2(host(Xd).reshape(op.T, op.N, cfg.d), want) < _tol(cfg)
 
 
 def test_block_partial_rejects_unknown_operations():
