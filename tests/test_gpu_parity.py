@@ -98,8 +98,9 @@ def test_gelu_epilogue_matches_exact_erf():
     assert np.max(np.abs(got - want) / np.maximum(1.0, np.abs(want))) < 2e-6
 
 
+# (2320, 2048, 512) and (2320, 512, 512): the 48 x 48 layer's MLP down and out-projection
 @pytest.mark.parametrize("M,K,N", [(300, 256, 512), (128, 512, 768), (129, 256, 192), (1, 256, 64), (2320, 512, 1536),
-                                   (777, 2048, 512)])
+                                   (777, 2048, 512), (2320, 2048, 512), (2320, 512, 512)])
 @pytest.mark.parametrize("epi", [B.TS_EPI_BIAS, B.TS_EPI_BIAS_GELU, B.TS_EPI_BIAS_RESID])
 def test_linear_bf16(M, K, N, epi):
     rng = np.random.default_rng(M * 7 + N + epi)
@@ -118,7 +119,7 @@ def test_linear_bf16(M, K, N, epi):
     assert rel_l2(host(y), want) < 3e-3
 
 
-@pytest.mark.parametrize("M,K,N", [(300, 256, 512), (129, 512, 256), (64, 1536, 4608)])
+@pytest.mark.parametrize("M,K,N", [(300, 256, 512), (129, 512, 256), (64, 1536, 4608), (300, 1024, 512)])
 def test_linear_fp8(M, K, N):
     from oracle import fp8 as F8
     rng = np.random.default_rng(M + K)
