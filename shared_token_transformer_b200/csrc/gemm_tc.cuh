@@ -314,13 +314,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int m0, n0;
       gemm_tile_origin(tile, mt, args.N / BN, BN, m0, n0);
       const int row = m0 + quarter * 32 + lane;
-      if (!mbar_wait(bar_tfull + 8 * acc, use & 1)) break;
-      tc_fence_after();
-      const uint32_t trow = tmem + acc * BN + (static_cast<uint32_t>(quarter * 32) << 16);
+      // the row's scale and coordinates are loaded while the accumulator fills
       float rs = 1.f;
       if (FP8 && row < args.M) rs = __ldg(args.a_scale + row);
       int4 pos = make_int4(0, 0, 0, 0);
       if (EPI == EPI_QKV && row < args.M) pos = __ldg(args.pos + row);
+      if (!mbar_wait(bar_tfull + 8 * acc, use & 1)) break;
+      tc_fence_after();
+      const uint32_t trow = tmem + acc * BN + (static_cast<uint32_t>(quarter * 32) << 16);
       int mine = 0;
 #pragma unroll 1
       for (int c = half; c < NCHUNK; c += 2) ++mine;

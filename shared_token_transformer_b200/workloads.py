@@ -68,6 +68,12 @@ CONFIGS = {
     "video44x80_fp8": Config("video44x80_fp8", (4, 44, 80), (4, 32, 32), (4, 24, 24), 1536, 24, 6144,
                              "fp8", L=24, k=6, rope_dims=(16, 24, 24), ks=(0, 4, 6, 24),
                              note="as video44x80_bf16 with e4m3 GEMMs; k in 0, 4, 6, 24"),
+    # spatio-temporal tiling: 8 latent frames, windows of 4 frames at temporal stride 2, so tiles
+    # overlap in time as well as in space (a token lies in up to 8 tiles)
+    "video88x80_st_bf16": Config("video88x80_st_bf16", (8, 44, 80), (4, 32, 32), (2, 24, 24), 1536, 24, 6144,
+                                 "bf16", L=24, k=6, rope_dims=(16, 24, 24),
+                                 note="8x44x80 grid, d=1536, 24 heads, MLP 6144, window 4x32x32 stride 2x24x24 "
+                                      "(temporal overlap), L=24 k=6, bf16"),
     # image-autoencoder-scale decode at 4K (256x256 tokens) and 2K (128x128 tokens)
     "image4k_bf16": Config("image4k_bf16", (1, 256, 256), (1, 32, 32), (1, 24, 24), 1024, 16, 4096, "bf16",
                            L=16, k=4, rope_dims=(0, 32, 32),

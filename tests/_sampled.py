@@ -21,15 +21,6 @@ def sample_tokens(op, rng, n=24):
     return sorted(set(int(u) for u in picks))
 
 
-
-    cfg = W.CONFIGS[name]
-    op = OP.make_plan(cfg.grid, cfg.win, cfg.stride)
-    dr = W.Draw(cfg, op.T, seed=seed, affine=True)
-    S0, G0 = dr.states()
-    layer = dr.layer()
-    return cfg, op, np.concatenate([S0, G0]), layer
-
-
 def oracle_shared_rows(S, layer, om, op, toks, globals_):
     """Rows `toks` (grid tokens) and U + t for t in globals_ of one shared layer."""
     U, N = op.U, op.N

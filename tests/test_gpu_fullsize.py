@@ -25,7 +25,7 @@ from _sampled import oracle_shared_rows, sample_tokens
 
 pytestmark = pytest.mark.gpu
 
-FULL = ["video44x80_bf16", "video44x80_fp8", "image4k_bf16", "image2k_bf16"]
+FULL = ["video44x80_bf16", "video44x80_fp8", "image4k_bf16", "image2k_bf16", "video88x80_st_bf16"]
 
 
 @pytest.fixture(scope="module", autouse=True)
