@@ -8,9 +8,10 @@ What the pages fix
         - Norm1, QKV projection and QK-RMSNorm run once per token on the shared
           state (exact: identical inputs give identical results);
         - RoPE runs per tile on tile coordinates, as released;
-        - attention is dense and per tile, with the tile's own registers (here one
-          global token per tile) that attend only to their own tile; keys and
-          values come from the shared states;
+        - attention is dense and per tile, with the tile's own registers (R per
+          tile, R14; one global token in the benchmark configurations) that
+          attend only to their own tile; keys and values come from the shared
+          states;
         - the blend of attention outputs of overlap tokens is the only
           approximation and happens in every shared layer.
     * [TileShare] Fig. 2: out-projection and MLP also run once per token; overlap
@@ -164,15 +165,16 @@ def qkv_project(x, p, m: Model):
 
 
 def tile_attention(q, k, v, slot_pos, m: Model):
-    """Attention of one tile: rows [global token, window slot 0..Nw-1].
+    """Attention of one tile: rows [its R registers, window slot 0..Nw-1].
 
-    RoPE on tile-local coordinates for the window rows only (R5, R6).
+    RoPE on tile-local coordinates for the window rows only (R5, R6, R14).
     Returns the attention output [N, d] before the out-projection.
     """
+    R = q.shape[0] - slot_pos.shape[0]
     q = q.copy()
     k = k.copy()
-    q[1:] = rope(q[1:], slot_pos, m)
-    k[1:] = rope(k[1:], slot_pos, m)
+    q[R:] = rope(q[R:], slot_pos, m)
+    k[R:] = rope(k[R:], slot_pos, m)
     return attention(q, k, v)
 
 
@@ -196,13 +198,19 @@ def mlp_residual(x, p, m: Model):
 # tile <-> token maps
 # ---------------------------------------------------------------------------
 
+def tile_rows(plan, t):
+    """Rows of the shared state that tile t attends over: its registers, then its window."""
+    U, R = plan.U, plan.R
+    return np.concatenate([np.arange(U + t * R, U + (t + 1) * R), plan.tile_tok[t]])
+
+
 def gather(S, plan):
-    """Per-tile copies X [T, N, d] of a shared state S [U + T, d]."""
-    T, N, U = plan.T, plan.N, plan.U
+    """Per-tile copies X [T, N, d] of a shared state S [U + T*R, d]."""
+    T, N, U, R = plan.T, plan.N, plan.U, plan.R
     X = np.empty((T, N, S.shape[1]), dtype=S.dtype)
     for t in range(T):
-        X[t, 0] = S[U + t]
-        X[t, 1:] = S[plan.tile_tok[t]]
+        X[t, :R] = S[U + t * R: U + (t + 1) * R]
+        X[t, R:] = S[plan.tile_tok[t]]
     return X
 
 
@@ -210,16 +218,16 @@ def merge(P, plan):
     """Blend per-tile rows P [T, N, d] into one row per token (Fig. 2, R8).
 
     S[u] = sum over the tiles t covering u, in ascending t, of w-bar[t, u] *
-    P[t, slot of u]; S[U + t] = P[t, 0] (each global token keeps its tile's row).
+    P[t, slot of u]; S[U + t*R + i] = P[t, i] (each register keeps its tile's row).
     """
-    T, N, U = plan.T, plan.N, plan.U
+    T, N, U, R = plan.T, plan.N, plan.U, plan.R
     flat = P.reshape(T * N, -1)
-    S = np.zeros((U + T, P.shape[2]), dtype=np.float64)
+    S = np.zeros((U + T * R, P.shape[2]), dtype=np.float64)
     for u in range(U):
         for e in range(plan.tok_ptr[u], plan.tok_ptr[u + 1]):
             S[u] += plan.tok_w[e] * flat[plan.tok_ent[e]]
     for t in range(T):
-        S[U + t] = P[t, 0]
+        S[U + t * R: U + (t + 1) * R] = P[t, :R]
     return S
 
 
@@ -240,22 +248,22 @@ def block_tiled(X, p, m: Model, plan):
 
 
 def shared_attention_outputs(S, p, m: Model, plan):
-    """Per-tile attention outputs O [T, N, d] of a shared layer on S [U + T, d].
+    """Per-tile attention outputs O [T, N, d] of a shared layer on S [U + T*R, d].
 
-    Norm1/QKV/QK-norm once per token; then, per tile, the rows of the tile's global
-    token and window tokens are taken from the shared q, k, v (Tab. S1).
+    Norm1/QKV/QK-norm once per token; then, per tile, the rows of the tile's
+    registers and window tokens are taken from the shared q, k, v (Tab. S1).
     """
-    U, T, N = plan.U, plan.T, plan.N
+    T, N = plan.T, plan.N
     q, k, v = qkv_project(S, p, m)
     O = np.empty((T, N, m.d), dtype=np.float64)
     for t in range(T):
-        rows = np.concatenate([[U + t], plan.tile_tok[t]])
+        rows = tile_rows(plan, t)
         O[t] = tile_attention(q[rows], k[rows], v[rows], plan.slot_pos, m)
     return O
 
 
 def block_shared(S, p, m: Model, plan):
-    """One TileShare shared layer on the shared state S [U + T, d] (Fig. 2, Tab. S1)."""
+    """One TileShare shared layer on the shared state S [U + T*R, d] (Fig. 2, Tab. S1)."""
     S = S.astype(np.float64)
     O = shared_attention_outputs(S, p, m, plan)
     A = merge(O, plan)
@@ -286,7 +294,7 @@ def block_partial(X, p, m: Model, plan, shared):
     if "qkv" in shared:
         q, k, v = qkv_project(merge(X, plan), p, m)
         for t in range(T):
-            rows = np.concatenate([[U + t], plan.tile_tok[t]])
+            rows = tile_rows(plan, t)
             O[t] = tile_attention(q[rows], k[rows], v[rows], plan.slot_pos, m)
     else:
         for t in range(T):
@@ -308,7 +316,8 @@ def block_partial(X, p, m: Model, plan, shared):
 def decode_stack(S0, G0, layers, m: Model, plan, k: int):
     """TileShare-k: layers 0..k-1 per tile, the rest shared; returns the U token rows.
 
-    S0 [U, d] are the grid tokens entering layer 0, G0 [T, d] the global tokens.
+    S0 [U, d] are the grid tokens entering layer 0, G0 [T*R, d] the registers
+    (tile t's register i in row t*R + i).
     With k = L this is overlapping tiled decoding with the tiles blended by w-bar at
     the end (abstract; R8).
     """

@@ -26,7 +26,13 @@ Readings taken where the pages are silent (stated here and in the design doc)
        tile-local raster order (f, y, x); grid tokens u = (f*H + y)*W + x.  The
        per-tile state of tile t has N = Nw + 1 rows: row 0 is the tile's global
        token, row 1 + j its window slot j.  A (tile, slot) entry is addressed as
-       t*N + 1 + j.
+       t*N + 1 + j (R registers per tile: see R14).
+    R14 registers ([TileShare] Tab. S1: "one set per tile, as released"; in shared
+       layers they stay per tile and attend only to their own tile): each tile has
+       R register tokens (R = 1: the one global token of the benchmark
+       configurations).  The per-tile state has N = Nw + R rows, rows 0 .. R-1 the
+       tile's registers and row R + j its window slot j, so an entry is t*N + R + j;
+       the shared state has U + T*R rows, tile t's register i at U + t*R + i.
     R11 hard stitching (blend rule "hard"; [TileShare] Tab. 2 and Tab. S2 list a
        "Hard stitching" baseline, Tab. S11 describes it as each pixel taken from its
        dominant tile): applied to the blend of overlap tokens, each token takes its
@@ -81,9 +87,10 @@ class Plan:
     wraw: np.ndarray     # [T, Nw] float64, unnormalised weight of slot j of tile t
     wbar: np.ndarray     # [T, Nw] float64, normalised blend weight
     tok_ptr: np.ndarray  # [U + 1] int64, CSR row pointer over grid tokens
-    tok_ent: np.ndarray  # [nnz] int64, entry t*N + 1 + j, ascending t per token
+    tok_ent: np.ndarray  # [nnz] int64, entry t*N + R + j, ascending t per token
     tok_w: np.ndarray    # [nnz] float64, w-bar of that entry
     coverage: np.ndarray = field(default=None)  # [U] int64, tiles per token
+    R: int = 1           # register tokens per tile (R14)
 
     @property
     def T(self):
@@ -95,7 +102,12 @@ class Plan:
 
     @property
     def N(self):
-        return self.Nw + 1
+        return self.Nw + self.R
+
+    @property
+    def G(self):
+        """Register rows of the shared state, T * R."""
+        return self.T * self.R
 
     @property
     def U(self):
@@ -107,13 +119,16 @@ class Plan:
         return int(self.tok_ent.shape[0])
 
 
-def make_plan(grid, win, stride, rule: str = "ramp") -> Plan:
+def make_plan(grid, win, stride, rule: str = "ramp", registers: int = 1) -> Plan:
     """Tile plan for a token grid (F, H, W); 2-D grids use F = wf = sf = 1.
 
     rule "ramp": w-bar of R2 (normalised ramp weights); rule "hard": R11.
+    registers: register tokens per tile (R14).
     """
     if rule not in ("ramp", "hard"):
         raise ValueError(f"unknown blend rule {rule!r}")
+    if registers < 1:
+        raise ValueError("a tile has at least one register token")
     F, H, W = (int(v) for v in grid)
     wf, wh, ww = (int(v) for v in win)
     sf, sh, sw = (int(v) for v in stride)
@@ -138,7 +153,7 @@ def make_plan(grid, win, stride, rule: str = "ramp") -> Plan:
             wraw[t, j] = rf[a, lf] * rh[b, ly] * rw[c, lx]
 
     U = F * H * W
-    N = Nw + 1
+    N = Nw + registers
     total = np.zeros(U, dtype=np.float64)
     coverage = np.zeros(U, dtype=np.int64)
     for t in range(T):
@@ -172,7 +187,7 @@ def make_plan(grid, win, stride, rule: str = "ramp") -> Plan:
         for j in range(Nw):
             if rule == "hard" and wbar[t, j] == 0.0:
                 continue
-            lists[tile_tok[t, j]].append((t * N + 1 + j, wbar[t, j]))
+            lists[tile_tok[t, j]].append((t * N + registers + j, wbar[t, j]))
     tok_ptr = np.zeros(U + 1, dtype=np.int64)
     for u in range(U):
         tok_ptr[u + 1] = tok_ptr[u] + len(lists[u])
@@ -180,7 +195,7 @@ def make_plan(grid, win, stride, rule: str = "ramp") -> Plan:
     tok_w = np.array([wv for lst in lists for _, wv in lst], dtype=np.float64)
     return Plan(grid=(F, H, W), win=(wf, wh, ww), stride=(sf, sh, sw), origins=origins,
                 tile_tok=tile_tok, slot_pos=slot_pos, wraw=wraw, wbar=wbar, tok_ptr=tok_ptr,
-                tok_ent=tok_ent, tok_w=tok_w, coverage=coverage)
+                tok_ent=tok_ent, tok_w=tok_w, coverage=coverage, R=registers)
 
 
 def duplicated_fraction(p: Plan) -> float:

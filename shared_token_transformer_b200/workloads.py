@@ -36,6 +36,7 @@ class Config:
     rope_dims: tuple      # channels of the head dimension given to the (f, y, x) axes
     note: str = ""
     ks: tuple = field(default=())   # further k values the configuration compares
+    R: int = 1                      # register tokens per tile (one global token in the benchmarks)
     block: str = "ln_gelu"          # "ln_gelu" or "rms_swiglu" (MLP up of 2 x mlp rows: gate, then up)
 
     @property
@@ -123,10 +124,10 @@ class Draw:
         self.rng = np.random.Generator(np.random.PCG64(seed))
 
     def states(self):
-        """(S0 [U, d], G0 [T, d]) rounded to the working dtype, as float64."""
+        """(S0 [U, d], G0 [T*R, d]) rounded to the working dtype, as float64."""
         c = self.cfg
         S0 = self.rng.standard_normal((c.U, c.d))
-        G0 = self.rng.standard_normal((self.T, c.d))
+        G0 = self.rng.standard_normal((self.T * c.R, c.d))
         return round_to(S0, c.dtype), round_to(G0, c.dtype)
 
     def layer(self):

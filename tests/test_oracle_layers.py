@@ -30,7 +30,7 @@ def _model(cfg):
 
 
 def _setup(cfg, seed=0, affine=True):
-    p = P.make_plan(cfg.grid, cfg.win, cfg.stride)
+    p = P.make_plan(cfg.grid, cfg.win, cfg.stride, registers=cfg.R)
     dr = W.Draw(cfg, p.T, seed=seed, affine=affine)
     S0, G0 = dr.states()
     return p, np.concatenate([S0, G0]), dr.layers()
@@ -41,10 +41,12 @@ def _setup(cfg, seed=0, affine=True):
 # ---------------------------------------------------------------------------
 
 def _torch_block(x, prm, m, pos):
-    """One pre-LN ViT block; row 0 is unrotated, rows 1.. use positions pos."""
+    """One pre-LN ViT block; the first len(x) - len(pos) rows (registers) are
+    unrotated, the others use positions pos."""
     t = {k: torch.from_numpy(np.asarray(v)) for k, v in prm.items()}
     x = torch.from_numpy(x)
     n, d, h, hd = x.shape[0], m.d, m.heads, m.hd
+    R = n - pos.shape[0]
     swiglu = m.block == "rms_swiglu"
 
     def norm(z, g, b):
@@ -64,10 +66,10 @@ def _torch_block(x, prm, m, pos):
             if half:
                 j = torch.arange(half, dtype=torch.float64)
                 ang = torch.from_numpy(pos[:, ax].astype(np.float64))[:, None] * m.rope_base ** (-2 * j / D)
-                zc = torch.complex(z[1:, :, off:off + half], z[1:, :, off + half:off + D])
+                zc = torch.complex(z[R:, :, off:off + half], z[R:, :, off + half:off + D])
                 zr = zc * torch.polar(torch.ones_like(ang), ang)[:, None, :]
-                out[1:, :, off:off + half] = zr.real
-                out[1:, :, off + half:off + D] = zr.imag
+                out[R:, :, off:off + half] = zr.real
+                out[R:, :, off + half:off + D] = zr.imag
             off += D
         return out
 
@@ -86,10 +88,10 @@ def _torch_block(x, prm, m, pos):
     return x.numpy()
 
 
-@pytest.mark.parametrize("block", ["ln_gelu", "rms_swiglu"])
+@pytest.mark.parametrize("block,R", [("ln_gelu", 1), ("rms_swiglu", 1), ("ln_gelu", 4)])
 @pytest.mark.parametrize("grid,rope", [((1, 6, 7), (0, 8, 8)), ((2, 3, 4), (4, 6, 6))])
-def test_single_tile_equals_library_block(grid, rope, block):
-    cfg = W.Config("one_tile", grid, grid, grid, 64, 4, 96, "f32", 1, 0, rope, block=block)
+def test_single_tile_equals_library_block(grid, rope, block, R):
+    cfg = W.Config("one_tile", grid, grid, grid, 64, 4, 96, "f32", 1, 0, rope, block=block, R=R)
     m = _model(cfg)
     p, S, layers = _setup(cfg)
     assert p.T == 1
@@ -163,7 +165,7 @@ def _loop_layer_shared(S, prm, m, p):
     A = [[0.0] * d for _ in range(n)]
     for t in range(T):
         of, oy, ox = (int(c) for c in p.origins[t])
-        rows, poss = [U + t], [None]
+        rows, poss = [U + t * p.R + i for i in range(p.R)], [None] * p.R
         for lf in range(wf):
             for ly in range(wh):
                 for lx in range(ww):
@@ -178,10 +180,10 @@ def _loop_layer_shared(S, prm, m, p):
                 ex = [math.exp(s - mx) for s in sc]
                 z = sum(ex)
                 o = [sum(ex[j] / z * v[rows[j]][hh][c] for j in range(len(rows))) for c in range(hd)]
-                if i == 0:
+                if i < p.R:
                     wgt = 1.0
                 else:
-                    wgt = p.wbar[t, i - 1]
+                    wgt = p.wbar[t, i - p.R]
                 for c in range(hd):
                     A[r][hh * hd + c] += wgt * o[c]
     out = np.empty_like(S)
@@ -192,13 +194,14 @@ def _loop_layer_shared(S, prm, m, p):
     return out
 
 
-@pytest.mark.parametrize("grid,win,stride,rope,block", [
-    ((1, 5, 5), (1, 3, 3), (1, 2, 2), (0, 2, 2), "ln_gelu"),
-    ((2, 4, 5), (2, 3, 3), (1, 1, 2), (2, 2, 4), "ln_gelu"),
-    ((1, 5, 5), (1, 3, 3), (1, 2, 2), (0, 2, 2), "rms_swiglu"),
+@pytest.mark.parametrize("grid,win,stride,rope,block,R", [
+    ((1, 5, 5), (1, 3, 3), (1, 2, 2), (0, 2, 2), "ln_gelu", 1),
+    ((2, 4, 5), (2, 3, 3), (1, 1, 2), (2, 2, 4), "ln_gelu", 1),
+    ((1, 5, 5), (1, 3, 3), (1, 2, 2), (0, 2, 2), "rms_swiglu", 1),
+    ((1, 5, 5), (1, 3, 3), (1, 2, 2), (0, 2, 2), "ln_gelu", 3),
 ])
-def test_shared_layer_brute_force(grid, win, stride, rope, block):
-    cfg = W.Config("bf", grid, win, stride, 16, 2, 24, "f32", 1, 0, rope, block=block)
+def test_shared_layer_brute_force(grid, win, stride, rope, block, R):
+    cfg = W.Config("bf", grid, win, stride, 16, 2, 24, "f32", 1, 0, rope, block=block, R=R)
     m = _model(cfg)
     p, S, layers = _setup(cfg, seed=3)
     prm = {k: (v.tolist() if v.ndim == 2 else list(v)) for k, v in layers[0].items()}
@@ -211,9 +214,9 @@ def test_shared_layer_brute_force(grid, win, stride, rope, block):
 # exactness statements of the pages
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("block", ["ln_gelu", "rms_swiglu"])
-def test_no_overlap_shared_equals_tiled(block):
-    cfg = dataclasses.replace(W.CONFIGS["vit16_nooverlap_fp32"], block=block)
+@pytest.mark.parametrize("block,R", [("ln_gelu", 1), ("rms_swiglu", 1), ("ln_gelu", 3)])
+def test_no_overlap_shared_equals_tiled(block, R):
+    cfg = dataclasses.replace(W.CONFIGS["vit16_nooverlap_fp32"], block=block, R=R)
     m = _model(cfg)
     p, S, layers = _setup(cfg)
     got = Lo.block_shared(S, layers[0], m, p)
@@ -238,25 +241,28 @@ def test_blend_before_or_after_out_projection():
     np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
 
 
-def test_identical_per_tile_states_stay_identical():
-    cfg = W.small_config(grid=(1, 9, 9), win=(1, 5, 5), stride=(1, 2, 2), d=32, heads=2, mlp=48, dtype="f32")
+@pytest.mark.parametrize("R", [1, 3])
+def test_identical_per_tile_states_stay_identical(R):
+    cfg = dataclasses.replace(W.small_config(grid=(1, 9, 9), win=(1, 5, 5), stride=(1, 2, 2), d=32, heads=2,
+                                             mlp=48, dtype="f32"), R=R)
     m = _model(cfg)
     p, S, layers = _setup(cfg, seed=7)
+    assert S.shape[0] == p.U + p.T * R
     X = Lo.gather(S, p)
     q, k, v = Lo.qkv_project(S, layers[0], m)
     for t in range(p.T):
         qt, kt, vt = Lo.qkv_project(X[t], layers[0], m)
-        rows = np.concatenate([[p.U + t], p.tile_tok[t]])
+        rows = np.concatenate([[p.U + t * R + i for i in range(R)], p.tile_tok[t]])
         for a, b in ((qt, q), (kt, k), (vt, v)):
             np.testing.assert_allclose(a, b[rows], rtol=0, atol=1e-14)
     # merging identical copies returns the state itself
     np.testing.assert_allclose(Lo.merge(X, p), S, rtol=0, atol=1e-14)
 
 
-@pytest.mark.parametrize("block", ["ln_gelu", "rms_swiglu"])
-def test_stack_k_equals_L_is_tiled_decoding_blended_at_the_end(block):
-    cfg = W.small_config(grid=(1, 10, 9), win=(1, 6, 5), stride=(1, 4, 3), d=32, heads=2, mlp=48,
-                         dtype="f32", L=3, k=3, block=block)
+@pytest.mark.parametrize("block,R", [("ln_gelu", 1), ("rms_swiglu", 1), ("ln_gelu", 2)])
+def test_stack_k_equals_L_is_tiled_decoding_blended_at_the_end(block, R):
+    cfg = dataclasses.replace(W.small_config(grid=(1, 10, 9), win=(1, 6, 5), stride=(1, 4, 3), d=32, heads=2,
+                                             mlp=48, dtype="f32", L=3, k=3, block=block), R=R)
     m = _model(cfg)
     p, S, layers = _setup(cfg, seed=11)
     got = Lo.decode_stack(S[:p.U], S[p.U:], layers, m, p, k=3)

@@ -197,3 +197,21 @@ def test_hard_stitch_equals_ramp_without_overlap():
         np.testing.assert_array_equal(a.tok_ptr, b.tok_ptr)
         np.testing.assert_array_equal(a.tok_ent, b.tok_ent)
         np.testing.assert_array_equal(a.tok_w, b.tok_w)
+
+
+@pytest.mark.parametrize("R", [2, 5])
+def test_registers_shift_the_entries_only(R):
+    """R register tokens per tile (R14): the window slots move to rows R.. of each
+    tile's state, so every entry t*N + 1 + j of the one-register plan becomes
+    t*(Nw + R) + R + j; weights, tiles and coverage do not change."""
+    g, w, st = (2, 9, 11), (2, 5, 6), (1, 3, 4)
+    one = P.make_plan(g, w, st)
+    p = P.make_plan(g, w, st, registers=R)
+    assert p.N == p.Nw + R and p.G == p.T * R
+    t, j = np.divmod(one.tok_ent, one.N)
+    np.testing.assert_array_equal(p.tok_ent, t * (one.Nw + R) + R + (j - 1))
+    np.testing.assert_array_equal(p.tok_ptr, one.tok_ptr)
+    np.testing.assert_array_equal(p.tok_w, one.tok_w)
+    np.testing.assert_array_equal(p.tile_tok, one.tile_tok)
+    with pytest.raises(ValueError):
+        P.make_plan(g, w, st, registers=0)
