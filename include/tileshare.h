@@ -25,9 +25,12 @@
  *   grid tokens  u = (f * H + y) * W + x for a grid of F x H x W tokens, U = F*H*W.
  *   tiles        T tiles in raster order of their (f, y, x) origins.
  *   window slot  j = (lf * wh + ly) * ww + lx, tile-local raster order, Nw = wf*wh*ww.
- *   shared state S [U + T, d]: the U grid tokens, then one global token per tile.
- *   per-tile state X [T, N, d], N = Nw + 1: row 0 of tile t is its global token,
- *                row 1 + j its window slot j.
+ *   registers    R register tokens per tile ([TileShare] Tab. S1: one set per
+ *                tile; R = 1, one global token, unless the plan says otherwise).
+ *   shared state S [U + T*R, d]: the U grid tokens, then tile t's registers at
+ *                rows U + t*R .. U + t*R + R - 1.
+ *   per-tile state X [T, N, d], N = Nw + R: rows 0 .. R-1 of tile t are its
+ *                registers, row R + j its window slot j.
  */
 #ifndef TILESHARE_H
 #define TILESHARE_H
@@ -90,7 +93,7 @@ typedef struct ts_plan_s* ts_plan_t;
 /* Read-only view of a plan.  Host arrays stay valid until ts_plan_destroy. */
 typedef struct {
   int grid[3], win[3], stride[3];  /* (F, H, W), (wf, wh, ww), (sf, sh, sw)          */
-  int T, U, Nw, N;                 /* tiles, grid tokens, window slots, Nw + 1        */
+  int T, U, Nw, N;                 /* tiles, grid tokens, window slots, Nw + R        */
   int nnz;                         /* CSR entries: T * Nw (ramp), U (hard stitching)  */
   int max_cover;                   /* most tiles covering one token                   */
   int device;                      /* CUDA device holding the plan's device arrays    */
@@ -101,8 +104,9 @@ typedef struct {
   const int* tile_tok;             /* host [T][Nw] grid token of slot j of tile t      */
   const int* slot_pos;             /* host [Nw][3] tile-local (f, y, x) of slot j      */
   const int* tok_ptr;              /* host [U + 1] CSR row pointer over grid tokens    */
-  const int* tok_ent;              /* host [nnz] entry t*N + 1 + j, ascending t        */
+  const int* tok_ent;              /* host [nnz] entry t*N + R + j, ascending t        */
   const float* wbar;               /* host [nnz] blend weight of that entry            */
+  int R;                           /* register tokens per tile                         */
 } ts_plan_desc;
 
 /* Model hyper-parameters ([TileShare] Tab. S1 block; readings in the comments). */
@@ -151,6 +155,14 @@ ts_status ts_plan_create(const int grid[3], const int win[3], const int stride[3
    ts_plan_desc reports device = -1. */
 ts_status ts_plan_create_host(const int grid[3], const int win[3], const int stride[3],
                               ts_blend_rule rule, ts_plan_t* out);
+/* The same two calls for R register tokens per tile, 1 <= registers <= 64
+   (TS_ERR_INVALID_ARG otherwise); ts_plan_create and ts_plan_create_host are
+   these with registers = 1.  The registers are not rotated by RoPE and attend,
+   and are attended by, their own tile only ([TileShare] Tab. S1). */
+ts_status ts_plan_create_registers(const int grid[3], const int win[3], const int stride[3],
+                                   ts_blend_rule rule, int registers, ts_plan_t* out);
+ts_status ts_plan_create_host_registers(const int grid[3], const int win[3], const int stride[3],
+                                        ts_blend_rule rule, int registers, ts_plan_t* out);
 ts_status ts_plan_info(ts_plan_t plan, ts_plan_desc* out);
 void ts_plan_destroy(ts_plan_t plan);
 
@@ -163,17 +175,17 @@ ts_status ts_workspace_size(ts_plan_t plan, const ts_model_desc* model, int L, i
 /* One released (per-tile) layer, in place on X [T, N, d] (device, model dtype; bf16
    for TS_FP8_E4M3).  [TileShare] Tab. S1, "Layer 0" column: every tile keeps its
    own residual stream; Norm1, QKV, QK-RMSNorm, RoPE on tile-local coordinates (the
-   global token is not rotated), dense attention over the tile's N rows,
+   registers are not rotated), dense attention over the tile's N rows,
    out-projection, Norm2 and MLP per tile row. */
 ts_status ts_block_tiled(ts_plan_t plan, const ts_model_desc* model, const ts_layer_weights* w,
                          void* X, void* workspace, size_t workspace_bytes, void* stream);
 
-/* One TileShare shared layer, in place on S [U + T, d] (device).  [TileShare]
+/* One TileShare shared layer, in place on S [U + T*R, d] (device).  [TileShare]
    Fig. 2 and Tab. S1 "Layers >= k": Norm1, QKV, QK-RMSNorm, out-projection and MLP
-   once per row of S; attention per tile over the rows [global token of t, window
+   once per row of S; attention per tile over the rows [registers of t, window
    tokens of t], with RoPE on tile-local coordinates; each grid token's attention
    output is the w-bar weighted sum, in ascending tile order, of its tiles' outputs
-   (the only approximate step); each global token keeps its own tile's output. */
+   (the only approximate step); each register keeps its own tile's output. */
 ts_status ts_block_shared(ts_plan_t plan, const ts_model_desc* model, const ts_layer_weights* w,
                           void* S, void* workspace, size_t workspace_bytes, void* stream);
 
@@ -182,7 +194,7 @@ ts_status ts_block_shared(ts_plan_t plan, const ts_model_desc* model, const ts_l
    plugin running inside a host application that owns every device buffer
    through its own pool and forbids the plugin from calling cudaMalloc, or code
    working inside a fixed, pre-partitioned memory budget.  It computes exactly
-   what ts_block_shared computes, in place on S [U + T, d], but its scratch
+   what ts_block_shared computes, in place on S [U + T*R, d], but its scratch
    (normalised rows, q/k/v, attention outputs, blend, MLP hidden) lives in one
    static device array of TS_NOALLOC_SCRATCH_BYTES (32 MiB) that every GPU
    loading the library holds until the process exits.
@@ -207,15 +219,15 @@ ts_status ts_block_shared_noalloc(ts_plan_t plan, const ts_model_desc* model, co
    (Fig. 3b), then layers k..L-1 shared.  With k = L this is overlapping tiled
    decoding blended with w-bar at the end.  w points to L host-side
    ts_layer_weights structs (whose members are device pointers).
-   S0 [U, d] grid tokens and G0 [T, d] global tokens in, out [U, d] grid tokens out
+   S0 [U, d] grid tokens and G0 [T*R, d] registers in, out [U, d] grid tokens out
    (device, model dtype).  0 <= k <= L. */
 ts_status ts_decode_stack(ts_plan_t plan, const ts_model_desc* model, const ts_layer_weights* w,
                           int L, int k, const void* S0, const void* G0, void* out,
                           void* workspace, size_t workspace_bytes, void* stream);
 
 /* Per-tile copies of the stack input, as ts_decode_stack makes before its first
-   per-tile layer: X[t*N] = G0[t], X[t*N + 1 + j] = S0[grid token of slot j of t].
-   S0 [U, d], G0 [T, d], X [T*N, d] (device, model dtype). */
+   per-tile layer: X[t*N + i] = G0[t*R + i], X[t*N + R + j] = S0[grid token of
+   slot j of t].  S0 [U, d], G0 [T*R, d], X [T*N, d] (device, model dtype). */
 ts_status ts_gather_tiles(ts_plan_t plan, const ts_model_desc* model, const void* S0, const void* G0,
                           void* X, void* stream);
 
@@ -239,7 +251,7 @@ typedef enum {
    tile keeps its own residual stream and only the listed operations are shared;
    attention always runs per tile).  In place on X [T, N, d] as ts_block_tiled.
    A shared operation takes, for each grid token, the w-bar blend of its tiles'
-   inputs (each tile's global token keeps its own row) and runs once per token;
+   inputs (each tile's registers keep their own rows) and runs once per token;
    shared q/k/v feed every tile's attention through the tile's rows, and the
    shared out-projection's and MLP's outputs are added to every tile's copy of the
    token.  shared_ops = 0 is ts_block_tiled; from identical per-tile copies, any set

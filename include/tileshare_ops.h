@@ -6,7 +6,7 @@
  * "TileShare: Training-Free Acceleration of Overlapping Tiled ViT Decoding".
  *
  * "rows mode" selects the row set a step works on:
- *   TS_ROWS_SHARED  the U + T rows of a shared state S (grid tokens, then globals)
+ *   TS_ROWS_SHARED  the U + T*R rows of a shared state S (grid tokens, then registers)
  *   TS_ROWS_TILED   the T * N rows of a per-tile state X
  */
 #ifndef TILESHARE_OPS_H
@@ -51,8 +51,8 @@ ts_status ts_op_linear(const ts_model_desc* model, const void* x, int rows, int 
    Tab. S1: Norm1, QKV, QK-RMSNorm once per token; RoPE on tile coordinates).
    state [rows, d] -> qkv [rows, 3d] (model dtype; bf16 for TS_FP8_E4M3).
    TS_ROWS_TILED rotates q and k of slot j of every tile by its tile-local
-   coordinates and leaves row 0 (the global token) unrotated.  TS_ROWS_SHARED
-   rotates grid token u by its grid coordinates and the global token of tile t by
+   coordinates and leaves rows 0 .. R-1 (the registers) unrotated.  TS_ROWS_SHARED
+   rotates grid token u by its grid coordinates and the registers of tile t by
    the tile's origin: attention scores then equal those of tile-local rotation
    exactly (RoPE scores depend on coordinate differences only), so the rotation
    can run once per token.  `scratch` holds, each region 256-byte aligned, the
@@ -63,8 +63,8 @@ ts_status ts_op_qkv(ts_plan_t plan, const ts_model_desc* model, const ts_layer_w
                     ts_rows_mode mode, const void* state, void* qkv, void* scratch, void* stream);
 
 /* Per-tile dense attention ([TileShare] Tab. S1 "Attention (dense, per tile)"; Fig.
-   2): for tile t and head h the rows are [global token of t, window slots of t]
-   taken from qkv ([U+T, 3d] rows for TS_ROWS_SHARED, gathered through the plan's
+   2): for tile t and head h the rows are [registers of t, window slots of t]
+   taken from qkv ([U+T*R, 3d] rows for TS_ROWS_SHARED, gathered through the plan's
    index map; [T*N, 3d] for TS_ROWS_TILED); O [T*N, d] (row t*N + s = slot s of
    tile t) = softmax(q k^T / sqrt(hd)) v, no mask.  bf16 needs hd == 64. */
 ts_status ts_op_attention(ts_plan_t plan, const ts_model_desc* model, ts_rows_mode mode,
@@ -73,8 +73,9 @@ ts_status ts_op_attention(ts_plan_t plan, const ts_model_desc* model, ts_rows_mo
 /* Blend ([TileShare] Fig. 2, Tab. S1 "Blend of attention outputs"; also the merge of
    per-tile states at layer k, Fig. 3b): for the first `rows` rows of the shared
    layout, A[u] = sum over the tiles covering u, in ascending tile order, of
-   wbar * P[t*N + 1 + j] (fp32 sum, one write per token, no atomics) and, for
-   rows >= U, A[U + t] = P[t*N].  P [T*N, d], A [rows, d]; rows is U or U + T. */
+   wbar * P[t*N + R + j] (fp32 sum, one write per token, no atomics) and, for
+   rows >= U, A[U + t*R + i] = P[t*N + i].  P [T*N, d], A [rows, d]; rows is U or
+   U + T*R. */
 ts_status ts_op_merge(ts_plan_t plan, const ts_model_desc* model, const void* P, int rows,
                       void* A, void* stream);
 

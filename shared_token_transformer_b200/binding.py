@@ -40,7 +40,8 @@ class PlanDesc(ctypes.Structure):
                 ("run", ctypes.c_int),
                 ("origins", ctypes.POINTER(ctypes.c_int)), ("tile_tok", ctypes.POINTER(ctypes.c_int)),
                 ("slot_pos", ctypes.POINTER(ctypes.c_int)), ("tok_ptr", ctypes.POINTER(ctypes.c_int)),
-                ("tok_ent", ctypes.POINTER(ctypes.c_int)), ("wbar", ctypes.POINTER(ctypes.c_float))]
+                ("tok_ent", ctypes.POINTER(ctypes.c_int)), ("wbar", ctypes.POINTER(ctypes.c_float)),
+                ("R", ctypes.c_int)]
 
 
 class ModelDesc(ctypes.Structure):
@@ -76,6 +77,9 @@ _lib = None
 _SIGS = {
     "ts_plan_create": [ctypes.POINTER(ctypes.c_int)] * 3 + [ctypes.c_int, ctypes.POINTER(_cp)],
     "ts_plan_create_host": [ctypes.POINTER(ctypes.c_int)] * 3 + [ctypes.c_int, ctypes.POINTER(_cp)],
+    "ts_plan_create_registers": [ctypes.POINTER(ctypes.c_int)] * 3 + [ctypes.c_int, ctypes.c_int, ctypes.POINTER(_cp)],
+    "ts_plan_create_host_registers": [ctypes.POINTER(ctypes.c_int)] * 3 + [ctypes.c_int, ctypes.c_int,
+                                                                            ctypes.POINTER(_cp)],
     "ts_plan_info": [_cp, ctypes.POINTER(PlanDesc)],
     "ts_plan_destroy": [_cp],
     "ts_workspace_size": [_cp, ctypes.POINTER(ModelDesc), ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)],
@@ -147,17 +151,17 @@ def _stream(stream=None):
 class Plan:
     """ts_plan_t with its host arrays as NumPy views (copied)."""
 
-    def __init__(self, grid, win, stride, host_only=False, rule=TS_BLEND_LINEAR_RAMP):
+    def __init__(self, grid, win, stride, host_only=False, rule=TS_BLEND_LINEAR_RAMP, registers=1):
         g, w, s = _int3(*grid), _int3(*win), _int3(*stride)
         h = _cp()
-        fn = "ts_plan_create_host" if host_only else "ts_plan_create"
-        _check(fn, getattr(lib(), fn)(g, w, s, rule, ctypes.byref(h)))
+        fn = "ts_plan_create_host_registers" if host_only else "ts_plan_create_registers"
+        _check(fn, getattr(lib(), fn)(g, w, s, rule, int(registers), ctypes.byref(h)))
         self.handle = h
         d = PlanDesc()
         _check("ts_plan_info", lib().ts_plan_info(h, ctypes.byref(d)))
         self.desc = d
         self.T, self.U, self.Nw, self.N, self.nnz = d.T, d.U, d.Nw, d.N, d.nnz
-        self.max_cover, self.device, self.run = d.max_cover, d.device, d.run
+        self.max_cover, self.device, self.run, self.R = d.max_cover, d.device, d.run, d.R
 
         def arr(p, n, dt):
             return np.ctypeslib.as_array(p, shape=(n,)).astype(dt).copy()

@@ -14,6 +14,9 @@
 //              and by (w - p) / (o_n + 1) for p >= w - o_n (product where both
 //              apply), 1 elsewhere; the tile weight is the product over axes,
 //              normalised to sum 1 over the tiles covering the token.
+//   registers  each tile has R register tokens ([TileShare] Tab. S1: one set per
+//              tile); the per-tile state is [R registers | Nw window slots] and the
+//              shared state [U grid tokens | T*R registers, tile t's at U + t*R].
 // Weights are computed in double and stored as float.
 #pragma once
 
@@ -24,12 +27,14 @@
 struct ts_plan_s {
   int grid[3], win[3], stride[3];
   int T, U, Nw, N, nnz, max_cover, device;
-  int run;                       // window slots 1 + k*run .. are runs of consecutive shared rows (0: none)
+  int R = 1;                     // register tokens per tile; N = Nw + R
+  int G = 0;                     // register rows of the shared state, T * R
+  int run;                       // slots 1 + k*run .. are runs of consecutive shared rows (0: none)
   int rule;                      // blend rule: 0 linear ramp (normalised), 1 hard stitching (one tile per token)
   std::vector<int> origins, tile_tok, slot_pos, tok_ptr, tok_ent;
   std::vector<float> wbar;
-  std::vector<int> rowmap;       // [T*N] shared-layout row of slot s of tile t (s = 0: U + t)
-  std::vector<int> pos_shared;   // [(U+T)*4] RoPE coordinates of shared rows
+  std::vector<int> rowmap;       // [T*N] shared-layout row of slot s of tile t (s < R: U + t*R + s)
+  std::vector<int> pos_shared;   // [(U+G)*4] RoPE coordinates of shared rows
   std::vector<int> pos_tiled;    // [(T*N)*4] RoPE coordinates of per-tile rows
   // device copies (on `device`)
   int* d_tok_ptr = nullptr;
@@ -81,7 +86,8 @@ inline bool build(ts_plan_s& P) {
   const int nf = static_cast<int>(of.size()), nh = static_cast<int>(oh.size()), nw = static_cast<int>(ow.size());
   P.T = nf * nh * nw;
   P.Nw = wf * wh * ww;
-  P.N = P.Nw + 1;
+  P.N = P.Nw + P.R;
+  P.G = P.T * P.R;
   P.U = F * H * W;
   P.nnz = P.T * P.Nw;
   P.slot_pos.assign(static_cast<size_t>(P.Nw) * 3, 0);
@@ -150,16 +156,16 @@ inline bool build(ts_plan_s& P) {
       const int u = P.tile_tok[e];
       if (P.rule == 1 && best_t[u] != t) continue;
       const int k = fill[u]++;
-      P.tok_ent[k] = t * P.N + 1 + j;
+      P.tok_ent[k] = t * P.N + P.R + j;
       P.wbar[k] = P.rule == 1 ? 1.0f : static_cast<float>(wraw[e] / total[u]);
     }
   // attention row map of the shared layout and RoPE coordinates
   P.rowmap.assign(static_cast<size_t>(P.T) * P.N, 0);
   P.pos_tiled.assign(static_cast<size_t>(P.T) * P.N * 4, 0);
   for (int t = 0; t < P.T; ++t) {
-    P.rowmap[static_cast<size_t>(t) * P.N] = P.U + t;
+    for (int i = 0; i < P.R; ++i) P.rowmap[static_cast<size_t>(t) * P.N + i] = P.U + t * P.R + i;
     for (int j = 0; j < P.Nw; ++j) {
-      const size_t r = static_cast<size_t>(t) * P.N + 1 + j;
+      const size_t r = static_cast<size_t>(t) * P.N + P.R + j;
       P.rowmap[r] = P.tile_tok[static_cast<size_t>(t) * P.Nw + j];
       for (int a = 0; a < 3; ++a) P.pos_tiled[4 * r + a] = P.slot_pos[3 * j + a];
     }
@@ -170,11 +176,11 @@ inline bool build(ts_plan_s& P) {
   for (int L = 64; L >= 8 && !P.run; L >>= 1) {
     bool ok = true;
     for (int t = 0; t < P.T && ok; ++t)
-      for (int j = 1; j < P.Nw && ok; ++j)
+      for (int j = 1; j < P.N - 1 && ok; ++j)
         if (j % L) ok = P.rowmap[static_cast<size_t>(t) * P.N + 1 + j] == P.rowmap[static_cast<size_t>(t) * P.N + j] + 1;
     if (ok) P.run = L;
   }
-  P.pos_shared.assign(static_cast<size_t>(P.U + P.T) * 4, 0);
+  P.pos_shared.assign(static_cast<size_t>(P.U + P.G) * 4, 0);
   for (int f = 0, u = 0; f < F; ++f)
     for (int y = 0; y < H; ++y)
       for (int x = 0; x < W; ++x, ++u) {
@@ -183,7 +189,9 @@ inline bool build(ts_plan_s& P) {
         P.pos_shared[4 * u + 2] = x;
       }
   for (int t = 0; t < P.T; ++t)
-    for (int a = 0; a < 3; ++a) P.pos_shared[4 * (static_cast<size_t>(P.U) + t) + a] = P.origins[3 * t + a];
+    for (int i = 0; i < P.R; ++i)
+      for (int a = 0; a < 3; ++a)
+        P.pos_shared[4 * (static_cast<size_t>(P.U) + t * P.R + i) + a] = P.origins[3 * t + a];
   return true;
 }
 

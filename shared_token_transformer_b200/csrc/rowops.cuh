@@ -144,11 +144,11 @@ __global__ void __launch_bounds__(256) layernorm_generic_kernel(const T* __restr
 // ---------------------------------------------------------------------------
 // Blend / merge ([TileShare] Fig. 2: overlap tokens' attention outputs blended with
 // w-bar; Fig. 3b: per-tile states merged).  Row u < U: fp32 sum over the token's
-// CSR entries in ascending tile order of wbar * P[ent]; row U + t: P[t*N].  One
+// CSR entries in ascending tile order of wbar * P[ent]; row U + t*R + i: P[t*N + i].  One
 // warp writes each output row once; no atomics, so the result is deterministic.
 // ---------------------------------------------------------------------------
 template <typename T, int NV, bool Q8>
-__global__ void __launch_bounds__(256) merge_kernel(const T* __restrict__ P, int rows, int U, int N, int d,
+__global__ void __launch_bounds__(256) merge_kernel(const T* __restrict__ P, int rows, int U, int N, int R, int d,
                                                     const int* __restrict__ tok_ptr, const int* __restrict__ tok_ent,
                                                     const float* __restrict__ wbar, T* __restrict__ A,
                                                     uint8_t* __restrict__ q8, float* __restrict__ qscale) {
@@ -177,7 +177,8 @@ __global__ void __launch_bounds__(256) merge_kernel(const T* __restrict__ P, int
       }
     }
   } else {
-    const T* src = P + (row - U) * static_cast<size_t>(N) * d;
+    const size_t reg = row - U;   // register i of tile t: row t*N + i of P
+    const T* src = P + ((reg / R) * static_cast<size_t>(N) + reg % R) * d;
 #pragma unroll
     for (int i = 0; i < NV; ++i) Vec<T>::load(src + (i * 32 + lane) * E, v[i]);
   }
@@ -188,12 +189,12 @@ __global__ void __launch_bounds__(256) merge_kernel(const T* __restrict__ P, int
 // buffers of `cover` rows (cover = most tiles on one token) and keeps two output
 // rows in flight; for each, the lanes read the token's entries (one per lane) and
 // issue one bulk copy per entry, so loads in flight hold no registers.  Row
-// U + t is the single entry t*N with weight 1.  Sums run in ascending entry order,
+// U + t*R + i is the single entry t*N + i with weight 1.  Sums run in ascending entry order,
 // as in merge_kernel.
 constexpr int kMergeWarps = 4;
 template <typename T, int NV, bool Q8>
 __global__ void __launch_bounds__(kMergeWarps * 32) merge_bulk_kernel(
-    const T* __restrict__ P, int rows, int U, int N, int d, const int* __restrict__ tok_ptr,
+    const T* __restrict__ P, int rows, int U, int N, int R, int d, const int* __restrict__ tok_ptr,
     const int* __restrict__ tok_ent, const float* __restrict__ wbar, int cover, T* __restrict__ A,
     uint8_t* __restrict__ q8, float* __restrict__ qscale) {
   extern __shared__ __align__(16) uint8_t smem[];
@@ -223,7 +224,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_bulk_kernel(
       }
     } else {
       n = 1;
-      ent = (r - U) * N;
+      ent = ((r - U) / R) * N + (r - U) % R;
       wl = 1.f;
     }
     fence_proxy_async_smem();   // this warp's reads of the buffer precede the copies that overwrite it
@@ -279,7 +280,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_bulk_kernel(
 
 // generic fallback of the blend for any d (scalar)
 template <typename T>
-__global__ void __launch_bounds__(256) merge_generic_kernel(const T* __restrict__ P, int rows, int U, int N, int d,
+__global__ void __launch_bounds__(256) merge_generic_kernel(const T* __restrict__ P, int rows, int U, int N, int R, int d,
                                                             const int* __restrict__ tok_ptr,
                                                             const int* __restrict__ tok_ent,
                                                             const float* __restrict__ wbar, T* __restrict__ A) {
@@ -292,7 +293,8 @@ __global__ void __launch_bounds__(256) merge_generic_kernel(const T* __restrict_
       for (int e = tok_ptr[row]; e < tok_ptr[row + 1]; ++e)
         acc = fmaf(wbar[e], static_cast<float>(P[static_cast<size_t>(tok_ent[e]) * d + c]), acc);
     } else {
-      acc = static_cast<float>(P[(row - U) * static_cast<size_t>(N) * d + c]);
+      const size_t reg = row - U;
+      acc = static_cast<float>(P[((reg / R) * static_cast<size_t>(N) + reg % R) * d + c]);
     }
     A[row * d + c] = static_cast<T>(acc);
   }
@@ -320,7 +322,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint8_t* __restr
 // ---------------------------------------------------------------------------
 // Partial sharing ([TileShare] Tab. 1 top): a per-token result R [U + T, d] of a
 // shared operation is added to every tile's copy of the token, X[r] += R[rowmap[r]]
-// for the T * N per-tile rows (row t*N of tile t takes R[U + t]).  fp32 add, one
+// for the T * N per-tile rows (a tile's registers take its register rows of R).  fp32 add, one
 // warp per row, 16-byte vectors; every X row is written by one warp.
 // ---------------------------------------------------------------------------
 template <typename T>

@@ -335,7 +335,7 @@ static ts::RopeTable make_rope_table(const ts_plan_s* p, const ts_model_desc* m,
 }
 
 static Workspace layout(const ts_plan_s* p, const ts_model_desc* m, bool stack, char* base) {
-  const size_t Mt = static_cast<size_t>(p->T) * p->N, Ms = static_cast<size_t>(p->U) + p->T;
+  const size_t Mt = static_cast<size_t>(p->T) * p->N, Ms = static_cast<size_t>(p->U) + p->G;
   const size_t Mx = std::max(Mt, Ms);
   const size_t e = esize(m->dtype), d = m->d, f = m->mlp;
   size_t off = 0;
@@ -449,7 +449,7 @@ static ts_status launch_merge_vec(const ts_plan_s* p, const void* P, int rows, i
       TS_CUDA_CHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));     \
       configured[dev] = 1;                                                                                    \
     }                                                                                                         \
-    launch_pdl(kern, dim3(grid), dim3(32 * ts::kMergeWarps), smem, st, pp, rows, p->U, p->N, d,                \
+    launch_pdl(kern, dim3(grid), dim3(32 * ts::kMergeWarps), smem, st, pp, rows, p->U, p->N, p->R, d,          \
                static_cast<const int*>(p->d_tok_ptr), static_cast<const int*>(p->d_tok_ent),                   \
                static_cast<const float*>(p->d_wbar), p->max_cover, aa, q8, qs);                              \
     break;                                                                                                    \
@@ -464,7 +464,8 @@ static ts_status launch_merge_vec(const ts_plan_s* p, const void* P, int rows, i
   trace_pre(st);
 #define TS_MG_CASE(NV)                                                                                    \
   case NV:                                                                                                \
-    launch_pdl(ts::merge_kernel<T, NV, Q8>, dim3(rows_grid(rows)), dim3(256), 0, st, pp, rows, p->U, p->N, d, \
+    launch_pdl(ts::merge_kernel<T, NV, Q8>, dim3(rows_grid(rows)), dim3(256), 0, st, pp, rows, p->U, p->N,    \
+               p->R, d,                                                                                     \
                static_cast<const int*>(p->d_tok_ptr), static_cast<const int*>(p->d_tok_ent),               \
                static_cast<const float*>(p->d_wbar), aa, q8, qs);                                           \
     break;
@@ -490,7 +491,7 @@ static ts_status run_merge(const char* name, const ts_plan_s* p, const ts_model_
   if (m->dtype == TS_F32) {
     if (d % 128 == 0 && d <= 1024) return launch_merge_vec<float, false>(p, P, rows, d, A, nullptr, nullptr, st);
     trace_pre(st);
-    ts::merge_generic_kernel<float><<<rows_grid(rows), 256, 0, st>>>(static_cast<const float*>(P), rows, p->U, p->N, d,
+    ts::merge_generic_kernel<float><<<rows_grid(rows), 256, 0, st>>>(static_cast<const float*>(P), rows, p->U, p->N, p->R, d,
                                                                     p->d_tok_ptr, p->d_tok_ent, p->d_wbar,
                                                                     static_cast<float*>(A));
     return trace_post(st, "merge_generic");
@@ -661,7 +662,7 @@ static ts_status run_attention(const ts_plan_s* p, const ts_model_desc* m, bool 
   a.rowmap = shared ? p->d_rowmap : nullptr;
   a.O = O;
   a.N = p->N;
-  a.Nw = p->Nw;
+  a.Nw = p->N - 1;    // slots after slot 0 (the tile's first register, handled apart)
   a.d = m->d;
   a.heads = m->heads;
   a.T = p->T;
@@ -681,7 +682,7 @@ static ts_status run_attention(const ts_plan_s* p, const ts_model_desc* m, bool 
     }
     return trace_post(st, "attn_f32");
   }
-  const int nqb = (p->Nw + ts::kAttnBQ - 1) / ts::kAttnBQ;
+  const int nqb = (p->N - 1 + ts::kAttnBQ - 1) / ts::kAttnBQ;
   static int configured[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -697,7 +698,7 @@ static ts_status run_attention(const ts_plan_s* p, const ts_model_desc* m, bool 
   // one box of a 3-D map over the grid; otherwise runs of consecutive rows are
   // 2-D boxes (the per-tile layout is one run per tile), else four-row gathers.
   const int wx = p->win[2], wy = p->win[1];
-  const bool grid_box = wx <= 64 ? (64 % wx == 0 && (wy * wx) % 64 == 0) : wx % 64 == 0;
+  const bool grid_box = p->R == 1 && (wx <= 64 ? (64 % wx == 0 && (wy * wx) % 64 == 0) : wx % 64 == 0);
   CUtensorMap tm;
   if (shared && grid_box) {
     a.load = 2;
@@ -707,7 +708,7 @@ static ts_status run_attention(const ts_plan_s* p, const ts_model_desc* m, bool 
   } else {
     a.run = shared ? p->run : 64;
     a.load = a.run > 0 ? 1 : 0;
-    TS_TRY(make_tmap(&tm, qkv, shared ? p->U + p->T : p->T * p->N, 3 * m->d, 2, a.run > 0 ? a.run : 1));
+    TS_TRY(make_tmap(&tm, qkv, shared ? p->U + p->G : p->T * p->N, 3 * m->d, 2, a.run > 0 ? a.run : 1));
   }
   dim3 grid(nqb, m->heads, p->T);
   launch_pdl(ts::attn_bf16_kernel, grid, dim3(ts::kAttnThreads), ts::AttnSmem::LAUNCH_BYTES, st, tm, a);
@@ -719,7 +720,7 @@ static ts_status run_attention(const ts_plan_s* p, const ts_model_desc* m, bool 
 // ---------------------------------------------------------------------------
 static ts_status run_qkv(const ts_plan_s* p, const ts_model_desc* m, const ts_layer_weights* w, bool shared,
                          const void* state, void* qkv, const Workspace& ws, cudaStream_t st) {
-  const int rows = shared ? p->U + p->T : p->T * p->N;
+  const int rows = shared ? p->U + p->G : p->T * p->N;
   const int* pos = shared ? p->d_pos_shared : p->d_pos_tiled;
   const int d = m->d;
   if (m->dtype == TS_F32) {
@@ -865,7 +866,7 @@ static ts_status layer_tiled(const ts_plan_s* p, const ts_model_desc* m, const t
 
 static ts_status layer_shared(const ts_plan_s* p, const ts_model_desc* m, const ts_layer_weights* w, void* S,
                               const Workspace& ws, cudaStream_t st) {
-  const int rows = p->U + p->T;
+  const int rows = p->U + p->G;
   TS_TRY(run_qkv(p, m, w, true, S, ws.qkv, ws, st));
   TS_TRY(run_attention(p, m, true, ws.qkv, ws.o, st));
   const bool q = m->dtype == TS_FP8_E4M3;
@@ -879,7 +880,7 @@ static ts_status layer_shared(const ts_plan_s* p, const ts_model_desc* m, const 
 // (QKV) or added to (out-projection, MLP) every tile's copy of the token.
 static ts_status layer_partial(const ts_plan_s* p, const ts_model_desc* m, const ts_layer_weights* w, unsigned ops,
                                void* X, const Workspace& ws, cudaStream_t st) {
-  const int rows_t = p->T * p->N, rows_s = p->U + p->T;
+  const int rows_t = p->T * p->N, rows_s = p->U + p->G;
   const bool q8 = m->dtype == TS_FP8_E4M3;
   if (ops & TS_SHARE_QKV) {
     TS_TRY(run_merge("merge", p, m, X, rows_s, ws.sm, nullptr, nullptr, st));
@@ -988,9 +989,10 @@ const char* ts_status_string(ts_status s) {
 const char* ts_last_error(void) { return g_last_error.c_str(); }
 
 static ts_status plan_build_host(const int grid[3], const int win[3], const int stride[3], ts_blend_rule rule,
-                                 ts_plan_s** out) {
+                                 int registers, ts_plan_s** out) {
   if (!grid || !win || !stride || !out) return fail(TS_ERR_INVALID_ARG, "NULL argument");
   *out = nullptr;
+  if (registers < 1 || registers > 64) return fail(TS_ERR_INVALID_ARG, "registers per tile must lie in [1, 64]");
   if (rule != TS_BLEND_LINEAR_RAMP && rule != TS_BLEND_HARD_STITCH)
     return fail(TS_ERR_INVALID_ARG, "unknown blend rule %d", static_cast<int>(rule));
   for (int a = 0; a < 3; ++a) {
@@ -1008,6 +1010,7 @@ static ts_status plan_build_host(const int grid[3], const int win[3], const int 
   }
   P->device = -1;
   P->rule = rule == TS_BLEND_HARD_STITCH ? 1 : 0;
+  P->R = registers;
   if (!tsplan::build(*P)) {
     delete P;
     return fail(TS_ERR_INVALID_ARG, "tiling leaves a token uncovered");
@@ -1022,13 +1025,23 @@ static ts_status plan_build_host(const int grid[3], const int win[3], const int 
 
 ts_status ts_plan_create_host(const int grid[3], const int win[3], const int stride[3], ts_blend_rule rule,
                               ts_plan_t* out) {
-  return plan_build_host(grid, win, stride, rule, out);
+  return plan_build_host(grid, win, stride, rule, 1, out);
+}
+
+ts_status ts_plan_create_host_registers(const int grid[3], const int win[3], const int stride[3], ts_blend_rule rule,
+                                        int registers, ts_plan_t* out) {
+  return plan_build_host(grid, win, stride, rule, registers, out);
 }
 
 ts_status ts_plan_create(const int grid[3], const int win[3], const int stride[3], ts_blend_rule rule,
                          ts_plan_t* out) {
+  return ts_plan_create_registers(grid, win, stride, rule, 1, out);
+}
+
+ts_status ts_plan_create_registers(const int grid[3], const int win[3], const int stride[3], ts_blend_rule rule,
+                                   int registers, ts_plan_t* out) {
   ts_plan_s* P = nullptr;
-  TS_TRY(plan_build_host(grid, win, stride, rule, &P));
+  TS_TRY(plan_build_host(grid, win, stride, rule, registers, &P));
   cudaError_t e = cudaGetDevice(&P->device);
   auto upload = [&](auto** dst, const auto& vec) -> bool {
     using E = typename std::decay<decltype(vec)>::type::value_type;
@@ -1067,6 +1080,7 @@ ts_status ts_plan_info(ts_plan_t p, ts_plan_desc* out) {
   out->max_cover = p->max_cover;
   out->device = p->device;
   out->run = p->run;
+  out->R = p->R;
   out->origins = p->origins.data();
   out->tile_tok = p->tile_tok.data();
   out->slot_pos = p->slot_pos.data();
@@ -1166,9 +1180,9 @@ static ts_status noalloc_scratch(void** out) {
   return TS_OK;
 }
 
-// Scratch regions of one shared layer only (rows U + T, attention outputs T * N).
+// Scratch regions of one shared layer only (rows U + T*R, attention outputs T * N).
 static Workspace layout_shared_scratch(const ts_plan_s* p, const ts_model_desc* m, char* base) {
-  const size_t Mt = static_cast<size_t>(p->T) * p->N, Ms = static_cast<size_t>(p->U) + p->T;
+  const size_t Mt = static_cast<size_t>(p->T) * p->N, Ms = static_cast<size_t>(p->U) + p->G;
   const size_t e = esize(m->dtype), d = m->d, f = m->mlp;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -1228,10 +1242,10 @@ ts_status ts_decode_stack(ts_plan_t p, const ts_model_desc* m, const ts_layer_we
     TS_TRY(run_gather(p, m, S0, G0, W.X, st));
     for (int l = 0; l < k; ++l) TS_TRY(layer_tiled(p, m, w + l, W.X, W, st));
     if (k == L) return run_merge("merge", p, m, W.X, p->U, out, nullptr, nullptr, st);
-    TS_TRY(run_merge("merge", p, m, W.X, p->U + p->T, W.S, nullptr, nullptr, st));
+    TS_TRY(run_merge("merge", p, m, W.X, p->U + p->G, W.S, nullptr, nullptr, st));
   } else {
     TS_CUDA_CHECK(cudaMemcpyAsync(W.S, S0, rb * p->U, cudaMemcpyDeviceToDevice, st));
-    TS_CUDA_CHECK(cudaMemcpyAsync(static_cast<char*>(W.S) + rb * p->U, G0, rb * p->T, cudaMemcpyDeviceToDevice, st));
+    TS_CUDA_CHECK(cudaMemcpyAsync(static_cast<char*>(W.S) + rb * p->U, G0, rb * p->G, cudaMemcpyDeviceToDevice, st));
   }
   for (int l = k; l < L; ++l) TS_TRY(layer_shared(p, m, w + l, W.S, W, st));
   TS_CUDA_CHECK(cudaMemcpyAsync(out, W.S, rb * p->U, cudaMemcpyDeviceToDevice, st));
@@ -1309,7 +1323,7 @@ ts_status ts_op_qkv(ts_plan_t p, const ts_model_desc* m, const ts_layer_weights*
   if (!state || !qkv || !scratch || !aligned16(state) || !aligned16(qkv) || !aligned16(scratch))
     return fail(TS_ERR_INVALID_ARG, "bad argument");
   const bool shared = mode == TS_ROWS_SHARED;
-  const size_t rows = shared ? p->U + p->T : static_cast<size_t>(p->T) * p->N;
+  const size_t rows = shared ? p->U + p->G : static_cast<size_t>(p->T) * p->N;
   Workspace ws{};
   ws.xn = scratch;
   ws.q8 = static_cast<uint8_t*>(scratch) + align256(rows * m->d * esize(m->dtype));
@@ -1330,7 +1344,7 @@ ts_status ts_op_merge(ts_plan_t p, const ts_model_desc* m, const void* P, int ro
   TS_TRY(check_plan(p));
   TS_TRY(check_model(m));
   if (!P || !A || !aligned16(P) || !aligned16(A)) return fail(TS_ERR_INVALID_ARG, "bad argument");
-  if (rows != p->U && rows != p->U + p->T) return fail(TS_ERR_INVALID_ARG, "rows must be U or U + T");
+  if (rows != p->U && rows != p->U + p->G) return fail(TS_ERR_INVALID_ARG, "rows must be U or U + T*R");
   return run_merge("merge", p, m, P, rows, A, nullptr, nullptr, static_cast<cudaStream_t>(stream));
 }
 

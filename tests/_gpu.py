@@ -59,9 +59,10 @@ class Case:
 
     def __init__(self, cfg, seed=0, affine=True, L=None, rule="ramp"):
         self.cfg = cfg
-        self.oplan = OP.make_plan(cfg.grid, cfg.win, cfg.stride, rule=rule)
+        self.oplan = OP.make_plan(cfg.grid, cfg.win, cfg.stride, rule=rule, registers=cfg.R)
         self.plan = B.Plan(cfg.grid, cfg.win, cfg.stride,
-                           rule=B.TS_BLEND_HARD_STITCH if rule == "hard" else B.TS_BLEND_LINEAR_RAMP)
+                           rule=B.TS_BLEND_HARD_STITCH if rule == "hard" else B.TS_BLEND_LINEAR_RAMP,
+                           registers=cfg.R)
         dr = W.Draw(cfg, self.oplan.T, seed=seed, affine=affine)
         self.S0, self.G0 = dr.states()
         self.layers = dr.layers(L)

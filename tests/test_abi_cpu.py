@@ -72,6 +72,26 @@ def test_host_planner_bit_exact_against_oracle(grid, win, stride):
         p.close()
 
 
+@pytest.mark.parametrize("R", [2, 5])
+def test_host_planner_registers_bit_exact_against_oracle(R):
+    grid, win, stride = (2, 9, 11), (2, 5, 6), (1, 3, 4)
+    o = OP.make_plan(grid, win, stride, registers=R)
+    p = B.Plan(grid, win, stride, host_only=True, registers=R)
+    try:
+        assert (p.T, p.U, p.Nw, p.N, p.nnz, p.R) == (o.T, o.U, o.Nw, o.N, o.nnz, R)
+        np.testing.assert_array_equal(p.tok_ptr, o.tok_ptr)
+        np.testing.assert_array_equal(p.tok_ent, o.tok_ent)
+        np.testing.assert_array_equal(p.wbar, o.tok_w.astype(np.float32))
+    finally:
+        p.close()
+
+
+@pytest.mark.parametrize("R", [0, 65])
+def test_plan_rejects_bad_register_count(R):
+    with pytest.raises(B.TileShareError):
+        B.Plan((1, 8, 8), (1, 4, 4), (1, 2, 2), host_only=True, registers=R)
+
+
 RUNS = {(1, 48, 48): 16, (4, 44, 80): 32, (1, 128, 128): 32, (1, 11, 13): 8, (3, 7, 9): 0, (1, 20, 9): 0,
         (1, 5, 5): 64, (1, 9, 40): 16, (1, 5, 200): 64}
 

@@ -454,6 +454,56 @@ def test_swiglu_block_partial(cfg, shared):
     assert rel_l2(host(Xd).reshape(op.T, op.N, cfg.d), want) < _tol(cfg)
 
 
+# ---------------------------------------------------------------------------
+# several register tokens per tile (Tab. S1: one set per tile)
+# ---------------------------------------------------------------------------
+SMALL_R4 = dataclasses.replace(SMALL, name="small_r4_bf16", R=4)
+VOL_R2 = dataclasses.replace(VOL, name="vol_r2_bf16", R=2)
+VIT14_R3 = dataclasses.replace(VIT14, name="vit14_r3_fp32", R=3)
+SMALL_FP8_R2 = dataclasses.replace(SMALL_FP8, name="small_r2_fp8", R=2)
+RUNS16_R8 = dataclasses.replace(RUNS16, name="runs16_r8_bf16", R=8)
+_REG = [SMALL_R4, VOL_R2, VIT14_R3, SMALL_FP8_R2, RUNS16_R8]
+
+
+@pytest.mark.parametrize("cfg", _REG, ids=lambda c: c.name)
+def test_registers_block_shared_and_tiled(cfg):
+    c = case(cfg)
+    assert c.plan.R == cfg.R and c.plan.N == c.plan.Nw + cfg.R
+    S_in = c.S
+    assert S_in.shape[0] == c.oplan.U + c.oplan.T * cfg.R
+    S = dev(S_in, c.dt)
+    B.block_shared(c.plan, c.m, c.wlist[0], S, c.workspace())
+    want = OL.block_shared(S_in, c.layers[0], c.om, c.oplan)
+    assert rel_l2(host(S), want) < _tol(cfg)
+    assert rel_l2(host(S) - S_in, want - S_in) < 3 * _tol(cfg)
+    X_in = OL.gather(S_in, c.oplan)
+    X = dev(X_in.reshape(c.oplan.T * c.oplan.N, -1), c.dt)
+    B.block_tiled(c.plan, c.m, c.wlist[0], X, c.workspace())
+    want = OL.block_tiled(X_in, c.layers[0], c.om, c.oplan).reshape(X.shape)
+    assert rel_l2(host(X), want) < _tol(cfg)
+
+
+@pytest.mark.parametrize("cfg", _REG, ids=lambda c: c.name)
+def test_registers_decode_stack(cfg):
+    c = case(cfg)
+    for k in (0, 1):
+        got = host(_run_stack(c, k))
+        want = OL.decode_stack(c.S0, c.G0, c.layers, c.om, c.oplan, k)
+        assert rel_l2(got, want) < _tol(cfg), k
+
+
+@pytest.mark.parametrize("cfg", [SMALL_R4, SMALL_FP8_R2], ids=lambda c: c.name)
+def test_registers_block_partial(cfg):
+    c = case(cfg)
+    op = c.oplan
+    X = OL.gather(c.S, op) + 0.1 * np.random.default_rng(23).standard_normal((op.T, op.N, cfg.d))
+    X = W.round_to(X, cfg.dtype if cfg.dtype != "fp8" else "bf16")
+    Xd = dev(X.reshape(op.T * op.N, cfg.d), c.dt)
+    B.block_partial(c.plan, c.m, c.wlist[0], B.TS_SHARE_QKV | B.TS_SHARE_OUT | B.TS_SHARE_MLP, Xd, c.workspace())
+    want = OL.block_partial(X, c.layers[0], c.om, op, ("qkv", "out", "mlp"))
+    assert rel_l2(host(Xd).reshape(op.T, op.N, cfg.d), want) < _tol(cfg)
+
+
 def test_block_partial_rejects_unknown_operations():
     c = case(SMALL)
     Xd = torch.zeros((c.oplan.T * c.oplan.N, SMALL.d), dtype=c.dt, device="cuda")
