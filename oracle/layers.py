@@ -21,7 +21,7 @@ What the pages fix
       tile (each tile its own residual stream), the rest shared.
     * [TileShare] Fig. 3b: the per-tile states can be merged into one state.
 
-Readings taken where the pages are silent (also listed in the design doc)
+Readings taken where the pages are silent
     R4 block: pre-LN ViT block  x += W_o Attn(RoPE(QKnorm(W_qkv LN1(x)))) + b_o;
        x += W_2 GELU(W_1 LN2(x) + b_1) + b_2; LayerNorm and QK-RMSNorm eps 1e-6
        with learnable gain (and LN bias); exact erf GELU; attention scale

@@ -10,7 +10,7 @@ What the pages fix
     * [TileShare] Fig. 2: a token in the overlap of two windows is stored once but
       attended in both windows; its attention outputs are blended with w-bar.
 
-Readings taken where the pages are silent (stated here and in the design doc)
+Readings taken where the pages are silent
     R1 tile placement: per axis, n = ceil((G - w) / s) + 1 tiles (1 if w == G), the
        i-th at origin min(i*s, G - w): the last tile sits flush with the far edge,
        no padding.
