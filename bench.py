@@ -474,7 +474,7 @@ def run_tileshare(args, rank, world, local):
         with open(tpath) as fh:
             tj = json.load(fh)
         ent = tj.get(args.config, {}).get(dom)
-        if ent and ent.get("kernel_source_sha") == kernel_source_sha():
+        if ent and ent.get("kernel_source_sha") == kernel_source_sha(kernel_class(dom)):
             traffic = ent.get("traffic_bytes_per_launch")
     roofline = {"bound": "tensor" if kd["unit"] == "TFLOP/s" else "hbm", "kernel": dom, "achieved": kd["achieved"],
                 "peak": round(tensor_peak_of(dom) if kd["unit"] == "TFLOP/s" else pk["hbm_gbs"], 1), "unit": kd["unit"],
@@ -542,14 +542,32 @@ def replica_rate(units_per_rank, world, ms):
     return units_per_rank * world / (ms / 1e3) if ms > 0 else 0.0
 
 
-def kernel_source_sha():
+# source files behind each kernel class: its own header, plus the shared device
+# helpers and the host code that sets its launches up
+_CLASS_SOURCES = {"attention": "attention.cuh", "gemm": "gemm_tc.cuh", "rows": "rowops.cuh"}
+
+
+def kernel_source_sha(kind=None):
+    """Hash of the sources a kernel class is built from (all of csrc/ when kind is None)."""
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "shared_token_transformer_b200", "csrc")
-    for fn in sorted(os.listdir(d)):
+    files = sorted(os.listdir(d))
+    if kind is not None:
+        files = sorted({"common.cuh", "plan.inl", "tileshare.cu", _CLASS_SOURCES[kind]})
+    for fn in files:
         with open(os.path.join(d, fn), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
+
+
+def kernel_class(name):
+    """Kernel class of a traced kernel name."""
+    if name.startswith("attention"):
+        return "attention"
+    if name.startswith(("gemm", "linear")):
+        return "gemm"
+    return "rows"
 
 
 def main():

@@ -211,22 +211,47 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_bulk_kernel(
   __syncwarp();
   pdl_wait();
   pdl_trigger();
-  // entries of row r (lane k < n holds entry k's weight) and their copies into buffer b
-  auto issue = [&](int r, int b, int& n, float& wl) {
-    int ent = 0;
+  // Row metadata runs ahead of the copies so that no dependent L2 round trip sits on
+  // a row's path: lane k holds the CSR row pointer and entry count of this warp's
+  // row base + k (refreshed every 32 rows), and the entries and weights of a row are
+  // loaded one row before its copies are issued.  A register row U + t*R + i is
+  // encoded as pointer -1 - (t*R + i), one entry t*N + i of weight 1.
+  const int stride = gridDim.x * kMergeWarps;
+  const int r0 = blockIdx.x * kMergeWarps + wib;
+  int my_e0 = 0, my_n = 0;
+  auto load_ptrs = [&](int base) {
+    const int r = r0 + (base + lane) * stride;
+    my_e0 = 0;
+    my_n = 0;
+    if (r < rows) {
+      if (r < U) {
+        my_e0 = __ldg(tok_ptr + r);
+        my_n = __ldg(tok_ptr + r + 1) - my_e0;
+      } else {
+        my_e0 = -1 - (r - U);
+        my_n = 1;
+      }
+    }
+  };
+  // entries (lane k < n: entry k and its weight) of this warp's i-th row
+  auto load_ents = [&](int i, int& ent, float& wl, int& n) {
+    const int e0 = __shfl_sync(0xffffffffu, my_e0, i & 31);
+    n = __shfl_sync(0xffffffffu, my_n, i & 31);
+    ent = 0;
     wl = 0.f;
-    if (r < U) {
-      const int e0 = __ldg(tok_ptr + r);
-      n = __ldg(tok_ptr + r + 1) - e0;
-      if (lane < n) {
+    if (lane < n) {
+      if (e0 >= 0) {
         ent = __ldg(tok_ent + e0 + lane);
         wl = __ldg(wbar + e0 + lane);
+      } else {
+        const int reg = -1 - e0;
+        ent = (reg / R) * N + reg % R;
+        wl = 1.f;
       }
-    } else {
-      n = 1;
-      ent = ((r - U) / R) * N + (r - U) % R;
-      wl = 1.f;
     }
+  };
+  // copies of a row's entries into buffer b
+  auto issue = [&](int b, int n, int ent) {
     fence_proxy_async_smem();   // this warp's reads of the buffer precede the copies that overwrite it
     __syncwarp();
     if (lane == 0) mbar_expect_tx(bar + 8 * b, n * rowbytes);
@@ -235,16 +260,26 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_bulk_kernel(
       bulk_load(smem_u32(wbuf + (static_cast<size_t>(b) * cover + lane) * rowbytes), P + static_cast<size_t>(ent) * d,
                 rowbytes, bar + 8 * b);
   };
-  const int stride = gridDim.x * kMergeWarps;
-  int row = blockIdx.x * kMergeWarps + wib;
-  int nc = 0, nn = 0;
+  int row = r0;
+  int nc = 0, nn = 0, entc = 0, entn = 0;
   float wc = 0.f, wn = 0.f;
   bool pending_next = false;
   int broke_at = -1;
-  if (row < rows) issue(row, 0, nc, wc);
+  load_ptrs(0);
+  if (row < rows) {
+    load_ents(0, entc, wc, nc);
+    issue(0, nc, entc);
+  }
+  if (row + stride < rows) load_ents(1, entn, wn, nn);
   for (int i = 0; row < rows; ++i, row += stride) {
     pending_next = row + stride < rows;
-    if (pending_next) issue(row + stride, (i + 1) & 1, nn, wn);
+    if (pending_next) issue((i + 1) & 1, nn, entn);
+    int n2 = 0, ent2 = 0;
+    float w2 = 0.f;
+    if (row + 2 * stride < rows) {
+      if (((i + 2) & 31) == 0) load_ptrs(i + 2);
+      load_ents(i + 2, ent2, w2, n2);
+    }
     if (!mbar_wait(bar + 8 * (i & 1), (i >> 1) & 1)) {
       broke_at = i;
       break;
@@ -270,6 +305,9 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_bulk_kernel(
     store_row<T, NV, Q8>(v, lane, A, q8, qscale, row, d);
     nc = nn;
     wc = wn;
+    nn = n2;
+    entn = ent2;
+    wn = w2;
   }
   // no copy may still be landing when the CTA exits (matters only after a timeout)
   if (broke_at >= 0) {
