@@ -1,0 +1,58 @@
+"""Host-side helpers of bench.py (CPU only): workload selection, FLOP counts, kernel classes
+and the source keys of the DRAM-traffic table."""
+
+import json
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from oracle import flops as Fo  # noqa: E402
+from oracle import plan as OP  # noqa: E402
+
+
+class _Args:
+    def __init__(self, config, block=None):
+        self.config, self.block = config, block
+
+
+def test_config_of_block_flavour():
+    assert bench.config_of(_Args("stack48_bf16")).block == "ln_gelu"
+    c = bench.config_of(_Args("stack48_bf16", "rms_swiglu"))
+    assert c.block == "rms_swiglu" and c.d == 512 and c.mlp == 2048
+
+
+@pytest.mark.parametrize("gated", [False, True])
+def test_bench_flops_match_the_oracle_count(gated):
+    # the bench's per-layer FLOPs equal the oracle's analytic count for both layer kinds
+    p = OP.make_plan((1, 48, 48), (1, 16, 16), (1, 12, 12))
+    d, f = 512, 2048
+    assert bench.flops_layer(p.T * p.N, p.T, p.N, d, f, gated) == Fo.tiled_layer_flops(p.T, p.N, d, f, gated)
+    assert bench.flops_layer(p.U + p.T, p.T, p.N, d, f, gated) == Fo.shared_layer_flops(p.U, p.T, p.N, d, f, gated)
+
+
+def test_kernel_classes():
+    assert bench.kernel_class("attention") == "attention"
+    assert bench.kernel_class("gemm_up") == "gemm" and bench.kernel_class("linear") == "gemm"
+    assert bench.kernel_class("blend") == "rows" and bench.kernel_class("layernorm") == "rows"
+
+
+def test_traffic_table_records():
+    """Every record of profiles/traffic.json names a traced kernel class, carries positive bytes
+    and a source hash of the form kernel_source_sha writes (the bench reports a record only
+    while that hash matches the current sources of the class)."""
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as fh:
+        tj = json.load(fh)
+    shas = {k: bench.kernel_source_sha(k) for k in ("attention", "gemm", "rows")}
+    assert len(set(shas.values())) == 3 and all(len(v) == 16 for v in shas.values())
+    for cfg, kinds in tj.items():
+        if cfg.startswith("_"):
+            continue
+        for kind, rec in kinds.items():
+            assert bench.kernel_class(kind) in shas
+            assert rec["traffic_bytes_per_launch"] > 0
+            assert len(rec["kernel_source_sha"]) == 16 and int(rec["kernel_source_sha"], 16) >= 0

@@ -12,7 +12,6 @@ scratch than the array holds is refused before anything runs.
 The file is named so that pytest collects it last.
 """
 
-import numpy as np
 import pytest
 import torch
 
