@@ -96,6 +96,14 @@ def flops_layer(rows, T, N, d, f, gated=False):
     return rows * 2.0 * (4 * d * d + (3 if gated else 2) * d * f) + 4.0 * T * N * N * d
 
 
+def flops_partial(U, T, N, d, f, qkv, out, mlp, gated=False):
+    """A partially shared layer: each shared operation on U + T rows, the others on T * N rows."""
+    def rows(shared):
+        return U + T if shared else T * N
+    return (2.0 * 3 * d * d * rows(qkv) + 2.0 * d * d * rows(out) + (6.0 if gated else 4.0) * d * f * rows(mlp)
+            + 4.0 * T * N * N * d)
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples of one GPU while running."""
 
@@ -487,11 +495,8 @@ def run_tileshare(args, rank, world, local):
     ft = flops_layer(T * N, T, N, d, f, gated)
     fs = flops_layer(U + T, T, N, d, f, gated)
     if share is not None:
-        # partial sharing: each shared operation on U + T rows, the others on T * N rows
-        def rows(bit):
-            return U + T if share & bit else T * N
-        fs = (2.0 * 3 * d * d * rows(B.TS_SHARE_QKV) + 2.0 * d * d * rows(B.TS_SHARE_OUT) +
-              (6.0 if gated else 4.0) * d * f * rows(B.TS_SHARE_MLP) + 4.0 * T * N * N * d)
+        fs = flops_partial(U, T, N, d, f, share & B.TS_SHARE_QKV, share & B.TS_SHARE_OUT, share & B.TS_SHARE_MLP,
+                           gated)
     flop_ratio = (k * ft + (L - k) * fs) / (L * ft)
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,

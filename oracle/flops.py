@@ -32,3 +32,16 @@ def stack_flop_ratio(U: int, T: int, N: int, d: int, f: int, L: int, k: int, gat
     tiled = tiled_layer_flops(T, N, d, f, gated)
     shared = shared_layer_flops(U, T, N, d, f, gated)
     return (k * tiled + (L - k) * shared) / (L * tiled)
+
+
+def partial_layer_flops(U: int, T: int, N: int, d: int, f: int, shared, gated: bool = False) -> int:
+    """A partially shared layer (Tab. 1 top, Tab. S7): the operations named in `shared`
+    ("qkv", "out", "mlp") run on the U + T shared rows, the others on the T * N tile rows;
+    attention is per tile either way."""
+    shared = set(shared)
+    if not shared <= {"qkv", "out", "mlp"}:
+        raise ValueError(f"unknown shared operations {shared}")
+    def rows(op):
+        return U + T if op in shared else T * N
+    return (2 * 3 * d * d * rows("qkv") + 2 * d * d * rows("out") + 2 * (3 if gated else 2) * d * f * rows("mlp")
+            + attention_flops(T, N, d))

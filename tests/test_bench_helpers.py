@@ -56,3 +56,11 @@ def test_traffic_table_records():
             assert bench.kernel_class(kind) in shas
             assert rec["traffic_bytes_per_launch"] > 0
             assert len(rec["kernel_source_sha"]) == 16 and int(rec["kernel_source_sha"], 16) >= 0
+
+
+@pytest.mark.parametrize("ops", [(), ("qkv",), ("out",), ("mlp",), ("qkv", "mlp"), ("qkv", "out", "mlp")])
+def test_bench_partial_flops_match_the_oracle_count(ops):
+    p = OP.make_plan((4, 44, 80), (4, 32, 32), (4, 24, 24))
+    d, f = 1536, 6144
+    got = bench.flops_partial(p.U, p.T, p.N, d, f, "qkv" in ops, "out" in ops, "mlp" in ops)
+    assert got == Fo.partial_layer_flops(p.U, p.T, p.N, d, f, ops)

@@ -5,6 +5,7 @@ import math
 import os
 
 import numpy as np
+import pytest
 import torch
 
 from oracle import flops as Fo
@@ -91,3 +92,24 @@ def test_flop_model_degenerates_and_matches_pages_structure():
     d, f = 512, 2048
     diff = Fo.tiled_layer_flops(p.T, p.N, d, f) - Fo.shared_layer_flops(p.U, p.T, p.N, d, f)
     assert diff == (p.T * p.Nw - p.U) * Fo.linear_flops_per_row(d, f)
+
+
+@pytest.mark.parametrize("gated", [False, True])
+def test_partial_sharing_flops(gated):
+    # nothing shared is the per-tile layer, everything shared is the shared layer, and the
+    # savings of the single operations add up (the structure of Tab. 1 and Tab. S7)
+    p = P.make_plan((4, 44, 80), (4, 32, 32), (4, 24, 24))
+    U, T, N, d, f = p.U, p.T, p.N, 1536, 6144
+    tiled = Fo.tiled_layer_flops(T, N, d, f, gated)
+    assert Fo.partial_layer_flops(U, T, N, d, f, (), gated) == tiled
+    assert Fo.partial_layer_flops(U, T, N, d, f, ("qkv", "out", "mlp"), gated) == \
+        Fo.shared_layer_flops(U, T, N, d, f, gated)
+    single = {op: tiled - Fo.partial_layer_flops(U, T, N, d, f, (op,), gated) for op in ("qkv", "out", "mlp")}
+    for combo in (("qkv", "out"), ("qkv", "mlp"), ("out", "mlp")):
+        assert tiled - Fo.partial_layer_flops(U, T, N, d, f, combo, gated) == sum(single[o] for o in combo)
+    # each operation's saving is its per-row FLOPs on the duplicated rows
+    dup = T * N - (U + T)
+    assert single["qkv"] == 6 * d * d * dup and single["out"] == 2 * d * d * dup
+    assert single["mlp"] == 2 * (3 if gated else 2) * d * f * dup
+    with pytest.raises(ValueError):
+        Fo.partial_layer_flops(U, T, N, d, f, ("attn",))
