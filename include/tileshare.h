@@ -256,7 +256,8 @@ typedef enum {
    shared out-projection's and MLP's outputs are added to every tile's copy of the
    token.  shared_ops = 0 is ts_block_tiled; from identical per-tile copies, any set
    with TS_SHARE_OUT gives the shared layer's result in every copy.  Workspace as
-   for ts_block_tiled. */
+   for ts_block_tiled (TS_ERR_WORKSPACE if smaller); bits other than the three
+   above give TS_ERR_INVALID_ARG. */
 ts_status ts_block_partial(ts_plan_t plan, const ts_model_desc* model, const ts_layer_weights* w,
                            unsigned shared_ops, void* X, void* workspace, size_t workspace_bytes, void* stream);
 
