@@ -228,3 +228,26 @@ def test_host_planner_matches_oracle_on_random_geometries():
             assert p.max_cover == int(o.coverage.max())
         finally:
             p.close()
+
+
+def test_plain_c_program_against_the_headers(tmp_path):
+    """The headers are plain C: a C11 program compiles against include/, links
+    libtileshare.so and uses the host-side calls (no GPU)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    so = B.lib()._name
+    exe = str(tmp_path / "abi_host")
+    r = subprocess.run([cc, "-std=c11", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        os.path.join(ROOT, "tests", "c", "abi_host.c"), so, "-o", exe,
+                        "-Wl,-rpath," + os.path.dirname(so)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, (r.stdout, r.stderr)
+    fields = dict(kv.split("=", 1) for kv in r.stdout.split()[:10])
+    o = OP.make_plan((1, 48, 48), (1, 16, 16), (1, 12, 12), registers=2)
+    assert (int(fields["T"]), int(fields["U"]), int(fields["N"]), int(fields["R"]), int(fields["nnz"])) == \
+        (o.T, o.U, o.N, 2, o.nnz)
+    assert fields["device"] == "-1" and int(fields["ws"]) > 0 and fields["bad"] == "1"
