@@ -251,3 +251,23 @@ def test_plain_c_program_against_the_headers(tmp_path):
     assert (int(fields["T"]), int(fields["U"]), int(fields["N"]), int(fields["R"]), int(fields["nnz"])) == \
         (o.T, o.U, o.N, 2, o.nnz)
     assert fields["device"] == "-1" and int(fields["ws"]) > 0 and fields["bad"] == "1"
+
+
+@pytest.mark.parametrize("grid,win,stride", [((4, 44, 80), (4, 32, 32), (4, 24, 24)),
+                                             ((8, 44, 80), (4, 32, 32), (2, 24, 24)),
+                                             ((1, 48, 48), (1, 16, 16), (1, 12, 12)),
+                                             ((1, 128, 128), (1, 32, 32), (1, 24, 24))])
+def test_host_wbar_sums_to_one_within_one_ulp(grid, win, stride):
+    """The planner's fp32 w-bar of each token, summed in fp32 in ascending tile order (the
+    blend's order), is 1 within one ulp of 1.0 (2^-23)."""
+    p = B.Plan(grid, win, stride, host_only=True)
+    try:
+        w = p.wbar.astype(np.float32)
+        acc = np.zeros(p.U, dtype=np.float32)
+        cnt = np.diff(p.tok_ptr)
+        for k in range(int(cnt.max())):
+            has = cnt > k
+            acc[has] = (acc[has] + w[p.tok_ptr[:-1][has] + k]).astype(np.float32)
+        assert np.max(np.abs(acc.astype(np.float64) - 1.0)) <= 2.0 ** -23
+    finally:
+        p.close()
