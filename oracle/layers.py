@@ -137,13 +137,19 @@ def linear(x, w, b, m: Model):
 
 
 def attention(q, k, v):
-    """Dense softmax attention of one tile, all heads: q, k, v [n, heads, hd] -> [n, heads*hd]."""
+    """Dense softmax attention of one tile, all heads: q, k, v [n, heads, hd] -> [n, heads*hd].
+
+    Head by head: scores q_j k_j^T / sqrt(hd), a softmax over the keys, then the
+    weighted sum of the values.
+    """
     n, h, hd = q.shape
-    s = np.einsum("qhc,khc->hqk", q, k) / math.sqrt(hd)
-    s = s - s.max(axis=-1, keepdims=True)
-    p = np.exp(s)
-    p = p / p.sum(axis=-1, keepdims=True)
-    o = np.einsum("hqk,khc->qhc", p, v)
+    o = np.empty((n, h, hd), dtype=np.float64)
+    for j in range(h):
+        s = (q[:, j] @ k[:, j].T) / math.sqrt(hd)          # [n, m] scores of head j
+        s -= s.max(axis=-1, keepdims=True)
+        p = np.exp(s)
+        p /= p.sum(axis=-1, keepdims=True)
+        o[:, j] = p @ v[:, j]
     return o.reshape(n, h * hd)
 
 
