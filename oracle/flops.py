@@ -7,6 +7,10 @@ layers relative to per-tile layers; Tab. S6 notes that per-token work shrinks
 with the token count while attention is unchanged.  Counted here: the four
 linear layers (2 FLOPs per multiply-add) and the two attention contractions;
 norms, softmax, GELU / SiLU gating and the blend are not counted.
+
+Pinned by tests/test_oracle_flop_count.py: every linear layer and attention call
+that the oracle's own layers and stacks make is intercepted and the FLOPs of its
+operand shapes are summed; the closed forms below must equal those sums exactly.
 """
 
 
