@@ -194,18 +194,28 @@ ts_status ts_block_shared(ts_plan_t plan, const ts_model_desc* model, const ts_l
    plugin running inside a host application that owns every device buffer
    through its own pool and forbids the plugin from calling cudaMalloc, or code
    working inside a fixed, pre-partitioned memory budget.  It computes exactly
-   what ts_block_shared computes, in place on S [U + T*R, d], but its scratch
-   (normalised rows, q/k/v, attention outputs, blend, MLP hidden) lives in one
-   static device array of TS_NOALLOC_SCRATCH_BYTES (32 MiB) that every GPU
-   loading the library holds until the process exits.
+   what ts_block_shared computes (the same kernels, bit for bit), in place on
+   S [U + T*R, d], but its scratch (normalised rows, q/k/v, attention outputs,
+   blend, MLP hidden) lives in one static device array of
+   TS_NOALLOC_SCRATCH_BYTES (32 MiB) instead of a caller workspace.
    - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+   - When the array is reserved: the array belongs to the library's device code,
+     which the CUDA driver loads into a context on the library's first use there.
+     Under lazy module loading (the default of recent CUDA releases) that can be
+     the first ts_block_shared_noalloc call itself.  A caller inside a fixed
+     budget should make that happen at set-up: any call that launches a library
+     kernel or reads its device status, e.g. ts_device_status(), loads the code
+     and reserves the 32 MiB in the current context; it is held until the
+     context is destroyed or the process exits.
    - Plans and models needing more scratch than the array holds are refused with
      TS_ERR_WORKSPACE before anything is launched (the 48x48-token, d = 512
      workload needs about 26 MB; large grids do not fit and must use
      ts_block_shared).
-   - The first call on a device looks up the array's device address
-     (cudaGetSymbolAddress) with that device current; make that first call
-     before any stream capture on the device.
+   - The first call in a CUDA context looks up the array's device address in that
+     context (cudaGetSymbolAddress, with the plan's device current) and caches it
+     under the context's unique ID, so non-primary contexts and a context
+     recreated after cudaDeviceReset get their own lookup; make that first call
+     before any stream capture in the context.
    - Every call shares the one array and leaves its contents behind.  No region
      has to start at zero: each is written before it is read within a call.
      Calls that overlap on the GPU (other streams, other threads) race on the

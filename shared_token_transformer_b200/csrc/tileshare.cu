@@ -334,9 +334,12 @@ static ts::RopeTable make_rope_table(const ts_plan_s* p, const ts_model_desc* m,
   return rt;
 }
 
-static Workspace layout(const ts_plan_s* p, const ts_model_desc* m, bool stack, char* base) {
+// Regions of the caller workspace (256-byte aligned, in this order).  With
+// shared_only the regions cover one shared layer alone (rows U + T*R; no stack
+// states, no partial-sharing buffer): the scratch of ts_block_shared_noalloc.
+static Workspace layout(const ts_plan_s* p, const ts_model_desc* m, bool stack, char* base, bool shared_only = false) {
   const size_t Mt = static_cast<size_t>(p->T) * p->N, Ms = static_cast<size_t>(p->U) + p->G;
-  const size_t Mx = std::max(Mt, Ms);
+  const size_t Mx = shared_only ? Ms : std::max(Mt, Ms);
   const size_t e = esize(m->dtype), d = m->d, f = m->mlp;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -354,12 +357,12 @@ static Workspace layout(const ts_plan_s* p, const ts_model_desc* m, bool stack, 
     w.q8 = reinterpret_cast<uint8_t*>(take(Mx * std::max(d, f)));
     w.qs = reinterpret_cast<float*>(take(Mx * 4));
   }
-  if (stack) {
+  if (stack && !shared_only) {
     w.X = take(Mt * d * e);
     w.S = take(Ms * d * e);
   }
   w.rope = reinterpret_cast<float2*>(take(rope_table_entries(p, m) * sizeof(float2)));
-  w.sm = take(Ms * d * e);
+  if (!shared_only) w.sm = take(Ms * d * e);
   w.bytes = off;
   return w;
 }
@@ -1159,50 +1162,65 @@ ts_status ts_block_partial(ts_plan_t p, const ts_model_desc* m, const ts_layer_w
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[TS_NOALLOC_SCRATCH_BYTES];
 
-static std::mutex g_noalloc_mu;
-static void* g_noalloc_ptr[64];
+// Device address of the static scratch in the current CUDA context.  The address
+// belongs to a context (the module holding the array is loaded per context), so it
+// is cached under the driver's unique context ID, which a process never reuses:
+// a non-primary context, or a primary context recreated after a device reset,
+// gets its own lookup.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
 
-// Device address of the static scratch on the current device, looked up once per
-// device (with that device current) and cached.
-static ts_status noalloc_scratch(void** out) {
-  int dev = -1;
-  TS_CUDA_CHECK(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 64) return fail(TS_ERR_UNSUPPORTED, "device index %d out of range", dev);
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || !p)
-      return fail(TS_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
-    g_noalloc_ptr[dev] = p;
+static std::mutex g_noalloc_mu;
+struct NoallocEntry {
+  unsigned long long ctx_id;
+  void* ptr;
+};
+static std::vector<NoallocEntry> g_noalloc_cache;
+
+static ts_status current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  if (!get_current || !get_id) {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) != cudaSuccess ||
+        qa != cudaDriverEntryPointSuccess || !a ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) != cudaSuccess ||
+        qb != cudaDriverEntryPointSuccess || !b)
+      return fail(TS_ERR_CUDA, "cuCtxGetCurrent / cuCtxGetId not available");
+    get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+    get_id = reinterpret_cast<CtxGetIdFn>(b);
   }
-  *out = g_noalloc_ptr[dev];
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return fail(TS_ERR_CUDA, "no current CUDA context");
+  if (get_id(ctx, id) != CUDA_SUCCESS) return fail(TS_ERR_CUDA, "cuCtxGetId failed");
   return TS_OK;
 }
 
-// Scratch regions of one shared layer only (rows U + T*R, attention outputs T * N).
-static Workspace layout_shared_scratch(const ts_plan_s* p, const ts_model_desc* m, char* base) {
-  const size_t Mt = static_cast<size_t>(p->T) * p->N, Ms = static_cast<size_t>(p->U) + p->G;
-  const size_t e = esize(m->dtype), d = m->d, f = m->mlp;
-  size_t off = 0;
-  auto take = [&](size_t bytes) {
-    char* r = base ? base + off : nullptr;
-    off += align256(bytes);
-    return r;
-  };
-  Workspace w{};
-  w.xn = take(Ms * d * e);
-  w.qkv = take(Ms * 3 * d * e);
-  w.o = take(Mt * d * e);
-  w.a = take(Ms * d * e);
-  w.h = take(Ms * f * e);
-  if (m->dtype == TS_FP8_E4M3) {
-    w.q8 = reinterpret_cast<uint8_t*>(take(Ms * std::max(d, f)));
-    w.qs = reinterpret_cast<float*>(take(Ms * 4));
+static ts_status noalloc_scratch(void** out) {
+  int dev = -1;
+  TS_CUDA_CHECK(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  unsigned long long id = 0;
+  // A thread with no current context yet gets the device's primary context from
+  // the runtime at the symbol lookup below; it is looked up (and cached) then.
+  if (current_context_id(&id) == TS_OK) {
+    for (const NoallocEntry& e : g_noalloc_cache)
+      if (e.ctx_id == id) {
+        *out = e.ptr;
+        return TS_OK;
+      }
   }
-  w.rope = reinterpret_cast<float2*>(take(rope_table_entries(p, m) * sizeof(float2)));
-  w.bytes = off;
-  return w;
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || !p)
+    return fail(TS_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed on device %d: %s", dev,
+                cudaGetErrorString(e));
+  TS_TRY(current_context_id(&id));
+  g_noalloc_cache.push_back({id, p});
+  *out = p;
+  return TS_OK;
 }
 
 extern "C" {
@@ -1213,7 +1231,7 @@ ts_status ts_block_shared_noalloc(ts_plan_t p, const ts_model_desc* m, const ts_
   TS_TRY(check_model(m));
   TS_TRY(check_weights(m, w));
   if (!S || !aligned16(S)) return fail(TS_ERR_INVALID_ARG, "S must be a 16-byte aligned device pointer");
-  const size_t need = layout_shared_scratch(p, m, nullptr).bytes;
+  const size_t need = layout(p, m, false, nullptr, true).bytes;
   if (need > TS_NOALLOC_SCRATCH_BYTES)
     return fail(TS_ERR_WORKSPACE,
                 "ts_block_shared_noalloc: this plan and model need %zu bytes of scratch, the static array holds %u; "
@@ -1221,7 +1239,11 @@ ts_status ts_block_shared_noalloc(ts_plan_t p, const ts_model_desc* m, const ts_
                 need, TS_NOALLOC_SCRATCH_BYTES);
   void* base = nullptr;
   TS_TRY(noalloc_scratch(&base));
-  const Workspace W = layout_shared_scratch(p, m, static_cast<char*>(base));
+  const Workspace W = layout(p, m, false, static_cast<char*>(base), true);
+  // layer_shared reads the regions xn, qkv, o, a, h, rope (and q8, qs for e4m3)
+  // and no others (not X, S or sm, which the shared-only layout leaves null)
+  if (!W.xn || !W.qkv || !W.o || !W.a || !W.h || !W.rope || (m->dtype == TS_FP8_E4M3 && (!W.q8 || !W.qs)))
+    return fail(TS_ERR_WORKSPACE, "ts_block_shared_noalloc: scratch layout incomplete");
   return layer_shared(p, m, w, S, W, static_cast<cudaStream_t>(stream));
 }
 

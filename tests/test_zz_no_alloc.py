@@ -5,9 +5,12 @@ example a plugin inside a host application that owns every device buffer through
 its own pool.  For them the library keeps the shared layer's scratch in one
 static device array and ts_block_shared_noalloc uses it instead of a caller
 workspace.  These tests call it through the C ABI and check its output against
-ts_block_shared (with a caller workspace) within the bf16 tolerance of the
-other parity tests, on two calls in a row, and check that a plan needing more
-scratch than the array holds is refused before anything runs.
+ts_block_shared (with a caller workspace) on two calls in a row.  Both run the
+same kernels on the same inputs, with no atomics and 256-byte aligned regions
+either way, so the outputs must be identical bit for bit: a scratch region that
+overlaps another, or stale contents of the previous call read back, would break
+the equality long before it reached a tolerance.  A plan needing more scratch
+than the array holds must be refused before anything runs.
 
 The file is named so that pytest collects it last.
 """
@@ -18,7 +21,7 @@ import torch
 from shared_token_transformer_b200 import binding as B
 from shared_token_transformer_b200 import workloads as W
 
-from _gpu import Case, dev, host, rel_l2
+from _gpu import Case, dev
 
 pytestmark = pytest.mark.gpu
 
@@ -33,6 +36,7 @@ def _cuda():
 
 @pytest.mark.parametrize("cfg", [
     W.CONFIGS["stack48_bf16"],
+    W.CONFIGS["vit14_fp32"],
     W.small_config("noalloc_fp8", grid=(1, 11, 13), win=(1, 8, 8), stride=(1, 5, 6), d=256, heads=4, mlp=512,
                    dtype="fp8", L=2, k=0),
 ], ids=lambda c: c.name)
@@ -41,12 +45,11 @@ def test_noalloc_matches_workspace_path_two_calls_in_a_row(cfg):
     S_ref = dev(c.S, c.dt)
     S_na = S_ref.clone()
     ws = c.workspace()
-    tol = 3e-2 if cfg.dtype == "fp8" else 1e-2
     for call in range(2):
         B.block_shared(c.plan, c.m, c.wlist[call], S_ref, ws)
         B.block_shared_noalloc(c.plan, c.m, c.wlist[call], S_na)
         torch.cuda.synchronize()
-        assert rel_l2(host(S_na), host(S_ref)) < tol, call
+        assert torch.equal(S_na, S_ref), call
     B.device_status()
     c.plan.close()
 
