@@ -4,9 +4,9 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tileshare|reference] [--config NAME]
 
 A step is one TileShare-k decode of the configuration's seeded synthetic input
-(default: the 48x48-token, d=512, L=8, k=2 bf16 stack): per-tile copies of the
-input, k per-tile layers, the merge of the per-tile states, L-k shared layers and
-the copy of the output rows.  It runs through the library's public calls,
+(default: the 4K image, 256x256 tokens, d=1024, L=16, k=4 bf16 stack; --k sets
+another k): per-tile copies of the input, k per-tile layers, the merge of the
+per-tile states, L-k shared layers and the copy of the output rows.  It runs through the library's public calls,
 captured as CUDA graphs (one for the per-tile part, one for the shared part) so
 that the shared layers are timed on their own by CUDA events on the launching
 stream; L2 is flushed (512 MiB write) before every step, outside the events.
@@ -15,12 +15,18 @@ value  = unique tokens per second per shared layer = U * (L - k) * K * N_ranks /
          (max over ranks of the summed shared-part time of the K steps).
 e2e    = the same metric through the public call with host buffers: pinned host
          state -> device, one ts_block_shared, device -> pinned host, timed with
-         CUDA events around the copies and the call.
+         CUDA events around the copies and the call; the value is the median step,
+         with the spread of the steps beside it.
 roofline  per kernel class from a traced pass (library kernel trace: CUDA events
          around each launch, algorithmic FLOPs / HBM bytes per launch); the
-         dominant class (most time) is reported against MEASURED_PEAKS.json.
+         dominant class (most time) is reported against MEASURED_PEAKS.json: the
+         burst bf16 figure when the traced pass lasts under a second, the
+         sustained one otherwise; fp32 kernels against the FP32 SIMT peak.
 cpu_baseline  the float64 CPU oracle's shared layer on the same inputs (rank 0,
-         N = 1).  --impl reference times that oracle alone as the reference arm.
+         N = 1): whole layers when one fits the budget, else a bounded sample
+         (per-token steps on blocks of rows, attention of whole tiles, the whole
+         blend) scaled to the layer.  --impl reference times that oracle alone as
+         the reference arm, each step a bounded sample of the same kind.
 
 Multi-GPU (torchrun): every rank decodes its own image (independent inputs, the
 same weights); there is no data-path collective, only a barrier and a max of the
@@ -51,10 +57,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="tileshare", choices=["tileshare", "reference"])
-    ap.add_argument("--config", default="stack48_bf16")
+    ap.add_argument("--config", default="image4k_bf16")
+    ap.add_argument("--k", type=int, default=None, help="per-tile layers before the merge (default: the workload's)")
     ap.add_argument("--no-graph", action="store_true", help="launch the calls eagerly instead of CUDA graphs")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -76,7 +83,23 @@ def config_of(args):
     cfg = W.CONFIGS[args.config]
     if args.block is not None and args.block != cfg.block:
         cfg = dataclasses.replace(cfg, block=args.block)
+    k = getattr(args, "k", None)
+    if k is not None:
+        if not 0 <= k <= cfg.L:
+            raise SystemExit(f"--k must lie in [0, {cfg.L}]")
+        cfg = dataclasses.replace(cfg, k=k)
     return cfg
+
+
+def workload_config(cfg, args, U, T, N, world):
+    """The `config` object of the JSON line (the same for both arms)."""
+    return {"workload": f"{cfg.name}: {cfg.note}", "grid": list(cfg.grid), "window": list(cfg.win),
+            "stride": list(cfg.stride), "blend": args.blend, "block": cfg.block,
+            "shared_ops": args.shared_ops or "TileShare shared layer",
+            "L": cfg.L, "k": cfg.k, "unique_tokens": U, "tiles": T, "rows_per_tile": N,
+            "l2": "flushed before every step (512 MiB write, outside the timed events)",
+            "launch": "eager public calls" if args.no_graph else "CUDA graphs of the public calls",
+            "parallelism": f"replicas x{world} (one image per GPU)"}
 
 
 # ---------------------------------------------------------------------------
@@ -178,8 +201,7 @@ def blas_threads():
     return os.cpu_count()
 
 
-def oracle_shared_layer_timing(cfg, budget_s, max_steps, warmup=1, rule="ramp"):
-    """Time the float64 oracle's shared layer on the configuration's seeded input."""
+def _oracle_inputs(cfg, rule):
     from oracle import layers as OL
     from oracle import plan as OP
     from shared_token_transformer_b200 import workloads as W
@@ -189,6 +211,59 @@ def oracle_shared_layer_timing(cfg, budget_s, max_steps, warmup=1, rule="ramp"):
     S = np.concatenate([S0, G0])
     layer = dr.layer()
     om = OL.Model(cfg.d, cfg.heads, cfg.mlp, cfg.rope_dims, fp8=(cfg.dtype == "fp8"), block=cfg.block)
+    return op, S, layer, om
+
+
+def oracle_layer_sample_seconds(op, S, layer, om, budget_s, row_block=1024):
+    """Seconds of one float64 oracle shared layer, estimated from a bounded sample.
+
+    The layer's work is per-token steps (Norm1, QKV, QK-RMSNorm, out-projection,
+    MLP) on its U + T rows, attention of each of its T tiles, and the blend.  Row
+    blocks and whole tiles are timed in turn until each kind has used half the
+    budget or all of its work; the blend over all tokens is timed once.  Each
+    kind's time is scaled by (all its units / units timed).  With a budget large
+    enough for the whole layer this is the whole layer, timed piece by piece.
+    Returns (seconds, description)."""
+    from oracle import layers as OL
+    M, T = S.shape[0], op.T
+    t_tok = t_att = 0.0
+    rows = tiles = 0
+    half = budget_s / 2
+    while rows < M and (rows == 0 or t_tok < half):
+        x = S[rows: rows + row_block]
+        t0 = time.perf_counter()
+        OL.qkv_project(x, layer, om)
+        y = x + OL.linear(x, layer["w_o"], layer["b_o"], om)      # out-projection of a block of rows
+        OL.mlp_residual(y, layer, om)
+        t_tok += time.perf_counter() - t0
+        rows += x.shape[0]
+    while tiles < T and (tiles == 0 or t_att < half):
+        r = OL.tile_rows(op, tiles)
+        q, k, v = OL.qkv_project(S[r], layer, om)                  # untimed: counted with the rows
+        t0 = time.perf_counter()
+        OL.tile_attention(q, k, v, op.slot_pos, om)
+        t_att += time.perf_counter() - t0
+        tiles += 1
+    O = np.zeros((T, op.N, S.shape[1]))
+    t0 = time.perf_counter()
+    OL.merge(O, op)
+    t_blend = time.perf_counter() - t0
+    sec = t_tok * M / rows + t_att * T / tiles + t_blend
+    what = (f"per-token steps on {rows} of {M} rows, attention of {tiles} of {T} tiles, the whole blend; "
+            f"each scaled by its share of the layer")
+    return sec, what
+
+
+def oracle_shared_layer_timing(cfg, budget_s, max_steps, warmup=1, rule="ramp"):
+    """Unique tokens/s of the float64 oracle's shared layer on the configuration's
+    seeded input: whole layers (block_shared) when one fits the budget, else one
+    bounded sample (oracle_layer_sample_seconds).  Returns (rate, steps, sample)."""
+    from oracle import layers as OL
+    op, S, layer, om = _oracle_inputs(cfg, rule)
+    est, what = oracle_layer_sample_seconds(op, S, layer, om, min(budget_s, 4.0))
+    if est * (max(1, warmup) + 1) > budget_s:
+        sec, what = oracle_layer_sample_seconds(op, S, layer, om, budget_s)
+        return op.U / sec, 1, f"one float64 oracle shared layer of {cfg.name}, timed on a bounded sample: {what}"
     for _ in range(warmup):
         OL.block_shared(S, layer, om, op)
     times = []
@@ -199,7 +274,8 @@ def oracle_shared_layer_timing(cfg, budget_s, max_steps, warmup=1, rule="ramp"):
         times.append(time.perf_counter() - t0)
         if time.perf_counter() - t_all > budget_s:
             break
-    return op.U, times
+    mean = float(np.mean(times))
+    return op.U / mean, len(times), f"{len(times)} whole float64 oracle shared layers of {cfg.name} (~{budget_s:.0f} s budget)"
 
 
 # ---------------------------------------------------------------------------
@@ -219,6 +295,7 @@ def run_tileshare(args, rank, world, local):
     cfg = config_of(args)
     L, k = cfg.L, cfg.k
     dt = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.bfloat16}[cfg.dtype]
+    num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
     plan = B.Plan(cfg.grid, cfg.win, cfg.stride,
                   rule=B.TS_BLEND_HARD_STITCH if args.blend == "hard" else B.TS_BLEND_LINEAR_RAMP)
     U, T, N, d, f = plan.U, plan.T, plan.N, cfg.d, cfg.mlp
@@ -393,7 +470,7 @@ def run_tileshare(args, rank, world, local):
     tiled_stack_ms = float(np.mean([a.elapsed_time(b) for a, b in tev]))
 
     # e2e: one shared layer through the public call with pinned host buffers
-    Ke = min(K, 200)
+    Ke = max(20, min(K, 200))
     if share is not None:
         # partial sharing: the per-tile state [T * N, d] goes in and out
         B.gather_tiles(plan, m, S0d, G0d, X)
@@ -432,12 +509,19 @@ def run_tileshare(args, rank, world, local):
         if i >= 3:
             eev[i - 3][1].record()
     torch.cuda.synchronize()
-    e2e_ms = float(np.mean([a.elapsed_time(b) for a, b in eev]))
+    e2e_all = np.array([a.elapsed_time(b) for a, b in eev])
+    e2e_ms = float(np.median(e2e_all))
     (e2e_max,) = max_over_ranks([e2e_ms], world)
     e2e_value = replica_rate(U, world, e2e_max)
+    e2e_spread = {"steps": int(len(e2e_all)), "ms_median": round(e2e_ms, 4),
+                  "ms_p10": round(float(np.percentile(e2e_all, 10)), 4),
+                  "ms_p90": round(float(np.percentile(e2e_all, 90)), 4),
+                  "ms_mean": round(float(e2e_all.mean()), 4)}
     state_bytes = S_host.numel() * S_host.element_size()
 
     # traced pass: per-kernel times of the same step, eagerly launched
+    torch.cuda.synchronize()
+    t_tr0 = time.perf_counter()
     B.trace_begin(100000)
     for _ in range(args.trace_steps):
         flush.zero_()
@@ -445,16 +529,33 @@ def run_tileshare(args, rank, world, local):
         part_shared()
         part_out()
     tr = B.trace_end()
+    trace_s = time.perf_counter() - t_tr0
     sampler.stop()
     clocks = sampler.summary(t_wall0, t_wall1)
 
     pk, pk_src = peaks()
-    bf16_peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    # a traced pass under a second runs at burst clocks; a longer one settles
+    # under the power cap, where the sustained figure applies
+    burst = trace_s < 1.0 or "bf16_tflops_sustained" not in pk
+    bf16_key = "bf16_tflops" if burst else "bf16_tflops_sustained"
+    bf16_peak = pk[bf16_key]
+    # fp32 path: SIMT FMA lanes x 2 FLOPs x clock (148 SMs x 128 FP32 lanes)
+    f32_peak = num_sms * 128 * 2 * float(pk.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
 
     def tensor_peak_of(name):
         # e4m3 GEMMs against the bf16 peak x the nominal e4m3 : bf16 dense ratio;
         # attention computes in bf16 in every configuration
+        if cfg.dtype == "f32":
+            return f32_peak
         return 2.0 * bf16_peak if cfg.dtype == "fp8" and not name.startswith("attention") else bf16_peak
+
+    def peak_source(name, unit):
+        if unit != "TFLOP/s":
+            return f"{pk_src} hbm_gbs"
+        if cfg.dtype == "f32":
+            return f"fp32 SIMT: {num_sms} SMs x 128 lanes x 2 FLOP x {pk.get('sm_max_mhz', 1965.0):.0f} MHz"
+        src = f"{pk_src} {bf16_key} (traced pass {trace_s:.2f} s)"
+        return src + (" x2 (e4m3:bf16 nominal)" if tensor_peak_of(name) > bf16_peak else "")
     total_ms = sum(v["ms"] for v in tr.values()) or 1.0
     kernels = {}
     for name, v in tr.items():
@@ -484,12 +585,10 @@ def run_tileshare(args, rank, world, local):
         ent = tj.get(args.config, {}).get(dom)
         if ent and ent.get("kernel_source_sha") == kernel_source_sha(kernel_class(dom)):
             traffic = ent.get("traffic_bytes_per_launch")
-    roofline = {"bound": "tensor" if kd["unit"] == "TFLOP/s" else "hbm", "kernel": dom, "achieved": kd["achieved"],
+    bound = ("alu" if cfg.dtype == "f32" else "tensor") if kd["unit"] == "TFLOP/s" else "hbm"
+    roofline = {"bound": bound, "kernel": dom, "achieved": kd["achieved"],
                 "peak": round(tensor_peak_of(dom) if kd["unit"] == "TFLOP/s" else pk["hbm_gbs"], 1), "unit": kd["unit"],
-                "frac": kd["frac"], "traffic": traffic,
-                "peak_source": (f"{pk_src} " + ("bf16_tflops_sustained" + (" x2 (e4m3:bf16 nominal)"
-                                                                           if tensor_peak_of(dom) > bf16_peak else "")
-                                                if kd["unit"] == "TFLOP/s" else "hbm_gbs"))}
+                "frac": kd["frac"], "traffic": traffic, "peak_source": peak_source(dom, kd["unit"])}
 
     gated = cfg.block == "rms_swiglu"
     ft = flops_layer(T * N, T, N, d, f, gated)
@@ -503,13 +602,7 @@ def run_tileshare(args, rank, world, local):
         "warmup": args.warmup, "ms_per_step": round(step_ms, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": {"bf16": "bf16", "f32": "f32", "fp8": "e4m3"}[cfg.dtype],
         "data": "synthetic (seeded N(0,1) states, N(0,0.02) weights, random init)",
-        "config": {"workload": f"{cfg.name}: {cfg.note}", "grid": list(cfg.grid), "window": list(cfg.win),
-                   "stride": list(cfg.stride), "blend": args.blend, "block": cfg.block,
-                   "shared_ops": (args.shared_ops or "none") if share is not None else "TileShare shared layer",
-                   "L": L, "k": k, "unique_tokens": U, "tiles": T, "rows_per_tile": N,
-                   "l2": "flushed before every step (512 MiB write, outside the timed events)",
-                   "launch": "CUDA graphs of the public calls" if use_graph else "eager public calls",
-                   "parallelism": f"replicas x{world} (one image per GPU)"},
+        "config": workload_config(cfg, args, U, T, N, world),
         "shared_layer_ms": round(shared_total_ms / K / max(1, L - k), 5),
         "per_tile_part_ms": round(tiled_ms, 5),
         "tiled_stack_ms": round(tiled_stack_ms, 5),
@@ -517,7 +610,7 @@ def run_tileshare(args, rank, world, local):
         "flop_ratio": round(flop_ratio, 4),
         "speedup_bar": round(0.85 / flop_ratio, 4),
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": state_bytes,
-                "d2h_bytes_per_step": state_bytes, "call": ("ts_block_partial" if share is not None else "ts_block_shared") + " with pinned host state in/out" +
+                "d2h_bytes_per_step": state_bytes, "spread": e2e_spread, "call": ("ts_block_partial" if share is not None else "ts_block_shared") + " with pinned host state in/out, value from the median step" +
                         (", copies and call replayed as one CUDA graph per step" if use_graph else "")},
         "gpu_launches": int(gpu_launches),
         "roofline": roofline,
@@ -575,6 +668,42 @@ def kernel_class(name):
     return "rows"
 
 
+def run_reference(args, cfg, world):
+    """The reference arm: the float64 CPU oracle's shared layer on this arm's
+    workload, W untimed and K timed steps, each a whole layer when one fits the
+    per-step budget, else a bounded sample of it, so that the run ends within a
+    few minutes."""
+    from oracle import layers as OL
+    op, S, layer, om = _oracle_inputs(cfg, args.blend)
+    K, Wm = max(1, args.steps), max(0, args.warmup)
+    per = max(1.0, 90.0 / (K + Wm))
+    est, what = oracle_layer_sample_seconds(op, S, layer, om, min(per, 4.0))
+    whole = est <= per
+    times = []
+    for i in range(Wm + K):
+        if whole:
+            t0 = time.perf_counter()
+            OL.block_shared(S, layer, om, op)
+            sec = time.perf_counter() - t0
+        else:
+            sec, what = oracle_layer_sample_seconds(op, S, layer, om, per)
+        if i >= Wm:
+            times.append(sec)
+    mean = float(np.mean(times))
+    v = op.U / mean
+    sample = (f"each step one whole float64 oracle shared layer of {cfg.name}" if whole else
+              f"each step one float64 oracle shared layer of {cfg.name} timed on a bounded sample "
+              f"(~{per:.0f} s): {what}")
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": UNIT, "n_gpus": world,
+            "steps": K, "warmup": Wm, "ms_per_step": round(mean * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded, same draws as the tileshare arm)",
+            "config": workload_config(cfg, args, op.U, op.T, op.N, world),
+            "cpu_baseline": {"value": round(v, 2), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(v, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -586,20 +715,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        budget = 150.0
-        U, times = oracle_shared_layer_timing(cfg, budget, args.steps, warmup=min(args.warmup, 1), rule=args.blend)
-        mean = float(np.mean(times))
-        v = U / mean
-        res = {"impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": UNIT, "n_gpus": world,
-               "steps": len(times), "warmup": min(args.warmup, 1), "ms_per_step": round(mean * 1e3, 3),
-               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-               "data": "synthetic (seeded, same draws as the tileshare arm)",
-               "config": {"workload": f"{cfg.name}: {cfg.note}", "grid": list(cfg.grid), "L": cfg.L, "k": cfg.k, "block": cfg.block},
-               "cpu_baseline": {"value": round(v, 2), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                                "sample": f"{len(times)} float64 oracle shared layers of {cfg.name} "
-                                          f"(steps capped at a {budget:.0f} s budget)"},
-               "e2e": {"value": round(v, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-        print(json.dumps(res))
+        print(json.dumps(run_reference(args, cfg, world)))
         return
 
     import torch.distributed as dist
@@ -610,15 +726,9 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     res, cfg = run_tileshare(args, rank, world, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        if flops_layer(cfg.U + 1, 1, 1, cfg.d, cfg.mlp, cfg.block == "rms_swiglu") < 5e11:
-            U, times = oracle_shared_layer_timing(cfg, args.cpu_seconds, 1000, rule=args.blend)
-            mean = float(np.mean(times))
-            res["cpu_baseline"] = {"value": round(U / mean, 2), "unit": UNIT, "cores": blas_threads(),
-                                   "kind": "oracle",
-                                   "sample": f"{len(times)} float64 oracle shared layers of {cfg.name} "
-                                             f"(~{args.cpu_seconds:.0f} s budget)"}
-        else:
-            res["cpu_baseline"] = None
+        rate, n, what = oracle_shared_layer_timing(cfg, args.cpu_seconds, 1000, rule=args.blend)
+        res["cpu_baseline"] = {"value": round(rate, 2), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                               "sample": what}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -19,3 +19,24 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+def pytest_collection_finish(session):
+    """Start the oracle runs of the selected full-size stack tests in worker
+    processes, so that they overlap the GPU tests collected before them."""
+    keys = [item.callspec.params["job"] for item in session.items
+            if getattr(item, "module", None) is not None and item.module.__name__ == "test_gpu_stack_fullsize"
+            and hasattr(item, "callspec")]
+    if not keys:
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    import _oracle_jobs
+    _oracle_jobs.start(keys)
+
+
+def pytest_sessionfinish(session, exitstatus):
+    mod = sys.modules.get("_oracle_jobs")
+    if mod is not None:
+        mod.shutdown()

@@ -64,3 +64,25 @@ def test_bench_partial_flops_match_the_oracle_count(ops):
     d, f = 1536, 6144
     got = bench.flops_partial(p.U, p.T, p.N, d, f, "qkv" in ops, "out" in ops, "mlp" in ops)
     assert got == Fo.partial_layer_flops(p.U, p.T, p.N, d, f, ops)
+
+
+def test_config_of_k_override():
+    a = _Args("video44x80_fp8")
+    a.k = 0
+    assert bench.config_of(a).k == 0 and bench.config_of(a).L == 24
+    a.k = 25
+    with pytest.raises(SystemExit):
+        bench.config_of(a)
+
+
+def test_oracle_sample_covers_the_whole_layer_when_the_budget_allows():
+    # with room for everything the sample is the whole layer, piece by piece: every
+    # row block and every tile timed once, and no scaling
+    cfg = bench.config_of(_Args("vit14_fp32"))
+    op, S, layer, om = bench._oracle_inputs(cfg, "ramp")
+    sec, what = bench.oracle_layer_sample_seconds(op, S, layer, om, budget_s=1e9, row_block=64)
+    assert sec > 0
+    assert f"{S.shape[0]} of {S.shape[0]} rows" in what and f"{op.T} of {op.T} tiles" in what
+    # a tiny budget still times one row block and one tile
+    sec, what = bench.oracle_layer_sample_seconds(op, S, layer, om, budget_s=1e-9, row_block=64)
+    assert f"64 of {S.shape[0]} rows" in what and f"1 of {op.T} tiles" in what
