@@ -8,7 +8,10 @@
 // (RoPE runs once per row in the QKV epilogue), so this is a plain gathered
 // attention.
 //
-// bf16 kernel (hd = 64), grid (nqb, heads, T), 256 threads, 2 CTAs per SM:
+// bf16 kernel (hd = 64), grid (nqb, T, heads), 256 threads, 2 CTAs per SM.  The
+// head index is the slowest grid dimension: CTAs in flight together work on one
+// head of neighbouring tiles, whose overlapping q/k/v rows (one head's slice of
+// the whole shared state: a few MB) then come from L2 instead of DRAM.
 //   blocks qb < nqb: 128 window queries, keys in blocks of 64.
 //     warp 4     TMA producer of Q (once) and of K/V blocks into 128-byte-
 //                swizzled shared rows: one box of a 3-D map over the grid per
@@ -65,6 +68,10 @@ constexpr int kAttnBK = 64;              // keys per block
 constexpr int kAttnKV = 4;               // K/V buffers
 constexpr int kAttnS = 3;                // S / P buffers in TMEM
 constexpr float kAttnRescale = 8.0f;     // lazy rescale threshold (log2 units)
+#ifndef TS_ATTN_EMU_EVERY
+#define TS_ATTN_EMU_EVERY 4
+#endif
+constexpr int kAttnEmuEvery = TS_ATTN_EMU_EVERY;   // one score pair in this many: 2^x on the FMA pipe
 
 struct AttnSmem {
   static constexpr int Q = 0;                 // 16 KB: 128 rows x 128 B
@@ -149,6 +156,27 @@ __device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
+}
+// 2^x of a pair of exponents on the FMA pipe, for x <= 2^7 (x below -125 is
+// taken as -125, whose power is below every probability that matters here).
+// Range reduction by the round-to-nearest addition of 1.5 * 2^23: the sum's low
+// mantissa bits hold the integer j nearest to x, and f = x - j lies in
+// [-1/2, 1/2] exactly.  2^f is a cubic fitted here for least maximum relative
+// error on [-1/2, 1/2] (Lawson's iteration; 7.5e-5, far below the 2^-9 of the
+// bf16 rounding of P), evaluated by Horner's rule on pairs; 2^j enters by adding
+// j to the result's exponent field (j << 23 wraps the 1.5 * 2^23 offset away).
+__device__ __forceinline__ void exp2_fma2(uint64_t x2, float& e0, float& e1) {
+  const float x0 = fmaxf(lo_f32(x2), -125.f), x1 = fmaxf(hi_f32(x2), -125.f);
+  const uint64_t xc = pack_f32x2(x0, x1);
+  const uint64_t t = add_f32x2(xc, pack_f32x2(12582912.f, 12582912.f));
+  const uint64_t j = add_f32x2(t, pack_f32x2(-12582912.f, -12582912.f));
+  const uint64_t f = fma_f32x2(j, pack_f32x2(-1.f, -1.f), xc);
+  uint64_t p = fma_f32x2(pack_f32x2(0.0551716685295105f, 0.0551716685295105f), f,
+                         pack_f32x2(0.2426111251115799f, 0.2426111251115799f));
+  p = fma_f32x2(p, f, pack_f32x2(0.6932609677314758f, 0.6932609677314758f));
+  p = fma_f32x2(p, f, pack_f32x2(0.9999280571937561f, 0.9999280571937561f));
+  e0 = __uint_as_float(__float_as_uint(lo_f32(p)) + (__float_as_uint(lo_f32(t)) << 23));
+  e1 = __uint_as_float(__float_as_uint(hi_f32(p)) + (__float_as_uint(hi_f32(t)) << 23));
 }
 // true in exactly one lane of the (fully active) warp
 __device__ __forceinline__ bool elect_one() {
@@ -567,30 +595,11 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
           for (int i = 0; i < kAttnBK; ++i)
             if (kbase + i >= a.Nw) sv[i] = -INFINITY;
         }
-        // The exponentials are taken against the current reference maximum m right
-        // away; the block's maximum is formed alongside them (independent chains).
-        // The reference moves only when a score exceeds it by more than 2^8 (lazy
-        // rescale: probabilities stay below 256 and O is rarely touched); such a row
-        // takes its exponentials again against the new reference.
-        const uint64_t sc2 = pack_f32x2(a.scale_log2, a.scale_log2);
-        uint64_t sp2[4];
-        uint32_t pw[kAttnBK / 2];
-        // pairs of scores through packed f32x2 arithmetic: one FMA per pair forms the
-        // exponents, the SFU takes each exponential, four packed partial sums; P goes
-        // back into the S columns as packed bf16 pairs (the A operand of P V)
-        auto exps = [&](float mref) {
-          const uint64_t nm2 = pack_f32x2(-mref, -mref);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) sp2[q] = 0ull;
-#pragma unroll
-          for (int i = 0; i < kAttnBK; i += 2) {
-            const uint64_t x2 = fma_f32x2(pack_f32x2(sv[i], sv[i + 1]), sc2, nm2);
-            const float e0 = ex2_approx(lo_f32(x2)), e1 = ex2_approx(hi_f32(x2));
-            sp2[(i >> 1) & 3] = add_f32x2(sp2[(i >> 1) & 3], pack_f32x2(e0, e1));
-            pw[i >> 1] = pack_bf16(e0, e1);
-          }
-        };
-        float mp[8];   // eight independent partial maxima keep the dependency chains short
+        // Block maximum first (eight independent partial maxima keep the chains
+        // short).  The reference maximum m moves only when a score exceeds it by
+        // more than 2^8 (lazy rescale: probabilities stay below 256 and O is rarely
+        // touched); then the exponentials are taken once, against m.
+        float mp[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           mp[q] = fmax3(sv[q], sv[8 + q], sv[16 + q]);
@@ -598,7 +607,6 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
           mp[q] = fmax3(mp[q], sv[40 + q], sv[48 + q]);
           mp[q] = fmaxf(mp[q], sv[56 + q]);
         }
-        exps(m);
         const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7])) * a.scale_log2;
         const bool grow = mx > m + kAttnRescale;
         const bool warp_grow = __any_sync(0xffffffffu, grow);
@@ -608,7 +616,40 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
           l *= alpha;
           gcoef *= alpha;
           m = mx;
-          exps(m);
+        }
+        // Pairs of scores through packed f32x2 arithmetic: one FMA per pair forms the
+        // exponents x = s * log2(e) / sqrt(hd) - m, four packed partial sums, P back
+        // into the S columns as packed bf16 pairs (the A operand of P V).  In a full
+        // block one pair in kAttnEmuEvery takes 2^x on the FMA pipe (exp2_fma2), the
+        // others on the SFU; the SFU alone would bound the block at twice the tensor
+        // time.  The last, partial block keeps every exponential on the SFU, whose
+        // 2^-inf = 0 removes its padding keys exactly.
+        const uint64_t sc2 = pack_f32x2(a.scale_log2, a.scale_log2);
+        const uint64_t nm2 = pack_f32x2(-m, -m);
+        uint64_t sp2[4] = {0ull, 0ull, 0ull, 0ull};
+        uint32_t pw[kAttnBK / 2];
+        if (kbase + kAttnBK <= a.Nw) {
+#pragma unroll
+          for (int i = 0; i < kAttnBK; i += 2) {
+            const uint64_t x2 = fma_f32x2(pack_f32x2(sv[i], sv[i + 1]), sc2, nm2);
+            float e0, e1;
+            if ((i >> 1) % kAttnEmuEvery == kAttnEmuEvery - 1) {
+              exp2_fma2(x2, e0, e1);
+            } else {
+              e0 = ex2_approx(lo_f32(x2));
+              e1 = ex2_approx(hi_f32(x2));
+            }
+            sp2[(i >> 1) & 3] = add_f32x2(sp2[(i >> 1) & 3], pack_f32x2(e0, e1));
+            pw[i >> 1] = pack_bf16(e0, e1);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < kAttnBK; i += 2) {
+            const uint64_t x2 = fma_f32x2(pack_f32x2(sv[i], sv[i + 1]), sc2, nm2);
+            const float e0 = ex2_approx(lo_f32(x2)), e1 = ex2_approx(hi_f32(x2));
+            sp2[(i >> 1) & 3] = add_f32x2(sp2[(i >> 1) & 3], pack_f32x2(e0, e1));
+            pw[i >> 1] = pack_bf16(e0, e1);
+          }
         }
         const uint64_t s01 = add_f32x2(sp2[0], sp2[1]), s23 = add_f32x2(sp2[2], sp2[3]);
         const uint64_t s0123 = add_f32x2(s01, s23);
@@ -672,7 +713,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     if (threadIdx.x == 0) set_status(kStatusDeviceCheck);
     return;
   }
-  attn_window_block_tc(&tm, a, blockIdx.x, blockIdx.y, blockIdx.z, smem);
+  attn_window_block_tc(&tm, a, blockIdx.x, blockIdx.z, blockIdx.y, smem);
 }
 
 // ---------------------------------------------------------------------------

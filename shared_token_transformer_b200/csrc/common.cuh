@@ -92,7 +92,13 @@ __device__ __noinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, uint64
     }
   }
 }
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) { return mbar_wait_for(bar, parity, kWaitLimitNs); }
+// Fast path inline (one potentially blocking try_wait); the bounded loop is a call.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+#ifndef TS_MBAR_NOFAST
+  if (mbar_try_wait(bar, parity)) return true;
+#endif
+  return mbar_wait_for(bar, parity, kWaitLimitNs);
+}
 
 // Self-test of the bounded wait: one thread initialises an mbarrier that nothing
 // arrives at and waits for it with a short limit; the wait must give up, write

@@ -713,7 +713,7 @@ static ts_status run_attention(const ts_plan_s* p, const ts_model_desc* m, bool 
     a.load = a.run > 0 ? 1 : 0;
     TS_TRY(make_tmap(&tm, qkv, shared ? p->U + p->G : p->T * p->N, 3 * m->d, 2, a.run > 0 ? a.run : 1));
   }
-  dim3 grid(nqb, m->heads, p->T);
+  dim3 grid(nqb, p->T, m->heads);   // head slowest: neighbouring tiles of one head share L2
   launch_pdl(ts::attn_bf16_kernel, grid, dim3(ts::kAttnThreads), ts::AttnSmem::LAUNCH_BYTES, st, tm, a);
   return trace_post(st, "attn_bf16");
 }
