@@ -9,6 +9,16 @@ within the test run (it runs in worker processes while the other GPU tests
 use the device, see _oracle_jobs).  The whole output is compared with the
 oracle's decode_stack on the same seeded inputs (relative L2 1e-2 for bf16,
 3e-2 for e4m3), and the worst row of every coverage class within 1.5 times that.
+
+e4m3 stacks: every e4m3 code is a rounding decision, and a bf16-level change of
+a quantiser's input moves a few per cent of the codes by one e4m3 step; the
+flips feed the next quantiser.  The oracle's own output therefore drifts by
+about 3e-2 over two layers when only the precision in which it stores its
+attention outputs and layer outputs changes (its "floor", computed in the same
+run).  The kernels store those tensors in bf16 and compute attention in bf16,
+so their distance to the oracle cannot fall below that floor: the e4m3 bound is
+max(3e-2, 1.5 x floor), and the per-layer parity of the e4m3 layers at full size
+(no compounding) stays at 3e-2 in test_gpu_fullsize.
 """
 
 import numpy as np
@@ -51,6 +61,11 @@ def test_decode_stack_full_geometry(job):
     want = J.result(job, timeout=900)
     assert want.shape == got.shape
     tol = TOL[cfg.dtype]
-    assert rel_l2(got, want) < tol
+    if J.needs_floor(job):
+        floor = rel_l2(J.result(job + J.FLOOR, timeout=900), want)
+        tol = max(tol, 1.5 * floor)
+    err = rel_l2(got, want)
+    print(f"{job}: relative L2 {err:.4e}, bound {tol:.4e}")
+    assert err < tol, f"relative L2 {err:.4e}, bound {tol:.4e}"
     assert_rows(got, want, op, "tokens", tol)
     c.plan.close()
