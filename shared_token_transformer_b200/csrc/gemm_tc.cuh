@@ -114,7 +114,18 @@ __device__ __forceinline__ void qk_norm_rope64(float* v, const float* __restrict
 // scales, bias, then GELU or QK-RMSNorm + RoPE (the residual is added by the caller).
 template <int EPI, bool FP8, int R0, int R1, int R2>
 __device__ __forceinline__ void gemm_epilogue64(float* v, int col, float rs, const int4 pos, const GemmArgs& args) {
-  if (FP8) {
+  if (FP8 && args.bias) {
+    // dequantisation scale and bias in one FMA per value
+#pragma unroll
+    for (int i = 0; i < 64; i += 4) {
+      const float4 ws = __ldg(reinterpret_cast<const float4*>(args.w_scale + col + i));
+      const float4 b = __ldg(reinterpret_cast<const float4*>(args.bias + col + i));
+      v[i] = fmaf(v[i], rs * ws.x, b.x);
+      v[i + 1] = fmaf(v[i + 1], rs * ws.y, b.y);
+      v[i + 2] = fmaf(v[i + 2], rs * ws.z, b.z);
+      v[i + 3] = fmaf(v[i + 3], rs * ws.w, b.w);
+    }
+  } else if (FP8) {
 #pragma unroll
     for (int i = 0; i < 64; i += 4) {
       const float4 ws = __ldg(reinterpret_cast<const float4*>(args.w_scale + col + i));
@@ -123,8 +134,7 @@ __device__ __forceinline__ void gemm_epilogue64(float* v, int col, float rs, con
       v[i + 2] *= rs * ws.z;
       v[i + 3] *= rs * ws.w;
     }
-  }
-  if (args.bias) {
+  } else if (args.bias) {
 #pragma unroll
     for (int i = 0; i < 64; i += 4) {
       const float4 b = __ldg(reinterpret_cast<const float4*>(args.bias + col + i));
@@ -136,7 +146,7 @@ __device__ __forceinline__ void gemm_epilogue64(float* v, int col, float rs, con
   }
   if (EPI == EPI_GELU) {
 #pragma unroll
-    for (int i = 0; i < 64; ++i) v[i] = gelu_erf(v[i]);
+    for (int i = 0; i < 64; ++i) v[i] = FP8 ? gelu_erf_one_sfu(v[i]) : gelu_erf(v[i]);
   } else if (EPI == EPI_QKV) {
     if (col < 2 * args.d)
       qk_norm_rope64<R0, R1, R2>(v, col < args.d ? args.q_g : args.k_g, args.eps_qk, pos, args);

@@ -101,6 +101,34 @@ def test_gelu_epilogue_matches_exact_erf():
     assert np.max(np.abs(got - want) / np.maximum(1.0, np.abs(want))) < 2e-6
 
 
+def test_gelu_epilogue_e4m3_matches_exact_erf():
+    """The e4m3 GEMMs' GELU epilogue evaluates erf by Abramowitz & Stegun 7.1.28
+    (one approximate reciprocal raised to the 16th power).  Inputs on the e4m3
+    grid times a power of two and an identity weight make the scaled product
+    exact, so every bf16 output must be exact-erf GELU of its input within one
+    bf16 rounding (2^-8 relative to max(1, |GELU|)), over both signs, zero and
+    the tails."""
+    import math
+    from oracle import fp8 as F8
+    K = N = 128
+    grid = np.array(sorted({F8.decode_e4m3(c) for c in range(127)}))
+    rng = np.random.default_rng(9)
+    x = rng.choice(grid, (256, K)) * rng.choice([-1.0, 1.0], (256, K)) / 32.0
+    x[:, 0] = 448.0 / 32.0                       # row absmax 14: scale 1/32, the row quantises exactly
+    x[0, 1:] = 0.0
+    w = np.eye(N, K)
+    m = B.model_desc(256, 4, 256, "fp8", (0, 32, 32))
+    q = torch.empty((N, K), dtype=torch.uint8, device="cuda")
+    s = torch.empty(N, dtype=torch.float32, device="cuda")
+    B.quantize_rows_e4m3(dev(w, torch.bfloat16), q, s)
+    y = torch.empty((256, N), dtype=torch.bfloat16, device="cuda")
+    scratch = torch.empty(256 * K + 4 * 256 + 512, dtype=torch.uint8, device="cuda")
+    B.op_linear(m, dev(x, torch.bfloat16), q, dev(np.zeros(N), torch.float32), y, epi=B.TS_EPI_BIAS_GELU,
+                w_scale=s, scratch=scratch)
+    want = np.vectorize(lambda v: 0.5 * v * (1.0 + math.erf(v / math.sqrt(2.0))))(x)
+    assert np.max(np.abs(host(y) - want) / np.maximum(1.0, np.abs(want))) <= 2.0 ** -8
+
+
 # (2320, 2048, 512) and (2320, 512, 512): the 48 x 48 layer's MLP down and out-projection
 @pytest.mark.parametrize("M,K,N", [(300, 256, 512), (128, 512, 768), (129, 256, 192), (1, 256, 64), (2320, 512, 1536),
                                    (777, 2048, 512), (2320, 2048, 512), (2320, 512, 512)])
