@@ -391,13 +391,14 @@ def run_tileshare(args, rank, world, local):
         with torch.cuda.stream(side):
             with torch.cuda.graph(g1, stream=side):
                 part_tiled()
-            with torch.cuda.graph(g2, stream=side):
-                part_shared()
+            if k < L:                      # with k = L there is no shared layer to capture
+                with torch.cuda.graph(g2, stream=side):
+                    part_shared()
             with torch.cuda.graph(g3, stream=side):
                 part_out()
         torch.cuda.current_stream().wait_stream(side)
         launches_per_step = B.launch_count() - n0
-        run1, run2, run3 = g1.replay, g2.replay, g3.replay
+        run1, run2, run3 = g1.replay, (g2.replay if k < L else (lambda: None)), g3.replay
         for _ in range(max(3, args.warmup)):
             run1(); run2(); run3()
     else:
@@ -613,6 +614,7 @@ def run_tileshare(args, rank, world, local):
                 "d2h_bytes_per_step": state_bytes, "spread": e2e_spread, "call": ("ts_block_partial" if share is not None else "ts_block_shared") + " with pinned host state in/out, value from the median step" +
                         (", copies and call replayed as one CUDA graph per step" if use_graph else "")},
         "gpu_launches": int(gpu_launches),
+        **({"note": "k = L: every layer per tile, no shared layer (value 0 by definition)"} if L == k else {}),
         "roofline": roofline,
         "kernels": kernels,
         "clocks": clocks,
@@ -727,6 +729,8 @@ def main():
     res, cfg = run_tileshare(args, rank, world, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, n, what = oracle_shared_layer_timing(cfg, args.cpu_seconds, 1000, rule=args.blend)
+        if args.shared_ops is not None:
+            what += "; the oracle's fully shared layer (partial sharing is not timed on the CPU)"
         res["cpu_baseline"] = {"value": round(rate, 2), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                                "sample": what}
     if world > 1:
