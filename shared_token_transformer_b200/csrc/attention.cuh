@@ -8,10 +8,13 @@
 // (RoPE runs once per row in the QKV epilogue), so this is a plain gathered
 // attention.
 //
-// bf16 kernel (hd = 64), grid (nqb, T, heads), 256 threads, 2 CTAs per SM.  The
-// head index is the slowest grid dimension: CTAs in flight together work on one
+// bf16 kernel (hd = 64), 256 threads, 2 CTAs per SM.  Shared layer: grid
+// (nqb, T, heads), the head slowest, so that CTAs in flight together work on one
 // head of neighbouring tiles, whose overlapping q/k/v rows (one head's slice of
-// the whole shared state: a few MB) then come from L2 instead of DRAM.
+// the whole shared state: a few MB) then come from L2 instead of DRAM.  Per-tile
+// layer (no rows shared between tiles): grid (nqb, heads, T), the tile slowest, so
+// that the heads of one tile run together and each tile's q/k/v rows (all heads'
+// column slices of the same rows) leave DRAM once.
 //   blocks qb < nqb: 128 window queries, keys in blocks of 64.
 //     warp 4     TMA producer of Q (once) and of K/V blocks into 128-byte-
 //                swizzled shared rows: one box of a 3-D map over the grid per
@@ -53,6 +56,7 @@ struct AttnArgs {
   int gw;             // load 2: grid width; shared row u is grid row u / gw, column u % gw
   float scale_log2;   // log2(e) / sqrt(hd)
   float scale;        // 1 / sqrt(hd)
+  int head_major;     // bf16 grid: 1 (nqb, T, heads), head slowest; 0 (nqb, heads, T), tile slowest
 };
 
 __device__ __forceinline__ int attn_row(const AttnArgs& a, int t, int s) {
@@ -713,7 +717,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     if (threadIdx.x == 0) set_status(kStatusDeviceCheck);
     return;
   }
-  attn_window_block_tc(&tm, a, blockIdx.x, blockIdx.z, blockIdx.y, smem);
+  const int h = a.head_major ? blockIdx.z : blockIdx.y, t = a.head_major ? blockIdx.y : blockIdx.z;
+  attn_window_block_tc(&tm, a, blockIdx.x, h, t, smem);
 }
 
 // ---------------------------------------------------------------------------

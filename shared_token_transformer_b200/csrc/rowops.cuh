@@ -66,56 +66,70 @@ __device__ __forceinline__ void store_row(const float (&v)[NV][Vec<T>::E], int l
 // two passes over the row held in registers.  NV = d / (32 * E) vectors per lane.
 // With rms set it is RMSNorm (Tab. S6 "RMSNorm"): no centring and no bias.
 // ---------------------------------------------------------------------------
-// Blocks past the rows (when rt.cs is set) fill the RoPE table that the next
-// QKV GEMM reads.
+// The first `row_blocks` blocks walk the rows grid-stride (one row per warp at a
+// time, the warp's next row loaded before the current one is normalised, so two
+// rows per warp are in flight); blocks past them (when rt.cs is set) fill the RoPE
+// table that the next QKV GEMM reads.
 template <typename T, int NV, bool Q8>
 __global__ void __launch_bounds__(256) layernorm_kernel(const T* __restrict__ x, int rows, int d,
                                                         const float* __restrict__ g, const float* __restrict__ b,
                                                         float eps, int rms, T* __restrict__ y, uint8_t* __restrict__ q8,
-                                                        float* __restrict__ qscale, const RopeTable rt) {
+                                                        float* __restrict__ qscale, const RopeTable rt,
+                                                        unsigned row_blocks) {
   pdl_wait();
   pdl_trigger();
   constexpr int E = Vec<T>::E;
   const int lane = threadIdx.x & 31;
-  const unsigned row_blocks = (static_cast<unsigned>(rows) + 7) / 8;
   if (blockIdx.x >= row_blocks) {
     rope_table_fill(rt, static_cast<int>((blockIdx.x - row_blocks) * blockDim.x + threadIdx.x));
     return;
   }
-  const size_t row = static_cast<size_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (row >= static_cast<size_t>(rows)) return;
-  float v[NV][E];
-  float s = 0.f;
+  const size_t step = static_cast<size_t>(row_blocks) * (blockDim.x >> 5);
+  size_t row = static_cast<size_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  // the next row waits in registers as raw 16-byte vectors
+  uint4 nx[NV];
+  if (row < static_cast<size_t>(rows)) {
 #pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    Vec<T>::load(x + row * d + (i * 32 + lane) * E, v[i]);
-#pragma unroll
-    for (int e = 0; e < E; ++e) s += v[i][e];
+    for (int i = 0; i < NV; ++i) nx[i] = *reinterpret_cast<const uint4*>(x + row * d + (i * 32 + lane) * E);
   }
-  const float mean = rms ? 0.f : warp_sum(s) / d;
-  float q = 0.f;
+  for (; row < static_cast<size_t>(rows); row += step) {
+    float v[NV][E];
 #pragma unroll
-  for (int i = 0; i < NV; ++i)
+    for (int i = 0; i < NV; ++i) Vec<T>::load(reinterpret_cast<const T*>(&nx[i]), v[i]);
+    if (row + step < static_cast<size_t>(rows)) {
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const float c = v[i][e] - mean;
-      q = fmaf(c, c, q);
+      for (int i = 0; i < NV; ++i) nx[i] = *reinterpret_cast<const uint4*>(x + (row + step) * d + (i * 32 + lane) * E);
     }
-  const float rstd = rsqrtf(warp_sum(q) / d + eps);
+    float s = 0.f;
 #pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int c0 = (i * 32 + lane) * E;
+    for (int i = 0; i < NV; ++i)
 #pragma unroll
-    for (int e = 0; e < E; e += 4) {   // gains and biases as 16-byte vectors
-      const float4 gg = __ldg(reinterpret_cast<const float4*>(g + c0 + e));
-      const float4 bb = rms ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldg(reinterpret_cast<const float4*>(b + c0 + e));
-      v[i][e] = (v[i][e] - mean) * rstd * gg.x + bb.x;
-      v[i][e + 1] = (v[i][e + 1] - mean) * rstd * gg.y + bb.y;
-      v[i][e + 2] = (v[i][e + 2] - mean) * rstd * gg.z + bb.z;
-      v[i][e + 3] = (v[i][e + 3] - mean) * rstd * gg.w + bb.w;
+      for (int e = 0; e < E; ++e) s += v[i][e];
+    const float mean = rms ? 0.f : warp_sum(s) / d;
+    float q = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float c = v[i][e] - mean;
+        q = fmaf(c, c, q);
+      }
+    const float rstd = rsqrtf(warp_sum(q) / d + eps);
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int c0 = (i * 32 + lane) * E;
+#pragma unroll
+      for (int e = 0; e < E; e += 4) {   // gains and biases as 16-byte vectors
+        const float4 gg = __ldg(reinterpret_cast<const float4*>(g + c0 + e));
+        const float4 bb = rms ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldg(reinterpret_cast<const float4*>(b + c0 + e));
+        v[i][e] = (v[i][e] - mean) * rstd * gg.x + bb.x;
+        v[i][e + 1] = (v[i][e + 1] - mean) * rstd * gg.y + bb.y;
+        v[i][e + 2] = (v[i][e + 2] - mean) * rstd * gg.z + bb.z;
+        v[i][e + 3] = (v[i][e + 3] - mean) * rstd * gg.w + bb.w;
+      }
     }
+    store_row<T, NV, Q8>(v, lane, y, q8, qscale, row, d);
   }
-  store_row<T, NV, Q8>(v, lane, y, q8, qscale, row, d);
 }
 
 // generic fallback: any d (one warp per row, scalar, two passes over global memory)

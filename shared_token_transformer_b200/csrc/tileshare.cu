@@ -392,11 +392,19 @@ static ts_status launch_layernorm_vec(const void* x, int rows, int d, const floa
   const T* xx = static_cast<const T*>(x);
   T* yy = static_cast<T*>(y);
   trace_pre(st);
-#define TS_LN_CASE(NV) \
-  case NV:                                                                                                  \
-    launch_pdl(ts::layernorm_kernel<T, NV, Q8>, dim3(rows_grid(rows) + fill_blocks), dim3(256), 0, st, xx, rows, d, \
-               g, b, eps, rms, yy, q8, qs, rt);                                                               \
-    break;
+  // row blocks: as many as are resident at once (all of them walk the rows grid-stride)
+#define TS_LN_CASE(NV)                                                                                      \
+  case NV: {                                                                                                \
+    auto kern = ts::layernorm_kernel<T, NV, Q8>;                                                            \
+    static int occ = 0;                                                                                     \
+    if (occ <= 0) {                                                                                         \
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 256, 0) != cudaSuccess || occ < 1) occ = 1; \
+    }                                                                                                       \
+    const unsigned row_blocks = std::min<unsigned>(rows_grid(rows), static_cast<unsigned>(occ * num_sms())); \
+    launch_pdl(kern, dim3(row_blocks + fill_blocks), dim3(256), 0, st, xx, rows, d, g, b, eps, rms, yy, q8, qs, rt, \
+               row_blocks);                                                                                 \
+    break;                                                                                                  \
+  }
   switch (nv) {
     TS_LN_CASE(1) TS_LN_CASE(2) TS_LN_CASE(3) TS_LN_CASE(4) TS_LN_CASE(5) TS_LN_CASE(6) TS_LN_CASE(7) TS_LN_CASE(8)
     default: return fail(TS_ERR_UNSUPPORTED, "layernorm width %d", d);
@@ -713,7 +721,9 @@ static ts_status run_attention(const ts_plan_s* p, const ts_model_desc* m, bool 
     a.load = a.run > 0 ? 1 : 0;
     TS_TRY(make_tmap(&tm, qkv, shared ? p->U + p->G : p->T * p->N, 3 * m->d, 2, a.run > 0 ? a.run : 1));
   }
-  dim3 grid(nqb, p->T, m->heads);   // head slowest: neighbouring tiles of one head share L2
+  a.head_major = shared ? 1 : 0;
+  dim3 grid = shared ? dim3(nqb, p->T, m->heads)    // head slowest: neighbouring tiles of one head share L2
+                     : dim3(nqb, m->heads, p->T);   // tile slowest: a tile's rows are read once for all heads
   launch_pdl(ts::attn_bf16_kernel, grid, dim3(ts::kAttnThreads), ts::AttnSmem::LAUNCH_BYTES, st, tm, a);
   return trace_post(st, "attn_bf16");
 }
