@@ -59,10 +59,10 @@ constexpr int kGemmThreads = 320;   // 8 epilogue warps + TMA warp + MMA warp
 constexpr int kGemmTmaWarp = 8;
 constexpr int kGemmMmaWarp = 9;
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int CG = 1>
 struct GemmSmem {
   static constexpr int A_BYTES = 128 * 128;
-  static constexpr int B_BYTES = BN * 128;
+  static constexpr int B_BYTES = (BN / CG) * 128;   // a CTA of a two-SM pair holds half of W's tile rows
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int EPI_OFFSET = STAGES * STAGE_BYTES;   // 8 x 4 KB: one 32 x 64 output chunk per epilogue warp
   static constexpr int BAR_OFFSET = EPI_OFFSET + 8 * 4096;
@@ -194,23 +194,33 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 // column tiles with the row tile fastest.  The CTAs in flight then share one or
 // two bands of A and the whole of W, which stay in L2 even when A does not.
 constexpr int kGemmBand = 16;
-__device__ __forceinline__ void gemm_tile_origin(int tile, int mt, int nt, int bn, int& m0, int& n0) {
+__device__ __forceinline__ void gemm_tile_origin(int tile, int mt, int nt, int bn, int& m0, int& n0, int tm = 128) {
   const int band = tile / (kGemmBand * nt);
   const int first = band * kGemmBand;
   const int rows = min(kGemmBand, mt - first);
   const int r = tile - first * nt;
-  m0 = (first + r % rows) * 128;
+  m0 = (first + r % rows) * tm;
   n0 = (r / rows) * bn;
 }
 
-template <int BN, int STAGES, int EPI, bool FP8, int R0, int R1, int R2>
+// CG = 2: a two-SM pair (cluster of two CTAs) computes 256 x BN tiles with
+// tcgen05 cta_group::2.  Each CTA loads its own 128 rows of A and half of the
+// tile's W rows into its own shared memory (no multicast), both CTAs' loads
+// completing on the even CTA's ring barriers; the even CTA's MMA warp issues the
+// M = 256 MMAs, and its commits arrive on the ring and accumulator barriers of both
+// CTAs.  Each CTA's TMEM holds the accumulators of its own 128 rows, which its
+// epilogue warps read as in a single CTA; they release an accumulator on the even
+// CTA's barrier.  Half the W bytes per CTA leave room for deeper rings.
+template <int BN, int STAGES, int EPI, bool FP8, int R0, int R1, int R2, int CG = 1>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmD, const GemmArgs args) {
-  using SM = GemmSmem<BN, STAGES>;
+  static_assert(CG == 1 || CG == 2, "one CTA or a two-SM pair");
+  using SM = GemmSmem<BN, STAGES, CG>;
   constexpr int NMMA = 128 / 32;                  // MMAs per 128-byte K slice (32 bytes each)
   constexpr uint32_t TMEM_COLS = 2 * BN;          // two accumulators: 128, 256 or 512 columns
-  constexpr uint32_t IDESC = idesc_make(FP8 ? 0u : 1u, BN);
+  constexpr uint32_t IDESC = idesc_make(FP8 ? 0u : 1u, BN, 128 * CG);
+  constexpr int TM = 128 * CG;                    // output rows per tile
   constexpr int KE = FP8 ? 128 : 64;              // K elements per slice
   constexpr bool GLU = EPI == EPI_SWIGLU;
   static_assert(!GLU || BN >= 128, "SwiGLU tiles need 64-column output chunks");
@@ -228,9 +238,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int mt = (args.M + 127) / 128;
+  const int mt = (args.M + TM - 1) / TM;
   const int ntiles = mt * (args.N / BN);
   const int KB = args.K / KE;
+  // tiles are walked per CTA, or per pair (the two CTAs of a pair walk the same tiles)
+  const uint32_t rank = CG == 2 ? cluster_rank() : 0u;
+  const int unit = CG == 2 ? static_cast<int>(blockIdx.x) / 2 : static_cast<int>(blockIdx.x);
+  const int units = CG == 2 ? static_cast<int>(gridDim.x) / 2 : static_cast<int>(gridDim.x);
+  const bool leader = rank == 0;
 
   if (warp == kGemmTmaWarp && lane == 0) {
     tma_prefetch_desc(&tmA);
@@ -242,17 +257,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_tfull + 8 * b, 1);
-      mbar_init(bar_tempty + 8 * b, 8);           // one arrival per epilogue warp
+      mbar_init(bar_tempty + 8 * b, 8 * CG);      // one arrival per epilogue warp (of both CTAs of a pair)
     }
     for (int w = 0; w < 8; ++w) mbar_init(bar_resid + 8 * w, 1);
     fence_barrier_init();
   }
   if (warp == kGemmMmaWarp) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-    tmem_relinquish();
+    if (CG == 2) {
+      tmem_alloc2(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_relinquish2();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if (CG == 2) cluster_sync();      // the pair's barriers exist before either CTA touches the other's
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   pdl_wait();        // A and the output/residual belong to the previous kernel
@@ -262,29 +283,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      for (int tile = unit; tile < ntiles && ok; tile += units) {
         int m0, n0;
-        gemm_tile_origin(tile, mt, args.N / BN, BN, m0, n0);
+        gemm_tile_origin(tile, mt, args.N / BN, BN, m0, n0, TM);
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const uint32_t s = it % STAGES;
           if (it >= STAGES && !mbar_wait(bar_empty + 8 * s, ((it / STAGES) - 1) & 1)) { ok = false; break; }
           const uint32_t sa = sbase + s * SM::STAGE_BYTES;
-          mbar_expect_tx(bar_full + 8 * s, SM::STAGE_BYTES);
-          tma_load_2d(sa, &tmA, bar_full + 8 * s, kb * KE, m0);
-          if (GLU) {    // BN/2 gate rows, then the BN/2 up rows of the same outputs
-            tma_load_2d(sa + SM::A_BYTES, &tmB, bar_full + 8 * s, kb * KE, n0 / 2);
-            tma_load_2d(sa + SM::A_BYTES + (BN / 2) * 128, &tmB, bar_full + 8 * s, kb * KE, args.N / 2 + n0 / 2);
+          if (CG == 2) {
+            // both CTAs' bytes complete on the even CTA's barrier, which expects them all
+            const uint32_t fb = cluster_map(bar_full + 8 * s, 0);
+            if (leader) mbar_expect_tx(bar_full + 8 * s, 2 * SM::STAGE_BYTES);
+            tma_load_2d_pair(sa, &tmA, fb, kb * KE, m0 + static_cast<int>(rank) * 128);
+            if (GLU)    // the even CTA holds the BN/2 gate rows, the odd one the BN/2 up rows
+              tma_load_2d_pair(sa + SM::A_BYTES, &tmB, fb, kb * KE, (rank ? args.N / 2 : 0) + n0 / 2);
+            else
+              tma_load_2d_pair(sa + SM::A_BYTES, &tmB, fb, kb * KE, n0 + static_cast<int>(rank) * (BN / 2));
           } else {
-            tma_load_2d(sa + SM::A_BYTES, &tmB, bar_full + 8 * s, kb * KE, n0);
+            mbar_expect_tx(bar_full + 8 * s, SM::STAGE_BYTES);
+            tma_load_2d(sa, &tmA, bar_full + 8 * s, kb * KE, m0);
+            if (GLU) {    // BN/2 gate rows, then the BN/2 up rows of the same outputs
+              tma_load_2d(sa + SM::A_BYTES, &tmB, bar_full + 8 * s, kb * KE, n0 / 2);
+              tma_load_2d(sa + SM::A_BYTES + (BN / 2) * 128, &tmB, bar_full + 8 * s, kb * KE, args.N / 2 + n0 / 2);
+            } else {
+              tma_load_2d(sa + SM::A_BYTES, &tmB, bar_full + 8 * s, kb * KE, n0);
+            }
           }
         }
       }
     }
   } else if (warp == kGemmMmaWarp) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {        // the odd CTA of a pair issues no MMA
       uint32_t it = 0, j = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++j) {
+      for (int tile = unit; tile < ntiles && ok; tile += units, ++j) {
         const uint32_t acc = j & 1, use = j >> 1;
         if (j >= 2 && !mbar_wait(bar_tempty + 8 * acc, (use - 1) & 1)) { ok = false; break; }
         tc_fence_after();
@@ -299,14 +331,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int k = 0; k < NMMA; ++k) {
             // +32 bytes of K = +2 in the descriptor's (address >> 4) field
-            if (FP8)
-              tc_mma_f8(dt, da + 2 * k, db + 2 * k, IDESC, (kb | k) != 0);
-            else
-              tc_mma_f16(dt, da + 2 * k, db + 2 * k, IDESC, (kb | k) != 0);
+            if (CG == 2) {
+              if (FP8)
+                tc_mma_f8_pair(dt, da + 2 * k, db + 2 * k, IDESC, (kb | k) != 0);
+              else
+                tc_mma_f16_pair(dt, da + 2 * k, db + 2 * k, IDESC, (kb | k) != 0);
+            } else {
+              if (FP8)
+                tc_mma_f8(dt, da + 2 * k, db + 2 * k, IDESC, (kb | k) != 0);
+              else
+                tc_mma_f16(dt, da + 2 * k, db + 2 * k, IDESC, (kb | k) != 0);
+            }
           }
-          tc_commit(bar_empty + 8 * s);
+          if (CG == 2)
+            tc_commit_pair(bar_empty + 8 * s);
+          else
+            tc_commit(bar_empty + 8 * s);
         }
-        tc_commit(bar_tfull + 8 * acc);
+        if (CG == 2)
+          tc_commit_pair(bar_tfull + 8 * acc);
+        else
+          tc_commit(bar_tfull + 8 * acc);
       }
     }
   } else {
@@ -319,10 +364,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     bool store_pending = false;        // a tile store may still be reading the staging buffer
     bool eok = true;
     uint32_t j = 0;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++j) {
+    // accumulator release: on this CTA's barrier, or on the even CTA's for a pair
+    const uint32_t tempty = CG == 2 ? cluster_map(bar_tempty, 0) : bar_tempty;
+    auto release = [&](uint32_t acc) {
+      if (CG == 2)
+        mbar_arrive_cluster(tempty + 8 * acc);
+      else
+        mbar_arrive(tempty + 8 * acc);
+    };
+    for (int tile = unit; tile < ntiles; tile += units, ++j) {
       const uint32_t acc = j & 1, use = j >> 1;
       int m0, n0;
-      gemm_tile_origin(tile, mt, args.N / BN, BN, m0, n0);
+      gemm_tile_origin(tile, mt, args.N / BN, BN, m0, n0, TM);
+      m0 += static_cast<int>(rank) * 128;      // this CTA's rows of the tile
       const int row = m0 + quarter * 32 + lane;
       // the row's scale and coordinates are loaded while the accumulator fills
       float rs = 1.f;
@@ -338,7 +392,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (mine == 0) {
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_tempty + 8 * acc);
+        if (lane == 0) release(acc);
       }
 #pragma unroll 1
       for (int c = half, k = 0; c < NCHUNK; c += 2, ++k) {
@@ -368,14 +422,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (k == mine - 1) {         // last TMEM read of this warp for this tile
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar_tempty + 8 * acc);
+            if (lane == 0) release(acc);
           }
           swiglu32<FP8>(v + 32, u, col + 32, args.N / 2, rs, args);
         } else {
           if (k == mine - 1) {         // last TMEM read of this warp for this tile
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar_tempty + 8 * acc);
+            if (lane == 0) release(acc);
           }
           gemm_epilogue64<EPI, FP8, R0, R1, R2>(v, col, rs, pos, args);
         }
@@ -410,9 +464,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if (CG == 2) cluster_sync();      // neither CTA leaves while the pair's MMAs or arrivals may still touch it
   if (warp == kGemmMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    if (CG == 2)
+      tmem_dealloc2(tmem, TMEM_COLS);
+    else
+      tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 

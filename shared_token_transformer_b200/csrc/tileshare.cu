@@ -217,6 +217,27 @@ static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
+// The same launch as clusters of two CTAs (two-SM MMA pairs); grid.x is even.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl_pair(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                   Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // ============================================================================
 // model checks and RoPE tables
 // ============================================================================
@@ -525,11 +546,11 @@ static ts_status run_quantize(const void* x, int rows, int cols, uint8_t* q, flo
 // ---------------------------------------------------------------------------
 
 
-template <int BN, int STAGES, int EPI, bool FP8, int R0, int R1, int R2>
+template <int BN, int STAGES, int EPI, bool FP8, int R0, int R1, int R2, int CG = 1>
 static ts_status launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
                                 const ts::GemmArgs& args, cudaStream_t st) {
-  using SM = ts::GemmSmem<BN, STAGES>;
-  auto kern = ts::gemm_tc_kernel<BN, STAGES, EPI, FP8, R0, R1, R2>;
+  using SM = ts::GemmSmem<BN, STAGES, CG>;
+  auto kern = ts::gemm_tc_kernel<BN, STAGES, EPI, FP8, R0, R1, R2, CG>;
   static int configured[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -537,18 +558,26 @@ static ts_status launch_gemm_tc(const CUtensorMap& ta, const CUtensorMap& tb, co
     TS_CUDA_CHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::LAUNCH_BYTES));
     configured[dev] = 1;
   }
-  const int tiles = ((args.M + 127) / 128) * (args.N / BN);
-  dim3 grid(std::min(tiles, num_sms()));
+  const int tiles = ((args.M + 128 * CG - 1) / (128 * CG)) * (args.N / BN);
   trace_pre(st);
-  launch_pdl(kern, grid, dim3(ts::kGemmThreads), SM::LAUNCH_BYTES, st, ta, tb, td, args);
+  if (CG == 2) {
+    // one pair per two SMs, both CTAs of a pair walking the same tiles
+    dim3 grid(2 * std::min(tiles, num_sms() / 2));
+    launch_pdl_pair(kern, grid, dim3(ts::kGemmThreads), SM::LAUNCH_BYTES, st, ta, tb, td, args);
+  } else {
+    dim3 grid(std::min(tiles, num_sms()));
+    launch_pdl(kern, grid, dim3(ts::kGemmThreads), SM::LAUNCH_BYTES, st, ta, tb, td, args);
+  }
   return trace_post(st, "gemm_tc");
 }
 
 template <int EPI, bool FP8, int R0, int R1, int R2>
-static ts_status dispatch_gemm_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
-                                  const ts::GemmArgs& args, cudaStream_t st) {
+static ts_status dispatch_gemm_bn(int bn, bool pair, const CUtensorMap& ta, const CUtensorMap& tb,
+                                  const CUtensorMap& td, const ts::GemmArgs& args, cudaStream_t st) {
   switch (bn) {
-    case 256: return launch_gemm_tc<256, 4, EPI, FP8, R0, R1, R2>(ta, tb, td, args, st);
+    case 256:
+      if (pair) return launch_gemm_tc<256, 6, EPI, FP8, R0, R1, R2, 2>(ta, tb, td, args, st);
+      return launch_gemm_tc<256, 4, EPI, FP8, R0, R1, R2>(ta, tb, td, args, st);
     case 128: return launch_gemm_tc<128, 6, EPI, FP8, R0, R1, R2>(ta, tb, td, args, st);
     default:
       if constexpr (EPI == ts::EPI_SWIGLU)   // SwiGLU tiles are at least 128 wide
@@ -556,6 +585,17 @@ static ts_status dispatch_gemm_bn(int bn, const CUtensorMap& ta, const CUtensorM
       else
         return launch_gemm_tc<64, 8, EPI, FP8, R0, R1, R2>(ta, tb, td, args, st);
   }
+}
+
+// Two-SM pairs (256-row tiles) for GEMMs of at least this many rows with 256-wide
+// tiles; TS_GEMM_PAIR=0 in the environment turns them off (for comparisons).
+static constexpr int kGemmPairMinRows = 2048;
+static bool gemm_pairs_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("TS_GEMM_PAIR");
+    return !(e && e[0] == '0');
+  }();
+  return on;
 }
 
 // Output tile width for the persistent GEMM: the persistent CTAs walk the tiles
@@ -604,9 +644,11 @@ static ts_status run_gemm_tc(const char* name, const ts_model_desc* m, int epi, 
   if (K % (fp8 ? 128 : 64) || N % 64) return fail(TS_ERR_UNSUPPORTED, "GEMM sizes K=%d N=%d not tiled", K, N);
   int bn = pick_bn(M, NA);
   if (glu && bn < 128) bn = 128;    // NA = 2N is a multiple of 128
+  // 256-wide tiles of tall GEMMs run as two-SM pairs of 256 x 256 tiles
+  const bool pair = bn == 256 && M >= kGemmPairMinRows && gemm_pairs_enabled();
   CUtensorMap ta, tb, td;
   TS_TRY(make_tmap(&ta, A, M, K, fp8 ? 1 : 2, 128));
-  TS_TRY(make_tmap(&tb, W, NA, K, fp8 ? 1 : 2, glu ? bn / 2 : bn));
+  TS_TRY(make_tmap(&tb, W, NA, K, fp8 ? 1 : 2, (glu || pair) ? bn / 2 : bn));
   TS_TRY(make_tmap(&td, out, M, N, 2, 32));   // output (and residual): 32 x 64 chunks of the epilogue warps
   ts::GemmArgs g{};
   g.M = M;
@@ -628,8 +670,8 @@ static ts_status run_gemm_tc(const char* name, const ts_model_desc* m, int epi, 
   }
   const bool r3 = m->rope_dims[0] == 16;
 #define TS_GEMM_EPI(E, R0, R1, R2) \
-  (fp8 ? dispatch_gemm_bn<E, true, R0, R1, R2>(bn, ta, tb, td, g, st)     \
-       : dispatch_gemm_bn<E, false, R0, R1, R2>(bn, ta, tb, td, g, st))
+  (fp8 ? dispatch_gemm_bn<E, true, R0, R1, R2>(bn, pair, ta, tb, td, g, st)     \
+       : dispatch_gemm_bn<E, false, R0, R1, R2>(bn, pair, ta, tb, td, g, st))
   switch (epi) {
     case ts::EPI_BIAS: return TS_GEMM_EPI(ts::EPI_BIAS, 0, 32, 32);
     case ts::EPI_GELU: return TS_GEMM_EPI(ts::EPI_GELU, 0, 32, 32);
