@@ -313,6 +313,39 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// packed pairs of floats (low = first) and the sm_100 f32x2 arithmetic on them
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float lo_f32(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return lo;
+}
+__device__ __forceinline__ float hi_f32(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return hi;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t splat_f32x2(float v) { return pack_f32x2(v, v); }
+
 // Exact-erf GELU, 0.5 x (1 + erf(x / sqrt 2)).  erf by Abramowitz & Stegun,
 // Handbook of Mathematical Functions, formula 7.1.26 (|error| <= 1.5e-7 for
 // z >= 0, odd extension), evaluated with the approximate reciprocal and base-2
@@ -328,6 +361,24 @@ __device__ __forceinline__ float gelu_erf(float x) {
   const float e = ex2_approx(-1.4426950408889634f * z * z);
   const float erf_z = fmaf(-p * t, e, 1.0f);
   return 0.5f * x * (1.0f + copysignf(erf_z, x));
+}
+// gelu_erf of a pair of values (low = first) in packed f32x2 arithmetic: the same
+// formula and the same two SFU operations per value, half the FMA-pipe
+// instructions.  The bf16 GEMM epilogue, bound by its issue slots, uses it.
+__device__ __forceinline__ uint64_t gelu_erf2(uint64_t x2) {
+  const float x0 = lo_f32(x2), x1 = hi_f32(x2);
+  const uint64_t z = mul_f32x2(pack_f32x2(fabsf(x0), fabsf(x1)), splat_f32x2(0.70710678118654752f));
+  const uint64_t den = fma_f32x2(splat_f32x2(0.3275911f), z, splat_f32x2(1.0f));
+  const uint64_t t = pack_f32x2(__fdividef(1.0f, lo_f32(den)), __fdividef(1.0f, hi_f32(den)));
+  uint64_t p = fma_f32x2(splat_f32x2(1.061405429f), t, splat_f32x2(-1.453152027f));
+  p = fma_f32x2(p, t, splat_f32x2(1.421413741f));
+  p = fma_f32x2(p, t, splat_f32x2(-0.284496736f));
+  p = fma_f32x2(p, t, splat_f32x2(0.254829592f));
+  const uint64_t ea = mul_f32x2(mul_f32x2(z, z), splat_f32x2(-1.4426950408889634f));
+  const uint64_t e = pack_f32x2(ex2_approx(lo_f32(ea)), ex2_approx(hi_f32(ea)));
+  const uint64_t erf = fma_f32x2(mul_f32x2(p, t), pack_f32x2(-lo_f32(e), -hi_f32(e)), splat_f32x2(1.0f));
+  const uint64_t s = pack_f32x2(copysignf(lo_f32(erf), x0), copysignf(hi_f32(erf), x1));
+  return mul_f32x2(mul_f32x2(x2, splat_f32x2(0.5f)), add_f32x2(s, splat_f32x2(1.0f)));
 }
 // The same GELU with erf by Abramowitz & Stegun formula 7.1.28: for z >= 0,
 // erf z = 1 - (1 + a1 z + a2 z^2 + ... + a6 z^6)^-16 with |error| <= 3e-7 (odd

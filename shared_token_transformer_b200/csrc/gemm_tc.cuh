@@ -145,8 +145,17 @@ __device__ __forceinline__ void gemm_epilogue64(float* v, int col, float rs, con
     }
   }
   if (EPI == EPI_GELU) {
+    if (FP8) {
 #pragma unroll
-    for (int i = 0; i < 64; ++i) v[i] = FP8 ? gelu_erf_one_sfu(v[i]) : gelu_erf(v[i]);
+      for (int i = 0; i < 64; ++i) v[i] = gelu_erf_one_sfu(v[i]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 64; i += 2) {
+        const uint64_t y = gelu_erf2(pack_f32x2(v[i], v[i + 1]));
+        v[i] = lo_f32(y);
+        v[i + 1] = hi_f32(y);
+      }
+    }
   } else if (EPI == EPI_QKV) {
     if (col < 2 * args.d)
       qk_norm_rope64<R0, R1, R2>(v, col < args.d ? args.q_g : args.k_g, args.eps_qk, pos, args);

@@ -101,6 +101,25 @@ def test_gelu_epilogue_matches_exact_erf():
     assert np.max(np.abs(got - want) / np.maximum(1.0, np.abs(want))) < 2e-6
 
 
+def test_gelu_epilogue_bf16_matches_exact_erf():
+    """The bf16 GEMMs' GELU epilogue (Abramowitz & Stegun 7.1.26 on pairs of values
+    in packed f32x2 arithmetic): bf16 inputs through an identity weight are exact
+    in the fp32 accumulator, so every bf16 output must be exact-erf GELU of its
+    input within one bf16 rounding (2^-8 relative to max(1, |GELU|)), over
+    [-10, 10] with zero, both signs and the tails, at a size that takes the
+    two-SM pair path (2304 rows, 256-wide tiles)."""
+    import math
+    M = K = N = 256
+    x = W.round_to(np.linspace(-10.0, 10.0, 2304 * K).reshape(2304, K), "bf16")
+    x[0, 0] = 0.0
+    m = B.model_desc(256, 4, 256, "bf16", (0, 32, 32))
+    y = torch.empty((2304, N), dtype=torch.bfloat16, device="cuda")
+    B.op_linear(m, dev(x, torch.bfloat16), dev(np.eye(N, K), torch.bfloat16), dev(np.zeros(N), torch.float32), y,
+                epi=B.TS_EPI_BIAS_GELU)
+    want = np.vectorize(lambda v: 0.5 * v * (1.0 + math.erf(v / math.sqrt(2.0))))(x)
+    assert np.max(np.abs(host(y) - want) / np.maximum(1.0, np.abs(want))) <= 2.0 ** -8
+
+
 def test_gelu_epilogue_e4m3_matches_exact_erf():
     """The e4m3 GEMMs' GELU epilogue evaluates erf by Abramowitz & Stegun 7.1.28
     (one approximate reciprocal raised to the 16th power).  Inputs on the e4m3
