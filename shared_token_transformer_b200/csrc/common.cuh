@@ -383,24 +383,27 @@ __device__ __forceinline__ uint64_t gelu_erf2(uint64_t x2) {
 // The same GELU with erf by Abramowitz & Stegun formula 7.1.28: for z >= 0,
 // erf z = 1 - (1 + a1 z + a2 z^2 + ... + a6 z^6)^-16 with |error| <= 3e-7 (odd
 // extension).  One approximate reciprocal and four squarings: a single SFU
-// operation per value where 7.1.26 needs two, at a few more FMA-pipe operations.
-// Evaluated in fp32 it stays within 6e-7 of exact-erf GELU relative to
-// max(1, |GELU|).  The e4m3 GEMMs use it: their MMAs run at twice the bf16 rate,
-// so their GELU epilogue is bound by the SFU.
-__device__ __forceinline__ float gelu_erf_one_sfu(float x) {
-  const float z = fabsf(x) * 0.70710678118654752f;
-  float p = fmaf(0.0000430638f, z, 0.0002765672f);
-  p = fmaf(p, z, 0.0001520143f);
-  p = fmaf(p, z, 0.0092705272f);
-  p = fmaf(p, z, 0.0422820123f);
-  p = fmaf(p, z, 0.0705230784f);
-  p = fmaf(p, z, 1.0f);
-  float r = __fdividef(1.0f, p);
-  r *= r;
-  r *= r;
-  r *= r;
-  r *= r;
-  return 0.5f * x * (1.0f + copysignf(1.0f - r, x));
+// operation per value where 7.1.26 needs two.  Evaluated in fp32 it stays within
+// 6e-7 of exact-erf GELU relative to max(1, |GELU|).  On a pair of values (low =
+// first) in packed f32x2 arithmetic; the e4m3 GEMMs use it, since at twice the
+// bf16 MMA rate their GELU epilogue is bound by the SFU and the issue slots.
+__device__ __forceinline__ uint64_t gelu_erf_one_sfu2(uint64_t x2) {
+  const float x0 = lo_f32(x2), x1 = hi_f32(x2);
+  const uint64_t z = mul_f32x2(pack_f32x2(fabsf(x0), fabsf(x1)), splat_f32x2(0.70710678118654752f));
+  uint64_t p = fma_f32x2(splat_f32x2(0.0000430638f), z, splat_f32x2(0.0002765672f));
+  p = fma_f32x2(p, z, splat_f32x2(0.0001520143f));
+  p = fma_f32x2(p, z, splat_f32x2(0.0092705272f));
+  p = fma_f32x2(p, z, splat_f32x2(0.0422820123f));
+  p = fma_f32x2(p, z, splat_f32x2(0.0705230784f));
+  p = fma_f32x2(p, z, splat_f32x2(1.0f));
+  uint64_t r = pack_f32x2(__fdividef(1.0f, lo_f32(p)), __fdividef(1.0f, hi_f32(p)));
+  r = mul_f32x2(r, r);
+  r = mul_f32x2(r, r);
+  r = mul_f32x2(r, r);
+  r = mul_f32x2(r, r);
+  const uint64_t erf = add_f32x2(splat_f32x2(1.0f), pack_f32x2(-lo_f32(r), -hi_f32(r)));
+  const uint64_t s = pack_f32x2(copysignf(lo_f32(erf), x0), copysignf(hi_f32(erf), x1));
+  return mul_f32x2(mul_f32x2(x2, splat_f32x2(0.5f)), add_f32x2(s, splat_f32x2(1.0f)));
 }
 
 __device__ __forceinline__ float warp_sum(float v) {

@@ -147,7 +147,11 @@ __device__ __forceinline__ void gemm_epilogue64(float* v, int col, float rs, con
   if (EPI == EPI_GELU) {
     if (FP8) {
 #pragma unroll
-      for (int i = 0; i < 64; ++i) v[i] = gelu_erf_one_sfu(v[i]);
+      for (int i = 0; i < 64; i += 2) {
+        const uint64_t y = gelu_erf_one_sfu2(pack_f32x2(v[i], v[i + 1]));
+        v[i] = lo_f32(y);
+        v[i + 1] = hi_f32(y);
+      }
     } else {
 #pragma unroll
       for (int i = 0; i < 64; i += 2) {
