@@ -402,32 +402,52 @@ __global__ void __launch_bounds__(256) scatter_add_rows_kernel(const T* __restri
 // Per-row e4m3 quantisation of a bf16 matrix: scale = absmax / 448 (1 if zero),
 // q = e4m3(x / scale), nearest-even, saturating.  cols % 8 == 0.
 // ---------------------------------------------------------------------------
+// Each lane walks its 16-byte vectors eight at a time (eight loads in flight, so
+// the pass is not bound by one load's latency); the second pass reads the row again
+// (from L1 / L2) to quantise it.
 __global__ void __launch_bounds__(256) quantize_rows_kernel(const bf16* __restrict__ x, int rows, int cols,
                                                             uint8_t* __restrict__ q, float* __restrict__ scale) {
   pdl_wait();
   pdl_trigger();
+  constexpr int U = 8;   // vectors in flight per lane
   const int lane = threadIdx.x & 31;
   const size_t row = static_cast<size_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= static_cast<size_t>(rows)) return;
   const bf16* xr = x + row * cols;
   float amax = 0.f;
-  for (int c = lane * 8; c < cols; c += 256) {
-    float f[8];
-    bf16x8_to_f32(*reinterpret_cast<const uint4*>(xr + c), f);
+  for (int c0 = lane * 8; c0 < cols; c0 += 256 * U) {
+    uint4 v[U];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+    for (int u = 0; u < U; ++u)
+      if (c0 + u * 256 < cols) v[u] = *reinterpret_cast<const uint4*>(xr + c0 + u * 256);
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (c0 + u * 256 < cols) {
+        float f[8];
+        bf16x8_to_f32(v[u], f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+      }
   }
   amax = warp_max(amax);
   const float s = amax > 0.f ? amax / 448.0f : 1.0f;
   const float inv = 1.0f / s;   // one division per row; x / s becomes x * (1 / s) (within an fp32 ulp)
   if (lane == 0) scale[row] = s;
-  for (int c = lane * 8; c < cols; c += 256) {
-    float f[8];
-    bf16x8_to_f32(*reinterpret_cast<const uint4*>(xr + c), f);
-    uint16_t pk[4];
+  for (int c0 = lane * 8; c0 < cols; c0 += 256 * U) {
+    uint4 v[U];
 #pragma unroll
-    for (int e = 0; e < 8; e += 2) pk[e / 2] = f32x2_to_e4m3x2(f[e] * inv, f[e + 1] * inv);
-    *reinterpret_cast<uint2*>(q + row * cols + c) = *reinterpret_cast<const uint2*>(pk);
+    for (int u = 0; u < U; ++u)
+      if (c0 + u * 256 < cols) v[u] = *reinterpret_cast<const uint4*>(xr + c0 + u * 256);
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (c0 + u * 256 < cols) {
+        float f[8];
+        bf16x8_to_f32(v[u], f);
+        uint16_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) pk[e / 2] = f32x2_to_e4m3x2(f[e] * inv, f[e + 1] * inv);
+        *reinterpret_cast<uint2*>(q + row * cols + c0 + u * 256) = *reinterpret_cast<const uint2*>(pk);
+      }
   }
 }
 
