@@ -8,36 +8,40 @@
 // (RoPE runs once per row in the QKV epilogue), so this is a plain gathered
 // attention.
 //
-// bf16 kernel (hd = 64), 256 threads, 2 CTAs per SM.  Shared layer: grid
-// (nqb, T, heads), the head slowest, so that CTAs in flight together work on one
-// head of neighbouring tiles, whose overlapping q/k/v rows (one head's slice of
-// the whole shared state: a few MB) then come from L2 instead of DRAM.  Per-tile
-// layer (no rows shared between tiles): grid (nqb, heads, T), the tile slowest, so
-// that the heads of one tile run together and each tile's q/k/v rows (all heads'
-// column slices of the same rows) leave DRAM once.
-//   blocks qb < nqb: 128 window queries, keys in blocks of 64.
-//     warp 4     TMA producer of Q (once) and of K/V blocks into 128-byte-
+// bf16 kernel (hd = 64), 320 threads, 2 CTAs per SM, each CTA two query tiles of
+// 128 rows that share one K/V stream: eight softmax warps per CTA, so that four
+// softmax warps share each scheduler and one tile's softmax runs while the other
+// tile's MMAs do.  Shared layer: grid (nqb + 1, T, heads), the head slowest, so that
+// CTAs in flight together work on one head of neighbouring tiles, whose overlapping
+// q/k/v rows (one head's slice of the whole shared state: a few MB) then come from
+// L2 instead of DRAM.  Per-tile layer (no rows shared between tiles): grid
+// (nqb + 1, heads, T), the tile slowest, so that the heads of one tile run together
+// and each tile's q/k/v rows (all heads' column slices of the same rows) leave DRAM
+// once.
+//   blocks qb < nqb: 256 window queries (two tiles), keys in blocks of 64.
+//     warp 8     TMA producer of Q (once) and of K/V blocks into 128-byte-
 //                swizzled shared rows: one box of a 3-D map over the grid per
 //                block when a block is whole window rows of one frame, else one
 //                2-D box per run of consecutive rows, else tile::gather4 loads
 //                through the row map (four rows per instruction); four K/V
 //                buffers, completion by transaction bytes on one mbarrier each;
-//     warp 5     MMA issuer (one lane): S = Q K^T (tcgen05 kind::f16, M = 128,
-//                N = 64) into one of three TMEM S buffers, then O += P V with P
-//                read from TMEM (A operand) and V from shared memory as an
-//                MN-major operand; S of block j+3 reuses the columns of P of
-//                block j and is issued after P V of block j (tcgen05.mma runs
-//                in issue order);
-//     warps 0-3  softmax, one query row per thread (TMEM lane = row): one tcgen05
-//                round trip brings the row's 64 scores into registers; online
-//                softmax in the exp2 domain with a lazily moved reference maximum
-//                (O rescaled in TMEM only when a score exceeds it by 2^8); P goes
-//                back over the scores as packed bf16; the global key (slot 0)
-//                seeds the running max and sum and is added back at the end with
-//                its running coefficient;
-//     warps 6-7  in query block 0 only: the global token's own query row (slot 0),
-//                an online softmax over the K/V blocks in shared memory (each
-//                warp every other block), merged at the end.
+//     warp 9     MMA issuer (one lane): per tile S = Q K^T (tcgen05 kind::f16,
+//                M = 128, N = 64) into the tile's TMEM S buffer, then O += P V
+//                with P read from TMEM (A operand) and V from shared memory as an
+//                MN-major operand; S of block j+1 overwrites P of block j and is
+//                issued after its P V (tcgen05.mma runs in issue order); the two
+//                tiles alternate;
+//     warps 0-7  softmax, one query row per thread (warps 0-3 tile 0, 4-7 tile 1;
+//                TMEM lane = row): one tcgen05 round trip brings the row's 64
+//                scores into registers; online softmax in the exp2 domain with a
+//                lazily moved reference maximum (O rescaled in TMEM only when a
+//                score exceeds it by 2^8); P goes back over the scores as packed
+//                bf16; the global key (slot 0) seeds the running max and sum and
+//                is added back at the end with its running coefficient.
+//   block qb = nqb: the global token's own query row (slot 0) of the tile and
+//                head: warp 8 streams the K/V blocks as for a window block, eight
+//                warps score them from shared memory (lane = key) with an online
+//                softmax each, merged at the end.
 // fp32 kernel (any hd <= 64, multiple of 4): one thread per query row, keys in
 //   shared memory, online softmax; for the fp32 reference-precision path.
 #pragma once
@@ -56,7 +60,8 @@ struct AttnArgs {
   int gw;             // load 2: grid width; shared row u is grid row u / gw, column u % gw
   float scale_log2;   // log2(e) / sqrt(hd)
   float scale;        // 1 / sqrt(hd)
-  int head_major;     // bf16 grid: 1 (nqb, T, heads), head slowest; 0 (nqb, heads, T), tile slowest
+  int head_major;     // bf16 grid: 1 (nqb + 1, T, heads), head slowest; 0 (nqb + 1, heads, T), tile slowest
+  int nqb;            // bf16: window query blocks (256 queries) per tile; block x = nqb is the global row
 };
 
 __device__ __forceinline__ int attn_row(const AttnArgs& a, int t, int s) {
@@ -66,11 +71,14 @@ __device__ __forceinline__ int attn_row(const AttnArgs& a, int t, int s) {
 // byte offset of 16-byte chunk `ch` of row `r` in a 128-byte-swizzled tile
 __device__ __forceinline__ uint32_t swz(int r, int ch) { return r * 128 + ((ch ^ (r & 7)) << 4); }
 
-constexpr int kAttnThreads = 256;        // 4 softmax, TMA producer, MMA issuer, 2 global-row warps
-constexpr int kAttnBQ = 128;             // queries per CTA
+constexpr int kAttnThreads = 320;        // 8 softmax warps (two query tiles), TMA producer, MMA issuer
+constexpr int kAttnCtasPerSm = 2;
+constexpr int kAttnTileQ = 128;          // queries per tile (M of the MMAs)
+constexpr int kAttnBQ = 2 * kAttnTileQ;  // queries per CTA
 constexpr int kAttnBK = 64;              // keys per block
 constexpr int kAttnKV = 4;               // K/V buffers
-constexpr int kAttnS = 3;                // S / P buffers in TMEM
+constexpr int kAttnTmemCols = 256;       // per tile: S / P (64 columns), then O (64 columns)
+constexpr int kAttnTmemTile = 128;       // TMEM columns of one query tile
 constexpr float kAttnRescale = 8.0f;     // lazy rescale threshold (log2 units)
 #ifndef TS_ATTN_EMU_EVERY
 #define TS_ATTN_EMU_EVERY 4
@@ -78,15 +86,18 @@ constexpr float kAttnRescale = 8.0f;     // lazy rescale threshold (log2 units)
 constexpr int kAttnEmuEvery = TS_ATTN_EMU_EVERY;   // one score pair in this many: 2^x on the FMA pipe
 
 struct AttnSmem {
-  static constexpr int Q = 0;                 // 16 KB: 128 rows x 128 B
-  static constexpr int K = 16384;                       // kAttnKV x 8 KB: 64 rows x 128 B
-  static constexpr int V = K + kAttnKV * 8192;          // kAttnKV x 8 KB
-  static constexpr int KG = V + kAttnKV * 8192;         // 64 floats k_g, 64 floats v_g
-  static constexpr int GR = KG + 512;         // 2 x 66 floats: partial states of the global query row
-  static constexpr int BAR = GR + 1024;       // barriers
-  static constexpr int NBAR = 2 * kAttnKV + 2 * kAttnS + 3;
+  static constexpr int KV_BYTES = kAttnBK * 128;       // one K or V block: 64 rows x 128 B
+  static constexpr int Q = 0;                          // 32 KB: 2 tiles x 128 rows x 128 B
+  static constexpr int K = kAttnBQ * 128;              // kAttnKV x 8 KB
+  static constexpr int V = K + kAttnKV * KV_BYTES;     // kAttnKV x 8 KB
+  static constexpr int KG = V + kAttnKV * KV_BYTES;    // 64 floats k_g, 64 floats v_g
+  static constexpr int BAR = KG + 512;                 // barriers
+  static constexpr int NBAR = 2 * kAttnKV + 2 + 2 + 2 + 1; // kvfull, kvempty, sfull[2], pfull[2], ofinal[2], qfull1
   static constexpr int BYTES = BAR + NBAR * 8 + 8;
-  static constexpr int LAUNCH_BYTES = BYTES;  // base must be 1024-aligned (checked): two CTAs per SM
+  static_assert((8 * 66 + 8 + 64) * 4 <= kAttnBQ * 128, "global-row states and query in the Q region");
+  // the base is rounded up to 1024 bytes inside the kernel (swizzled tiles)
+  static constexpr int LAUNCH_BYTES = BYTES + 1024;
+  static_assert(kAttnCtasPerSm * (LAUNCH_BYTES + 1024) <= 228 * 1024, "shared memory for 2 CTAs per SM");
 };
 
 // Shared-memory descriptor of an MN-major operand with the 128-byte swizzle: rows
@@ -102,15 +113,12 @@ __device__ __forceinline__ uint64_t sdesc_sw128_mn(uint32_t saddr) {
   return d;
 }
 
-__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* v) {
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* v) {
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
       "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
-      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
-      "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
-      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
 }
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
@@ -196,18 +204,25 @@ __device__ __forceinline__ void tc_mma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tm
 // What the three load variants of the producer warp share.
 struct AttnLoad {
   const CUtensorMap* tm;
-  uint32_t sb, bar_kvfull, bar_kvempty;
+  uint32_t sb, bar_kvfull, bar_kvempty, bar_q1;   // bar_q1 = 0: K/V only (global-row block), no Q
   int q0, nkb, t, h, lane;
 };
+
+// Tile 0's Q (128 rows) travels with K/V block 0 on its barrier, tile 1's Q on a
+// barrier of its own.
+constexpr uint32_t kAttnTxFirst = kAttnTileQ * 128 + 2 * AttnSmem::KV_BYTES;
+constexpr uint32_t kAttnTxQ1 = kAttnTileQ * 128;
+constexpr uint32_t kAttnTxBlock = 2 * AttnSmem::KV_BYTES;
 
 __device__ __forceinline__ void attn_load_grid(const AttnArgs& a, const AttnLoad& c) {
   const CUtensorMap* tm = c.tm;
   const uint32_t sb = c.sb, bar_kvfull = c.bar_kvfull, bar_kvempty = c.bar_kvempty;
   const int q0 = c.q0, nkb = c.nkb, t = c.t, h = c.h, lane = c.lane;
   // ---------------- TMA producer, one grid box per 64 slots ----------------
-  // A block of 64 window slots is 64 / bx whole window rows of one frame: one
-  // box of the 3-D map (channels, grid column, grid row) starting at the row
-  // of its first slot.  Blocks past the tile's last slot load block 0 again.
+  // A block of 64 window slots is 64 / bx whole window rows of one frame (or a
+  // part of one row): one box of the 3-D map (channels, grid column, grid row)
+  // starting at the grid position of its first slot.  Blocks past the tile's
+  // last slot load block 0 again.
   auto box_at = [&](int slot, int& x, int& y) {
     const int u = attn_row(a, t, slot < a.N ? slot : 1);
     x = u % a.gw;
@@ -216,11 +231,18 @@ __device__ __forceinline__ void attn_load_grid(const AttnArgs& a, const AttnLoad
   if (lane == 0) {
     const int xq = h * 64, xk = a.d + h * 64, xv = 2 * a.d + h * 64;
     int x, y;
-    mbar_expect_tx(bar_kvfull, 2 * 16384);   // Q rows travel with K/V block 0
-    box_at(q0, x, y);
-    tma_load_3d(sb + AttnSmem::Q, tm, bar_kvfull, xq, x, y);
-    box_at(q0 + 64, x, y);
-    tma_load_3d(sb + AttnSmem::Q + 8192, tm, bar_kvfull, xq, x, y);
+    if (c.bar_q1) {
+      mbar_expect_tx(bar_kvfull, kAttnTxFirst);
+      mbar_expect_tx(c.bar_q1, kAttnTxQ1);
+#pragma unroll
+      for (int i = 0; i < kAttnBQ / kAttnBK; ++i) {
+        box_at(q0 + i * kAttnBK, x, y);
+        tma_load_3d(sb + AttnSmem::Q + i * AttnSmem::KV_BYTES, tm, i < kAttnTileQ / kAttnBK ? bar_kvfull : c.bar_q1,
+                    xq, x, y);
+      }
+    } else {
+      mbar_expect_tx(bar_kvfull, kAttnTxBlock);
+    }
     int xn, yn;
     box_at(1, xn, yn);
     int armed = 0;
@@ -230,14 +252,15 @@ __device__ __forceinline__ void attn_load_grid(const AttnArgs& a, const AttnLoad
       if (j + 1 < nkb) box_at(1 + (j + 1) * kAttnBK, xn, yn);
       if (j > 0) {
         if (j >= kAttnKV && !mbar_wait(bar_kvempty + 8 * b, ((j / kAttnKV) - 1) & 1)) break;
-        mbar_expect_tx(bar_kvfull + 8 * b, 16384);
+        mbar_expect_tx(bar_kvfull + 8 * b, kAttnTxBlock);
       }
-      tma_load_3d(sb + AttnSmem::K + b * 8192, tm, bar_kvfull + 8 * b, xk, xc, yc);
-      tma_load_3d(sb + AttnSmem::V + b * 8192, tm, bar_kvfull + 8 * b, xv, xc, yc);
+      tma_load_3d(sb + AttnSmem::K + b * AttnSmem::KV_BYTES, tm, bar_kvfull + 8 * b, xk, xc, yc);
+      tma_load_3d(sb + AttnSmem::V + b * AttnSmem::KV_BYTES, tm, bar_kvfull + 8 * b, xv, xc, yc);
       armed = j + 1;
     }
     // no copy may still be landing when the CTA exits (matters only after a timeout)
     for (int j = max(0, armed - kAttnKV); j < armed; ++j) mbar_wait(bar_kvfull + 8 * (j % kAttnKV), (j / kAttnKV) & 1);
+    if (c.bar_q1) mbar_wait(c.bar_q1, 0);
   }
 }
 
@@ -246,21 +269,26 @@ __device__ __forceinline__ void attn_load_runs(const AttnArgs& a, const AttnLoad
   const uint32_t sb = c.sb, bar_kvfull = c.bar_kvfull, bar_kvempty = c.bar_kvempty;
   const int q0 = c.q0, nkb = c.nkb, t = c.t, h = c.h, lane = c.lane;
   // ---------------- TMA producer, runs of consecutive rows ----------------
-  // Each run of `run` slots is one tiled box (128 bytes x run rows) of the q/k/v
-  // columns of head h.  Runs past the tile's last slot (padding of the last key
-  // or query block) load the first run again: their scores are masked and their
-  // outputs are not stored.  Lane i looks up the row of run i one block ahead;
-  // lane 0 issues the copies.
+  // Each run of `run` slots (8, 16, 32 or 64) is one tiled box (128 bytes x run rows)
+  // of the q/k/v columns of head h.  Runs past the tile's last slot (padding of
+  // the last key or query block) load the first run again: their scores are
+  // masked and their outputs are not stored.  Lane i looks up the row of run i one
+  // block ahead; lane 0 issues the copies.
   const int L = a.run, nrun = kAttnBK / L;
   auto run_row = [&](int slot) { return attn_row(a, t, slot < a.N ? slot : 1); };
   const int xq = h * 64, xk = a.d + h * 64, xv = 2 * a.d + h * 64;
-  {
+  if (c.bar_q1) {
     const int rq = lane < kAttnBQ / L ? run_row(q0 + lane * L) : 0;
-    if (lane == 0) mbar_expect_tx(bar_kvfull, 2 * 16384);   // Q rows travel with K/V block 0
+    if (lane == 0) {
+      mbar_expect_tx(bar_kvfull, kAttnTxFirst);
+      mbar_expect_tx(c.bar_q1, kAttnTxQ1);
+    }
     for (int i = 0; i < kAttnBQ / L; ++i) {
       const int r = __shfl_sync(0xffffffffu, rq, i);
-      if (lane == 0) tma_load_2d(sb + AttnSmem::Q + i * L * 128, tm, bar_kvfull, xq, r);
+      if (lane == 0) tma_load_2d(sb + AttnSmem::Q + i * L * 128, tm, i < kAttnTileQ / L ? bar_kvfull : c.bar_q1, xq, r);
     }
+  } else if (lane == 0) {
+    mbar_expect_tx(bar_kvfull, kAttnTxBlock);
   }
   int rnext = lane < nrun ? run_row(1 + lane * L) : 0;
   int armed = 0;
@@ -272,20 +300,22 @@ __device__ __forceinline__ void attn_load_runs(const AttnArgs& a, const AttnLoad
       int ok = 1;
       if (lane == 0 && j >= kAttnKV) ok = mbar_wait(bar_kvempty + 8 * b, ((j / kAttnKV) - 1) & 1);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      if (lane == 0) mbar_expect_tx(bar_kvfull + 8 * b, 16384);
+      if (lane == 0) mbar_expect_tx(bar_kvfull + 8 * b, kAttnTxBlock);
     }
     for (int i = 0; i < nrun; ++i) {
       const int r = __shfl_sync(0xffffffffu, rcur, i);
       if (lane == 0) {
-        tma_load_2d(sb + AttnSmem::K + b * 8192 + i * L * 128, tm, bar_kvfull + 8 * b, xk, r);
-        tma_load_2d(sb + AttnSmem::V + b * 8192 + i * L * 128, tm, bar_kvfull + 8 * b, xv, r);
+        tma_load_2d(sb + AttnSmem::K + b * AttnSmem::KV_BYTES + i * L * 128, tm, bar_kvfull + 8 * b, xk, r);
+        tma_load_2d(sb + AttnSmem::V + b * AttnSmem::KV_BYTES + i * L * 128, tm, bar_kvfull + 8 * b, xv, r);
       }
     }
     armed = j + 1;
   }
   // no copy may still be landing when the CTA exits (matters only after a timeout)
-  if (lane == 0)
+  if (lane == 0) {
     for (int j = max(0, armed - kAttnKV); j < armed; ++j) mbar_wait(bar_kvfull + 8 * (j % kAttnKV), (j / kAttnKV) & 1);
+    if (c.bar_q1) mbar_wait(c.bar_q1, 0);
+  }
 }
 
 __device__ __forceinline__ void attn_load_gather(const AttnArgs& a, const AttnLoad& c) {
@@ -296,47 +326,59 @@ __device__ __forceinline__ void attn_load_gather(const AttnArgs& a, const AttnLo
   // Rows are gathered four at a time (tile::gather4) from the q/k/v columns of
   // head h.  Slots past the tile's last one (padding of the last key or query
   // block) repeat the last slot's row, so every coordinate is in range; their
-  // scores are masked and their outputs are not stored.
+  // scores are masked and their outputs are not stored.  Lane i holds the rows of
+  // slots i and 32 + i of the block.
   auto row_of = [&](int slot) { return attn_row(a, t, min(slot, a.N - 1)); };
   const int xq = h * 64, xk = a.d + h * 64, xv = 2 * a.d + h * 64;
-  int vq[4];
+  int vq[kAttnBQ / 32];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) vq[k] = row_of(q0 + 32 * k + lane);
-  int v0 = row_of(1 + lane), v1 = row_of(33 + lane);
-  if (lane == 0) mbar_expect_tx(bar_kvfull, 2 * 16384);   // Q rows travel with K/V block 0
+  for (int k = 0; k < kAttnBQ / 32; ++k) vq[k] = row_of(q0 + 32 * k + lane);
+  if (c.bar_q1) {
+    if (lane == 0) {
+      mbar_expect_tx(bar_kvfull, kAttnTxFirst);
+      mbar_expect_tx(c.bar_q1, kAttnTxQ1);
+    }
 #pragma unroll
-  for (int g = 0; g < 32; ++g) {
-    int r[4];
+    for (int g = 0; g < kAttnBQ / 4; ++g) {
+      int r[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) r[i] = __shfl_sync(0xffffffffu, vq[g >> 3], (4 * g + i) & 31);
-    if (lane == 0) tma_gather4(sb + AttnSmem::Q + g * 512, tm, bar_kvfull, xq, r[0], r[1], r[2], r[3]);
+      for (int i = 0; i < 4; ++i) r[i] = __shfl_sync(0xffffffffu, vq[g >> 3], (4 * g + i) & 31);
+      if (lane == 0)
+        tma_gather4(sb + AttnSmem::Q + g * 512, tm, g < kAttnTileQ / 4 ? bar_kvfull : c.bar_q1, xq, r[0], r[1], r[2],
+                    r[3]);
+    }
+  } else if (lane == 0) {
+    mbar_expect_tx(bar_kvfull, kAttnTxBlock);
   }
   int armed = 0;
   for (int j = 0; j < nkb; ++j) {
     const int b = j % kAttnKV;
+    const int v0 = row_of(1 + j * kAttnBK + lane), v1 = row_of(1 + j * kAttnBK + 32 + lane);
     if (j > 0) {
-      v0 = row_of(1 + j * kAttnBK + lane);
-      v1 = row_of(1 + j * kAttnBK + 32 + lane);
       int ok = 1;
       if (lane == 0 && j >= kAttnKV) ok = mbar_wait(bar_kvempty + 8 * b, ((j / kAttnKV) - 1) & 1);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      if (lane == 0) mbar_expect_tx(bar_kvfull + 8 * b, 16384);
+      if (lane == 0) mbar_expect_tx(bar_kvfull + 8 * b, kAttnTxBlock);
     }
 #pragma unroll
-    for (int g = 0; g < 16; ++g) {
+    for (int g = 0; g < kAttnBK / 4; ++g) {
       int r[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) r[i] = __shfl_sync(0xffffffffu, g < 8 ? v0 : v1, (4 * g + i) & 31);
       if (lane == 0) {
-        tma_gather4(sb + AttnSmem::K + b * 8192 + g * 512, tm, bar_kvfull + 8 * b, xk, r[0], r[1], r[2], r[3]);
-        tma_gather4(sb + AttnSmem::V + b * 8192 + g * 512, tm, bar_kvfull + 8 * b, xv, r[0], r[1], r[2], r[3]);
+        tma_gather4(sb + AttnSmem::K + b * AttnSmem::KV_BYTES + g * 512, tm, bar_kvfull + 8 * b, xk, r[0], r[1], r[2],
+                    r[3]);
+        tma_gather4(sb + AttnSmem::V + b * AttnSmem::KV_BYTES + g * 512, tm, bar_kvfull + 8 * b, xv, r[0], r[1], r[2],
+                    r[3]);
       }
     }
     armed = j + 1;
   }
   // no copy may still be landing when the CTA exits (matters only after a timeout)
-  if (lane == 0)
+  if (lane == 0) {
     for (int j = max(0, armed - kAttnKV); j < armed; ++j) mbar_wait(bar_kvfull + 8 * (j % kAttnKV), (j / kAttnKV) & 1);
+    if (c.bar_q1) mbar_wait(c.bar_q1, 0);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -349,36 +391,33 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sb = smem_u32(smem);
   const uint32_t bar_kvfull = sb + AttnSmem::BAR;        // kAttnKV, count 1 (producer's expect_tx) + TMA bytes
-  const uint32_t bar_kvempty = bar_kvfull + 8 * kAttnKV; // kAttnKV, count 1 (commit after P V) [+1 global-row warp]
-  const uint32_t bar_sfull = bar_kvempty + 8 * kAttnKV;  // kAttnS, count 1 (commit after Q K^T)
-  const uint32_t bar_pfull = bar_sfull + 8 * kAttnS;     // kAttnS, count 4 (softmax warps wrote P into TMEM)
-  const uint32_t bar_odone = bar_pfull + 8 * kAttnS;     // 2, count 1 (commit after P V)
-  const uint32_t bar_ofinal = bar_odone + 16;            // 1, count 1 (commit after the last P V)
+  const uint32_t bar_kvempty = bar_kvfull + 8 * kAttnKV; // kAttnKV, count 1 (commit after tile 1's P V)
+  const uint32_t bar_sfull = bar_kvempty + 8 * kAttnKV;  // 2 (one per tile), count 1 (commit after Q K^T)
+  const uint32_t bar_pfull = bar_sfull + 16;             // 2 (one per tile), count 4 (the tile's softmax warps)
+  const uint32_t bar_ofinal = bar_pfull + 16;            // 2 (one per tile), count 1 (commit after its last P V)
+  const uint32_t bar_q1 = bar_ofinal + 16;               // 1, count 1 (producer's expect_tx) + TMA bytes of tile 1's Q
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + AttnSmem::BAR + AttnSmem::NBAR * 8);
   float* sKg = reinterpret_cast<float*>(smem + AttnSmem::KG);
   float* sVg = sKg + 64;
   const int nkb = (a.Nw + kAttnBK - 1) / kAttnBK;
-  const int q0 = 1 + qb * kAttnBQ;  // first slot of this query block
-  // The CTA of query block 0 also computes the global token's own query row
-  // (slot 0) in warps 6 and 7, which then co-own the K/V buffers they read.
-  const bool grow_row = qb == 0;
+  const int q0 = 1 + qb * kAttnBQ;  // first slot of this query block (tile 0; tile 1 follows)
 
   uint32_t tmem = 0;
-  if (warp == 4) {
+  if (warp == 8) {
     // ---------------- TMA producer ----------------
     // Its copies start as soon as the barriers exist; the other warps learn of
     // the initialisation through a named barrier that this warp only arrives at.
-    if (warp == 4 && lane == 0) {
+    if (lane == 0) {
       for (int i = 0; i < kAttnKV; ++i) {
         mbar_init(bar_kvfull + 8 * i, 1);
-        mbar_init(bar_kvempty + 8 * i, grow_row ? 2 : 1);
+        mbar_init(bar_kvempty + 8 * i, 1);
       }
-      for (int i = 0; i < kAttnS; ++i) {
+      for (int i = 0; i < 2; ++i) {
         mbar_init(bar_sfull + 8 * i, 1);
         mbar_init(bar_pfull + 8 * i, 4);
       }
-      for (int i = 0; i < 2; ++i) mbar_init(bar_odone + 8 * i, 1);
-      mbar_init(bar_ofinal, 1);
+      for (int i = 0; i < 2; ++i) mbar_init(bar_ofinal + 8 * i, 1);
+      mbar_init(bar_q1, 1);
       fence_barrier_init();
       tma_prefetch_desc(tm);
     }
@@ -386,7 +425,7 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
     asm volatile("bar.arrive 2, %0;" ::"n"(kAttnThreads) : "memory");
     pdl_wait();
     pdl_trigger();
-    const AttnLoad c{tm, sb, bar_kvfull, bar_kvempty, q0, nkb, t, h, lane};
+    const AttnLoad c{tm, sb, bar_kvfull, bar_kvempty, bar_q1, q0, nkb, t, h, lane};
     if (a.load == 2)
       attn_load_grid(a, c);
     else if (a.load == 1)
@@ -394,8 +433,8 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
     else
       attn_load_gather(a, c);
   } else {
-    if (warp == 5) {
-      tmem_alloc(smem_u32(tmem_slot), 256);    // S / P buffer k: cols 64k .. 64k + 63 (k < 3), O: 192-255
+    if (warp == 9) {
+      tmem_alloc(smem_u32(tmem_slot), kAttnTmemCols);   // tile i: S / P at 128i .. 128i + 63, O at 128i + 64 ..
       tmem_relinquish();
     }
     pdl_wait();
@@ -409,147 +448,93 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
     asm volatile("bar.sync 2, %0;" ::"n"(kAttnThreads) : "memory");
     tc_fence_after();
     tmem = *tmem_slot;
-    const uint32_t tO = tmem + 64 * kAttnS;
-    if (warp == 5) {
+    if (warp == 9) {
       // ---------------- MMA issuer ----------------
-      // S of block j+3 goes into the TMEM columns that hold P of block j; it is
-      // issued after P V of block j, and tcgen05.mma runs in issue order.  The whole
-      // warp waits on the barriers (lane 0's outcome decides for all); one elected
-      // lane issues the MMAs and commits.
+      // Per tile one S / P buffer: S of block j+1 goes into the columns that hold
+      // P of block j and is issued after P V of block j (tcgen05.mma runs in issue
+      // order), so the commit that announces S of block j+1 also means that O
+      // holds the sum up to block j.  The two tiles alternate: P V and the next S
+      // of tile 0, then of tile 1, whose P V commit also releases the K/V buffer.
+      // The whole warp waits on the barriers (lane 0's outcome decides for all);
+      // one elected lane issues the MMAs and commits.
       constexpr uint32_t IDESC_S = idesc_make(1u, kAttnBK);             // Q K^T: M 128, N 64
       constexpr uint32_t IDESC_O = idesc_make(1u, 64) | (1u << 16);     // P V: M 128, N 64, B MN-major
-      const uint64_t dq = sdesc_sw128(sb + AttnSmem::Q);
       const bool leader = elect_one();
-      auto issue_s = [&](int j) -> bool {
-        const int b = j % kAttnKV, sbuf = j % kAttnS;
-        if (!__shfl_sync(0xffffffffu, mbar_wait(bar_kvfull + 8 * b, (j / kAttnKV) & 1) ? 1 : 0, 0)) return false;
-        tc_fence_after();
-        if (leader) {
-          const uint64_t dk = sdesc_sw128(sb + AttnSmem::K + b * 8192);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) tc_mma_f16(tmem + sbuf * 64, dq + 2 * k, dk + 2 * k, IDESC_S, k != 0);
-          tc_commit(bar_sfull + 8 * sbuf);
-        }
-        __syncwarp();
-        return true;
+      auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
+        return __shfl_sync(0xffffffffu, mbar_wait(bar, parity) ? 1 : 0, 0) != 0;
       };
-      bool ok = true;
-      for (int j = 0; j < kAttnS && j < nkb && ok; ++j) ok = issue_s(j);
-      for (int j = 0; j < nkb && ok; ++j) {
-        const int pb = j % kAttnS, b = j % kAttnKV;
-        if (!__shfl_sync(0xffffffffu, mbar_wait(bar_pfull + 8 * pb, (j / kAttnS) & 1) ? 1 : 0, 0)) { ok = false; break; }
-        tc_fence_after();
+      auto issue_s = [&](int i, int j) {   // S of tile i, block j (K block j is in shared memory)
         if (leader) {
+          const int b = j % kAttnKV;
+          const uint64_t dq = sdesc_sw128(sb + AttnSmem::Q + i * kAttnTileQ * 128);
+          const uint64_t dk = sdesc_sw128(sb + AttnSmem::K + b * AttnSmem::KV_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t dv = sdesc_sw128_mn(sb + AttnSmem::V + b * 8192 + kk * 2048);
-            tc_mma_f16_tmem_a(tO, tmem + pb * 64 + kk * 8, dv, IDESC_O, (j | kk) != 0);
-          }
-          tc_commit(bar_odone + 8 * (j & 1));
-          tc_commit(bar_kvempty + 8 * b);
+          for (int k = 0; k < 4; ++k) tc_mma_f16(tmem + i * kAttnTmemTile, dq + 2 * k, dk + 2 * k, IDESC_S, k != 0);
+          tc_commit(bar_sfull + 8 * i);
         }
         __syncwarp();
-        if (j + kAttnS < nkb) ok = issue_s(j + kAttnS);
-      }
-      // single-phase barrier: waiters may arrive any number of phases early
-      if (ok && leader) tc_commit(bar_ofinal);
-    } else if (warp >= 6) {
-      // ---------------- global token's query row (query block 0 only) ----------------
-      // Warp 6 + g takes blocks g, g + 2, ...: lane l scores keys l and l + 32 with
-      // the full query in registers, then accumulates channels 2l, 2l + 1 of P V.
-      // The two warps' online-softmax states are merged at the end.
-      if (grow_row) {
-        const int g = warp - 6;
-        float qf[64];
-        {
-          const uint4* qr = reinterpret_cast<const uint4*>(qkv + static_cast<size_t>(attn_row(a, t, 0)) * ld + h * 64);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) bf16x8_to_f32(qr[c], qf + 8 * c);
-        }
-        float gm = -INFINITY, gl = 0.f, ga0 = 0.f, ga1 = 0.f;
-        if (g == 0) {   // the global key itself
-          float sg = 0.f;
-#pragma unroll
-          for (int c = 0; c < 64; ++c) sg = fmaf(qf[c], sKg[c], sg);
-          gm = sg * a.scale_log2;
-          gl = lane == 0 ? 1.f : 0.f;
-          ga0 = sVg[2 * lane];
-          ga1 = sVg[2 * lane + 1];
-        }
-        for (int j = g; j < nkb; j += 2) {
+      };
+      auto issue_pv = [&](int i, int j) {  // O of tile i += P V of block j
+        if (leader) {
           const int b = j % kAttnKV;
-          if (!mbar_wait(bar_kvfull + 8 * b, (j / kAttnKV) & 1)) break;
-          const uint8_t* kbuf = smem + AttnSmem::K + b * 8192;
-          const uint8_t* vbuf = smem + AttnSmem::V + b * 8192;
-          float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            float f0[8], f1[8];
-            bf16x8_to_f32(*reinterpret_cast<const uint4*>(kbuf + swz(lane, c)), f0);
-            bf16x8_to_f32(*reinterpret_cast<const uint4*>(kbuf + swz(lane + 32, c)), f1);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              s0 = fmaf(qf[8 * c + e], f0[e], s0);
-              s1 = fmaf(qf[8 * c + e], f1[e], s1);
-            }
+          for (int kk = 0; kk < kAttnBK / 16; ++kk) {
+            const uint64_t dv = sdesc_sw128_mn(sb + AttnSmem::V + b * AttnSmem::KV_BYTES + kk * 2048);
+            tc_mma_f16_tmem_a(tmem + i * kAttnTmemTile + 64, tmem + i * kAttnTmemTile + kk * 8, dv, IDESC_O,
+                              (j | kk) != 0);
           }
-          const int nvalid = min(kAttnBK, a.Nw - j * kAttnBK);
-          const float x0 = lane < nvalid ? s0 * a.scale_log2 : -INFINITY;
-          const float x1 = lane + 32 < nvalid ? s1 * a.scale_log2 : -INFINITY;
-          const float mnew = fmaxf(gm, warp_max(fmaxf(x0, x1)));
-          const float al = ex2_approx(gm - mnew);
-          const float p0 = ex2_approx(x0 - mnew), p1 = ex2_approx(x1 - mnew);
-          gl = fmaf(gl, al, p0 + p1);
-          ga0 *= al;
-          ga1 *= al;
-#pragma unroll 8
-          for (int k = 0; k < kAttnBK; ++k) {
-            const float pk = __shfl_sync(0xffffffffu, k < 32 ? p0 : p1, k & 31);
-            const uint32_t off = swz(k, lane >> 2) + (lane & 3) * 4;
-            const float2 vv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vbuf + off));
-            ga0 = fmaf(pk, vv.x, ga0);
-            ga1 = fmaf(pk, vv.y, ga1);
-          }
-          gm = mnew;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar_kvempty + 8 * b);
+          if (i == 1) tc_commit(bar_kvempty + 8 * b);
         }
-        gl = warp_sum(gl);
-        float* gbuf = reinterpret_cast<float*>(smem + AttnSmem::GR);
-        if (lane == 0) {
-          gbuf[g * 66] = gm;
-          gbuf[g * 66 + 1] = gl;
-        }
-        gbuf[g * 66 + 2 + 2 * lane] = ga0;
-        gbuf[g * 66 + 3 + 2 * lane] = ga1;
-        asm volatile("bar.sync 1, 64;" ::: "memory");
-        if (g == 0) {
-          const float M = fmaxf(gbuf[0], gbuf[66]);
-          float L = 0.f, o0 = 0.f, o1 = 0.f;
-#pragma unroll
-          for (int w = 0; w < 2; ++w) {
-            const float f = gbuf[w * 66] == -INFINITY ? 0.f : ex2_approx(gbuf[w * 66] - M);
-            L += f * gbuf[w * 66 + 1];
-            o0 += f * gbuf[w * 66 + 2 + 2 * lane];
-            o1 += f * gbuf[w * 66 + 3 + 2 * lane];
-          }
-          bf16* O = reinterpret_cast<bf16*>(a.O) + static_cast<size_t>(t) * a.N * a.d + h * 64 + 2 * lane;
-          *reinterpret_cast<__nv_bfloat162*>(O) = __floats2bfloat162_rn(o0 / L, o1 / L);
-        }
+        __syncwarp();
+      };
+      // Tile 1 starts one softmax block after tile 0 (its first S follows tile 0's
+      // first P V), so that each tile's softmax runs while the other tile waits
+      // for its P V and next S.
+      bool ok = nkb > 0 && wait_all(bar_kvfull, 0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
       }
-    } else if (warp < 4) {
+      for (int j = 0; j < nkb && ok; ++j) {
+        const bool more = j + 1 < nkb;
+        if (!wait_all(bar_pfull, j & 1)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(0, j);
+        if (!more && leader) tc_commit(bar_ofinal);
+        if (j == 0) {
+          if (!wait_all(bar_q1, 0)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(1, 0);
+        }
+        if (more) {
+          if (!wait_all(bar_kvfull + 8 * ((j + 1) % kAttnKV), ((j + 1) / kAttnKV) & 1)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        if (!wait_all(bar_pfull + 8, j & 1)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(1, j);
+        if (more) issue_s(1, j + 1);
+      }
+      // single-phase barriers: waiters may arrive any number of phases early
+      if (ok && leader) tc_commit(bar_ofinal + 8);
+    } else {
       // ---------------- softmax: one query row per thread ----------------
-      const int row = tid;                     // 0..127, TMEM lane = row
-      const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-      bool ok = mbar_wait(bar_kvfull, 0);      // Q rows are in shared memory
+      const int tile = warp >> 2;              // warps 0-3: tile 0, warps 4-7: tile 1
+      const int row = tid & 127;               // TMEM lane = row of the tile
+      const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+      const uint32_t tS = tmem + tile * kAttnTmemTile, tO = tS + 64;
+      const uint32_t sfull = bar_sfull + 8 * tile, pfull = bar_pfull + 8 * tile;
+      bool ok = mbar_wait(tile ? bar_q1 : bar_kvfull, 0);   // the tile's Q rows are in shared memory
       float m = -INFINITY, l = 0.f, gcoef = 0.f;
       if (ok) {
         // score of the global key seeds the running maximum and sum
+        const uint8_t* qrow = smem + AttnSmem::Q + tile * kAttnTileQ * 128;
         float sg = 0.f;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           float f[8];
-          bf16x8_to_f32(*reinterpret_cast<const uint4*>(smem + AttnSmem::Q + swz(row, c)), f);
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(qrow + swz(row, c)), f);
 #pragma unroll
           for (int e = 0; e < 8; ++e) sg = fmaf(f[e], sKg[c * 8 + e], sg);
         }
@@ -558,12 +543,11 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
         gcoef = 1.f;
       }
       for (int j = 0; j < nkb && ok; ++j) {
-        const int sbuf = j % kAttnS;
-        if (!mbar_wait(bar_sfull + 8 * sbuf, (j / kAttnS) & 1)) { ok = false; break; }
+        if (!mbar_wait(sfull, j & 1)) { ok = false; break; }
         tc_fence_after();
         float sv[kAttnBK];
-        tmem_ld32(tmem + sbuf * 64 + lane_off, sv);
-        tmem_ld32(tmem + sbuf * 64 + lane_off + 32, sv + 32);
+        tmem_ld32(tS + lane_off, sv);
+        tmem_ld32(tS + lane_off + 32, sv + 32);
         tmem_wait_ld();
         const int kbase = j * kAttnBK;
         // row maximum of the raw scores (the scale is positive); keys beyond the
@@ -632,11 +616,10 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
         const uint64_t s01 = add_f32x2(sp2[0], sp2[1]), s23 = add_f32x2(sp2[2], sp2[3]);
         const uint64_t s0123 = add_f32x2(s01, s23);
         l += lo_f32(s0123) + hi_f32(s0123);
-        tmem_st32u(tmem + sbuf * 64 + lane_off, pw);
+        tmem_st16u(tS + lane_off, pw);
+        tmem_st16u(tS + lane_off + 16, pw + 16);
         if (warp_grow && j >= 1) {
-          // O holds the sum up to block j-1: wait for that P V, then rescale the row
-          if (!mbar_wait(bar_odone + 8 * ((j - 1) & 1), ((j - 1) >> 1) & 1)) { ok = false; break; }
-          tc_fence_after();
+          // O holds the sum up to block j-1 (its P V ran before this block's S): rescale the row
 #pragma unroll 1
           for (int hh = 0; hh < 4; ++hh) {
             float o[16];
@@ -650,11 +633,11 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_pfull + 8 * sbuf);
+        if (lane == 0) mbar_arrive(pfull);
       }
-      if (ok && mbar_wait(bar_ofinal, 0)) {
+      if (ok && mbar_wait(bar_ofinal + 8 * tile, 0)) {
         tc_fence_after();
-        const int slot = q0 + row;
+        const int slot = q0 + tile * kAttnTileQ + row;
         const float inv = 1.f / l;
         bf16* dst = reinterpret_cast<bf16*>(a.O) + (static_cast<size_t>(t) * a.N + slot) * a.d + h * 64;
 #pragma unroll 1
@@ -677,22 +660,155 @@ __device__ __forceinline__ void attn_window_block_tc(const CUtensorMap* tm, cons
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, kAttnTmemCols);
   }
 }
 
-__global__ void __launch_bounds__(kAttnThreads, 2)
+// ---------------------------------------------------------------------------
+// the global token's own query row (slot 0) of tile t, head h
+// ---------------------------------------------------------------------------
+// Warp 8 streams the K/V blocks into the four shared buffers exactly as for a
+// window block (no Q); warps w and w + 4 (w < 4) take the blocks of buffer w, w + 4,
+// ..., keys 0-31 and 32-63 of each: lane l scores one key against the query (in
+// shared memory), the warp's online softmax moves by the maximum over its 32 keys,
+// and lane l accumulates channels 2l, 2l + 1 of P V from the shared V rows.  The
+// eight warps' states are merged in warp order.
+__device__ __forceinline__ void attn_global_block(const CUtensorMap* tm, const AttnArgs& a, int h, int t,
+                                                  uint8_t* smem) {
+  const bf16* qkv = reinterpret_cast<const bf16*>(a.qkv);
+  const size_t ld = static_cast<size_t>(3) * a.d;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t bar_kvfull = sb + AttnSmem::BAR;        // kAttnKV, count 1 (producer's expect_tx) + TMA bytes
+  const uint32_t bar_kvempty = bar_kvfull + 8 * kAttnKV; // kAttnKV, count 2 (the two warps that read the block)
+  float* sKg = reinterpret_cast<float*>(smem + AttnSmem::KG);
+  float* sVg = sKg + 64;
+  float* gbuf = reinterpret_cast<float*>(smem + AttnSmem::Q);   // 8 x 66 floats: the warps' states
+  float* sQg = gbuf + 8 * 66 + 8;                                // 64 floats: the global query (16-byte aligned)
+  const int nkb = (a.Nw + kAttnBK - 1) / kAttnBK;
+  constexpr int kWarps = 8;
+  if (warp == 8) {
+    if (lane == 0) {
+      for (int i = 0; i < kAttnKV; ++i) {
+        mbar_init(bar_kvfull + 8 * i, 1);
+        mbar_init(bar_kvempty + 8 * i, 2);
+      }
+      fence_barrier_init();
+      tma_prefetch_desc(tm);
+    }
+    __syncwarp();
+    asm volatile("bar.arrive 2, %0;" ::"n"(kAttnThreads) : "memory");
+    pdl_wait();
+    pdl_trigger();
+    const AttnLoad c{tm, sb, bar_kvfull, bar_kvempty, 0u, 1, nkb, t, h, lane};
+    if (a.load == 2)
+      attn_load_grid(a, c);
+    else if (a.load == 1)
+      attn_load_runs(a, c);
+    else
+      attn_load_gather(a, c);
+  } else {
+    pdl_wait();
+    pdl_trigger();
+    const size_t grow = static_cast<size_t>(attn_row(a, t, 0)) * ld + h * 64;
+    if (tid < 64) {
+      sQg[tid] = __bfloat162float(qkv[grow + tid]);
+      sKg[tid] = __bfloat162float(qkv[grow + a.d + tid]);
+      sVg[tid] = __bfloat162float(qkv[grow + 2 * a.d + tid]);
+    }
+    asm volatile("bar.sync 2, %0;" ::"n"(kAttnThreads) : "memory");
+    if (warp < kWarps) {
+      float gm = -INFINITY, gl = 0.f, ga0 = 0.f, ga1 = 0.f;
+      if (warp == 0) {   // the global key itself
+        float sg = 0.f;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) sg = fmaf(sQg[c], sKg[c], sg);
+        gm = sg * a.scale_log2;
+        gl = lane == 0 ? 1.f : 0.f;
+        ga0 = sVg[2 * lane];
+        ga1 = sVg[2 * lane + 1];
+      }
+      // warps w and w + 4 share the blocks of buffer w % 4, keys 0-31 and 32-63:
+      // each waits on every phase of its buffer's barrier, in order
+      const int half = warp >> 2, key = half * 32 + lane;
+      for (int j = warp & 3; j < nkb; j += kAttnKV) {
+        const int b = j % kAttnKV;
+        if (!mbar_wait(bar_kvfull + 8 * b, (j / kAttnKV) & 1)) break;
+        const uint8_t* kbuf = smem + AttnSmem::K + b * AttnSmem::KV_BYTES;
+        const uint8_t* vbuf = smem + AttnSmem::V + b * AttnSmem::KV_BYTES;
+        float s0 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float f0[8];
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(kbuf + swz(key, c)), f0);
+          const float4 qa = *reinterpret_cast<const float4*>(sQg + 8 * c);
+          const float4 qb = *reinterpret_cast<const float4*>(sQg + 8 * c + 4);
+          const float q8[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) s0 = fmaf(q8[e], f0[e], s0);
+        }
+        const int nvalid = min(kAttnBK, a.Nw - j * kAttnBK);
+        const float x0 = key < nvalid ? s0 * a.scale_log2 : -INFINITY;
+        const float bm = warp_max(x0);
+        if (bm != -INFINITY) {           // the second half of a last, short block may hold no key
+          const float mnew = fmaxf(gm, bm);
+          const float al = ex2_approx(gm - mnew);
+          const float p0 = ex2_approx(x0 - mnew);
+          gl = fmaf(gl, al, p0);
+          ga0 *= al;
+          ga1 *= al;
+#pragma unroll 8
+          for (int k = 0; k < 32; ++k) {
+            const float pk = __shfl_sync(0xffffffffu, p0, k);
+            const uint32_t off = swz(half * 32 + k, lane >> 2) + (lane & 3) * 4;
+            const float2 vv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vbuf + off));
+            ga0 = fmaf(pk, vv.x, ga0);
+            ga1 = fmaf(pk, vv.y, ga1);
+          }
+          gm = mnew;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_kvempty + 8 * b);
+      }
+      gl = warp_sum(gl);
+      if (lane == 0) {
+        gbuf[warp * 66] = gm;
+        gbuf[warp * 66 + 1] = gl;
+      }
+      gbuf[warp * 66 + 2 + 2 * lane] = ga0;
+      gbuf[warp * 66 + 3 + 2 * lane] = ga1;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, gbuf[w * 66]);
+    float L = 0.f, o0 = 0.f, o1 = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float f = gbuf[w * 66] == -INFINITY ? 0.f : ex2_approx(gbuf[w * 66] - M);
+      L = fmaf(f, gbuf[w * 66 + 1], L);
+      o0 = fmaf(f, gbuf[w * 66 + 2 + 2 * lane], o0);
+      o1 = fmaf(f, gbuf[w * 66 + 3 + 2 * lane], o1);
+    }
+    bf16* O = reinterpret_cast<bf16*>(a.O) + static_cast<size_t>(t) * a.N * a.d + h * 64 + 2 * lane;
+    *reinterpret_cast<__nv_bfloat162*>(O) = __floats2bfloat162_rn(o0 / L, o1 / L);
+  }
+}
+
+__global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
     attn_bf16_kernel(const __grid_constant__ CUtensorMap tm, const AttnArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = smem_raw;
-  if (smem_u32(smem) & 1023u) {          // swizzled tiles need a 1024-byte aligned base
-    if (threadIdx.x == 0) set_status(kStatusDeviceCheck);
-    return;
-  }
+  // swizzled tiles need a 1024-byte aligned base: round up inside the launch's slack
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int h = a.head_major ? blockIdx.z : blockIdx.y, t = a.head_major ? blockIdx.y : blockIdx.z;
-  attn_window_block_tc(&tm, a, blockIdx.x, h, t, smem);
+  if (static_cast<int>(blockIdx.x) == a.nqb)
+    attn_global_block(&tm, a, h, t, smem);
+  else
+    attn_window_block_tc(&tm, a, blockIdx.x, h, t, smem);
 }
 
 // ---------------------------------------------------------------------------

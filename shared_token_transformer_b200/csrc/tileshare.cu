@@ -742,30 +742,34 @@ static ts_status run_attention(const ts_plan_s* p, const ts_model_desc* m, bool 
   if (dev < 64 && !configured[dev]) {
     TS_CUDA_CHECK(cudaFuncSetAttribute(ts::attn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        ts::AttnSmem::LAUNCH_BYTES));
+    // four CTAs per SM need the largest shared-memory carveout
+    TS_CUDA_CHECK(cudaFuncSetAttribute(ts::attn_bf16_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                       cudaSharedmemCarveoutMaxShared));
     configured[dev] = 1;
   }
-  // map over the q/k/v rows: a 128-byte column box, `run` rows high for runs of
-  // consecutive rows (the per-tile layout is one run per tile), one row high for
-  // four-row gathers
-  // Loads: a block of 64 window slots that is whole window rows of one frame is
-  // one box of a 3-D map over the grid; otherwise runs of consecutive rows are
-  // 2-D boxes (the per-tile layout is one run per tile), else four-row gathers.
+  // Loads: a block of 32 window slots that is whole window rows of one frame (or
+  // a part of one row) is one box of a 3-D map over the grid; otherwise runs of
+  // consecutive rows are 2-D boxes of `run` rows (the per-tile layout is one run
+  // per block), else four-row gathers through a map with one-row boxes.
   const int wx = p->win[2], wy = p->win[1];
-  const bool grid_box = p->R == 1 && (wx <= 64 ? (64 % wx == 0 && (wy * wx) % 64 == 0) : wx % 64 == 0);
+  const int bk = ts::kAttnBK;
+  const bool grid_box = p->R == 1 && (wx <= bk ? (bk % wx == 0 && (wy * wx) % bk == 0) : wx % bk == 0);
   CUtensorMap tm;
   if (shared && grid_box) {
     a.load = 2;
     a.gw = p->grid[2];
-    const int bx = std::min(wx, 64);
-    TS_TRY(make_tmap_grid(&tm, qkv, 3 * m->d, p->grid[2], p->grid[0] * p->grid[1], bx, 64 / bx));
+    const int bx = std::min(wx, bk);
+    TS_TRY(make_tmap_grid(&tm, qkv, 3 * m->d, p->grid[2], p->grid[0] * p->grid[1], bx, bk / bx));
   } else {
-    a.run = shared ? p->run : 64;
+    a.run = shared ? std::min(p->run, bk) : bk;   // runs of 64 consecutive rows are runs of 32 as well
     a.load = a.run > 0 ? 1 : 0;
     TS_TRY(make_tmap(&tm, qkv, shared ? p->U + p->G : p->T * p->N, 3 * m->d, 2, a.run > 0 ? a.run : 1));
   }
   a.head_major = shared ? 1 : 0;
-  dim3 grid = shared ? dim3(nqb, p->T, m->heads)    // head slowest: neighbouring tiles of one head share L2
-                     : dim3(nqb, m->heads, p->T);   // tile slowest: a tile's rows are read once for all heads
+  a.nqb = nqb;
+  // block x = nqb of each tile and head computes the global token's query row
+  dim3 grid = shared ? dim3(nqb + 1, p->T, m->heads)    // head slowest: neighbouring tiles of one head share L2
+                     : dim3(nqb + 1, m->heads, p->T);   // tile slowest: a tile's rows are read once for all heads
   launch_pdl(ts::attn_bf16_kernel, grid, dim3(ts::kAttnThreads), ts::AttnSmem::LAUNCH_BYTES, st, tm, a);
   return trace_post(st, "attn_bf16");
 }
