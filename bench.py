@@ -21,7 +21,8 @@ roofline  per kernel class from a traced pass (library kernel trace: CUDA events
          around each launch, algorithmic FLOPs / HBM bytes per launch); the
          dominant class (most time) is reported against MEASURED_PEAKS.json: the
          burst bf16 figure when the traced pass lasts under a second, the
-         sustained one otherwise; fp32 kernels against the FP32 SIMT peak.
+         sustained one otherwise (frac_vs_burst and frac_vs_sustained give
+         both); fp32 kernels against the FP32 SIMT peak.
 cpu_baseline  the float64 CPU oracle's shared layer on the same inputs (rank 0,
          N = 1): whole layers when one fits the budget, else a bounded sample
          (per-token steps on blocks of rows, attention of whole tiles, the whole
@@ -620,6 +621,11 @@ def run_tileshare(args, rank, world, local):
     roofline = {"bound": bound, "kernel": dom, "achieved": kd["achieved"],
                 "peak": round(tensor_peak_of(dom) if kd["unit"] == "TFLOP/s" else pk["hbm_gbs"], 1), "unit": kd["unit"],
                 "frac": kd["frac"], "traffic": traffic, "peak_source": peak_source(dom, kd["unit"])}
+    if kd["unit"] == "TFLOP/s" and cfg.dtype != "f32" and "bf16_tflops_sustained" in pk:
+        # both measured bf16 figures, since a traced pass near one second could take either
+        scale = tensor_peak_of(dom) / bf16_peak
+        roofline["frac_vs_burst"] = round(kd["achieved"] / (scale * pk["bf16_tflops"]), 4)
+        roofline["frac_vs_sustained"] = round(kd["achieved"] / (scale * pk["bf16_tflops_sustained"]), 4)
 
     gated = cfg.block == "rms_swiglu"
     ft = flops_layer(T * N, T, N, d, f, gated)
