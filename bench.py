@@ -28,6 +28,9 @@ cpu_baseline  the float64 CPU oracle's shared layer on the same inputs (rank 0,
          (per-token steps on blocks of rows, attention of whole tiles, the whole
          blend) scaled to the layer.  --impl reference times that oracle alone as
          the reference arm, each step a bounded sample of the same kind.
+         --cpu-detail times the oracle alone on the host cores (no GPU): one
+         shared and one per-tile layer, and the whole stack where it ends within
+         15 minutes.
 
 Multi-GPU (torchrun): every rank decodes its own image (independent inputs, the
 same weights); there is no data-path collective, only a barrier and a max of the
@@ -66,6 +69,8 @@ def parse():
     ap.add_argument("--no-graph", action="store_true", help="launch the calls eagerly instead of CUDA graphs")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-detail", action="store_true",
+                    help="oracle timings only (host cores, no GPU): shared and per-tile layer, whole stack")
     ap.add_argument("--trace-steps", type=int, default=20)
     ap.add_argument("--shared-ops", default=None,
                     help="partial sharing from layer k on: comma list of qkv,out,mlp ('none': nothing shared) run "
@@ -253,6 +258,82 @@ def oracle_layer_sample_seconds(op, S, layer, om, budget_s, row_block=1024):
     what = (f"per-token steps on {rows} of {M} rows, attention of {tiles} of {T} tiles, the whole blend; "
             f"each scaled by its share of the layer")
     return sec, what
+
+
+def oracle_tiled_layer_sample_seconds(op, X, layer, om, budget_s, row_block=1024):
+    """Seconds of one float64 oracle per-tile layer on X [T, N, d], estimated from a
+    bounded sample: per-token steps (Norm1, QKV, QK-RMSNorm, out-projection, MLP) on
+    blocks of the T*N tile rows and attention of whole tiles, each timed in turn until
+    it has used half the budget or all of its work and scaled by (all its units /
+    units timed).  Returns (seconds, description)."""
+    from oracle import layers as OL
+    T, N = X.shape[0], X.shape[1]
+    R = X.reshape(T * N, X.shape[2])
+    t_tok = t_att = 0.0
+    rows = tiles = 0
+    half = budget_s / 2
+    while rows < R.shape[0] and (rows == 0 or t_tok < half):
+        x = R[rows: rows + row_block]
+        t0 = time.perf_counter()
+        OL.qkv_project(x, layer, om)
+        y = x + OL.linear(x, layer["w_o"], layer["b_o"], om)
+        OL.mlp_residual(y, layer, om)
+        t_tok += time.perf_counter() - t0
+        rows += x.shape[0]
+    while tiles < T and (tiles == 0 or t_att < half):
+        q, k, v = OL.qkv_project(X[tiles], layer, om)               # untimed: counted with the rows
+        t0 = time.perf_counter()
+        OL.tile_attention(q, k, v, op.slot_pos, om)
+        t_att += time.perf_counter() - t0
+        tiles += 1
+    sec = t_tok * (T * N) / rows + t_att * T / tiles
+    return sec, (f"per-token steps on {rows} of {T * N} tile rows, attention of {tiles} of {T} tiles; "
+                 f"each scaled by its share of the layer")
+
+
+def run_cpu_detail(args, cfg, budget_s=300.0, stack_limit_s=900.0):
+    """Oracle timings of the workload on the host cores (no GPU): one shared layer and
+    one per-tile layer, whole when the estimate fits budget_s, else a bounded sample,
+    and the whole TileShare-k stack when its estimate is under stack_limit_s."""
+    from oracle import layers as OL
+    from shared_token_transformer_b200 import workloads as W
+    op, S, layer, om = _oracle_inputs(cfg, args.blend)
+    res = {"impl": "oracle-detail", "config": cfg.name, "L": cfg.L, "k": cfg.k, "unique_tokens": op.U,
+           "tiles": op.T, "rows_per_tile": op.N, "dtype": "f64", "cores": os.cpu_count(),
+           "blas_threads": blas_threads(),
+           "note": "the oracle computes in float64 by definition; it has no float32 form to time"}
+    est, _ = oracle_layer_sample_seconds(op, S, layer, om, min(budget_s, 4.0))
+    if est <= budget_s:
+        t0 = time.perf_counter()
+        OL.block_shared(S, layer, om, op)
+        sh, how = time.perf_counter() - t0, "one whole layer"
+    else:
+        sh, how = oracle_layer_sample_seconds(op, S, layer, om, budget_s)
+        how = "bounded sample: " + how
+    res.update(shared_layer_s=round(sh, 3), shared_layer_unique_tok_s=round(op.U / sh, 2), shared_layer_how=how)
+    X = OL.gather(S, op)
+    est, _ = oracle_tiled_layer_sample_seconds(op, X, layer, om, min(budget_s, 4.0))
+    if est <= budget_s:
+        t0 = time.perf_counter()
+        OL.block_tiled(X, layer, om, op)
+        ti, how = time.perf_counter() - t0, "one whole layer"
+    else:
+        ti, how = oracle_tiled_layer_sample_seconds(op, X, layer, om, budget_s)
+        how = "bounded sample: " + how
+    res.update(tiled_layer_s=round(ti, 3), tiled_layer_how=how)
+    est_stack = cfg.k * ti + (cfg.L - cfg.k) * sh
+    res["stack_estimate_s"] = round(est_stack, 1)
+    if est_stack <= stack_limit_s:
+        dr = W.Draw(cfg, op.T, seed=0)
+        S0, G0 = dr.states()
+        layers = dr.layers()
+        t0 = time.perf_counter()
+        OL.decode_stack(S0, G0, layers, om, op, cfg.k)
+        res["stack_s"] = round(time.perf_counter() - t0, 3)
+    else:
+        res["stack_s"] = None
+        res["stack_note"] = f"not run: estimated {est_stack:.0f} s, above {stack_limit_s:.0f} s"
+    return res
 
 
 def oracle_shared_layer_timing(cfg, budget_s, max_steps, warmup=1, rule="ramp"):
@@ -757,6 +838,10 @@ def main():
         if rank != 0:
             return
         print(json.dumps(run_reference(args, cfg, world)))
+        return
+    if args.cpu_detail:
+        if rank == 0:
+            print(json.dumps(run_cpu_detail(args, cfg)))
         return
 
     import torch.distributed as dist

@@ -86,3 +86,28 @@ def test_oracle_sample_covers_the_whole_layer_when_the_budget_allows():
     # a tiny budget still times one row block and one tile
     sec, what = bench.oracle_layer_sample_seconds(op, S, layer, om, budget_s=1e-9, row_block=64)
     assert f"64 of {S.shape[0]} rows" in what and f"1 of {op.T} tiles" in what
+
+
+def test_oracle_tiled_sample_covers_the_whole_layer_when_the_budget_allows():
+    cfg = bench.config_of(_Args("vit14_fp32"))
+    op, S, layer, om = bench._oracle_inputs(cfg, "ramp")
+    from oracle import layers as OL
+    X = OL.gather(S, op)
+    sec, what = bench.oracle_tiled_layer_sample_seconds(op, X, layer, om, budget_s=1e9, row_block=64)
+    assert sec > 0
+    assert f"{op.T * op.N} of {op.T * op.N} tile rows" in what and f"{op.T} of {op.T} tiles" in what
+    sec, what = bench.oracle_tiled_layer_sample_seconds(op, X, layer, om, budget_s=1e-9, row_block=64)
+    assert f"64 of {op.T * op.N} tile rows" in what and f"1 of {op.T} tiles" in what
+
+
+def test_cpu_detail_times_both_layers_and_the_stack():
+    a = _Args("vit14_fp32")
+    a.blend = "ramp"
+    cfg = bench.config_of(a)
+    res = bench.run_cpu_detail(a, cfg, budget_s=60.0, stack_limit_s=60.0)
+    assert res["dtype"] == "f64" and res["cores"] >= 1
+    assert res["shared_layer_s"] > 0 and res["tiled_layer_s"] > 0 and res["stack_s"] > 0
+    assert res["shared_layer_how"] == "one whole layer" and res["tiled_layer_how"] == "one whole layer"
+    res = bench.run_cpu_detail(a, cfg, budget_s=1e-9, stack_limit_s=0.0)
+    assert res["shared_layer_how"].startswith("bounded sample") and res["tiled_layer_how"].startswith("bounded sample")
+    assert res["stack_s"] is None and "not run" in res["stack_note"]
