@@ -28,9 +28,8 @@ cpu_baseline  the float64 CPU oracle's shared layer on the same inputs (rank 0,
          (per-token steps on blocks of rows, attention of whole tiles, the whole
          blend) scaled to the layer.  --impl reference times that oracle alone as
          the reference arm, each step a bounded sample of the same kind.
-         --cpu-detail times the oracle alone on the host cores (no GPU): one
-         shared and one per-tile layer, and the whole stack where it ends within
-         15 minutes.
+         With --cpu-detail the reference arm times one shared and one per-tile
+         oracle layer and the whole stack where it ends within 15 minutes.
 
 Multi-GPU (torchrun): every rank decodes its own image (independent inputs, the
 same weights); there is no data-path collective, only a barrier and a max of the
@@ -70,7 +69,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-detail", action="store_true",
-                    help="oracle timings only (host cores, no GPU): shared and per-tile layer, whole stack")
+                    help="with --impl reference: the oracle's shared and per-tile layer and whole stack")
     ap.add_argument("--trace-steps", type=int, default=20)
     ap.add_argument("--shared-ops", default=None,
                     help="partial sharing from layer k on: comma list of qkv,out,mlp ('none': nothing shared) run "
@@ -292,13 +291,14 @@ def oracle_tiled_layer_sample_seconds(op, X, layer, om, budget_s, row_block=1024
 
 
 def run_cpu_detail(args, cfg, budget_s=300.0, stack_limit_s=900.0):
-    """Oracle timings of the workload on the host cores (no GPU): one shared layer and
-    one per-tile layer, whole when the estimate fits budget_s, else a bounded sample,
-    and the whole TileShare-k stack when its estimate is under stack_limit_s."""
+    """The reference arm's detailed form (--impl reference --cpu-detail): oracle timings
+    of the workload on the host cores, one shared layer and one per-tile layer, whole
+    when the estimate fits budget_s, else a bounded sample, and the whole TileShare-k
+    stack when its estimate is under stack_limit_s."""
     from oracle import layers as OL
     from shared_token_transformer_b200 import workloads as W
     op, S, layer, om = _oracle_inputs(cfg, args.blend)
-    res = {"impl": "oracle-detail", "config": cfg.name, "L": cfg.L, "k": cfg.k, "unique_tokens": op.U,
+    res = {"impl": "reference", "kind": "oracle-detail", "config": cfg.name, "L": cfg.L, "k": cfg.k, "unique_tokens": op.U,
            "tiles": op.T, "rows_per_tile": op.N, "dtype": "f64", "cores": os.cpu_count(),
            "blas_threads": blas_threads(),
            "note": "the oracle computes in float64 by definition; it has no float32 form to time"}
@@ -834,14 +834,12 @@ def main():
     from shared_token_transformer_b200 import workloads as W
     cfg = config_of(args)
 
+    if args.cpu_detail and args.impl != "reference":
+        raise SystemExit("--cpu-detail is a form of the reference arm: add --impl reference")
     if args.impl == "reference":
         if rank != 0:
             return
-        print(json.dumps(run_reference(args, cfg, world)))
-        return
-    if args.cpu_detail:
-        if rank == 0:
-            print(json.dumps(run_cpu_detail(args, cfg)))
+        print(json.dumps(run_cpu_detail(args, cfg) if args.cpu_detail else run_reference(args, cfg, world)))
         return
 
     import torch.distributed as dist
